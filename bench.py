@@ -1,0 +1,595 @@
+"""Benchmark of the FSDP2 per-parameter sharding step on B200.
+
+One step = for every parameter group of the model, in order:
+  copy-in (fp32 shards -> bf16 rank-major all-gather buffer),
+  copy-out (all-gather buffer -> unsharded bf16 parameters),
+  reduce-scatter (N ranks' bf16 gradients -> fp32 reduced shards, AVG, fused
+  pack + rank-ordered fold),
+  AdamW (fp32 master, m, v shards),
+with the N data-parallel ranks emulated as N virtual ranks in one GPU's HBM.
+The default workload is the 7B-shaped model: 32 Llama-2-7B blocks plus the
+root group (embedding, final norm, LM head), N = 8, 6.74 G parameters.
+
+Byte model (algorithmic bytes a group step must move, each once):
+  B = 6*Pp (copy-in) + 2*Pp + 2*P (copy-out) + 2*N*P + 4*Pp (reduce-scatter)
+      + 28*Pp (AdamW),     Pp = N*S padded elements, P real elements.
+Reported value = total bytes of the step / step time (GB/s, 1e9 bytes).
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs its own full workload (no data-path
+collective; weak scaling) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FSDP2 step GB/s and params/s over N virtual ranks; % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+KERNELS_SRC = os.path.join(ROOT, "fully_sharded_shard_b200", "csrc", "fsdpk_kernels.cu")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "dram_traffic.json")
+
+
+# ---------------------------------------------------------------------------
+# byte model
+# ---------------------------------------------------------------------------
+def stage_bytes(N: int, S: int, P: int) -> dict:
+    Pp = N * S
+    return {
+        "copy_in": 6 * Pp,
+        "copy_out": 2 * Pp + 2 * P,
+        "rs_reduce": 2 * N * P + 4 * Pp,
+        "adamw": 28 * Pp,
+    }
+
+
+def group_bytes(N: int, S: int, P: int) -> int:
+    return sum(stage_bytes(N, S, P).values())
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str):
+    import datetime
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, traffic record
+# ---------------------------------------------------------------------------
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        maxp = max(r[2] for r in rows)
+        load = [r for r in rows if r[2] >= 0.5 * maxp] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in load for k in range(4) if r[3][k].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": maxp}
+
+
+def kernels_hash() -> str:
+    with open(KERNELS_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
+    when it is absent or the kernels changed since it was captured."""
+    try:
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernels_sha256_16") != kernels_hash() or rec.get("workload") != workload:
+        return None
+    k = rec.get("per_launch_bytes", {}).get(kernel)
+    return float(k) if k is not None else None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Model:
+    """Device state of one workload replica: plans, fp32 sharded state per
+    group instance, shared working buffers and a pool of gradient buffers."""
+
+    def __init__(self, wl, device, grad_pool: int, rank: int):
+        import torch
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200 import workloads as W
+        self.wl = wl
+        self.device = device
+        self.plans = []            # one abi.Group per distinct group
+        self.instances = []        # (plan index, master, m, v, grad pool index)
+        N = wl.N
+        max_NS = 0
+        max_A = 0
+        for gi, grp in enumerate(wl.groups):
+            g = abi.fsdp_plan_group(grp.shapes, N)
+            self.plans.append(g)
+            max_NS = max(max_NS, N * g.S)
+            max_A = max(max_A, g.P_arena)
+        self.ag = torch.empty(max(max_NS, 1), dtype=torch.bfloat16, device=device)
+        self.arena = torch.empty(max(max_A, 1), dtype=torch.bfloat16, device=device)
+        self.reduced = torch.empty(max(max_NS, 1), dtype=torch.float32, device=device)
+        full = torch.empty(max(max_A, 1), dtype=torch.float32, device=device)
+        # gradient pools: per plan, up to `grad_pool` distinct seeded buffers
+        self.grads = []
+        for gi, grp in enumerate(wl.groups):
+            g = self.plans[gi]
+            k = max(1, min(grad_pool, grp.repeat))
+            pool = []
+            for j in range(k):
+                t = torch.empty(N, g.P_arena, dtype=torch.bfloat16, device=device)
+                for r in range(N):
+                    W.fill_grads_bf16(t[r], wl, grp.name, "rank", rank, "pool", j, r)
+                    if grp.zero_grad:
+                        W.zero_param_ranges(t[r], g.arena_off, g.numel, grp.zero_grad)
+                pool.append(t)
+            self.grads.append(pool)
+        for gi, grp in enumerate(wl.groups):
+            g = self.plans[gi]
+            for rep in range(grp.repeat):
+                NS = N * g.S
+                master = torch.empty(NS, dtype=torch.float32, device=device)
+                W.fill_master(full[:g.P_arena], wl, grp.name, "rank", rank, "layer", rep)
+                abi.fsdp_shard_params(self.plans[gi], full, master)
+                m = torch.zeros(NS, dtype=torch.float32, device=device)
+                v = torch.zeros(NS, dtype=torch.float32, device=device)
+                self.instances.append((gi, master, m, v, rep % len(self.grads[gi])))
+        del full
+        torch.cuda.synchronize(device)
+        self.step_count = 0
+        self.P_total = sum(self.plans[i[0]].P for i in self.instances)
+        self.bytes_per_step = sum(group_bytes(N, self.plans[i[0]].S, self.plans[i[0]].P)
+                                  for i in self.instances)
+        self.stage_bytes = {k: 0 for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
+        for i in self.instances:
+            g = self.plans[i[0]]
+            for k, b in stage_bytes(N, g.S, g.P).items():
+                self.stage_bytes[k] += b
+        self.launches_per_step = 4 * len(self.instances)
+
+    def run_group(self, idx, stream, step, grads=None, events=None):
+        """Enqueue the four stages of group instance `idx` on `stream`.
+        events: optional dict stage -> list receiving (start, end) events."""
+        import torch
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200 import workloads as W
+        gi, master, m, v, pj = self.instances[idx]
+        g = self.plans[gi]
+        if grads is None:
+            grads = self.grads[gi][pj]
+        hp = dict(W.ADAMW_DEFAULTS)
+        calls = (
+            ("copy_in", lambda: abi.fsdp_copy_in(g, master, self.ag, stream)),
+            ("copy_out", lambda: abi.fsdp_copy_out(g, self.ag, self.arena, stream)),
+            ("rs_reduce", lambda: abi.fsdp_rs_reduce(g, grads, self.wl.op, self.reduced,
+                                                     stream=stream)),
+            ("adamw", lambda: abi.fsdp_adamw_step(g, master, m, v, self.reduced, step=step,
+                                                  stream=stream, **hp)),
+        )
+        for name, fn in calls:
+            if events is None:
+                fn()
+            else:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                events[name].append((e0, e1))
+
+    def step(self, stream, events=None):
+        """Enqueue one full step (every group, in order) on `stream`."""
+        self.step_count += 1
+        for idx in range(len(self.instances)):
+            self.run_group(idx, stream, self.step_count, events=events)
+
+
+def run_ours(args, wl, device, rank, ws):
+    import torch
+    from fully_sharded_shard_b200 import workloads as W
+    stream = torch.cuda.Stream(device)
+    t_setup = time.time()
+    model = Model(wl, device, args.grad_pool, rank)
+    setup_s = time.time() - t_setup
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            model.step(stream)
+    torch.cuda.synchronize(device)
+
+    # timed region: K whole steps between two events on the launching stream
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        model.step(stream)
+    e_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    ms_total = e_start.elapsed_time(e_end)
+    ms_total = max_over_ranks(ms_total, device)
+    ms_step = ms_total / args.steps
+
+    # per-stage times: the same steps again with events around every launch
+    events = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
+    stage_steps = max(1, min(args.steps, 3))
+    for _ in range(stage_steps):
+        model.step(stream, events=events)
+    torch.cuda.synchronize(device)
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / stage_steps for k, v in events.items()}
+
+    peak, peak_kind = hbm_peak()
+    gbs = ws * model.bytes_per_step / (ms_step * 1e-3) / 1e9
+    params_s = ws * model.P_total / (ms_step * 1e-3)
+    dom = max(stage_ms, key=stage_ms.get)
+    dom_launch_ms = stage_ms[dom] / len(model.instances)
+    dom_achieved = model.stage_bytes[dom] / (stage_ms[dom] * 1e-3) / 1e9
+    kernel_names = {"copy_in": "k_copy_in", "copy_out": "k_copy_out",
+                    "rs_reduce": "k_reduce_units", "adamw": "k_adamw"}
+    traffic = recorded_traffic(kernel_names[dom], wl.name)
+    roofline = {
+        "bound": "hbm", "kernel": kernel_names[dom], "achieved": round(dom_achieved, 1),
+        "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+        "frac": round(dom_achieved / peak, 4),
+        "algorithmic_bytes_per_launch": int(model.stage_bytes[dom] / len(model.instances)),
+        "avg_launch_ms": round(dom_launch_ms, 4),
+        "traffic": traffic,
+    }
+    stages = {k: {"ms_per_step": round(stage_ms[k], 3),
+                  "GBps": round(model.stage_bytes[k] / (stage_ms[k] * 1e-3) / 1e9, 1),
+                  "frac_of_peak": round(model.stage_bytes[k] / (stage_ms[k] * 1e-3) / 1e9 / peak, 4)}
+              for k in stage_ms}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, model, device, stream, ws)
+
+    out = {
+        "metric": METRIC,
+        "value": round(gbs, 1),
+        "unit": "GB/s",
+        "params_per_s": round(params_s, 1),
+        "hbm_frac_of_measured": round(gbs / ws / peak, 4),
+        "hbm_frac_of_spec_8TBs": round(gbs / ws / SPEC_HBM_GBS, 4),
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32+bf16",
+        "data": "synthetic: seeded N(0,0.02) fp32 master, N(0,1e-3) bf16 per-rank grads",
+        "config": {
+            "workload": wl.name,
+            "N_virtual_ranks": wl.N,
+            "groups_per_step": len(model.instances),
+            "params": model.P_total,
+            "bytes_per_step": model.bytes_per_step,
+            "reduce_op": W.OP_NAMES[wl.op],
+            "grad_pool_per_plan": args.grad_pool,
+            "l2": "inputs larger than L2 (every group's state >> 126 MB)",
+            "parallelism": f"{ws} GPU(s), each a full {wl.N}-virtual-rank replica",
+        },
+        "stages": stages,
+        "roofline": roofline,
+        "gpu_launches": model.launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "setup_s": round(setup_s, 1),
+    }
+    return out, model
+
+
+def run_e2e(args, model, device, stream, ws):
+    """The same step through the public API with the gradients starting in
+    pinned host memory: every group's H2D copy (on a copy stream, double
+    buffered so group g+1's copy overlaps group g's kernels) and a D2H read
+    of the step's last updated parameter are inside the timed region."""
+    import torch
+    N = model.wl.N
+    host = []
+    dev = []
+    for gi, g in enumerate(model.plans):
+        h = torch.empty(N, g.P_arena, dtype=torch.bfloat16, pin_memory=True)
+        h.copy_(model.grads[gi][0])
+        host.append(h)
+        dev.append([torch.empty_like(model.grads[gi][0]) for _ in range(2)])
+    copy_stream = torch.cuda.Stream(device)
+    result = torch.empty(1, dtype=torch.float32, pin_memory=True)
+    n_inst = len(model.instances)
+    h2d_bytes = sum(host[gi].numel() * 2 for gi, *_ in model.instances)
+
+    def one_step():
+        model.step_count += 1
+        ready = [None] * n_inst   # H2D of group idx done (copy stream)
+        freed = [None] * n_inst   # group idx's kernels done with its buffer
+
+        def issue(idx):
+            gi = model.instances[idx][0]
+            buf = dev[gi][idx % 2]
+            if idx >= 2:
+                copy_stream.wait_event(freed[idx - 2])
+            with torch.cuda.stream(copy_stream):
+                buf.copy_(host[gi], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(copy_stream)
+            ready[idx] = ev
+            return buf
+
+        # the previous step's kernels may still read both buffers
+        prev_done = torch.cuda.Event()
+        prev_done.record(stream)
+        copy_stream.wait_event(prev_done)
+        bufs = [None] * n_inst
+        for idx in range(min(2, n_inst)):
+            bufs[idx] = issue(idx)
+        for idx in range(n_inst):
+            stream.wait_event(ready[idx])
+            model.run_group(idx, stream, model.step_count, grads=bufs[idx])
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            freed[idx] = ev
+            if idx + 2 < n_inst:
+                bufs[idx + 2] = issue(idx + 2)
+        last = model.instances[-1][1]
+        with torch.cuda.stream(stream):
+            result.copy_(last[:1], non_blocking=True)
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    with torch.cuda.stream(stream):
+        one_step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            one_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    _ = float(result.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, device)
+    return {"value": round(ws * model.bytes_per_step / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(ms, 2), "steps": steps,
+            "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": 4}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(wl):
+    """One block group of the workload (the unit the step repeats)."""
+    from fully_sharded_shard_b200 import workloads as W
+    grp = max(wl.groups, key=lambda g: g.repeat)
+    return grp
+
+
+def oracle_pass(O, p, full, grads, wl, state, step):
+    """One oracle step over one group: copy-in, copy-out, reduce-scatter
+    (direct form), AdamW."""
+    master, m, v = state
+    ag = O.copy_in(p, master)
+    O.copy_out(p, ag)
+    red = O.reduce_scatter_direct(p, grads, wl.op)
+    O.adamw(master, m, v, red, step=step, lr=3e-4, beta1=0.9, beta2=0.999, eps=1e-8,
+            weight_decay=0.01)
+
+
+def oracle_setup(wl):
+    import numpy as np
+    import oracle as O
+    O.build()
+    grp = oracle_sample(wl)
+    p = O.plan(grp.shapes, wl.N)
+    rng = np.random.default_rng(0)
+    full = (rng.standard_normal(p.P_arena, dtype=np.float32) * np.float32(0.02))
+    bits = (rng.standard_normal(wl.N * p.P_arena, dtype=np.float32) * np.float32(1e-3)).view(np.uint32)
+    grads = O.bf16_bits_from_u32(bits)
+    del bits
+    master = O.shard(p, full)
+    state = (master, np.zeros_like(master), np.zeros_like(master))
+    return O, grp, p, full, grads, state
+
+
+def cpu_baseline(wl, min_seconds: float):
+    O, grp, p, full, grads, state = oracle_setup(wl)
+    cores = O.get_threads()
+    t0 = time.time()
+    passes = 0
+    while True:
+        passes += 1
+        oracle_pass(O, p, full, grads, wl, state, passes)
+        if time.time() - t0 >= min_seconds:
+            break
+    dt = (time.time() - t0) / passes
+    b = group_bytes(wl.N, p.S, p.P)
+    return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "params_per_s": round(p.P / dt, 1),
+            "sample": f"{passes} oracle pass(es) over one '{grp.name}' group of {wl.name} "
+                      f"({p.P} params, N={wl.N}): copy-in, copy-out, reduce-scatter, AdamW; "
+                      f"{dt:.2f} s per pass, OpenMP over {cores} threads"}
+
+
+def run_reference(args, wl):
+    O, grp, p, full, grads, state = oracle_setup(wl)
+    cores = O.get_threads()
+    for k in range(args.warmup):
+        oracle_pass(O, p, full, grads, wl, state, k + 1)
+    t0 = time.time()
+    for k in range(args.steps):
+        oracle_pass(O, p, full, grads, wl, state, args.warmup + k + 1)
+    dt = (time.time() - t0) / args.steps
+    b = group_bytes(wl.N, p.S, p.P)
+    val = round(b / dt / 1e9, 3)
+    sample = (f"each step: one oracle pass over one '{grp.name}' group of {wl.name} "
+              f"({p.P} params, N={wl.N}) on {cores} host threads")
+    return {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s",
+        "params_per_s": round(p.P / dt, 1), "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32+bf16",
+        "data": "synthetic: seeded N(0,0.02) fp32 master, N(0,1e-3) bf16 per-rank grads",
+        "config": {"workload": wl.name, "N_virtual_ranks": wl.N,
+                   "sample_group": grp.name, "params_per_sample": p.P},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b")
+    ap.add_argument("--grad-pool", type=int, default=8)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    from fully_sharded_shard_b200 import workloads as W
+    wl = W.by_name(args.workload)
+    ws, rank, local = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if ws > 1:
+        init_dist("nccl")
+    out, model = run_ours(args, wl, device, rank, ws)
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,211 @@
+"""Thin ctypes binding of libfsdpk.so (declared in include/fsdpk.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are passed by ``data_ptr()``; the stream defaults to torch's
+current stream on the tensors' device.  There is no fallback: importing this
+module without the built library raises, and every non-OK status raises
+``FsdpError``.
+
+Function names follow the C entry points:
+``fsdp_plan_group``, ``fsdp_shard_params``, ``fsdp_copy_in``,
+``fsdp_copy_out``, ``fsdp_rs_reduce``, ``fsdp_adamw_step``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfsdpk.so")
+
+FSDP_MAX_NDIM = 8
+FSDP_MAX_WORLD = 1024
+
+FSDP_OK, FSDP_EINVAL, FSDP_ENOMEM, FSDP_ECUDA, FSDP_EALIGN, FSDP_ESTATE = 0, -1, -2, -3, -4, -5
+FSDP_SUM, FSDP_AVG, FSDP_SUM_THEN_DIV = 0, 1, 2
+
+EXPORTED = (
+    "fsdp_plan_group", "fsdp_group_sizes", "fsdp_group_param_offsets",
+    "fsdp_destroy_group", "fsdp_shard_params", "fsdp_copy_in", "fsdp_copy_out",
+    "fsdp_rs_reduce", "fsdp_adamw_step", "fsdp_status_string",
+    "fsdp_last_cuda_error", "fsdp_abi_version",
+)
+
+
+class FsdpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.fsdp_status_string(status).decode()
+        if status == FSDP_ECUDA:
+            msg += f" (cudaError {_lib.fsdp_last_cuda_error()})"
+        super().__init__(f"{where}: {msg} [{status}]")
+        self.status = status
+
+
+class ParamDesc(ctypes.Structure):
+    _fields_ = [("ndim", ctypes.c_int32), ("shape", ctypes.c_int64 * FSDP_MAX_NDIM)]
+
+
+class AdamWHparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double),
+                ("beta2", ctypes.c_double), ("eps", ctypes.c_double),
+                ("weight_decay", ctypes.c_double), ("step", ctypes.c_int64)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libfsdpk.so is not built ({LIB_PATH}); run "
+            "`python -m fully_sharded_shard_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    L.fsdp_plan_group.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, ctypes.POINTER(vp)]
+    L.fsdp_group_sizes.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    L.fsdp_group_param_offsets.argtypes = [vp, vp, vp, vp]
+    L.fsdp_destroy_group.argtypes = [vp]
+    L.fsdp_destroy_group.restype = None
+    L.fsdp_shard_params.argtypes = [vp, vp, vp, vp]
+    L.fsdp_copy_in.argtypes = [vp, vp, vp, vp]
+    L.fsdp_copy_out.argtypes = [vp, vp, vp, vp]
+    L.fsdp_rs_reduce.argtypes = [vp, vp, i32, vp, vp, vp]
+    L.fsdp_adamw_step.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp]
+    L.fsdp_status_string.argtypes = [ctypes.c_int]
+    L.fsdp_status_string.restype = ctypes.c_char_p
+    for name in ("fsdp_plan_group", "fsdp_group_sizes", "fsdp_group_param_offsets",
+                 "fsdp_shard_params", "fsdp_copy_in", "fsdp_copy_out", "fsdp_rs_reduce",
+                 "fsdp_adamw_step", "fsdp_last_cuda_error", "fsdp_abi_version"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != FSDP_OK:
+        raise FsdpError(status, where)
+
+
+class Group:
+    """A plan of one parameter group (one fully_shard call) over N ranks."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], world_size: int):
+        shapes = [tuple(int(d) for d in s) for s in shapes]
+        arr = (ParamDesc * max(1, len(shapes)))()
+        for i, s in enumerate(shapes):
+            if len(s) > FSDP_MAX_NDIM:
+                raise ValueError(f"parameter {i}: more than {FSDP_MAX_NDIM} dims")
+            arr[i].ndim = len(s)
+            for k, d in enumerate(s):
+                arr[i].shape[k] = d
+        h = ctypes.c_void_p()
+        _check(_lib.fsdp_plan_group(arr, len(shapes), int(world_size), ctypes.byref(h)),
+               "fsdp_plan_group")
+        self._h = h
+        self.shapes = shapes
+        self.N = int(world_size)
+        self.n = len(shapes)
+        S, P, A = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib.fsdp_group_sizes(h, ctypes.byref(S), ctypes.byref(P), ctypes.byref(A)),
+               "fsdp_group_sizes")
+        self.S, self.P, self.P_arena = S.value, P.value, A.value
+        n = max(1, self.n)
+        off, arena, rows = (ctypes.c_int64 * n)(), (ctypes.c_int64 * n)(), (ctypes.c_int64 * n)()
+        _check(_lib.fsdp_group_param_offsets(h, off, arena, rows), "fsdp_group_param_offsets")
+        self.shard_off = list(off)[:self.n]
+        self.arena_off = list(arena)[:self.n]
+        self.chunk_rows = list(rows)[:self.n]
+        self.numel = [int(torch.Size(s).numel()) if len(s) else 1 for s in shapes]
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise ValueError("group destroyed")
+        return self._h
+
+    def destroy(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            _lib.fsdp_destroy_group(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def fsdp_plan_group(shapes: Sequence[Sequence[int]], world_size: int) -> Group:
+    return Group(shapes, world_size)
+
+
+def _stream(stream, t: torch.Tensor):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor], dtypes, numel: int, name: str):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements < required {numel}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+_F32 = (torch.float32,)
+_B16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def fsdp_shard_params(g: Group, full_arena: torch.Tensor, master: torch.Tensor, stream=None):
+    _check(_lib.fsdp_shard_params(g.handle, _ptr(full_arena, _F32, g.P_arena, "full_arena"),
+                                  _ptr(master, _F32, g.N * g.S, "master"),
+                                  _stream(stream, master)), "fsdp_shard_params")
+
+
+def fsdp_copy_in(g: Group, master: torch.Tensor, ag: torch.Tensor, stream=None):
+    _check(_lib.fsdp_copy_in(g.handle, _ptr(master, _F32, g.N * g.S, "master"),
+                             _ptr(ag, _B16, g.N * g.S, "ag"), _stream(stream, master)),
+           "fsdp_copy_in")
+
+
+def fsdp_copy_out(g: Group, ag: torch.Tensor, arena: torch.Tensor, stream=None):
+    _check(_lib.fsdp_copy_out(g.handle, _ptr(ag, _B16, g.N * g.S, "ag"),
+                              _ptr(arena, _B16, g.P_arena, "arena"), _stream(stream, ag)),
+           "fsdp_copy_out")
+
+
+def fsdp_rs_reduce(g: Group, grads: torch.Tensor, op: int, reduced: torch.Tensor,
+                   packed: Optional[torch.Tensor] = None, stream=None):
+    _check(_lib.fsdp_rs_reduce(g.handle, _ptr(grads, _B16, g.N * g.P_arena, "grads"), int(op),
+                               _ptr(packed, _F32, g.N * g.N * g.S, "packed"),
+                               _ptr(reduced, _F32, g.N * g.S, "reduced"),
+                               _stream(stream, reduced)), "fsdp_rs_reduce")
+
+
+def fsdp_adamw_step(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                    grad: torch.Tensor, *, lr: float, beta1: float, beta2: float, eps: float,
+                    weight_decay: float, step: int, stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = g.N * g.S
+    _check(_lib.fsdp_adamw_step(g.handle, _ptr(master, _F32, n, "master"),
+                                _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                _ptr(grad, _F32, n, "grad"), ctypes.byref(hp),
+                                _stream(stream, master)), "fsdp_adamw_step")

@@ -1,0 +1,358 @@
+// fsdpk_api.cu -- host side of libfsdpk.so: the parameter-group plan and the
+// extern "C" entry points declared in include/fsdpk.h.
+//
+// The plan restates the Shard(0) placement of "Sharded Training: FSDP2,
+// DTensor, Tensor and Pipeline Parallelism" (fully_shard paragraph): rank r
+// keeps chunk r of torch.chunk(param, N, dim=0), i.e. rows
+// [r*c, r*c + v_r) with c = ceil(d0 / N), and every rank's shard is padded
+// to c rows.  One call = one parameter group = one communication unit.
+//
+// Everything that can be decided once per group is decided here, on the
+// host, and uploaded once: the work units of the segment kernels and the pad
+// intervals of the copy-in.  The data calls then only validate pointers and
+// launch.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <new>
+#include <vector>
+
+#include "fsdpk.h"
+#include "fsdpk_internal.h"
+
+using fsdpk::Interval;
+using fsdpk::TileRange;
+using fsdpk::Unit;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return FSDP_ECUDA;
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > std::numeric_limits<int64_t>::max() / a) return false;
+    *out = a * b;
+    return true;
+}
+
+bool add_ok(int64_t a, int64_t b, int64_t* out) {
+    if (b > std::numeric_limits<int64_t>::max() - a) return false;
+    *out = a + b;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Split [pos, pos+len) of a (rank, parameter) run into units of at most
+// kUnitElems elements.
+void push_units(std::vector<Unit>& out, int64_t shard_pos, int64_t arena_pos, int64_t len,
+                int32_t is_pad) {
+    for (int64_t done = 0; done < len; done += fsdpk::kUnitElems) {
+        const int64_t l = std::min<int64_t>(fsdpk::kUnitElems, len - done);
+        out.push_back(Unit{shard_pos + done, is_pad ? 0 : arena_pos + done, (int32_t)l, is_pad});
+    }
+}
+
+// Check the current device is the plan's device.
+int check_device(const fsdp_group* g) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return dev == g->device ? FSDP_OK : FSDP_ESTATE;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fsdp_abi_version(void) { return FSDP_ABI_VERSION; }
+
+int fsdp_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* fsdp_status_string(int status) {
+    switch (status) {
+        case FSDP_OK: return "ok";
+        case FSDP_EINVAL: return "invalid argument";
+        case FSDP_ENOMEM: return "out of memory";
+        case FSDP_ECUDA: return "CUDA error";
+        case FSDP_EALIGN: return "pointer not 16-byte aligned";
+        case FSDP_ESTATE: return "plan used on a different device";
+        default: return "unknown status";
+    }
+}
+
+int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t world_size,
+                    fsdp_group_t* out) {
+    if (out == nullptr) return FSDP_EINVAL;
+    *out = nullptr;
+    if (n_params < 0 || (n_params > 0 && params == nullptr)) return FSDP_EINVAL;
+    if (world_size < 1 || world_size > FSDP_MAX_WORLD) return FSDP_EINVAL;
+
+    fsdp_group* g = new (std::nothrow) fsdp_group();
+    if (g == nullptr) return FSDP_ENOMEM;
+    auto fail = [&](int st) {
+        delete g;
+        return st;
+    };
+    const int64_t N = world_size;
+    g->N = world_size;
+    g->n = n_params;
+    try {
+        g->d0.resize(n_params);
+        g->cols.resize(n_params);
+        g->c.resize(n_params);
+        g->s.resize(n_params);
+        g->off.resize(n_params);
+        g->u.resize(n_params);
+    } catch (...) {
+        return fail(FSDP_ENOMEM);
+    }
+
+    // per-parameter tables
+    int64_t S = 0, P = 0, A = 0;
+    for (int32_t i = 0; i < n_params; ++i) {
+        const fsdp_param_desc& d = params[i];
+        if (d.ndim < 0 || d.ndim > FSDP_MAX_NDIM) return fail(FSDP_EINVAL);
+        int64_t d0 = 1, cols = 1;
+        for (int k = 0; k < d.ndim; ++k) {
+            if (d.shape[k] < 0) return fail(FSDP_EINVAL);
+            if (k == 0) d0 = d.shape[0];
+            else if (!mul_ok(cols, d.shape[k], &cols)) return fail(FSDP_EINVAL);
+        }
+        const int64_t c = d0 == 0 ? 0 : (d0 + N - 1) / N;  // torch.chunk rows
+        int64_t s, numel;
+        if (!mul_ok(c, cols, &s) || !mul_ok(d0, cols, &numel)) return fail(FSDP_EINVAL);
+        g->d0[i] = d0;
+        g->cols[i] = cols;
+        g->c[i] = c;
+        g->s[i] = s;
+        g->off[i] = S;
+        if (!add_ok(S, s, &S) || !add_ok(P, numel, &P)) return fail(FSDP_EINVAL);
+        // arena: each parameter starts on a multiple of 8 elements (16 bytes)
+        int64_t ui;
+        if (!add_ok(A, 7, &ui)) return fail(FSDP_EINVAL);
+        ui = ui / 8 * 8;
+        g->u[i] = ui;
+        if (!add_ok(ui, numel, &A)) return fail(FSDP_EINVAL);
+    }
+    int64_t Aup;
+    if (!add_ok(A, 7, &Aup)) return fail(FSDP_EINVAL);
+    g->S = S;
+    g->P = P;
+    g->P_arena = Aup / 8 * 8;
+    // every buffer size the data calls imply must fit int64 indexing
+    int64_t NS, NA, NNS, tmp;
+    if (!mul_ok(N, S, &NS) || !mul_ok(N, g->P_arena, &NA) || !mul_ok(NS, N, &NNS) ||
+        !mul_ok(NNS, 4, &tmp) || !mul_ok(NA, 2, &tmp))
+        return fail(FSDP_EINVAL);
+    if (NS / fsdpk::kCopyInTile + 1 > std::numeric_limits<int32_t>::max()) return fail(FSDP_EINVAL);
+    g->pad_elems = NS - P;
+
+    // work units: real runs for every (rank j, parameter i), then pad runs
+    try {
+        for (int64_t j = 0; j < N; ++j)
+            for (int32_t i = 0; i < n_params; ++i) {
+                const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
+                push_units(g->units, j * S + g->off[i], g->u[i] + j * g->c[i] * g->cols[i],
+                           v * g->cols[i], 0);
+            }
+        g->n_real_units = (int64_t)g->units.size();
+        for (int64_t j = 0; j < N; ++j)
+            for (int32_t i = 0; i < n_params; ++i) {
+                const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
+                const int64_t lo = j * S + g->off[i] + v * g->cols[i];
+                const int64_t len = (g->c[i] - v) * g->cols[i];
+                push_units(g->units, lo, 0, len, 1);
+                if (len > 0) {
+                    if (!g->intervals.empty() && g->intervals.back().hi == lo)
+                        g->intervals.back().hi = lo + len;  // merge adjacent pads
+                    else
+                        g->intervals.push_back(Interval{lo, lo + len});
+                }
+            }
+        if (g->intervals.size() > (size_t)std::numeric_limits<int32_t>::max())
+            return fail(FSDP_EINVAL);
+        g->n_tiles = (NS + fsdpk::kCopyInTile - 1) / fsdpk::kCopyInTile;
+        if (!g->intervals.empty()) {
+            g->tile_ranges.resize((size_t)g->n_tiles);
+            size_t a = 0, b = 0;
+            for (int64_t t = 0; t < g->n_tiles; ++t) {
+                const int64_t lo = t * fsdpk::kCopyInTile;
+                const int64_t hi = lo + fsdpk::kCopyInTile;
+                while (a < g->intervals.size() && g->intervals[a].hi <= lo) ++a;
+                if (b < a) b = a;
+                while (b < g->intervals.size() && g->intervals[b].lo < hi) ++b;
+                g->tile_ranges[(size_t)t] = TileRange{(int32_t)a, (int32_t)b};
+            }
+        }
+    } catch (...) {
+        return fail(FSDP_ENOMEM);
+    }
+
+    // device tables, one allocation, uploaded once
+    cudaError_t e = cudaGetDevice(&g->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e));
+    e = cudaDeviceGetAttribute(&g->sm_count, cudaDevAttrMultiProcessorCount, g->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e));
+    const size_t b_units = g->units.size() * sizeof(Unit);
+    const size_t b_iv = g->intervals.size() * sizeof(Interval);
+    const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
+    auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr);
+    if (total > 0) {
+        e = cudaMalloc(&g->dev_mem, total);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            g->dev_mem = nullptr;
+            return fail(e == cudaErrorMemoryAllocation ? FSDP_ENOMEM : cuda_fail(e));
+        }
+        char* base = static_cast<char*>(g->dev_mem);
+        g->d_units = reinterpret_cast<const Unit*>(base);
+        g->d_intervals = reinterpret_cast<const Interval*>(base + up256(b_units));
+        g->d_tile_ranges = reinterpret_cast<const TileRange*>(base + up256(b_units) + up256(b_iv));
+        if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && b_iv)
+            e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && b_tr)
+            e = cudaMemcpy((void*)g->d_tile_ranges, g->tile_ranges.data(), b_tr,
+                           cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            cudaFree(g->dev_mem);
+            return fail(cuda_fail(e));
+        }
+    }
+    *out = g;
+    return FSDP_OK;
+}
+
+int fsdp_group_sizes(fsdp_group_t g, int64_t* S, int64_t* P, int64_t* P_arena) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if (S) *S = g->S;
+    if (P) *P = g->P;
+    if (P_arena) *P_arena = g->P_arena;
+    return FSDP_OK;
+}
+
+int fsdp_group_param_offsets(fsdp_group_t g, int64_t* shard_off, int64_t* arena_off,
+                             int64_t* chunk_rows) {
+    if (g == nullptr) return FSDP_EINVAL;
+    for (int32_t i = 0; i < g->n; ++i) {
+        if (shard_off) shard_off[i] = g->off[i];
+        if (arena_off) arena_off[i] = g->u[i];
+        if (chunk_rows) chunk_rows[i] = g->c[i];
+    }
+    return FSDP_OK;
+}
+
+void fsdp_destroy_group(fsdp_group_t g) {
+    if (g == nullptr) return;
+    if (g->dev_mem) {
+        int prev = -1;
+        bool switched = false;
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != g->device)
+            switched = cudaSetDevice(g->device) == cudaSuccess;
+        cudaFree(g->dev_mem);
+        if (switched) cudaSetDevice(prev);
+    }
+    delete g;
+}
+
+int fsdp_shard_params(fsdp_group_t g, const float* full_arena, float* master,
+                      fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if ((int64_t)g->N * g->S > 0 && master == nullptr) return FSDP_EINVAL;
+    if (g->P > 0 && full_arena == nullptr) return FSDP_EINVAL;
+    if (!aligned16(full_arena) || !aligned16(master)) return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_shard(*g, full_arena, master, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_copy_in(fsdp_group_t g, const float* master, uint16_t* ag, fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if ((int64_t)g->N * g->S > 0 && (master == nullptr || ag == nullptr)) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(ag)) return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_copy_in(*g, master, ag, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_copy_out(fsdp_group_t g, const uint16_t* ag, uint16_t* arena, fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if (g->P > 0 && (ag == nullptr || arena == nullptr)) return FSDP_EINVAL;
+    if (!aligned16(ag) || !aligned16(arena)) return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_copy_out(*g, ag, arena, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_rs_reduce(fsdp_group_t g, const uint16_t* grads, int32_t op, float* packed_or_null,
+                   float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && reduced == nullptr) return FSDP_EINVAL;
+    if (g->P > 0 && grads == nullptr) return FSDP_EINVAL;
+    if (!aligned16(grads) || !aligned16(reduced) || !aligned16(packed_or_null))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (packed_or_null == nullptr) {
+        e = fsdpk::launch_rs_fused(*g, grads, op, reduced, s);
+    } else {
+        // staged: materialise every rank's reduce-scatter input, reduce it,
+        // and for SUM_THEN_DIV divide in a separate pass
+        e = fsdpk::launch_rs_pack(*g, grads, packed_or_null, s);
+        if (e == cudaSuccess)
+            e = fsdpk::launch_rs_reduce_packed(*g, packed_or_null, op == FSDP_AVG ? FSDP_AVG : FSDP_SUM,
+                                               reduced, s);
+        if (e == cudaSuccess && op == FSDP_SUM_THEN_DIV) e = fsdpk::launch_div_inplace(*g, reduced, s);
+    }
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_adamw_step(fsdp_group_t g, float* master, float* m, float* v, const float* grad,
+                    const fsdp_adamw_hparams* hp, fsdp_stream_t stream) {
+    if (g == nullptr || hp == nullptr) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr || grad == nullptr))
+        return FSDP_EINVAL;
+    if (!(hp->step >= 1) || !(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
+        !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) ||
+        !std::isfinite(hp->weight_decay) || !std::isfinite(hp->lr))
+        return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    const double t = (double)hp->step;
+    const double bc1 = 1.0 - std::pow(hp->beta1, t);
+    const double bc2 = 1.0 - std::pow(hp->beta2, t);
+    fsdpk::AdamScalars sc;
+    sc.decay = (float)(1.0 - hp->lr * hp->weight_decay);
+    sc.beta1 = (float)hp->beta1;
+    sc.omb1 = (float)(1.0 - hp->beta1);
+    sc.beta2 = (float)hp->beta2;
+    sc.omb2 = (float)(1.0 - hp->beta2);
+    sc.step_size = (float)(hp->lr / bc1);
+    sc.inv_bc2_sqrt = (float)(1.0 / std::sqrt(bc2));
+    sc.eps = (float)hp->eps;
+    cudaError_t e = fsdpk::launch_adamw(*g, master, m, v, grad, sc, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+// fsdpk_internal.h -- types shared by the plan builder, the kernels and the
+// C-ABI entry points of libfsdpk.so.  Not part of the public interface.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "fsdpk.h"
+
+namespace fsdpk {
+
+// Elements per work unit of the segment kernels (copy-out, reduce-scatter,
+// pack, shard).  Large enough that a unit's head/tail peeling is noise,
+// small enough that the largest parameter splits into thousands of units.
+constexpr int64_t kUnitElems = 8192;
+
+// Elements per tile of the flat copy-in kernel (256 threads x 8 x 4).
+constexpr int64_t kCopyInTile = 8192;
+
+// One contiguous run of a (rank j, parameter i) shard segment.
+//   shard_pos: first element in the rank-major [N][S] index space
+//   arena_pos: first element of the matching rows in an unsharded arena
+//              (real runs only)
+//   len:       elements in the run
+//   is_pad:    1 for a run of pad rows (written as +0), 0 for real rows
+struct Unit {
+    int64_t shard_pos;
+    int64_t arena_pos;
+    int32_t len;
+    int32_t is_pad;
+};
+static_assert(sizeof(Unit) == 24, "Unit layout");
+
+// A half-open range [lo, hi) of pad elements in the [N][S] index space.
+struct Interval {
+    int64_t lo;
+    int64_t hi;
+};
+
+// For each copy-in tile, the half-open index range of the pad intervals that
+// intersect it.
+struct TileRange {
+    int32_t begin;
+    int32_t end;
+};
+
+}  // namespace fsdpk
+
+// The opaque plan behind fsdp_group_t.
+struct fsdp_group {
+    int device = -1;
+    int sm_count = 0;
+    int32_t N = 0;
+    int32_t n = 0;
+    std::vector<int64_t> d0, cols, c, s, off, u;
+    int64_t S = 0, P = 0, P_arena = 0;
+    int64_t pad_elems = 0;  // N*S - P
+
+    // host copies (kept for inspection and tests of the plan)
+    std::vector<fsdpk::Unit> units;  // real units first, then pad units
+    int64_t n_real_units = 0;
+    std::vector<fsdpk::Interval> intervals;
+    std::vector<fsdpk::TileRange> tile_ranges;  // empty when no padding
+    int64_t n_tiles = 0;                        // copy-in tiles over N*S
+
+    // one device allocation holding the three tables
+    void* dev_mem = nullptr;
+    const fsdpk::Unit* d_units = nullptr;
+    const fsdpk::Interval* d_intervals = nullptr;
+    const fsdpk::TileRange* d_tile_ranges = nullptr;
+};
+
+namespace fsdpk {
+
+// Scalars of one AdamW step, precomputed on the host in binary64.
+struct AdamScalars {
+    float decay;         // 1 - lr*wd
+    float beta1, omb1;   // b1, 1 - b1
+    float beta2, omb2;   // b2, 1 - b2
+    float step_size;     // lr / (1 - b1^t)
+    float inv_bc2_sqrt;  // 1 / sqrt(1 - b2^t)
+    float eps;
+};
+
+// Kernel launchers (fsdpk_kernels.cu).  They enqueue work and return the
+// cudaError_t of the launch.
+cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* ag,
+                           cudaStream_t st);
+cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* arena,
+                            cudaStream_t st);
+cudaError_t launch_rs_fused(const fsdp_group& g, const uint16_t* grads, int op,
+                            float* reduced, cudaStream_t st);
+cudaError_t launch_rs_pack(const fsdp_group& g, const uint16_t* grads, float* packed,
+                           cudaStream_t st);
+cudaError_t launch_rs_reduce_packed(const fsdp_group& g, const float* packed, int op,
+                                    float* reduced, cudaStream_t st);
+cudaError_t launch_div_inplace(const fsdp_group& g, float* reduced, cudaStream_t st);
+cudaError_t launch_adamw(const fsdp_group& g, float* master, float* m, float* v,
+                         const float* grad, const AdamScalars& sc, cudaStream_t st);
+cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
+                         cudaStream_t st);
+
+}  // namespace fsdpk

@@ -1,0 +1,207 @@
+/*
+ * fsdpk.h -- C ABI of libfsdpk.so, the B200 (sm_100a) kernels of the FSDP2
+ * per-parameter sharding step, with the N data-parallel ranks of one
+ * parameter group emulated as N virtual ranks resident in one GPU's memory.
+ *
+ * Sources, by page title and section:
+ *   [ML] "Sharded Training: FSDP2, DTensor, Tensor and Pipeline Parallelism":
+ *        fully_shard paragraph (Shard(0): rank r keeps chunk r of
+ *        torch.chunk(param, world, dim=0), padded internally when rows do not
+ *        divide evenly; one fully_shard call = one parameter group = one unit
+ *        of communication), Mixed precision paragraph (param_dtype bf16
+ *        all-gather, reduce_dtype fp32 reduction), Other controls paragraph
+ *        (set_force_sum_reduction_for_comms: SUM plus FSDP's own division),
+ *        opening paragraph (2 + 2 + 12 bytes per parameter).
+ *   [MS] "Introduction to PyTorch FSDP2 Backend Features": Working Principle
+ *        (all-gather -> compute -> reduce-scatter -> sharded update) and
+ *        Mixed Precision.
+ *
+ * Notation for a group of n parameters over N ranks (registration order i):
+ *   d0_i = rows, cols_i = product of the remaining dims (1 for 1-D tensors)
+ *   c_i  = ceil(d0_i / N)              rows of every rank's padded shard
+ *   v_ir = clamp(d0_i - r*c_i, 0, c_i) real rows on rank r (the rest: pad)
+ *   s_i  = c_i*cols_i; off_i = s_0 + ... + s_{i-1}; S = sum of s_i
+ *   u_i  = unsharded ("arena") offset of parameter i: the previous
+ *          parameter's end rounded up to a multiple of 8 elements (16 bytes);
+ *          P_arena = last end rounded up to a multiple of 8.
+ *   P    = sum of d0_i*cols_i (real elements of the group).
+ *
+ * Buffer layouts (element counts; all row-major, no strides):
+ *   sharded fp32 state (master, m, v, reduced grad): [N][S], rank-major;
+ *       rank r's shard of parameter i is rows [0, c_i) x cols_i at
+ *       r*S + off_i; rows >= v_ir are padding and hold +0.
+ *   all-gather buffer (bf16): [N][S], same layout as the sharded state.
+ *   unsharded arena (bf16 params, fp32 full params): [P_arena], parameter i
+ *       as a dense [d0_i][cols_i] block at u_i; gap elements are never
+ *       read or written.
+ *   per-rank full gradients (bf16): [N][P_arena], rank r's arena at
+ *       r*P_arena.
+ *   packed reduce-scatter input (fp32, optional): [N][N][S]; packed[r][j] is
+ *       what rank r contributes to destination rank j.
+ * bf16 values are passed as their uint16_t bit patterns.
+ *
+ * Ownership: the caller allocates and owns every data buffer and stream.  The
+ * library owns only the plan (host tables and one device table, allocated in
+ * fsdp_plan_group on the device current at that time, freed by
+ * fsdp_destroy_group).  A plan is used on the device it was made on.
+ *
+ * Execution: every data call validates its arguments on the host, enqueues
+ * kernels on `stream` and returns without synchronising.  Data pointers are
+ * device pointers (or managed memory) and must be 16-byte aligned.  Buffers
+ * of one call must not overlap unless stated.  Calls on the same group may run
+ * concurrently on different streams only if their buffers are disjoint.
+ *
+ * Errors: every call returns an fsdp_status.  Invalid arguments are detected
+ * before any launch and nothing is enqueued; FSDP_ECUDA reports a failed
+ * launch (cudaGetLastError after the launch).  No kernel traps or waits.
+ */
+#ifndef FSDPK_H
+#define FSDPK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FSDP_MAX_NDIM 8
+#define FSDP_MAX_WORLD 1024
+#define FSDP_ABI_VERSION 1
+
+/* One parameter's shape; dims must be >= 0, ndim in [0, FSDP_MAX_NDIM].
+ * ndim == 0 (a scalar) is treated as shape [1]. */
+typedef struct {
+    int32_t ndim;
+    int64_t shape[FSDP_MAX_NDIM];
+} fsdp_param_desc;
+
+/* Opaque plan of one parameter group (one fully_shard call). */
+typedef struct fsdp_group* fsdp_group_t;
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* fsdp_stream_t;
+
+typedef enum {
+    FSDP_OK = 0,
+    FSDP_EINVAL = -1, /* bad argument (null, size, count, op, hparams)     */
+    FSDP_ENOMEM = -2, /* host or device allocation of the plan failed      */
+    FSDP_ECUDA = -3,  /* a CUDA runtime call or kernel launch failed       */
+    FSDP_EALIGN = -4, /* a data pointer is not 16-byte aligned             */
+    FSDP_ESTATE = -5  /* plan used on a device other than its own          */
+} fsdp_status;
+
+/* Reduce-scatter reduction ([ML] Other controls; The bug Adam hid). */
+typedef enum {
+    FSDP_SUM = 0,          /* ((g_0 + g_1) + ...) + g_{N-1}, binary32 RN   */
+    FSDP_AVG = 1,          /* the SUM divided once by N (IEEE binary32 /)  */
+    FSDP_SUM_THEN_DIV = 2  /* SUM, then FSDP's own division by N; the same
+                              bits as FSDP_AVG                             */
+} fsdp_reduce_op;
+
+/* AdamW hyper-parameters (decoupled weight decay).  step is the 1-based
+ * step count t used in the bias corrections 1 - beta^t. */
+typedef struct {
+    double lr;
+    double beta1;
+    double beta2;
+    double eps;
+    double weight_decay;
+    int64_t step;
+} fsdp_adamw_hparams;
+
+/* ------------------------------------------------------------------------ */
+/* Plan                                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Build the plan of one group: chunk rows, padded shard offsets, arena
+ * offsets and the device work tables ([ML] fully_shard paragraph).
+ * params: n_params descriptors (host memory, read only during the call).
+ * n_params >= 0; world_size in [1, FSDP_MAX_WORLD].  On success *out owns a
+ * new plan.  Errors: EINVAL (bad descriptor, sizes overflow int64),
+ * ENOMEM, ECUDA (device table upload). */
+int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params,
+                    int32_t world_size, fsdp_group_t* out);
+
+/* S (per-rank padded shard elements), P (real elements), P_arena.
+ * Any output pointer may be NULL. */
+int fsdp_group_sizes(fsdp_group_t group, int64_t* S, int64_t* P,
+                     int64_t* P_arena);
+
+/* Per-parameter tables, each an int64 array of n_params entries supplied by
+ * the caller (any may be NULL): off_i, u_i and c_i. */
+int fsdp_group_param_offsets(fsdp_group_t group, int64_t* shard_off,
+                             int64_t* arena_off, int64_t* chunk_rows);
+
+/* Free a plan (NULL is ignored).  Work already enqueued that uses the plan
+ * must have completed. */
+void fsdp_destroy_group(fsdp_group_t group);
+
+/* ------------------------------------------------------------------------ */
+/* Data path (asynchronous on `stream`)                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Shard(0) placement: fp32 full parameters in arena layout [P_arena] ->
+ * padded fp32 master [N][S] (pad rows written as +0).  This is fully_shard's
+ * initial sharding ([ML] fully_shard paragraph). */
+int fsdp_shard_params(fsdp_group_t group, const float* full_arena,
+                      float* master, fsdp_stream_t stream);
+
+/* Stage 1, all-gather copy-in: ag[r][k] = bf16_rn(master[r][k]) for real
+ * elements and +0 for pad elements ([ML] Mixed precision: bf16 copies are
+ * all-gathered; [MS] Mixed Precision).  master: fp32 [N][S] (read);
+ * ag: bf16 [N][S] (written). */
+int fsdp_copy_in(fsdp_group_t group, const float* master, uint16_t* ag,
+                 fsdp_stream_t stream);
+
+/* Stage 2, all-gather copy-out: the rank-major buffer is split into the
+ * unsharded parameters with the padding stripped ([MS] Working Principle,
+ * All-Gather state): arena[u_i + row*cols_i + col] =
+ * ag[r*S + off_i + (row - r*c_i)*cols_i + col] with r = row / c_i.
+ * ag: bf16 [N][S] (read); arena: bf16 [P_arena] (written, gaps untouched). */
+int fsdp_copy_out(fsdp_group_t group, const uint16_t* ag, uint16_t* arena,
+                  fsdp_stream_t stream);
+
+/* Stages 3 + 4, reduce-scatter: each rank's bf16 full gradients are cast to
+ * fp32 (reduce_dtype), packed per destination rank and reduced over the N
+ * ranks in rank order ([ML] Mixed precision, Other controls).
+ * grads: bf16 [N][P_arena] (read).  reduced: fp32 [N][S] (written; pads +0).
+ * op: an fsdp_reduce_op.  packed_or_null: NULL runs the fused path (no
+ * packed buffer is materialised); otherwise fp32 [N][N][S] receives the packed
+ * reduce-scatter inputs and the reduction reads them back (staged path; for
+ * FSDP_SUM_THEN_DIV the division is a separate pass).  Both paths give the
+ * same bits. */
+int fsdp_rs_reduce(fsdp_group_t group, const uint16_t* grads, int32_t op,
+                   float* packed_or_null, float* reduced,
+                   fsdp_stream_t stream);
+
+/* Stage 5, sharded AdamW on all N*S elements (decoupled weight decay,
+ * PyTorch's documented AdamW; [ML] Fence 4 and opening paragraph: 12 bytes
+ * of fp32 state per parameter):
+ *   p <- p*(1 - lr*wd);  m <- b1*m + (1-b1)*g;  v <- b2*v + (1-b2)*g*g
+ *   p <- p - (lr/(1-b1^t)) * m / (sqrt(v)/sqrt(1-b2^t) + eps)
+ * master, m, v: fp32 [N][S] updated in place; grad: fp32 [N][S] (read).
+ * A zero pad stays +0.  hparams: host pointer; step >= 1, lr >= 0,
+ * 0 <= beta < 1, eps > 0.  Computed in binary32. */
+int fsdp_adamw_step(fsdp_group_t group, float* master, float* m, float* v,
+                    const float* grad, const fsdp_adamw_hparams* hparams,
+                    fsdp_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Misc                                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Static description of a status code. */
+const char* fsdp_status_string(int status);
+
+/* The cudaError_t of the most recent FSDP_ECUDA on this thread (0 if none). */
+int fsdp_last_cuda_error(void);
+
+/* FSDP_ABI_VERSION of the loaded library. */
+int fsdp_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FSDPK_H */

@@ -19,6 +19,8 @@ Every function follows a definition from the pages (see the C file's header):
 * ``copy_out``    -- rank-major buffer -> unsharded views, padding stripped;
 * ``pack``        -- per-rank bf16 gradients -> fp32 reduce-scatter input;
 * ``reduce_packed`` -- rank-ordered binary32 fold, SUM / AVG / SUM_THEN_DIV;
+* ``reduce_scatter_direct`` -- pack + fold from the per-rank gradients with no
+  packed intermediate (same definitions, for full-size groups);
 * ``adamw``       -- decoupled-weight-decay AdamW in binary64.
 
 Parity status: every function above is pinned by tests under ``tests/``
@@ -79,6 +81,7 @@ def lib() -> ctypes.CDLL:
         for name in ("or_shard", "or_copy_in", "or_copy_out", "or_pack"):
             getattr(L, name).argtypes = [vp, vp, i32, i32, vp, vp]
         L.or_reduce_packed.argtypes = [i32, i64, vp, i32, vp]
+        L.or_reduce_scatter_direct.argtypes = [vp, vp, i32, i32, vp, i32, vp]
         L.or_adamw.argtypes = [vp, vp, vp, vp, i64, f64, f64, f64, f64, f64, i64]
         _lib = L
     return _lib
@@ -214,6 +217,17 @@ def reduce_packed(p: Plan, packed: np.ndarray, op: int) -> np.ndarray:
 def reduce_scatter(p: Plan, grads: np.ndarray, op: int) -> np.ndarray:
     """pack followed by the rank-ordered reduction."""
     return reduce_packed(p, pack(p, grads), op)
+
+
+def reduce_scatter_direct(p: Plan, grads: np.ndarray, op: int) -> np.ndarray:
+    """The same reduce-scatter straight from the per-rank gradients, without
+    the [N][N][S] packed intermediate (for groups too large to pack)."""
+    grads = np.ascontiguousarray(grads, np.uint16)
+    assert grads.size == p.N * p.P_arena
+    out = np.empty(p.N * p.S, np.float32)
+    lib().or_reduce_scatter_direct(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(grads),
+                                   int(op), _ptr(out))
+    return out
 
 
 def adamw(master, m, v, grad, *, lr, beta1, beta2, eps, weight_decay, step):

@@ -1,0 +1,213 @@
+"""Helpers for the GPU parity tests: run one parameter group through the
+C-ABI kernels and through the CPU oracle on identical seeded inputs, and
+compare (bit-exact for data movement and reduction, 1e-6 * (1 + |x|) for
+AdamW).
+
+Buffers are allocated with guard bands on both sides, filled with a
+sentinel and checked after every call, so an out-of-range write shows up
+as a failure.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from fully_sharded_shard_b200 import abi
+from fully_sharded_shard_b200 import workloads as W
+
+GUARD = 64  # elements on each side (a multiple of 16 bytes for every dtype here)
+ADAM_TOL = 1e-6
+
+
+class Guarded:
+    """A device buffer with sentinel guard bands before and after it."""
+
+    SENT = {torch.float32: -12345.5, torch.bfloat16: None, torch.int16: 0x3BEF}
+
+    def __init__(self, n: int, dtype, device="cuda", fill=None):
+        self.n = n
+        self.full = torch.empty(n + 2 * GUARD, dtype=dtype, device=device)
+        if dtype == torch.float32:
+            self.full.fill_(-12345.5)
+        else:
+            self.full.view(torch.int16).fill_(0x3BEF)
+        self.t = self.full[GUARD:GUARD + n]
+        if fill is not None:
+            self.t.copy_(fill)
+
+    def guards_intact(self) -> bool:
+        if self.full.dtype == torch.float32:
+            s = torch.tensor(-12345.5, dtype=torch.float32, device=self.full.device)
+            lo, hi = self.full[:GUARD], self.full[GUARD + self.n:]
+            return bool((lo == s).all() and (hi == s).all())
+        v = self.full.view(torch.int16)
+        return bool((v[:GUARD] == 0x3BEF).all() and (v[GUARD + self.n:] == 0x3BEF).all())
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
+
+
+def f32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy().reshape(-1)
+
+
+def bits_equal(a: np.ndarray, b: np.ndarray) -> bool:
+    a = np.asarray(a)
+    b = np.asarray(b)
+    if a.dtype == np.float32:
+        a = a.view(np.uint32)
+    if b.dtype == np.float32:
+        b = b.view(np.uint32)
+    return a.shape == b.shape and bool(np.array_equal(a, b))
+
+
+def first_mismatch(a, b) -> str:
+    a = np.asarray(a).reshape(-1)
+    b = np.asarray(b).reshape(-1)
+    if a.dtype == np.float32:
+        a, b = a.view(np.uint32), b.view(np.uint32)
+    bad = np.nonzero(a != b)[0]
+    if bad.size == 0:
+        return "no mismatch"
+    k = int(bad[0])
+    return f"{bad.size} mismatches, first at {k}: gpu={a[k]:#x} oracle={b[k]:#x}"
+
+
+def bf16_within_ulp(a: np.ndarray, b: np.ndarray) -> bool:
+    """Elementwise |a - b| <= 1 bf16 ulp of b (bit patterns as uint16)."""
+    fa = oracle.bf16_to_f32(a).astype(np.float64)
+    fb = oracle.bf16_to_f32(b).astype(np.float64)
+    e = np.floor(np.log2(np.maximum(np.abs(fb), 2.0 ** -126)))
+    return bool(np.all(np.abs(fa - fb) <= 2.0 ** (e - 7)))
+
+
+def adam_close(gpu: np.ndarray, ref: np.ndarray, tol: float = ADAM_TOL):
+    d = np.abs(gpu.astype(np.float64) - ref.astype(np.float64))
+    lim = tol * (1.0 + np.abs(ref.astype(np.float64)))
+    ok = bool(np.all(d <= lim))
+    return ok, float(np.max(d / lim)) if d.size else 0.0
+
+
+def check_plan(g: abi.Group, p: oracle.Plan) -> None:
+    assert (g.S, g.P, g.P_arena) == (p.S, p.P, p.P_arena)
+    assert list(g.shard_off) == [int(x) for x in p.shard_off]
+    assert list(g.arena_off) == [int(x) for x in p.arena_off]
+    assert list(g.chunk_rows) == [int(x) for x in p.chunk_rows]
+
+
+def make_grads(g: abi.Group, wl: W.Workload, group: W.Group, step: int, tag=()) -> torch.Tensor:
+    """Per-rank bf16 gradients [N][P_arena] on the device, seeded per rank."""
+    grads = torch.empty(g.N, g.P_arena, dtype=torch.bfloat16, device="cuda")
+    for r in range(g.N):
+        W.fill_grads_bf16(grads[r], wl, group.name, *tag, step, r)
+        if group.zero_grad:
+            W.zero_param_ranges(grads[r], g.arena_off, g.numel, group.zero_grad)
+    return grads
+
+
+def run_group(wl: W.Workload, group: W.Group, *, steps: int = 1, ops=None, staged: bool = True,
+              direct_oracle: bool = False, tag=()) -> dict:
+    """Run shard -> copy-in -> copy-out -> reduce-scatter -> AdamW on the GPU and
+    in the oracle for `steps` steps; assert parity at every stage.  Returns a
+    small report."""
+    N = wl.N
+    g = abi.fsdp_plan_group(group.shapes, N)
+    p = oracle.plan(group.shapes, N)
+    check_plan(g, p)
+    NS = N * g.S
+    report = {"S": g.S, "P": g.P, "N": N, "adam_max_ratio": 0.0}
+    ops = [wl.op] if ops is None else list(ops)
+
+    # shard the full fp32 parameters
+    full = torch.empty(max(g.P_arena, 1), dtype=torch.float32, device="cuda")
+    W.fill_master(full, wl, group.name, *tag)
+    master = Guarded(NS, torch.float32)
+    abi.fsdp_shard_params(g, full, master.t)
+    torch.cuda.synchronize()
+    assert master.guards_intact(), "shard wrote outside master"
+    master_o = oracle.shard(p, f32(full)[:p.P_arena] if p.P_arena else np.zeros(0, np.float32))
+    assert bits_equal(f32(master.t), master_o), "shard: " + first_mismatch(f32(master.t), master_o)
+
+    m = Guarded(NS, torch.float32, fill=torch.zeros(NS))
+    v = Guarded(NS, torch.float32, fill=torch.zeros(NS))
+    m_o = np.zeros(NS, np.float32)
+    v_o = np.zeros(NS, np.float32)
+    hp = dict(W.ADAMW_DEFAULTS)
+
+    for step in range(1, steps + 1):
+        # stage 1: copy-in.  At step 1 both sides start from the same seeded
+        # master and must agree bit for bit.  Later steps start from each
+        # side's own AdamW result, which may differ within the AdamW
+        # tolerance; a bf16 copy may then differ by one ulp, and only where
+        # the fp32 masters differ.
+        ag = Guarded(NS, torch.bfloat16)
+        abi.fsdp_copy_in(g, master.t, ag.t)
+        torch.cuda.synchronize()
+        assert ag.guards_intact(), "copy-in wrote outside ag"
+        ag_o = oracle.copy_in(p, master_o)
+        ag_h = u16(ag.t)
+        if step == 1:
+            assert bits_equal(ag_h, ag_o), f"copy-in: " + first_mismatch(ag_h, ag_o)
+        else:
+            diff = ag_h != ag_o
+            assert not np.any(diff & (f32(master.t).view(np.uint32) == master_o.view(np.uint32)))
+            assert bf16_within_ulp(ag_h[diff], ag_o[diff])
+
+        # stage 2: copy-out (gaps keep their sentinel on both sides)
+        arena = Guarded(g.P_arena, torch.bfloat16)
+        abi.fsdp_copy_out(g, ag.t, arena.t)
+        torch.cuda.synchronize()
+        assert arena.guards_intact(), "copy-out wrote outside the arena"
+        arena_o = oracle.copy_out(p, ag_o, np.full(p.P_arena, 0x3BEF, np.uint16))
+        arena_h = u16(arena.t)
+        if step == 1:
+            assert bits_equal(arena_h, arena_o), "copy-out: " + first_mismatch(arena_h, arena_o)
+        else:
+            # copy-out moves every real element once: differences carry over
+            # one for one from the copy-in (pads are equal on both sides)
+            assert int(np.sum(arena_h != arena_o)) == int(np.sum(ag_h != ag_o))
+            assert bf16_within_ulp(arena_h[arena_h != arena_o], arena_o[arena_h != arena_o])
+        del ag, arena
+
+        # stages 3 + 4: reduce-scatter
+        grads = make_grads(g, wl, group, step, tag)
+        grads_h = u16(grads)
+        red = None
+        red_o = None
+        for op in ops:
+            red = Guarded(NS, torch.float32)
+            abi.fsdp_rs_reduce(g, grads, op, red.t)
+            torch.cuda.synchronize()
+            assert red.guards_intact(), "reduce wrote outside reduced"
+            if direct_oracle:
+                red_o = oracle.reduce_scatter_direct(p, grads_h, op)
+            else:
+                red_o = oracle.reduce_scatter(p, grads_h, op)
+            assert bits_equal(f32(red.t), red_o), \
+                f"rs fused {W.OP_NAMES[op]}: " + first_mismatch(f32(red.t), red_o)
+            if staged:
+                packed = Guarded(N * NS, torch.float32)
+                red2 = Guarded(NS, torch.float32)
+                abi.fsdp_rs_reduce(g, grads, op, red2.t, packed=packed.t)
+                torch.cuda.synchronize()
+                assert packed.guards_intact() and red2.guards_intact()
+                packed_o = oracle.pack(p, grads_h)
+                assert bits_equal(f32(packed.t), packed_o), "pack: " + first_mismatch(f32(packed.t), packed_o)
+                assert bits_equal(f32(red2.t), red_o), \
+                    f"rs staged {W.OP_NAMES[op]}: " + first_mismatch(f32(red2.t), red_o)
+                del packed, red2
+        del grads
+
+        # stage 5: AdamW on the last op's reduced gradient (same bits both sides)
+        abi.fsdp_adamw_step(g, master.t, m.t, v.t, red.t, step=step, **hp)
+        torch.cuda.synchronize()
+        assert master.guards_intact() and m.guards_intact() and v.guards_intact()
+        oracle.adamw(master_o, m_o, v_o, red_o, step=step, **hp)
+        for name, gbuf, obuf in (("master", master, master_o), ("m", m, m_o), ("v", v, v_o)):
+            ok, ratio = adam_close(f32(gbuf.t), obuf)
+            report["adam_max_ratio"] = max(report["adam_max_ratio"], ratio)
+            assert ok, f"adamw {name} step {step}: max |d|/tol = {ratio}"
+    g.destroy()
+    return report

@@ -1,0 +1,125 @@
+"""GPU parity: the C-ABI kernels against the CPU oracle on seeded inputs.
+
+Bit-exact for the Shard(0) placement, copy-in, copy-out, packing and the
+rank-ordered reduction; max |gpu - oracle| <= 1e-6 * (1 + |x|) for AdamW on
+parameters and both moments.  Every buffer carries guard bands that must
+survive each call.
+
+Small cases span several units and tiles with ragged heads and tails and
+misaligned segments; the full-size cases are the five workloads at their
+real shapes, in the same launch configuration the benchmark times (the 7B
+model's 32 block groups share one plan, so one block group plus the root
+group covers every launch it makes).
+"""
+import pytest
+import torch
+
+from fully_sharded_shard_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+ALL_OPS = [W.SUM, W.AVG, W.SUM_THEN_DIV]
+
+
+@pytest.fixture(scope="module")
+def H():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from tests import _harness
+    return _harness
+
+
+def _wl(name, shapes, N, op=W.AVG, steps=2, dist="normal", scale=0.02, sigma=1e-3, zero=()):
+    g = W.Group(name, [tuple(s) for s in shapes], [f"p{i}" for i in range(len(shapes))],
+                zero_grad=list(zero))
+    return W.Workload(name, N, [g], op, 0, dist, scale, sigma, steps=steps)
+
+
+SMALL = [
+    _wl("ragged_n4", [(7, 3), (5,), (1, 32), (1,), (0, 4), (13, 9), (2, 2)], 4),
+    _wl("one_rank", [(5, 3), (4,), (1000, 7)], 1),
+    _wl("n3_odd", [(1001, 3), (17,), (3, 4099), (8191, 1)], 3),
+    _wl("n9_generic", [(3, 5), (9,), (17, 2), (4000, 13), (123, 77)], 9),
+    _wl("n12_generic", [(37, 100), (6,), (1999, 31)], 12),
+    _wl("n2_shift", [(3,), (9001, 5), (7, 1), (16385,)], 2, zero=[1]),
+    _wl("n8_tiny_rows", [(3, 1), (1, 1), (7, 8), (5, 3)], 8),
+    _wl("empty_params", [(0, 5), (0,)], 4),
+    _wl("no_params", [], 3),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
+def test_small_groups_all_ops_two_steps(H, wl):
+    H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=True)
+
+
+def test_tiny_mlp_three_steps(H):
+    wl = W.tiny_mlp()
+    rep = H.run_group(wl, wl.groups[0], steps=wl.steps, ops=ALL_OPS, staged=True)
+    assert rep["S"] == 338
+
+
+SCALED = [W.llama_block(16), W.uneven(8), W.moe(8), W.llama7b(16, layers=1)]
+
+
+@pytest.mark.parametrize("wl", SCALED, ids=[w.name for w in SCALED])
+def test_scaled_workloads(H, wl):
+    for g in wl.groups:
+        H.run_group(wl, g, steps=2, ops=ALL_OPS, staged=True)
+
+
+FULL = [W.tiny_mlp(), W.llama_block(), W.uneven(), W.moe()]
+
+
+@pytest.mark.parametrize("wl", FULL, ids=[w.name for w in FULL])
+def test_full_size_workloads(H, wl):
+    for g in wl.groups:
+        H.run_group(wl, g, steps=1, ops=[wl.op], staged=False, direct_oracle=True)
+
+
+def test_full_size_llama7b_block_and_root(H):
+    wl = W.llama7b()
+    for g in wl.groups:
+        H.run_group(wl, g, steps=1, ops=[wl.op], staged=False, direct_oracle=True)
+
+
+def test_fused_and_staged_reduce_are_deterministic(H):
+    from fully_sharded_shard_b200 import abi
+    wl = W.uneven(8)
+    grp = wl.groups[0]
+    g = abi.fsdp_plan_group(grp.shapes, wl.N)
+    grads = H.make_grads(g, wl, grp, 1)
+    outs = []
+    for packed in (None, torch.empty(wl.N * wl.N * g.S, device="cuda")):
+        for _ in range(2):
+            red = torch.empty(wl.N * g.S, device="cuda")
+            abi.fsdp_rs_reduce(g, grads, W.SUM_THEN_DIV, red, packed=packed)
+            outs.append(red)
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int32), outs[0].view(torch.int32))
+
+
+def test_host_validation_rejects_before_launch(H):
+    from fully_sharded_shard_b200 import abi
+    g = abi.fsdp_plan_group([(33, 5), (7,)], 4)
+    NS = g.N * g.S
+    buf = torch.zeros(NS + 8, device="cuda")
+    ag = torch.zeros(NS + 16, dtype=torch.bfloat16, device="cuda")
+    L = abi.lib()
+    import ctypes
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    p = lambda t, off=0: ctypes.c_void_p(t.data_ptr() + off)
+    # misaligned pointers
+    assert L.fsdp_copy_in(g.handle, p(buf, 4), p(ag), s) == abi.FSDP_EALIGN
+    assert L.fsdp_copy_out(g.handle, p(ag, 2), p(ag), s) == abi.FSDP_EALIGN
+    # null pointers, bad op, bad hyper-parameters
+    assert L.fsdp_copy_in(g.handle, None, p(ag), s) == abi.FSDP_EINVAL
+    assert L.fsdp_rs_reduce(g.handle, p(ag), 7, None, p(buf), s) == abi.FSDP_EINVAL
+    hp = abi.AdamWHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 0)   # step 0
+    assert L.fsdp_adamw_step(g.handle, p(buf), p(buf), p(buf), p(buf), ctypes.byref(hp), s) == abi.FSDP_EINVAL
+    hp = abi.AdamWHparams(1e-3, 1.0, 0.999, 1e-8, 0.0, 1)   # beta1 == 1
+    assert L.fsdp_adamw_step(g.handle, p(buf), p(buf), p(buf), p(buf), ctypes.byref(hp), s) == abi.FSDP_EINVAL
+    with pytest.raises(abi.FsdpError):
+        abi.fsdp_rs_reduce(g, ag, 5, buf)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(buf) == 0 and torch.count_nonzero(ag.view(torch.int16)) == 0

@@ -70,12 +70,14 @@ def _gather_reduced(p, red, i):
     return np.concatenate(parts)
 
 
+@pytest.mark.parametrize("form", ["packed", "direct"])
 @pytest.mark.parametrize("op", [W.SUM, W.AVG, W.SUM_THEN_DIV], ids=["SUM", "AVG", "SUM_THEN_DIV"])
 @pytest.mark.parametrize("name,shapes,N", GROUPS, ids=[g[0] for g in GROUPS])
-def test_reduce_scatter_then_all_gather_equals_all_reduce(oracle, name, shapes, N, op):
+def test_reduce_scatter_then_all_gather_equals_all_reduce(oracle, name, shapes, N, op, form):
     p = oracle.plan(shapes, N)
     grads = _rank_grads(shapes, N, seed=11)
-    red = oracle.reduce_scatter(p, _arena(p, grads), op)
+    rs = oracle.reduce_scatter if form == "packed" else oracle.reduce_scatter_direct
+    red = rs(p, _arena(p, grads), op)
     for i in range(p.n):
         want = _allreduce(grads, i, op).numpy()
         got = _gather_reduced(p, red, i)
@@ -104,6 +106,16 @@ def test_avg_sum_relations(oracle, name, shapes, N):
         assert np.array_equal(s.view(np.uint32), (avg * np.float32(N)).view(np.uint32))
     if N == 1:
         assert np.array_equal(s.view(np.uint32), avg.view(np.uint32))
+
+
+@pytest.mark.parametrize("op", [W.SUM, W.AVG, W.SUM_THEN_DIV], ids=["SUM", "AVG", "SUM_THEN_DIV"])
+@pytest.mark.parametrize("name,shapes,N", GROUPS, ids=[g[0] for g in GROUPS])
+def test_direct_form_equals_packed_form(oracle, name, shapes, N, op):
+    p = oracle.plan(shapes, N)
+    a = _arena(p, _rank_grads(shapes, N, seed=15))
+    x = oracle.reduce_scatter(p, a, op)
+    y = oracle.reduce_scatter_direct(p, a, op)
+    assert np.array_equal(x.view(np.uint32), y.view(np.uint32))
 
 
 def test_world_size_one_is_a_cast(oracle):
