@@ -119,7 +119,10 @@ def test_host_validation_rejects_before_launch(H):
     assert L.fsdp_adamw_step(g.handle, p(buf), p(buf), p(buf), p(buf), ctypes.byref(hp), s) == abi.FSDP_EINVAL
     hp = abi.AdamWHparams(1e-3, 1.0, 0.999, 1e-8, 0.0, 1)   # beta1 == 1
     assert L.fsdp_adamw_step(g.handle, p(buf), p(buf), p(buf), p(buf), ctypes.byref(hp), s) == abi.FSDP_EINVAL
+    grads = torch.zeros(g.N * g.P_arena, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(abi.FsdpError):
-        abi.fsdp_rs_reduce(g, ag, 5, buf)
+        abi.fsdp_rs_reduce(g, grads, 5, buf)
+    with pytest.raises(ValueError):
+        abi.fsdp_rs_reduce(g, grads[:5], W.AVG, buf)      # too small: caught in the binding
     torch.cuda.synchronize()
     assert torch.count_nonzero(buf) == 0 and torch.count_nonzero(ag.view(torch.int16)) == 0
