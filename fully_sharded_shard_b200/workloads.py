@@ -148,6 +148,9 @@ def llama7b(scale: int = 1, layers: int = 32) -> Workload:
 
 
 def by_name(name: str) -> Workload:
+    """A workload by name; ``<name>_div<k>`` divides its dims by k and
+    ``llama7b..._l<L>`` keeps L blocks (small cases for profiling)."""
+    import re
     table = {
         "tiny_mlp": tiny_mlp,
         "llama_block": llama_block,
@@ -155,7 +158,20 @@ def by_name(name: str) -> Workload:
         "moe": moe,
         "llama7b": llama7b,
     }
-    return table[name]()
+    if name in table:
+        return table[name]()
+    m = re.fullmatch(r"(llama_block|uneven|moe|llama7b)(?:_div(\d+))?(?:_l(\d+))?", name)
+    if not m:
+        raise KeyError(name)
+    base, div, layers = m.group(1), int(m.group(2) or 1), m.group(3)
+    if base == "llama7b":
+        wl = llama7b(div, layers=int(layers)) if layers else llama7b(div)
+    else:
+        if layers:
+            raise KeyError(name)
+        wl = table[base](div) if div != 1 else table[base]()
+    wl.name = name
+    return wl
 
 
 # ---------------------------------------------------------------------------
