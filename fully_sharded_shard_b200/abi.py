@@ -71,6 +71,8 @@ def _load() -> ctypes.CDLL:
     L.fsdp_copy_out.argtypes = [vp, vp, vp, vp]
     L.fsdp_rs_reduce.argtypes = [vp, vp, i32, vp, vp, vp]
     L.fsdp_adamw_step.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp]
+    L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
+    L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
     L.fsdp_status_string.argtypes = [ctypes.c_int]
     L.fsdp_status_string.restype = ctypes.c_char_p
     for name in ("fsdp_plan_group", "fsdp_group_sizes", "fsdp_group_param_offsets",
@@ -90,6 +92,18 @@ def lib() -> ctypes.CDLL:
 def _check(status: int, where: str) -> None:
     if status != FSDP_OK:
         raise FsdpError(status, where)
+
+
+def _descs(shapes):
+    shapes = [tuple(int(d) for d in s) for s in shapes]
+    arr = (ParamDesc * max(1, len(shapes)))()
+    for i, s in enumerate(shapes):
+        if len(s) > FSDP_MAX_NDIM:
+            raise ValueError(f"parameter {i}: more than {FSDP_MAX_NDIM} dims")
+        arr[i].ndim = len(s)
+        for k, d in enumerate(s):
+            arr[i].shape[k] = d
+    return shapes, arr
 
 
 class Group:
@@ -209,3 +223,20 @@ def fsdp_adamw_step(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Te
                                 _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
                                 _ptr(grad, _F32, n, "grad"), ctypes.byref(hp),
                                 _stream(stream, master)), "fsdp_adamw_step")
+
+
+FSDP_NOALLOC_MAX_UNITS = 131072
+
+
+def fsdp_rs_reduce_noalloc(shapes: Sequence[Sequence[int]], world_size: int,
+                           grads: torch.Tensor, op: int, reduced: torch.Tensor,
+                           *, P_arena: int, S: int, stream=None):
+    """The fused reduce-scatter without any allocation (no plan object): for
+    callers that cannot allocate device memory.  P_arena and S size-check the
+    tensors here; the library derives them again from the shapes."""
+    shapes, arr = _descs(shapes)
+    N = int(world_size)
+    _check(_lib.fsdp_rs_reduce_noalloc(arr, len(shapes), N,
+                                       _ptr(grads, _B16, N * P_arena, "grads"), int(op),
+                                       _ptr(reduced, _F32, N * S, "reduced"),
+                                       _stream(stream, reduced)), "fsdp_rs_reduce_noalloc")

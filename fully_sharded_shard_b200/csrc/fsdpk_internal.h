@@ -101,5 +101,10 @@ cudaError_t launch_adamw(const fsdp_group& g, float* master, float* m, float* v,
                          const float* grad, const AdamScalars& sc, cudaStream_t st);
 cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
                          cudaStream_t st);
+// The fused reduce-scatter over a caller-supplied unit table (device memory)
+// instead of a plan's own table.
+cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Unit* units,
+                                  int64_t n_units, const uint16_t* grads, int op, float* reduced,
+                                  cudaStream_t st);
 
 }  // namespace fsdpk

@@ -624,6 +624,25 @@ cudaError_t launch_rs_fused(const fsdp_group& g, const uint16_t* grads, int op, 
     }
 }
 
+cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Unit* units,
+                                  int64_t n_units, const uint16_t* grads, int op, float* reduced,
+                                  cudaStream_t st) {
+    if (n_units == 0) return cudaSuccess;
+    fsdp_group g;  // only the SM count is read when sizing the grid
+    g.sm_count = sm_count;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    switch (N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_reduce_nr<K>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_reduce_nr<0>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg,
+                                       st);
+    }
+}
+
 cudaError_t launch_rs_pack(const fsdp_group& g, const uint16_t* grads, float* packed,
                            cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();

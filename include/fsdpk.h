@@ -188,6 +188,47 @@ int fsdp_adamw_step(fsdp_group_t group, float* master, float* m, float* v,
                     fsdp_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Reduce-scatter without any allocation                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Largest work table fsdp_rs_reduce_noalloc accepts: one table entry per run
+ * of at most 8192 elements of a (rank, parameter) shard segment, so this
+ * covers groups of up to about 1.07e9 padded elements (N*S) when the
+ * segments are large. */
+#define FSDP_NOALLOC_MAX_UNITS 131072
+
+/* The fused reduce-scatter of fsdp_rs_reduce (packed_or_null == NULL), for
+ * callers that cannot allocate device memory: a custom allocator or memory
+ * pool that owns every byte of the device, code running where cudaMalloc is
+ * forbidden or would synchronise (inside another library's critical
+ * section, a signal-free runtime, a process whose memory budget is fixed up
+ * front).  There is no plan object: the group is described by params /
+ * n_params / world_size exactly as for fsdp_plan_group, and the work table
+ * the kernel needs is written into a fixed array in the library's own
+ * device memory (FSDP_NOALLOC_MAX_UNITS entries of 24 bytes, 3 MiB on every
+ * GPU that loads the library, held until the process exits).  Nothing is
+ * allocated on the device or the host, by this library or any library it
+ * calls.  (The pages describe no counterpart of this entry point.)
+ *   grads: bf16 [N][P_arena] (read); reduced: fp32 [N][S] (written, pads
+ *   +0); op: an fsdp_reduce_op; results are bit-identical to fsdp_rs_reduce.
+ *   P_arena and S follow the layout rules at the top of this file.
+ * The first call on each device looks up the array's device address on the
+ * device current at that time; make that first call before any stream
+ * capture.  The table is copied from host memory with cudaMemcpyAsync on
+ * `stream` before the kernel, so the call returns once the copy is staged.
+ * Every call shares the one array and leaves its last table there: calls on
+ * the same device that overlap on the GPU (different streams without
+ * ordering between them) race; serialise them on one stream.  Host threads
+ * are serialised inside the call.
+ * Errors: FSDP_EINVAL for the same argument errors as fsdp_plan_group and
+ * fsdp_rs_reduce, and for a group that needs more than
+ * FSDP_NOALLOC_MAX_UNITS table entries (nothing is enqueued then);
+ * FSDP_EALIGN; FSDP_ECUDA. */
+int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_params,
+                           int32_t world_size, const uint16_t* grads, int32_t op,
+                           float* reduced, fsdp_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Misc                                                                     */
 /* ------------------------------------------------------------------------ */
 
