@@ -1,0 +1,77 @@
+"""Host-side logic of bench.py without a GPU: the byte model, the
+max-over-ranks timing reduction across two gloo ranks, the clock-sample
+parser and the reference arm (the oracle on the host cores)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from fully_sharded_shard_b200 import workloads as W  # noqa: E402
+
+
+def test_byte_model_is_42_plus_2n_per_unpadded_param(oracle):
+    for N in (2, 6, 8):
+        assert bench.group_bytes(N, 1000, N * 1000) == (42 + 2 * N) * N * 1000
+    wl = W.llama7b()
+    total = 0
+    for g in wl.groups:
+        p = oracle.plan(g.shapes, wl.N)
+        total += g.repeat * bench.group_bytes(wl.N, p.S, p.P)
+    assert total == 58 * 6_738_415_616 == 390_828_105_728
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank(rank, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE="2", LOCAL_RANK=str(rank))
+    bench.init_dist("gloo")
+    v = bench.max_over_ranks(10.0 + 5.0 * rank)
+    bench.barrier()
+    with open(os.path.join(out, f"{rank}.txt"), "w") as f:
+        f.write(repr(v))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks(tmp_path):
+    mp.spawn(_rank, args=(_free_port(), str(tmp_path)), nprocs=2, join=True)
+    for r in range(2):
+        assert float(open(tmp_path / f"{r}.txt").read()) == 15.0
+
+
+def test_clock_sampler_parses_nvidia_smi_rows(tmp_path):
+    cs = bench.ClockSampler(0)
+    with open(cs.out.name, "w") as f:
+        f.write("0, 1965, 1965, 650.2, 0x0, Not Active, Not Active, Not Active, Active\n")
+        f.write("0, 1950, 1965, 700.1, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("0, 345, 1965, 90.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    cs.proc = type("P", (), {"terminate": lambda s: None, "wait": lambda s, timeout=None: 0})()
+    rep = cs.stop()
+    assert rep["sm_max_mhz"] == 1965 and rep["samples"] == 3 and rep["samples_under_load"] == 2
+    assert rep["sm_mhz"] == 1957.5 and rep["reasons"] == ["sw_power_cap"]
+
+
+def test_reference_arm_prints_one_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "llama7b_div16_l1", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["unit"] == "GB/s" and out["value"] > 0
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["metric"] == bench.METRIC
