@@ -60,6 +60,18 @@ def group_bytes(N: int, S: int, P: int) -> int:
     return sum(stage_bytes(N, S, P).values())
 
 
+def fused_stage_bytes(N: int, S: int, P: int) -> dict:
+    """The step with the reduce-scatter, AdamW and the next step's copy-in
+    fused into one pass: copy-out, then one kernel that reads the N ranks'
+    gradients and master/m/v and writes master/m/v and the bf16 all-gather
+    input of the next step."""
+    Pp = N * S
+    return {
+        "copy_out": 2 * Pp + 2 * P,
+        "rs_adamw_copy_in": 2 * N * P + 24 * Pp + 2 * Pp,
+    }
+
+
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
@@ -247,6 +259,53 @@ class Model:
             for k, b in stage_bytes(N, g.S, g.P).items():
                 self.stage_bytes[k] += b
         self.launches_per_step = 4 * len(self.instances)
+        self.ag_groups = None
+
+    def enable_fused(self):
+        """Per-group bf16 all-gather buffers: the fused update writes the next
+        step's all-gather input for each group, so each group keeps its own."""
+        import torch
+        from fully_sharded_shard_b200 import abi
+        self.ag_groups = []
+        for gi, master, m, v, pj in self.instances:
+            g = self.plans[gi]
+            ag = torch.empty(max(g.N * g.S, 1), dtype=torch.bfloat16, device=self.device)
+            abi.fsdp_copy_in(g, master, ag)
+            self.ag_groups.append(ag)
+        torch.cuda.synchronize(self.device)
+        N = self.wl.N
+        self.fused_bytes = {k: 0 for k in ("copy_out", "rs_adamw_copy_in")}
+        for i in self.instances:
+            g = self.plans[i[0]]
+            for k, b in fused_stage_bytes(N, g.S, g.P).items():
+                self.fused_bytes[k] += b
+
+    def fused_step(self, stream, events=None):
+        """One step with the reduce-scatter, AdamW and next copy-in fused."""
+        import torch
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200 import workloads as W
+        self.step_count += 1
+        hp = dict(W.ADAMW_DEFAULTS)
+        for idx, (gi, master, m, v, pj) in enumerate(self.instances):
+            g = self.plans[gi]
+            ag = self.ag_groups[idx]
+            calls = (
+                ("copy_out", lambda: abi.fsdp_copy_out(g, ag, self.arena, stream)),
+                ("rs_adamw_copy_in", lambda: abi.fsdp_rs_adamw_step(
+                    g, self.grads[gi][pj], self.wl.op, master, m, v, step=self.step_count,
+                    ag_next=ag, stream=stream, **hp)),
+            )
+            for name, fn in calls:
+                if events is None:
+                    fn()
+                else:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                    events[name].append((e0, e1))
 
     def run_group(self, idx, stream, step, grads=None, events=None):
         """Enqueue the four stages of group instance `idx` on `stream`.
@@ -351,6 +410,10 @@ def run_ours(args, wl, device, rank, ws):
     if not args.no_e2e:
         e2e = run_e2e(args, model, device, stream, ws)
 
+    fused = None
+    if not args.no_fused:
+        fused = run_fused(args, model, device, stream, ws, ms_step, peak)
+
     out = {
         "metric": METRIC,
         "value": round(gbs, 1),
@@ -383,9 +446,50 @@ def run_ours(args, wl, device, rank, ws):
         "gpu_launches": model.launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
+        "fused_step": fused,
         "setup_s": round(setup_s, 1),
     }
     return out, model
+
+
+def run_fused(args, model, device, stream, ws, ms_unfused, peak):
+    """Time the fused step (copy-out, then reduce-scatter + AdamW + next
+    copy-in in one kernel per group) on the same state, under its own byte
+    model."""
+    import torch
+    model.enable_fused()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            model.fused_step(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        model.fused_step(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
+    events = {k: [] for k in ("copy_out", "rs_adamw_copy_in")}
+    model.fused_step(stream, events=events)
+    torch.cuda.synchronize(device)
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in events.items()}
+    total = sum(model.fused_bytes.values())
+    return {
+        "ms_per_step": round(ms, 3),
+        "bytes_per_step": total,
+        "bytes_per_param": round(total / model.P_total, 3),
+        "value": round(ws * total / (ms * 1e-3) / 1e9, 1),
+        "unit": "GB/s (own byte model)",
+        "frac_of_measured_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+        "params_per_s": round(ws * model.P_total / (ms * 1e-3), 1),
+        "speedup_vs_unfused_step": round(ms_unfused / ms, 3),
+        "stages": {k: {"ms_per_step": round(stage_ms[k], 3),
+                       "GBps": round(model.fused_bytes[k] / (stage_ms[k] * 1e-3) / 1e9, 1)}
+                   for k in stage_ms},
+        "launches_per_step": 2 * len(model.instances),
+    }
 
 
 def run_e2e(args, model, device, stream, ws):
@@ -556,6 +660,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--grad-pool", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -8,7 +8,9 @@ module without the built library raises, and every non-OK status raises
 
 Function names follow the C entry points:
 ``fsdp_plan_group``, ``fsdp_shard_params``, ``fsdp_copy_in``,
-``fsdp_copy_out``, ``fsdp_rs_reduce``, ``fsdp_adamw_step``.
+``fsdp_copy_out``, ``fsdp_rs_reduce``, ``fsdp_adamw_step``,
+``fsdp_rs_adamw_step`` (reduce-scatter + AdamW + next copy-in, fused) and
+``fsdp_rs_reduce_noalloc``.
 """
 from __future__ import annotations
 
@@ -71,6 +73,9 @@ def _load() -> ctypes.CDLL:
     L.fsdp_copy_out.argtypes = [vp, vp, vp, vp]
     L.fsdp_rs_reduce.argtypes = [vp, vp, i32, vp, vp, vp]
     L.fsdp_adamw_step.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp]
+    L.fsdp_rs_adamw_step.argtypes = [vp, vp, i32, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp,
+                                     vp, vp]
+    L.fsdp_rs_adamw_step.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
     L.fsdp_status_string.argtypes = [ctypes.c_int]
@@ -224,6 +229,22 @@ def fsdp_adamw_step(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Te
                                 _ptr(grad, _F32, n, "grad"), ctypes.byref(hp),
                                 _stream(stream, master)), "fsdp_adamw_step")
 
+
+
+def fsdp_rs_adamw_step(g: Group, grads: torch.Tensor, op: int, master: torch.Tensor,
+                       m: torch.Tensor, v: torch.Tensor, *, lr: float, beta1: float,
+                       beta2: float, eps: float, weight_decay: float, step: int,
+                       ag_next: Optional[torch.Tensor] = None,
+                       reduced: Optional[torch.Tensor] = None, stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = g.N * g.S
+    _check(_lib.fsdp_rs_adamw_step(g.handle, _ptr(grads, _B16, g.N * g.P_arena, "grads"),
+                                   int(op), _ptr(master, _F32, n, "master"),
+                                   _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                   ctypes.byref(hp), _ptr(ag_next, _B16, n, "ag_next"),
+                                   _ptr(reduced, _F32, n, "reduced"),
+                                   _stream(stream, master)), "fsdp_rs_adamw_step")
 
 FSDP_NOALLOC_MAX_UNITS = 131072
 

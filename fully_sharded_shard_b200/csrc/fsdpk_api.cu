@@ -72,7 +72,32 @@ int check_device(const fsdp_group* g) {
 
 }  // namespace
 
+namespace {
+
+// AdamW hyper-parameters -> the per-step scalars (binary64 on the host).
+bool adam_scalars(const fsdp_adamw_hparams* hp, fsdpk::AdamScalars* sc) {
+    if (!(hp->step >= 1) || !(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
+        !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) ||
+        !std::isfinite(hp->weight_decay) || !std::isfinite(hp->lr))
+        return false;
+    const double t = (double)hp->step;
+    const double bc1 = 1.0 - std::pow(hp->beta1, t);
+    const double bc2 = 1.0 - std::pow(hp->beta2, t);
+    sc->decay = (float)(1.0 - hp->lr * hp->weight_decay);
+    sc->beta1 = (float)hp->beta1;
+    sc->omb1 = (float)(1.0 - hp->beta1);
+    sc->beta2 = (float)hp->beta2;
+    sc->omb2 = (float)(1.0 - hp->beta2);
+    sc->step_size = (float)(hp->lr / bc1);
+    sc->inv_bc2_sqrt = (float)(1.0 / std::sqrt(bc2));
+    sc->eps = (float)hp->eps;
+    return true;
+}
+
+}  // namespace
+
 extern "C" {
+
 
 int fsdp_abi_version(void) { return FSDP_ABI_VERSION; }
 
@@ -331,27 +356,33 @@ int fsdp_adamw_step(fsdp_group_t g, float* master, float* m, float* v, const flo
     const int64_t NS = (int64_t)g->N * g->S;
     if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr || grad == nullptr))
         return FSDP_EINVAL;
-    if (!(hp->step >= 1) || !(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
-        !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) ||
-        !std::isfinite(hp->weight_decay) || !std::isfinite(hp->lr))
-        return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!adam_scalars(hp, &sc)) return FSDP_EINVAL;
     if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad))
         return FSDP_EALIGN;
     int st = check_device(g);
     if (st != FSDP_OK) return st;
-    const double t = (double)hp->step;
-    const double bc1 = 1.0 - std::pow(hp->beta1, t);
-    const double bc2 = 1.0 - std::pow(hp->beta2, t);
-    fsdpk::AdamScalars sc;
-    sc.decay = (float)(1.0 - hp->lr * hp->weight_decay);
-    sc.beta1 = (float)hp->beta1;
-    sc.omb1 = (float)(1.0 - hp->beta1);
-    sc.beta2 = (float)hp->beta2;
-    sc.omb2 = (float)(1.0 - hp->beta2);
-    sc.step_size = (float)(hp->lr / bc1);
-    sc.inv_bc2_sqrt = (float)(1.0 / std::sqrt(bc2));
-    sc.eps = (float)hp->eps;
     cudaError_t e = fsdpk::launch_adamw(*g, master, m, v, grad, sc, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_rs_adamw_step(fsdp_group_t g, const uint16_t* grads, int32_t op, float* master,
+                       float* m, float* v, const fsdp_adamw_hparams* hp, uint16_t* ag_next,
+                       float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr || hp == nullptr) return FSDP_EINVAL;
+    if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr)) return FSDP_EINVAL;
+    if (g->P > 0 && grads == nullptr) return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!adam_scalars(hp, &sc)) return FSDP_EINVAL;
+    if (!aligned16(grads) || !aligned16(master) || !aligned16(m) || !aligned16(v) ||
+        !aligned16(ag_next) || !aligned16(reduced))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_rs_adamw(*g, grads, op, master, m, v, sc, ag_next, reduced,
+                                           (cudaStream_t)stream);
     return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
 }
 

@@ -107,4 +107,10 @@ cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Un
                                   int64_t n_units, const uint16_t* grads, int op, float* reduced,
                                   cudaStream_t st);
 
+// Fused reduce-scatter + AdamW (+ optional next-step copy-in into ag_next and
+// optional reduced-gradient output).
+cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, float* master,
+                            float* m, float* v, const AdamScalars& sc, uint16_t* ag_next,
+                            float* reduced, cudaStream_t st);
+
 }  // namespace fsdpk

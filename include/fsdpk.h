@@ -187,6 +187,29 @@ int fsdp_adamw_step(fsdp_group_t group, float* master, float* m, float* v,
                     const float* grad, const fsdp_adamw_hparams* hparams,
                     fsdp_stream_t stream);
 
+/* Stages 3 + 4 + 5 fused, followed by the next step's stage 1: the
+ * reduce-scatter of fsdp_rs_reduce (fused path), the AdamW update of
+ * fsdp_adamw_step on the reduced gradient, and the copy-in of
+ * fsdp_copy_in on the updated master, in one pass over [N][S].  It follows the
+ * lifecycle of [MS] Working Principle (reduce-scatter, then the sharded
+ * update, then the next all-gather): the reduced gradient stays in registers
+ * and the updated fp32 master is cast while it is still in registers.
+ * Results are the same bits as running fsdp_rs_reduce, fsdp_adamw_step and
+ * fsdp_copy_in in turn.
+ *   grads: bf16 [N][P_arena] (read); op: an fsdp_reduce_op;
+ *   master, m, v: fp32 [N][S] (updated in place); hparams as for
+ *   fsdp_adamw_step;
+ *   ag_next_or_null: bf16 [N][S] receiving bf16_rn(updated master), +0 in
+ *   pad rows (the next all-gather's input), or NULL;
+ *   reduced_or_null: fp32 [N][S] receiving the reduced gradient, or NULL.
+ * Algorithmic bytes: 2N per real element + 24 (+2 with ag, +4 with reduced)
+ * per padded element.  Errors as for fsdp_rs_reduce and fsdp_adamw_step. */
+int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32_t op,
+                       float* master, float* m, float* v,
+                       const fsdp_adamw_hparams* hparams,
+                       uint16_t* ag_next_or_null, float* reduced_or_null,
+                       fsdp_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Reduce-scatter without any allocation                                    */
 /* ------------------------------------------------------------------------ */

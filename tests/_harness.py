@@ -214,3 +214,68 @@ def run_group(wl: W.Workload, group: W.Group, *, steps: int = 1, ops=None, stage
             assert ok, f"adamw {name} step {step}: max |d|/tol = {ratio}"
     g.destroy()
     return report
+
+
+def run_group_fused(wl: W.Workload, group: W.Group, *, steps: int = 1, op=None,
+                    direct_oracle: bool = False, tag=()) -> dict:
+    """The fused reduce-scatter + AdamW + next copy-in against (a) the three
+    separate GPU stages on a copy of the same state (bit for bit) and (b) the
+    oracle's composition reduce_scatter -> adamw -> copy_in (reduced gradient
+    bit for bit, AdamW within tolerance, bf16 copy within the AdamW band)."""
+    N = wl.N
+    op = wl.op if op is None else op
+    g = abi.fsdp_plan_group(group.shapes, N)
+    p = oracle.plan(group.shapes, N)
+    check_plan(g, p)
+    NS = N * g.S
+    full = torch.empty(max(g.P_arena, 1), dtype=torch.float32, device="cuda")
+    W.fill_master(full, wl, group.name, *tag)
+    master = Guarded(NS, torch.float32)
+    abi.fsdp_shard_params(g, full, master.t)
+    torch.cuda.synchronize()
+    master_o = oracle.shard(p, f32(full)[:p.P_arena] if p.P_arena else np.zeros(0, np.float32))
+    m = Guarded(NS, torch.float32, fill=torch.zeros(NS))
+    v = Guarded(NS, torch.float32, fill=torch.zeros(NS))
+    # the unfused GPU path on a copy of the same state
+    mu, vu = torch.zeros(NS, device="cuda"), torch.zeros(NS, device="cuda")
+    masteru = master.t.clone()
+    m_o = np.zeros(NS, np.float32)
+    v_o = np.zeros(NS, np.float32)
+    hp = dict(W.ADAMW_DEFAULTS)
+    report = {"adam_max_ratio": 0.0}
+    for step in range(1, steps + 1):
+        grads = make_grads(g, wl, group, step, tag)
+        grads_h = u16(grads)
+        ag = Guarded(NS, torch.bfloat16)
+        red = Guarded(NS, torch.float32)
+        abi.fsdp_rs_adamw_step(g, grads, op, master.t, m.t, v.t, step=step, ag_next=ag.t,
+                               reduced=red.t, **hp)
+        # unfused GPU stages
+        redu = torch.empty(NS, device="cuda")
+        agu = torch.empty(NS, dtype=torch.bfloat16, device="cuda")
+        abi.fsdp_rs_reduce(g, grads, op, redu)
+        abi.fsdp_adamw_step(g, masteru, mu, vu, redu, step=step, **hp)
+        abi.fsdp_copy_in(g, masteru, agu)
+        torch.cuda.synchronize()
+        for buf in (master, m, v, ag, red):
+            assert buf.guards_intact(), "fused kernel wrote outside a buffer"
+        for name, a, b in (("master", master.t, masteru), ("m", m.t, mu), ("v", v.t, vu),
+                           ("reduced", red.t, redu)):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32)), f"fused != unfused {name}"
+        assert torch.equal(ag.t.view(torch.int16), agu.view(torch.int16)), "fused != unfused ag"
+        # oracle composition
+        red_o = (oracle.reduce_scatter_direct if direct_oracle else oracle.reduce_scatter)(p, grads_h, op)
+        assert bits_equal(f32(red.t), red_o), "fused reduced: " + first_mismatch(f32(red.t), red_o)
+        oracle.adamw(master_o, m_o, v_o, red_o, step=step, **hp)
+        for name, gbuf, obuf in (("master", master, master_o), ("m", m, m_o), ("v", v, v_o)):
+            ok, ratio = adam_close(f32(gbuf.t), obuf)
+            report["adam_max_ratio"] = max(report["adam_max_ratio"], ratio)
+            assert ok, f"fused adamw {name} step {step}: max |d|/tol = {ratio}"
+        ag_o = oracle.copy_in(p, master_o)
+        ag_h = u16(ag.t)
+        diff = ag_h != ag_o
+        assert not np.any(diff & (f32(master.t).view(np.uint32) == master_o.view(np.uint32)))
+        assert bf16_within_adam_band(ag_h[diff], ag_o[diff])
+        del grads, ag, red, redu, agu
+    g.destroy()
+    return report

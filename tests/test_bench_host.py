@@ -75,3 +75,8 @@ def test_reference_arm_prints_one_json_line():
     assert out["impl"] == "reference" and out["unit"] == "GB/s" and out["value"] > 0
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["metric"] == bench.METRIC
+
+
+def test_fused_byte_model_is_30_plus_2n_per_unpadded_param():
+    for N in (2, 6, 8):
+        assert sum(bench.fused_stage_bytes(N, 1000, N * 1000).values()) == (30 + 2 * N) * N * 1000

@@ -82,6 +82,26 @@ def test_full_size_llama7b_block_and_root(H):
         H.run_group(wl, g, steps=1, ops=[wl.op], staged=False, direct_oracle=True)
 
 
+FUSED = [
+    _wl("fused_ragged_n4", [(7, 3), (5,), (1, 32), (1,), (0, 4), (13, 9), (2, 2)], 4, op=W.SUM),
+    _wl("fused_n3_odd", [(1001, 3), (17,), (3, 4099), (8191, 1)], 3, op=W.SUM_THEN_DIV),
+    _wl("fused_n12", [(37, 100), (6,), (1999, 31)], 12),
+    _wl("fused_n2_shift", [(3,), (9001, 5), (7, 1), (16385,)], 2, zero=[1]),
+]
+
+
+@pytest.mark.parametrize("wl", FUSED + [W.tiny_mlp(), W.uneven(8), W.moe(8)],
+                         ids=[w.name for w in FUSED] + ["tiny_mlp", "uneven_div8", "moe_div8"])
+def test_fused_rs_adamw_copy_in(H, wl):
+    for g in wl.groups:
+        H.run_group_fused(wl, g, steps=3)
+
+
+def test_fused_full_size_llama7b_block(H):
+    wl = W.llama7b()
+    H.run_group_fused(wl, wl.groups[0], steps=1, direct_oracle=True)
+
+
 def test_fused_and_staged_reduce_are_deterministic(H):
     from fully_sharded_shard_b200 import abi
     wl = W.uneven(8)
