@@ -194,7 +194,7 @@ __device__ __forceinline__ void zero_f32_run(float* __restrict__ dst, int64_t le
 template <bool SHIFTED>
 __device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_al,
                                               uint16_t* __restrict__ dst, int nvec, int D) {
-    constexpr int V = 4;
+    constexpr int V = SHIFTED ? 2 : 4;
     const uint4* s = reinterpret_cast<const uint4*>(src_al);
     uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll 1
@@ -221,7 +221,7 @@ __device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_a
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 5)
 k_copy_out(const uint16_t* __restrict__ ag, uint16_t* __restrict__ arena,
            const Unit* __restrict__ units, int64_t n_units) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
@@ -614,10 +614,12 @@ __device__ __forceinline__ void load_pmv8(const FusedOut& o, int64_t k, float4 (
 }
 
 // Rank-ordered fold of 8 elements; NR = N at compile time (1..8) or 0 (any).
+// A misaligned run folds its ranks in batches of 4 (two 16-byte vectors per
+// rank would otherwise be live at once next to master/m/v).
 template <int NR, bool SHIFTED>
 __device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64_t stride, int N,
                                       int q, int D, float (&acc)[8]) {
-    if constexpr (NR != 0) {
+    if constexpr (NR != 0 && !SHIFTED) {
         uint4 a[NR], b[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
