@@ -21,6 +21,8 @@ Every function follows a definition from the pages (see the C file's header):
 * ``reduce_packed`` -- rank-ordered binary32 fold, SUM / AVG / SUM_THEN_DIV;
 * ``reduce_scatter_direct`` -- pack + fold from the per-rank gradients with no
   packed intermediate (same definitions, for full-size groups);
+* ``accumulate``  -- gradient accumulation without sync, fp32 left fold;
+* ``reduce_scatter_f32`` -- reduce-scatter of fp32 (accumulated) arenas;
 * ``adamw``       -- decoupled-weight-decay AdamW in binary64.
 
 Parity status: every function above is pinned by tests under ``tests/``
@@ -82,6 +84,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).argtypes = [vp, vp, i32, i32, vp, vp]
         L.or_reduce_packed.argtypes = [i32, i64, vp, i32, vp]
         L.or_reduce_scatter_direct.argtypes = [vp, vp, i32, i32, vp, i32, vp]
+        L.or_accumulate.argtypes = [vp, vp, i64, i32]
+        L.or_reduce_scatter_f32.argtypes = [vp, vp, i32, i32, vp, i32, vp]
         L.or_adamw.argtypes = [vp, vp, vp, vp, i64, f64, f64, f64, f64, f64, i64]
         _lib = L
     return _lib
@@ -227,6 +231,25 @@ def reduce_scatter_direct(p: Plan, grads: np.ndarray, op: int) -> np.ndarray:
     out = np.empty(p.N * p.S, np.float32)
     lib().or_reduce_scatter_direct(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(grads),
                                    int(op), _ptr(out))
+    return out
+
+
+def accumulate(acc: np.ndarray, grads: np.ndarray, first: bool) -> np.ndarray:
+    """In place: acc = fp32(grads) (first microbatch) or acc + fp32(grads)."""
+    assert acc.dtype == np.float32 and acc.flags["C_CONTIGUOUS"]
+    grads = np.ascontiguousarray(grads, np.uint16)
+    assert acc.size == grads.size
+    lib().or_accumulate(_ptr(acc), _ptr(grads), acc.size, int(bool(first)))
+    return acc
+
+
+def reduce_scatter_f32(p: Plan, src: np.ndarray, op: int) -> np.ndarray:
+    """Reduce-scatter of fp32 per-rank arenas [N][P_arena]."""
+    src = np.ascontiguousarray(src, np.float32)
+    assert src.size == p.N * p.P_arena
+    out = np.empty(p.N * p.S, np.float32)
+    lib().or_reduce_scatter_f32(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(src), int(op),
+                                _ptr(out))
     return out
 
 

@@ -336,6 +336,58 @@ void or_reduce_scatter_direct(const int64_t* d0, const int64_t* cols, int32_t n,
 }
 
 /* ------------------------------------------------------------------ */
+/* Gradient accumulation without sync ([ML] Other controls:            */
+/* set_requires_gradient_sync(False) accumulates the unsharded         */
+/* gradients and skips the reduce-scatter).  Accumulated in             */
+/* reduce_dtype fp32, a left fold over microbatches:                    */
+/*   first: acc[k] = fp32(g[k]);  later: acc[k] = acc[k] + fp32(g[k])   */
+/* over every element of the per-rank arenas [N][P_arena].              */
+/* ------------------------------------------------------------------ */
+void or_accumulate(float* acc, const uint16_t* grads, int64_t count, int32_t first) {
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < count; ++k) {
+        float g = or_bf16_to_f32(grads[k]);
+        acc[k] = first ? g : acc[k] + g;
+    }
+}
+
+/* Reduce-scatter of fp32 per-rank arenas [N][P_arena] (the accumulated
+ * gradients): the same packing and rank-ordered fold as
+ * or_reduce_scatter_direct, with fp32 sources (no cast needed). */
+void or_reduce_scatter_f32(const int64_t* d0, const int64_t* cols, int32_t n, int32_t N,
+                           const float* src, int32_t op, float* red) {
+    int64_t c[n > 0 ? n : 1], s[n > 0 ? n : 1], off[n > 0 ? n : 1],
+        u[n > 0 ? n : 1], sz[3];
+    or_plan(d0, cols, n, N, c, s, off, u, sz);
+    int64_t S = sz[0], A = sz[2];
+    for (int32_t j = 0; j < N; ++j) {
+        for (int32_t i = 0; i < n; ++i) {
+            int64_t v = or_valid_rows(d0[i], N, j);
+#pragma omp parallel for schedule(static)
+            for (int64_t row = 0; row < c[i]; ++row) {
+                for (int64_t col = 0; col < cols[i]; ++col) {
+                    int64_t dst = (int64_t)j * S + off[i] + row * cols[i] + col;
+                    if (row >= v) {
+                        red[dst] = 0.0f;
+                        continue;
+                    }
+                    int64_t k = u[i] + ((int64_t)j * c[i] + row) * cols[i] + col;
+                    float acc = src[k];
+                    for (int32_t r = 1; r < N; ++r) acc = acc + src[(int64_t)r * A + k];
+                    if (op == OR_AVG) acc = acc / (float)N;
+                    red[dst] = acc;
+                }
+            }
+        }
+    }
+    if (op == OR_SUM_THEN_DIV) {
+        int64_t total = (int64_t)N * S;
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < total; ++k) red[k] = red[k] / (float)N;
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* a5 AdamW (decoupled weight decay), binary64, one rounding per store */
 /* [ML] Fence 4 (AdamW built after sharding steps each shard);          */
 /* [MS] "Working Principle" (update state uses gradient slices).       */
