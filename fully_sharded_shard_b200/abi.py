@@ -76,6 +76,10 @@ def _load() -> ctypes.CDLL:
     L.fsdp_rs_adamw_step.argtypes = [vp, vp, i32, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp,
                                      vp, vp]
     L.fsdp_rs_adamw_step.restype = ctypes.c_int
+    L.fsdp_grad_accumulate.argtypes = [vp, vp, vp, i32, vp]
+    L.fsdp_grad_accumulate.restype = ctypes.c_int
+    L.fsdp_rs_reduce_accumulated.argtypes = [vp, vp, vp, i32, vp, vp]
+    L.fsdp_rs_reduce_accumulated.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
     L.fsdp_status_string.argtypes = [ctypes.c_int]
@@ -245,6 +249,24 @@ def fsdp_rs_adamw_step(g: Group, grads: torch.Tensor, op: int, master: torch.Ten
                                    ctypes.byref(hp), _ptr(ag_next, _B16, n, "ag_next"),
                                    _ptr(reduced, _F32, n, "reduced"),
                                    _stream(stream, master)), "fsdp_rs_adamw_step")
+
+
+def fsdp_grad_accumulate(g: Group, grads: torch.Tensor, acc: torch.Tensor, first: bool,
+                         stream=None):
+    n = g.N * g.P_arena
+    _check(_lib.fsdp_grad_accumulate(g.handle, _ptr(grads, _B16, n, "grads"),
+                                     _ptr(acc, _F32, n, "acc"), int(bool(first)),
+                                     _stream(stream, acc)), "fsdp_grad_accumulate")
+
+
+def fsdp_rs_reduce_accumulated(g: Group, grads: Optional[torch.Tensor], acc: torch.Tensor,
+                               op: int, reduced: torch.Tensor, stream=None):
+    n = g.N * g.P_arena
+    _check(_lib.fsdp_rs_reduce_accumulated(g.handle, _ptr(grads, _B16, n, "grads"),
+                                           _ptr(acc, _F32, n, "acc"), int(op),
+                                           _ptr(reduced, _F32, g.N * g.S, "reduced"),
+                                           _stream(stream, reduced)),
+           "fsdp_rs_reduce_accumulated")
 
 FSDP_NOALLOC_MAX_UNITS = 131072
 

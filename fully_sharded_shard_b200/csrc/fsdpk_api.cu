@@ -386,4 +386,29 @@ int fsdp_rs_adamw_step(fsdp_group_t g, const uint16_t* grads, int32_t op, float*
     return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
 }
 
+int fsdp_grad_accumulate(fsdp_group_t g, const uint16_t* grads, float* acc, int32_t first,
+                         fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if ((int64_t)g->N * g->P_arena > 0 && (grads == nullptr || acc == nullptr)) return FSDP_EINVAL;
+    if (!aligned16(grads) || !aligned16(acc)) return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_accumulate(*g, grads, acc, first ? 1 : 0, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_rs_reduce_accumulated(fsdp_group_t g, const uint16_t* grads_or_null, const float* acc,
+                               int32_t op, float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
+    if ((int64_t)g->N * g->S > 0 && reduced == nullptr) return FSDP_EINVAL;
+    if (g->P > 0 && acc == nullptr) return FSDP_EINVAL;
+    if (!aligned16(grads_or_null) || !aligned16(acc) || !aligned16(reduced)) return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_rs_reduce_acc(*g, grads_or_null, acc, op, reduced,
+                                                (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
 }  // extern "C"

@@ -113,4 +113,12 @@ cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, 
                             float* m, float* v, const AdamScalars& sc, uint16_t* ag_next,
                             float* reduced, cudaStream_t st);
 
+// Gradient accumulation without sync over [N][P_arena] in fp32, and the
+// reduce-scatter of the accumulated arenas (+ the last microbatch's bf16
+// gradients when grads is not null).
+cudaError_t launch_accumulate(const fsdp_group& g, const uint16_t* grads, float* acc, int first,
+                              cudaStream_t st);
+cudaError_t launch_rs_reduce_acc(const fsdp_group& g, const uint16_t* grads, const float* acc,
+                                 int op, float* reduced, cudaStream_t st);
+
 }  // namespace fsdpk

@@ -731,6 +731,150 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o
 }
 
 // ---------------------------------------------------------------------------
+// gradient accumulation without sync, in reduce_dtype fp32
+//   first: acc[k] = fp32(g[k]);  later: acc[k] = acc[k] + fp32(g[k])
+// over the flat per-rank arenas [N][P_arena] (a multiple of 8 elements).
+// ---------------------------------------------------------------------------
+
+constexpr int kAccV = 2;  // 8-element vectors per thread per chunk
+constexpr int64_t kAccChunk8 = (int64_t)kThreads * kAccV;
+
+__global__ void __launch_bounds__(kThreads, 3)
+k_accumulate(const uint16_t* __restrict__ g, float* __restrict__ acc, int64_t n8, int first) {
+    const uint4* g8 = reinterpret_cast<const uint4*>(g);
+    float4* a4 = reinterpret_cast<float4*>(acc);
+    const int64_t n_chunks = (n8 + kAccChunk8 - 1) / kAccChunk8;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        const int64_t q0 = c * kAccChunk8 + threadIdx.x;
+        uint4 w[kAccV];
+        float4 A[kAccV][2];
+#pragma unroll
+        for (int k = 0; k < kAccV; ++k) {
+            const int64_t q = q0 + k * kThreads;
+            if (q < n8) {
+                w[k] = __ldcs(g8 + q);
+                if (!first) {
+                    A[k][0] = __ldcs(a4 + 2 * q);
+                    A[k][1] = __ldcs(a4 + 2 * q + 1);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kAccV; ++k) {
+            const int64_t q = q0 + k * kThreads;
+            if (q < n8) {
+                float x[8];
+                unpack8(w[k], x);
+                if (!first) {
+                    const float a[8] = {A[k][0].x, A[k][0].y, A[k][0].z, A[k][0].w,
+                                        A[k][1].x, A[k][1].y, A[k][1].z, A[k][1].w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = __fadd_rn(a[e], x[e]);
+                }
+                __stcs(a4 + 2 * q, make_float4(x[0], x[1], x[2], x[3]));
+                __stcs(a4 + 2 * q + 1, make_float4(x[4], x[5], x[6], x[7]));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// reduce-scatter of the accumulated gradients (the last microbatch)
+//   red[shard_pos + e] = fold over r of x_r, x_r = acc_r[k] (+ fp32(g_r[k]))
+// with k = arena_pos + e, the same rank-ordered fold and division as
+// k_reduce_units.  A run whose source and destination are congruent mod 8
+// moves 16-byte vectors; any other run goes element by element.
+// ---------------------------------------------------------------------------
+
+template <bool WITH_G>
+__device__ __forceinline__ float acc_src1(const float* __restrict__ acc,
+                                          const uint16_t* __restrict__ g, int64_t k) {
+    float x = acc[k];
+    if constexpr (WITH_G) x = __fadd_rn(x, bf16_bits_to_f32(g[k]));
+    return x;
+}
+
+template <bool WITH_G>
+__global__ void __launch_bounds__(kThreads, 2)
+k_reduce_acc(const float* __restrict__ acc, const uint16_t* __restrict__ g, int64_t stride, int N,
+             float* __restrict__ out, const Unit* __restrict__ units, int64_t n_units,
+             int op_avg) {
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        float* dst = out + u.shard_pos;
+        if (u.is_pad) {
+            zero_f32_run(dst, len);
+            continue;
+        }
+        const int64_t s0 = u.arena_pos;
+        const bool vec = ((s0 - u.shard_pos) & 7) == 0;
+        int head = vec ? (int)((8 - (s0 & 7)) & 7) : len;
+        if (head > len) head = len;
+        for (int e = threadIdx.x; e < head; e += blockDim.x) {
+            float a = acc_src1<WITH_G>(acc, g, s0 + e);
+            for (int r = 1; r < N; ++r)
+                a = __fadd_rn(a, acc_src1<WITH_G>(acc, g, (int64_t)r * stride + s0 + e));
+            dst[e] = finish(a, avg, fN);
+        }
+        const int nvec = (len - head) >> 3;
+#pragma unroll 1
+        for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+            const int64_t k = s0 + head + 8 * (int64_t)q;
+            float accv[8];
+#pragma unroll 1
+            for (int r0 = 0; r0 < N; r0 += 4) {
+                float4 A[4][2];
+                uint4 w[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r0 + r < N) {
+                        const int64_t kr = (int64_t)(r0 + r) * stride + k;
+                        A[r][0] = __ldcs(reinterpret_cast<const float4*>(acc + kr));
+                        A[r][1] = __ldcs(reinterpret_cast<const float4*>(acc + kr) + 1);
+                        if constexpr (WITH_G) w[r] = __ldcs(reinterpret_cast<const uint4*>(g + kr));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r0 + r < N) {
+                        float x[8] = {A[r][0].x, A[r][0].y, A[r][0].z, A[r][0].w,
+                                      A[r][1].x, A[r][1].y, A[r][1].z, A[r][1].w};
+                        if constexpr (WITH_G) {
+                            float y[8];
+                            unpack8(w[r], y);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = __fadd_rn(x[e], y[e]);
+                        }
+                        if (r0 + r == 0) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) accv[e] = x[e];
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) accv[e] = __fadd_rn(accv[e], x[e]);
+                        }
+                    }
+                }
+            }
+            if (avg) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) accv[e] = __fdiv_rn(accv[e], fN);
+            }
+            store8(dst + head + 8 * q, accv);
+        }
+        const int done = head + 8 * nvec;
+        for (int e = done + threadIdx.x; e < len; e += blockDim.x) {
+            float a = acc_src1<WITH_G>(acc, g, s0 + e);
+            for (int r = 1; r < N; ++r)
+                a = __fadd_rn(a, acc_src1<WITH_G>(acc, g, (int64_t)r * stride + s0 + e));
+            dst[e] = finish(a, avg, fN);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // launch geometry
 // ---------------------------------------------------------------------------
 
@@ -901,6 +1045,34 @@ cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, 
         default:
             return launch_rs_adamw_nr<0>(g, grads, o, avg, sc, st);
     }
+}
+
+}  // namespace fsdpk
+
+namespace fsdpk {
+
+cudaError_t launch_accumulate(const fsdp_group& g, const uint16_t* grads, float* acc, int first,
+                              cudaStream_t st) {
+    const int64_t n8 = (int64_t)g.N * g.P_arena / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int64_t chunks = (n8 + kAccChunk8 - 1) / kAccChunk8;
+    k_accumulate<<<grid_for(g, (const void*)k_accumulate, chunks), kThreads, 0, st>>>(grads, acc,
+                                                                                     n8, first);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rs_reduce_acc(const fsdp_group& g, const uint16_t* grads, const float* acc,
+                                 int op, float* reduced, cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu == 0) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    if (grads != nullptr)
+        k_reduce_acc<true><<<grid_for(g, (const void*)k_reduce_acc<true>, nu), kThreads, 0, st>>>(
+            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+    else
+        k_reduce_acc<false><<<grid_for(g, (const void*)k_reduce_acc<false>, nu), kThreads, 0, st>>>(
+            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+    return cudaGetLastError();
 }
 
 }  // namespace fsdpk

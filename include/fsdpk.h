@@ -210,6 +210,30 @@ int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32_t op,
                        uint16_t* ag_next_or_null, float* reduced_or_null,
                        fsdp_stream_t stream);
 
+/* Gradient accumulation without sync ([ML] Other controls:
+ * set_requires_gradient_sync(False) accumulates the unsharded gradients and
+ * skips the reduce-scatter).  Each rank's unsharded gradient is accumulated in
+ * reduce_dtype fp32, a left fold over microbatches:
+ *   first != 0: acc[k] = fp32(grads[k]);  first == 0: acc[k] += fp32(grads[k])
+ * over every element of [N][P_arena] (gap elements included; they are never
+ * read by the reduce-scatter).  grads: bf16 [N][P_arena] (read); acc: fp32
+ * [N][P_arena] (updated; not read when first != 0).  Algorithmic bytes per
+ * element: 6 (first) or 10. */
+int fsdp_grad_accumulate(fsdp_group_t group, const uint16_t* grads, float* acc,
+                         int32_t first, fsdp_stream_t stream);
+
+/* The reduce-scatter of the last microbatch when gradients were accumulated:
+ * for each rank, x_r = acc_r (+ fp32(grads_r) when grads_or_null is not
+ * NULL, the last microbatch's own gradient), then the packing and the
+ * rank-ordered fold of fsdp_rs_reduce on the fp32 x_r.  Equal to
+ * fsdp_grad_accumulate(grads) followed by a reduce-scatter of acc, without
+ * writing acc back.  acc: fp32 [N][P_arena] (read); reduced: fp32 [N][S]
+ * (written, pads +0).  Algorithmic bytes: 6N (4N without grads) per real
+ * element + 4 per padded element. */
+int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grads_or_null,
+                               const float* acc, int32_t op, float* reduced,
+                               fsdp_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Reduce-scatter without any allocation                                    */
 /* ------------------------------------------------------------------------ */

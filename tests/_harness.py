@@ -279,3 +279,42 @@ def run_group_fused(wl: W.Workload, group: W.Group, *, steps: int = 1, op=None,
         del grads, ag, red, redu, agu
     g.destroy()
     return report
+
+
+def run_group_accumulate(wl: W.Workload, group: W.Group, *, micro: int = 3, op=None,
+                         tag=()) -> None:
+    """Gradient accumulation without sync over `micro` microbatches: the
+    accumulated fp32 arenas after every microbatch and the final reduce-scatter
+    (fused with the last microbatch, and from the accumulated arenas alone)
+    against the oracle, bit for bit."""
+    assert micro >= 2, "one microbatch needs no accumulation: use fsdp_rs_reduce"
+    N = wl.N
+    op = wl.op if op is None else op
+    g = abi.fsdp_plan_group(group.shapes, N)
+    p = oracle.plan(group.shapes, N)
+    check_plan(g, p)
+    n = N * g.P_arena
+    acc = Guarded(n, torch.float32)
+    acc_o = np.zeros(n, np.float32)
+    for t in range(1, micro):
+        grads = make_grads(g, wl, group, t, ("micro",) + tuple(tag))
+        abi.fsdp_grad_accumulate(g, grads, acc.t, first=(t == 1))
+        torch.cuda.synchronize()
+        assert acc.guards_intact()
+        oracle.accumulate(acc_o, u16(grads), first=(t == 1))
+        assert bits_equal(f32(acc.t), acc_o), f"accumulate {t}: " + first_mismatch(f32(acc.t), acc_o)
+    last = make_grads(g, wl, group, micro, ("micro",) + tuple(tag))
+    red = Guarded(N * g.S, torch.float32)
+    abi.fsdp_rs_reduce_accumulated(g, last, acc.t, op, red.t)
+    torch.cuda.synchronize()
+    assert red.guards_intact() and acc.guards_intact()
+    oracle.accumulate(acc_o, u16(last), first=False)
+    red_o = oracle.reduce_scatter_f32(p, acc_o, op)
+    assert bits_equal(f32(red.t), red_o), "rs accumulated: " + first_mismatch(f32(red.t), red_o)
+    # the same through an explicit last accumulation and a reduce of acc alone
+    abi.fsdp_grad_accumulate(g, last, acc.t, first=False)
+    red2 = torch.empty(N * g.S, device="cuda")
+    abi.fsdp_rs_reduce_accumulated(g, None, acc.t, op, red2)
+    torch.cuda.synchronize()
+    assert bits_equal(f32(red2), red_o)
+    g.destroy()

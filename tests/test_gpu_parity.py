@@ -102,6 +102,21 @@ def test_fused_full_size_llama7b_block(H):
     H.run_group_fused(wl, wl.groups[0], steps=1, direct_oracle=True)
 
 
+ACCUM = SMALL[:4] + [W.tiny_mlp(), W.uneven(8), W.moe(16), W.llama7b(16, layers=1)]
+
+
+@pytest.mark.parametrize("wl", ACCUM, ids=[w.name for w in ACCUM])
+def test_gradient_accumulation_without_sync(H, wl):
+    for g in wl.groups:
+        for op in ALL_OPS:
+            H.run_group_accumulate(wl, g, micro=3, op=op)
+
+
+def test_gradient_accumulation_two_microbatches(H):
+    wl = W.uneven(16)
+    H.run_group_accumulate(wl, wl.groups[0], micro=2)
+
+
 def test_fused_and_staged_reduce_are_deterministic(H):
     from fully_sharded_shard_b200 import abi
     wl = W.uneven(8)
