@@ -414,6 +414,14 @@ def run_ours(args, wl, device, rank, ws):
     if not args.no_fused:
         fused = run_fused(args, model, device, stream, ws, ms_step, peak)
 
+    accum = None
+    if not args.no_accumulate:
+        accum = run_accumulate(args, model, device, stream)
+
+    latency = None
+    if not args.no_latency:
+        latency = run_latency(device)
+
     out = {
         "metric": METRIC,
         "value": round(gbs, 1),
@@ -447,6 +455,8 @@ def run_ours(args, wl, device, rank, ws):
         "clocks": clocks,
         "e2e": e2e,
         "fused_step": fused,
+        "grad_accumulation": accum,
+        "tiny_latency": latency,
         "setup_s": round(setup_s, 1),
     }
     return out, model
@@ -490,6 +500,91 @@ def run_fused(args, model, device, stream, ws, ms_unfused, peak):
                    for k in stage_ms},
         "launches_per_step": 2 * len(model.instances),
     }
+
+
+def run_accumulate(args, model, device, stream, micro: int = 4):
+    """Gradient accumulation without sync on the largest repeated group:
+    micro - 1 accumulations into fp32 per-rank arenas, then the reduce-scatter
+    fused with the last microbatch.  Own byte model: 6 (first) or 10 bytes per
+    arena element per accumulation; 6N per real element + 4 per padded
+    element for the last microbatch."""
+    import torch
+    from fully_sharded_shard_b200 import abi
+    gi = max(range(len(model.plans)), key=lambda i: model.wl.groups[i].repeat)
+    g = model.plans[gi]
+    pool = model.grads[gi]
+    N = g.N
+    acc = torch.empty(N * g.P_arena, dtype=torch.float32, device=device)
+
+    def one():
+        for t in range(micro - 1):
+            abi.fsdp_grad_accumulate(g, pool[t % len(pool)], acc, first=(t == 0), stream=stream)
+        abi.fsdp_rs_reduce_accumulated(g, pool[(micro - 1) % len(pool)], acc, model.wl.op,
+                                       model.reduced, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            one()
+    torch.cuda.synchronize(device)
+    reps = max(1, args.steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / reps
+    A = N * g.P_arena
+    b = 6 * A + 10 * A * (micro - 2) + 6 * N * g.P + 4 * N * g.S
+    del acc
+    return {"group": model.wl.groups[gi].name, "microbatches": micro, "params": g.P,
+            "ms_per_group_step": round(ms, 3), "bytes": b,
+            "value": round(b / (ms * 1e-3) / 1e9, 1), "unit": "GB/s (own byte model)",
+            "launches": micro}
+
+
+def run_latency(device, reps: int = 200):
+    """The tiny MLP group (4 parameters, N = 2) is launch-bound: report the
+    step latency in microseconds, eager and with the whole step captured in a
+    CUDA graph and replayed.  (A captured step replays the AdamW step count
+    it was captured with.)"""
+    import torch
+    from fully_sharded_shard_b200 import workloads as W
+    wl = W.tiny_mlp()
+    model = Model(wl, device, 1, 0)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            model.step(stream)
+    torch.cuda.synchronize(device)
+
+    def timed(fn):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    t0 = time.perf_counter()
+    eager_us = timed(lambda: model.step(stream))
+    host_us = (time.perf_counter() - t0) * 1e6 / reps
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        model.step(stream)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        graph_us = timed(graph.replay)
+    del graph
+    return {"workload": wl.name, "launches_per_step": model.launches_per_step,
+            "eager_us_per_step": round(eager_us, 2), "eager_host_us_per_step": round(host_us, 2),
+            "graph_us_per_step": round(graph_us, 2)}
 
 
 def run_e2e(args, model, device, stream, ws):
@@ -661,6 +756,8 @@ def main(argv=None):
     ap.add_argument("--grad-pool", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fused", action="store_true")
+    ap.add_argument("--no-accumulate", action="store_true")
+    ap.add_argument("--no-latency", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
