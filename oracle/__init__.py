@@ -23,6 +23,8 @@ Every function follows a definition from the pages (see the C file's header):
   packed intermediate (same definitions, for full-size groups);
 * ``accumulate``  -- gradient accumulation without sync, fp32 left fold;
 * ``reduce_scatter_f32`` -- reduce-scatter of fp32 (accumulated) arenas;
+* ``e4m3_bits``, ``fp8_scales``, ``copy_in_fp8``, ``copy_out_fp8`` -- the FP8
+  (E4M3, per-parameter tensorwise scale) all-gather copy-in and copy-out;
 * ``adamw``       -- decoupled-weight-decay AdamW in binary64.
 
 Parity status: every function above is pinned by tests under ``tests/``
@@ -85,6 +87,16 @@ def lib() -> ctypes.CDLL:
         L.or_reduce_packed.argtypes = [i32, i64, vp, i32, vp]
         L.or_reduce_scatter_direct.argtypes = [vp, vp, i32, i32, vp, i32, vp]
         L.or_accumulate.argtypes = [vp, vp, i64, i32]
+        L.or_e4m3_bits.argtypes = [ctypes.c_float]
+        L.or_e4m3_bits.restype = ctypes.c_uint8
+        L.or_fp8_scale.argtypes = [ctypes.c_float]
+        L.or_fp8_scale.restype = ctypes.c_float
+        L.or_fp8_quant_input.argtypes = [ctypes.c_float, ctypes.c_float]
+        L.or_fp8_quant_input.restype = ctypes.c_float
+        L.or_cast_e4m3.argtypes = [vp, vp, i64]
+        L.or_fp8_scales.argtypes = [vp, vp, i32, i32, vp, vp]
+        L.or_copy_in_fp8.argtypes = [vp, vp, i32, i32, vp, vp, vp]
+        L.or_copy_out_fp8.argtypes = [vp, vp, i32, i32, vp, vp]
         L.or_reduce_scatter_f32.argtypes = [vp, vp, i32, i32, vp, i32, vp]
         L.or_adamw.argtypes = [vp, vp, vp, vp, i64, f64, f64, f64, f64, f64, i64]
         _lib = L
@@ -251,6 +263,41 @@ def reduce_scatter_f32(p: Plan, src: np.ndarray, op: int) -> np.ndarray:
     lib().or_reduce_scatter_f32(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(src), int(op),
                                 _ptr(out))
     return out
+
+
+def e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """binary32 (|x| <= 448 or NaN) -> E4M3 bytes, round to nearest even."""
+    x = np.ascontiguousarray(x, np.float32)
+    y = np.empty(x.shape, np.uint8)
+    lib().or_cast_e4m3(_ptr(x), _ptr(y), x.size)
+    return y
+
+
+def fp8_scales(p: Plan, master: np.ndarray) -> np.ndarray:
+    master = np.ascontiguousarray(master, np.float32)
+    assert master.size == p.N * p.S
+    out = np.empty(max(p.n, 1), np.float32)
+    lib().or_fp8_scales(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(master), _ptr(out))
+    return out[:p.n]
+
+
+def copy_in_fp8(p: Plan, master: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    master = np.ascontiguousarray(master, np.float32)
+    scales = np.ascontiguousarray(scales, np.float32)
+    assert master.size == p.N * p.S and scales.size == p.n
+    out = np.empty(p.N * p.S, np.uint8)
+    lib().or_copy_in_fp8(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(master), _ptr(scales),
+                         _ptr(out))
+    return out
+
+
+def copy_out_fp8(p: Plan, ag8: np.ndarray, arena8: np.ndarray | None = None) -> np.ndarray:
+    ag8 = np.ascontiguousarray(ag8, np.uint8)
+    assert ag8.size == p.N * p.S
+    if arena8 is None:
+        arena8 = np.zeros(p.P_arena, np.uint8)
+    lib().or_copy_out_fp8(_ptr(p.d0), _ptr(p.cols), p.n, p.N, _ptr(ag8), _ptr(arena8))
+    return arena8
 
 
 def adamw(master, m, v, grad, *, lr, beta1, beta2, eps, weight_decay, step):

@@ -388,6 +388,117 @@ void or_reduce_scatter_f32(const int64_t* d0, const int64_t* cols, int32_t n, in
 }
 
 /* ------------------------------------------------------------------ */
+/* FP8 all-gather copy-in ("PyTorch FSDP2 Guide: Distributed LLM        */
+/* Training with DTensor", Deep Dive "2. Native FP8 Training with       */
+/* Float8Tensor": parameters in FP8 E4M3, the all-gather moves raw FP8  */
+/* bytes).  The pages leave scaling open; reading: per-parameter        */
+/* tensorwise dynamic scaling,                                          */
+/*   amax_i  = max |x| over the whole parameter (all ranks),            */
+/*   scale_i = 448 / max(amax_i, 1e-12)            (binary32),          */
+/*   q       = e4m3_rn(clamp(x * scale_i, -448, 448)), pads 0x00.       */
+/* E4M3 here is the "fn" encoding: bias 7, 3 mantissa bits, no          */
+/* infinities, S.1111.111 is NaN, largest finite 448.                   */
+/* ------------------------------------------------------------------ */
+
+/* Round a finite |x| <= 448 (or NaN) to E4M3, nearest even, from the
+ * format's definition. */
+uint8_t or_e4m3_bits(float x) {
+    if (x != x) return 0x7F; /* NaN */
+    uint8_t sign = (f32_bits(x) >> 31) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a < 0.015625) { /* below 2^-6: subnormal grid of 2^-9 */
+        double q = nearbyint(a * 512.0); /* 0..8; 8 is the smallest normal */
+        return (uint8_t)(sign | (uint8_t)q);
+    }
+    int e = 0;
+    double m = frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+    m *= 2.0;
+    e -= 1; /* a = m * 2^e, m in [1, 2) */
+    double r = nearbyint((m - 1.0) * 8.0);
+    if (r == 8.0) {
+        r = 0.0;
+        e += 1;
+    }
+    int field = e + 7; /* 1..15 for 2^-6 <= a <= 448 */
+    return (uint8_t)(sign | (uint8_t)(field << 3) | (uint8_t)r);
+}
+
+float or_fp8_scale(float amax) {
+    float a = amax > 1e-12f ? amax : 1e-12f;
+    return 448.0f / a;
+}
+
+float or_fp8_quant_input(float x, float scale) {
+    float y = x * scale;
+    if (y > 448.0f) y = 448.0f;
+    if (y < -448.0f) y = -448.0f;
+    return y;
+}
+
+void or_cast_e4m3(const float* x, uint8_t* y, int64_t n) {
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < n; ++k) y[k] = or_e4m3_bits(x[k]);
+}
+
+/* scales[i] = 448 / max(amax_i, 1e-12), amax over parameter i's real rows */
+void or_fp8_scales(const int64_t* d0, const int64_t* cols, int32_t n, int32_t N,
+                   const float* master, float* scales) {
+    int64_t c[n > 0 ? n : 1], s[n > 0 ? n : 1], off[n > 0 ? n : 1],
+        u[n > 0 ? n : 1], sz[3];
+    or_plan(d0, cols, n, N, c, s, off, u, sz);
+    int64_t S = sz[0];
+    for (int32_t i = 0; i < n; ++i) {
+        float amax = 0.0f;
+        for (int32_t r = 0; r < N; ++r) {
+            int64_t v = or_valid_rows(d0[i], N, r);
+            for (int64_t k = 0; k < v * cols[i]; ++k) {
+                float a = fabsf(master[(int64_t)r * S + off[i] + k]);
+                if (a > amax) amax = a;
+            }
+        }
+        scales[i] = or_fp8_scale(amax);
+    }
+}
+
+void or_copy_in_fp8(const int64_t* d0, const int64_t* cols, int32_t n, int32_t N,
+                    const float* master, const float* scales, uint8_t* ag8) {
+    int64_t c[n > 0 ? n : 1], s[n > 0 ? n : 1], off[n > 0 ? n : 1],
+        u[n > 0 ? n : 1], sz[3];
+    or_plan(d0, cols, n, N, c, s, off, u, sz);
+    int64_t S = sz[0];
+#pragma omp parallel for schedule(static)
+    for (int32_t r = 0; r < N; ++r) {
+        for (int32_t i = 0; i < n; ++i) {
+            int64_t v = or_valid_rows(d0[i], N, r);
+            for (int64_t row = 0; row < c[i]; ++row) {
+                for (int64_t col = 0; col < cols[i]; ++col) {
+                    int64_t k = (int64_t)r * S + off[i] + row * cols[i] + col;
+                    ag8[k] = (row < v) ? or_e4m3_bits(or_fp8_quant_input(master[k], scales[i]))
+                                       : (uint8_t)0;
+                }
+            }
+        }
+    }
+}
+
+void or_copy_out_fp8(const int64_t* d0, const int64_t* cols, int32_t n, int32_t N,
+                     const uint8_t* ag8, uint8_t* arena8) {
+    int64_t c[n > 0 ? n : 1], s[n > 0 ? n : 1], off[n > 0 ? n : 1],
+        u[n > 0 ? n : 1], sz[3];
+    or_plan(d0, cols, n, N, c, s, off, u, sz);
+    int64_t S = sz[0];
+    for (int32_t i = 0; i < n; ++i) {
+#pragma omp parallel for schedule(static)
+        for (int64_t row = 0; row < d0[i]; ++row) {
+            int64_t r = row / c[i];
+            int64_t local = row - r * c[i];
+            for (int64_t col = 0; col < cols[i]; ++col)
+                arena8[u[i] + row * cols[i] + col] = ag8[r * S + off[i] + local * cols[i] + col];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* a5 AdamW (decoupled weight decay), binary64, one rounding per store */
 /* [ML] Fence 4 (AdamW built after sharding steps each shard);          */
 /* [MS] "Working Principle" (update state uses gradient slices).       */
