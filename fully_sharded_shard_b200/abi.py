@@ -80,6 +80,10 @@ def _load() -> ctypes.CDLL:
     L.fsdp_grad_accumulate.restype = ctypes.c_int
     L.fsdp_rs_reduce_accumulated.argtypes = [vp, vp, vp, i32, vp, vp]
     L.fsdp_rs_reduce_accumulated.restype = ctypes.c_int
+    L.fsdp_copy_in_fp8.argtypes = [vp, vp, vp, vp, vp]
+    L.fsdp_copy_in_fp8.restype = ctypes.c_int
+    L.fsdp_copy_out_fp8.argtypes = [vp, vp, vp, vp]
+    L.fsdp_copy_out_fp8.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
     L.fsdp_status_string.argtypes = [ctypes.c_int]
@@ -194,6 +198,7 @@ def _ptr(t: Optional[torch.Tensor], dtypes, numel: int, name: str):
 
 _F32 = (torch.float32,)
 _B16 = (torch.bfloat16, torch.int16, torch.uint16)
+_U8 = (torch.uint8, torch.int8, torch.float8_e4m3fn)
 
 
 def fsdp_shard_params(g: Group, full_arena: torch.Tensor, master: torch.Tensor, stream=None):
@@ -267,6 +272,20 @@ def fsdp_rs_reduce_accumulated(g: Group, grads: Optional[torch.Tensor], acc: tor
                                            _ptr(reduced, _F32, g.N * g.S, "reduced"),
                                            _stream(stream, reduced)),
            "fsdp_rs_reduce_accumulated")
+
+
+def fsdp_copy_in_fp8(g: Group, master: torch.Tensor, ag8: torch.Tensor, scales: torch.Tensor,
+                     stream=None):
+    _check(_lib.fsdp_copy_in_fp8(g.handle, _ptr(master, _F32, g.N * g.S, "master"),
+                                 _ptr(ag8, _U8, g.N * g.S, "ag8"),
+                                 _ptr(scales, _F32, g.n, "scales"), _stream(stream, master)),
+           "fsdp_copy_in_fp8")
+
+
+def fsdp_copy_out_fp8(g: Group, ag8: torch.Tensor, arena8: torch.Tensor, stream=None):
+    _check(_lib.fsdp_copy_out_fp8(g.handle, _ptr(ag8, _U8, g.N * g.S, "ag8"),
+                                  _ptr(arena8, _U8, g.P_arena, "arena8"), _stream(stream, ag8)),
+           "fsdp_copy_out_fp8")
 
 FSDP_NOALLOC_MAX_UNITS = 131072
 

@@ -54,11 +54,12 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Split [pos, pos+len) of a (rank, parameter) run into units of at most
 // kUnitElems elements.
-void push_units(std::vector<Unit>& out, int64_t shard_pos, int64_t arena_pos, int64_t len,
-                int32_t is_pad) {
+void push_units(std::vector<Unit>& out, std::vector<int32_t>& out_param, int32_t param,
+                int64_t shard_pos, int64_t arena_pos, int64_t len, int32_t is_pad) {
     for (int64_t done = 0; done < len; done += fsdpk::kUnitElems) {
         const int64_t l = std::min<int64_t>(fsdpk::kUnitElems, len - done);
         out.push_back(Unit{shard_pos + done, is_pad ? 0 : arena_pos + done, (int32_t)l, is_pad});
+        out_param.push_back(param);
     }
 }
 
@@ -187,8 +188,8 @@ int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t wor
         for (int64_t j = 0; j < N; ++j)
             for (int32_t i = 0; i < n_params; ++i) {
                 const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
-                push_units(g->units, j * S + g->off[i], g->u[i] + j * g->c[i] * g->cols[i],
-                           v * g->cols[i], 0);
+                push_units(g->units, g->unit_param, i, j * S + g->off[i],
+                           g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);
             }
         g->n_real_units = (int64_t)g->units.size();
         for (int64_t j = 0; j < N; ++j)
@@ -196,7 +197,7 @@ int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t wor
                 const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
                 const int64_t lo = j * S + g->off[i] + v * g->cols[i];
                 const int64_t len = (g->c[i] - v) * g->cols[i];
-                push_units(g->units, lo, 0, len, 1);
+                push_units(g->units, g->unit_param, i, lo, 0, len, 1);
                 if (len > 0) {
                     if (!g->intervals.empty() && g->intervals.back().hi == lo)
                         g->intervals.back().hi = lo + len;  // merge adjacent pads
@@ -231,8 +232,9 @@ int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t wor
     const size_t b_units = g->units.size() * sizeof(Unit);
     const size_t b_iv = g->intervals.size() * sizeof(Interval);
     const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
+    const size_t b_up = g->unit_param.size() * sizeof(int32_t);
     auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr);
+    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up);
     if (total > 0) {
         e = cudaMalloc(&g->dev_mem, total);
         if (e != cudaSuccess) {
@@ -244,11 +246,16 @@ int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t wor
         g->d_units = reinterpret_cast<const Unit*>(base);
         g->d_intervals = reinterpret_cast<const Interval*>(base + up256(b_units));
         g->d_tile_ranges = reinterpret_cast<const TileRange*>(base + up256(b_units) + up256(b_iv));
+        g->d_unit_param = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
+                                                           up256(b_tr));
         if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
         if (e == cudaSuccess && b_iv)
             e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
         if (e == cudaSuccess && b_tr)
             e = cudaMemcpy((void*)g->d_tile_ranges, g->tile_ranges.data(), b_tr,
+                           cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && b_up)
+            e = cudaMemcpy((void*)g->d_unit_param, g->unit_param.data(), b_up,
                            cudaMemcpyHostToDevice);
         if (e != cudaSuccess) {
             cudaFree(g->dev_mem);
@@ -408,6 +415,29 @@ int fsdp_rs_reduce_accumulated(fsdp_group_t g, const uint16_t* grads_or_null, co
     if (st != FSDP_OK) return st;
     cudaError_t e = fsdpk::launch_rs_reduce_acc(*g, grads_or_null, acc, op, reduced,
                                                 (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_copy_in_fp8(fsdp_group_t g, const float* master, uint8_t* ag8, float* scales,
+                     fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if ((int64_t)g->N * g->S > 0 && (master == nullptr || ag8 == nullptr)) return FSDP_EINVAL;
+    if (g->n > 0 && scales == nullptr) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(ag8) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_copy_in_fp8(*g, master, ag8, scales, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_copy_out_fp8(fsdp_group_t g, const uint8_t* ag8, uint8_t* arena8, fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if (g->P > 0 && (ag8 == nullptr || arena8 == nullptr)) return FSDP_EINVAL;
+    if (!aligned16(ag8) || !aligned16(arena8)) return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_copy_out_fp8(*g, ag8, arena8, (cudaStream_t)stream);
     return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
 }
 

@@ -60,6 +60,7 @@ struct fsdp_group {
 
     // host copies (kept for inspection and tests of the plan)
     std::vector<fsdpk::Unit> units;  // real units first, then pad units
+    std::vector<int32_t> unit_param;  // parameter index of every unit
     int64_t n_real_units = 0;
     std::vector<fsdpk::Interval> intervals;
     std::vector<fsdpk::TileRange> tile_ranges;  // empty when no padding
@@ -70,6 +71,7 @@ struct fsdp_group {
     const fsdpk::Unit* d_units = nullptr;
     const fsdpk::Interval* d_intervals = nullptr;
     const fsdpk::TileRange* d_tile_ranges = nullptr;
+    const int32_t* d_unit_param = nullptr;
 };
 
 namespace fsdpk {
@@ -120,5 +122,12 @@ cudaError_t launch_accumulate(const fsdp_group& g, const uint16_t* grads, float*
                               cudaStream_t st);
 cudaError_t launch_rs_reduce_acc(const fsdp_group& g, const uint16_t* grads, const float* acc,
                                  int op, float* reduced, cudaStream_t st);
+
+// FP8 (E4M3) all-gather: per-parameter scales from the master's amax, the
+// quantising copy-in and the byte copy-out.
+cudaError_t launch_copy_in_fp8(const fsdp_group& g, const float* master, uint8_t* ag8,
+                               float* scales, cudaStream_t st);
+cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t* arena8,
+                                cudaStream_t st);
 
 }  // namespace fsdpk

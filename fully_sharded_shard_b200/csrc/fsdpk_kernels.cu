@@ -17,6 +17,7 @@
 //   AdamW     -- Sharded Training page, Fence 4: the optimizer steps the
 //                sharded fp32 parameters, its state sharded the same way.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -875,6 +876,162 @@ k_reduce_acc(const float* __restrict__ acc, const uint16_t* __restrict__ g, int6
 }
 
 // ---------------------------------------------------------------------------
+// FP8 (E4M3) all-gather copy-in and copy-out
+//   amax_i = max |x| over parameter i (NaN ignored), scale_i = 448 / max(amax_i,
+//   1e-12), ag8[k] = e4m3_rn(clamp(x * scale_i, -448, 448)), pads 0x00.
+// ---------------------------------------------------------------------------
+
+// Max |x| of each real unit, folded into its parameter's slot with an integer
+// atomicMax (non-negative floats order like their bit patterns).
+__global__ void __launch_bounds__(kThreads)
+k_fp8_amax(const float* __restrict__ master, unsigned* __restrict__ amax_bits,
+           const Unit* __restrict__ units, const int32_t* __restrict__ unit_param,
+           int64_t n_real) {
+    __shared__ float part[kThreads / 32];
+    for (int64_t ui = blockIdx.x; ui < n_real; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const float* src = master + u.shard_pos;
+        const int len = u.len;
+        const int head = (int)head_to_16B(src, len);
+        float mx = 0.0f;
+        for (int e = threadIdx.x; e < head; e += blockDim.x) mx = fmaxf(mx, fabsf(src[e]));
+        const int nv = (len - head) >> 2;
+        const float4* s4 = reinterpret_cast<const float4*>(src + head);
+#pragma unroll 4
+        for (int q = threadIdx.x; q < nv; q += blockDim.x) {
+            const float4 x = __ldcs(s4 + q);
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+        }
+        for (int e = head + 4 * nv + threadIdx.x; e < len; e += blockDim.x)
+            mx = fmaxf(mx, fabsf(src[e]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            mx = threadIdx.x < kThreads / 32 ? part[threadIdx.x] : 0.0f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (threadIdx.x == 0) atomicMax(amax_bits + unit_param[ui], __float_as_uint(mx));
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_fp8_scales(float* __restrict__ scales, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) scales[i] = __fdiv_rn(448.0f, fmaxf(scales[i], 1e-12f));
+}
+
+// x * scale clamped to the finite E4M3 range (NaN passes through).
+__device__ __forceinline__ float fp8_in(float x, float sc) {
+    float y = __fmul_rn(x, sc);
+    if (y > 448.0f) y = 448.0f;
+    if (y < -448.0f) y = -448.0f;
+    return y;
+}
+
+// Two floats -> two E4M3 bytes (lo in bits 0..7), round to nearest even.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ uint8_t e4m3(float x) {
+    return (uint8_t)(e4m3x2(x, 0.0f) & 0xFFu);
+}
+
+__device__ __forceinline__ void zero_u8_run(uint8_t* __restrict__ dst, int len) {
+    const int head = (int)head_to_16B(dst, len);
+    if ((int)threadIdx.x < head) dst[threadIdx.x] = 0;
+    const int nv = (len - head) >> 4;
+    uint4* d = reinterpret_cast<uint4*>(dst + head);
+    for (int q = threadIdx.x; q < nv; q += blockDim.x) __stcs(d + q, make_uint4(0u, 0u, 0u, 0u));
+    const int done = head + 16 * nv;
+    if ((int)threadIdx.x < len - done) dst[done + threadIdx.x] = 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
+k_fp8_copy_in(const float* __restrict__ master, uint8_t* __restrict__ ag8,
+              const float* __restrict__ scales, const Unit* __restrict__ units,
+              const int32_t* __restrict__ unit_param, int64_t n_units) {
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        uint8_t* dst = ag8 + u.shard_pos;
+        const int len = u.len;
+        if (u.is_pad) {
+            zero_u8_run(dst, len);
+            continue;
+        }
+        const float sc = scales[unit_param[ui]];
+        const float* src = master + u.shard_pos;
+        // 16-byte output vectors; the fp32 source of a vector is then 64-byte aligned
+        const int head = (int)head_to_16B(dst, len);
+        if ((int)threadIdx.x < head) dst[threadIdx.x] = e4m3(fp8_in(src[threadIdx.x], sc));
+        const int nv = (len - head) >> 4;
+        const float4* s4 = reinterpret_cast<const float4*>(src + head);
+        uint4* d = reinterpret_cast<uint4*>(dst + head);
+#pragma unroll 1
+        for (int q = threadIdx.x; q < nv; q += blockDim.x) {
+            float4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[k] = __ldcs(s4 + 4 * q + k);
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t lo = e4m3x2(fp8_in(x[k].x, sc), fp8_in(x[k].y, sc));
+                const uint32_t hi = e4m3x2(fp8_in(x[k].z, sc), fp8_in(x[k].w, sc));
+                w[k] = (lo & 0xFFFFu) | (hi << 16);
+            }
+            __stcs(d + q, make_uint4(w[0], w[1], w[2], w[3]));
+        }
+        const int done = head + 16 * nv;
+        if ((int)threadIdx.x < len - done)
+            dst[done + threadIdx.x] = e4m3(fp8_in(src[done + threadIdx.x], sc));
+    }
+}
+
+// The 16 bytes that start D (1..15) bytes into the 32 bytes a:b.
+__device__ __forceinline__ uint4 shift_bytes16(const uint4& a, const uint4& b, int D) {
+    const int s = D >> 2;
+    const uint32_t sh = 8u * (uint32_t)(D & 3);
+    const uint32_t w0 = s == 0 ? a.x : s == 1 ? a.y : s == 2 ? a.z : a.w;
+    const uint32_t w1 = s == 0 ? a.y : s == 1 ? a.z : s == 2 ? a.w : b.x;
+    const uint32_t w2 = s == 0 ? a.z : s == 1 ? a.w : s == 2 ? b.x : b.y;
+    const uint32_t w3 = s == 0 ? a.w : s == 1 ? b.x : s == 2 ? b.y : b.z;
+    const uint32_t w4 = s == 0 ? b.x : s == 1 ? b.y : s == 2 ? b.z : b.w;
+    return make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh),
+                      __funnelshift_r(w2, w3, sh), __funnelshift_r(w3, w4, sh));
+}
+
+__global__ void __launch_bounds__(kThreads, 5)
+k_fp8_copy_out(const uint8_t* __restrict__ ag8, uint8_t* __restrict__ arena8,
+               const Unit* __restrict__ units, int64_t n_units) {
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        uint8_t* dst = arena8 + u.arena_pos;
+        const uint8_t* src = ag8 + u.shard_pos;
+        const int head = (int)head_to_16B(dst, len);
+        if ((int)threadIdx.x < head) dst[threadIdx.x] = src[threadIdx.x];
+        const int nv = (len - head) >> 4;
+        const int D = (int)(reinterpret_cast<uintptr_t>(src + head) & 15u);
+        const uint4* sa = reinterpret_cast<const uint4*>(src + head - D);
+        uint4* d = reinterpret_cast<uint4*>(dst + head);
+        if (D == 0) {
+#pragma unroll 4
+            for (int q = threadIdx.x; q < nv; q += blockDim.x) __stcs(d + q, __ldcs(sa + q));
+        } else {
+#pragma unroll 2
+            for (int q = threadIdx.x; q < nv; q += blockDim.x)
+                __stcs(d + q, shift_bytes16(__ldg(sa + q), __ldg(sa + q + 1), D));
+        }
+        const int done = head + 16 * nv;
+        if ((int)threadIdx.x < len - done) dst[done + threadIdx.x] = src[done + threadIdx.x];
+    }
+}
+
+// ---------------------------------------------------------------------------
 // launch geometry
 // ---------------------------------------------------------------------------
 
@@ -1072,6 +1229,37 @@ cudaError_t launch_rs_reduce_acc(const fsdp_group& g, const uint16_t* grads, con
     else
         k_reduce_acc<false><<<grid_for(g, (const void*)k_reduce_acc<false>, nu), kThreads, 0, st>>>(
             acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+    return cudaGetLastError();
+}
+
+}  // namespace fsdpk
+
+namespace fsdpk {
+
+cudaError_t launch_copy_in_fp8(const fsdp_group& g, const float* master, uint8_t* ag8,
+                               float* scales, cudaStream_t st) {
+    if (g.n > 0) {
+        cudaError_t e = cudaMemsetAsync(scales, 0, (size_t)g.n * sizeof(float), st);
+        if (e != cudaSuccess) return e;
+        if (g.n_real_units > 0)
+            k_fp8_amax<<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
+                master, reinterpret_cast<unsigned*>(scales), g.d_units, g.d_unit_param,
+                g.n_real_units);
+        k_fp8_scales<<<(unsigned)((g.n + kThreads - 1) / kThreads), kThreads, 0, st>>>(scales, g.n);
+    }
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu > 0)
+        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(master, ag8, scales,
+                                                                     g.d_units, g.d_unit_param, nu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t* arena8,
+                                cudaStream_t st) {
+    if (g.n_real_units == 0) return cudaSuccess;
+    k_fp8_copy_out<<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(ag8, arena8,
+                                                                              g.d_units,
+                                                                              g.n_real_units);
     return cudaGetLastError();
 }
 

@@ -234,6 +234,28 @@ int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grads_or_null
                                const float* acc, int32_t op, float* reduced,
                                fsdp_stream_t stream);
 
+/* FP8 all-gather copy-in ("PyTorch FSDP2 Guide: Distributed LLM Training
+ * with DTensor", Deep Dive, "2. Native FP8 Training with Float8Tensor":
+ * parameters in FP8 E4M3, the all-gather moves raw FP8 bytes).  The page
+ * leaves the scaling open; this library uses per-parameter tensorwise
+ * dynamic scaling:
+ *   amax_i  = max |master| over parameter i, all ranks (NaN ignored)
+ *   scale_i = 448 / max(amax_i, 1e-12)                       (binary32)
+ *   ag8[r][k] = e4m3_rn(clamp(master[r][k] * scale_i, -448, 448)),
+ * 0x00 in pad rows; E4M3 is the "fn" encoding (no infinities, largest
+ * finite 448).  A consumer recovers x ~ e4m3_value(q) / scale_i.
+ * master: fp32 [N][S] (read); ag8: uint8 [N][S] (written); scales: fp32
+ * [n_params] (written; 4-byte aligned).  Algorithmic bytes: 4 (amax pass) +
+ * 4 + 1 per padded element. */
+int fsdp_copy_in_fp8(fsdp_group_t group, const float* master, uint8_t* ag8,
+                     float* scales, fsdp_stream_t stream);
+
+/* FP8 copy-out: the byte-for-byte counterpart of fsdp_copy_out.
+ * ag8: uint8 [N][S] (read); arena8: uint8 [P_arena] (written, gaps
+ * untouched).  Algorithmic bytes: 1 read + 1 written per real element. */
+int fsdp_copy_out_fp8(fsdp_group_t group, const uint8_t* ag8, uint8_t* arena8,
+                      fsdp_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Reduce-scatter without any allocation                                    */
 /* ------------------------------------------------------------------------ */

@@ -117,6 +117,20 @@ def test_gradient_accumulation_two_microbatches(H):
     H.run_group_accumulate(wl, wl.groups[0], micro=2)
 
 
+FP8 = SMALL + [W.tiny_mlp(), W.uneven(8), W.moe(8), W.llama7b(8, layers=1)]
+
+
+@pytest.mark.parametrize("wl", FP8, ids=[w.name for w in FP8])
+def test_fp8_all_gather_copy_in_and_out(H, wl):
+    for g in wl.groups:
+        H.run_group_fp8(wl, g)
+
+
+def test_fp8_full_size_llama7b_root(H):
+    wl = W.llama7b()
+    H.run_group_fp8(wl, wl.groups[1])
+
+
 def test_fused_and_staged_reduce_are_deterministic(H):
     from fully_sharded_shard_b200 import abi
     wl = W.uneven(8)
