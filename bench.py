@@ -418,6 +418,10 @@ def run_ours(args, wl, device, rank, ws):
     if not args.no_accumulate:
         accum = run_accumulate(args, model, device, stream)
 
+    fp8 = None
+    if not args.no_fp8:
+        fp8 = run_fp8(args, model, device, stream)
+
     latency = None
     if not args.no_latency:
         latency = run_latency(device)
@@ -456,6 +460,7 @@ def run_ours(args, wl, device, rank, ws):
         "e2e": e2e,
         "fused_step": fused,
         "grad_accumulation": accum,
+        "fp8_all_gather": fp8,
         "tiny_latency": latency,
         "setup_s": round(setup_s, 1),
     }
@@ -542,6 +547,60 @@ def run_accumulate(args, model, device, stream, micro: int = 4):
             "ms_per_group_step": round(ms, 3), "bytes": b,
             "value": round(b / (ms * 1e-3) / 1e9, 1), "unit": "GB/s (own byte model)",
             "launches": micro}
+
+
+def run_fp8(args, model, device, stream):
+    """The all-gather half of the step in FP8 (per-parameter scales, E4M3
+    copy-in, byte copy-out) against the same half in bf16, over every group
+    of the model.  Own byte models: FP8 = 4 B per real element (amax pass) +
+    5 B per padded element + 2 B per real element; bf16 = 6 + 4 B."""
+    import torch
+    from fully_sharded_shard_b200 import abi
+    max_NS = max(model.wl.N * g.S for g in model.plans)
+    max_A = max(g.P_arena for g in model.plans)
+    ag8 = torch.empty(max(max_NS, 1), dtype=torch.uint8, device=device)
+    ar8 = torch.empty(max(max_A, 1), dtype=torch.uint8, device=device)
+    scales = [torch.empty(max(g.n, 1), dtype=torch.float32, device=device) for g in model.plans]
+
+    def fp8_half():
+        for gi, master, m, v, pj in model.instances:
+            g = model.plans[gi]
+            abi.fsdp_copy_in_fp8(g, master, ag8, scales[gi], stream)
+            abi.fsdp_copy_out_fp8(g, ag8, ar8, stream)
+
+    def bf16_half():
+        for gi, master, m, v, pj in model.instances:
+            g = model.plans[gi]
+            abi.fsdp_copy_in(g, master, model.ag, stream)
+            abi.fsdp_copy_out(g, model.ag, model.arena, stream)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(max(1, args.steps)):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / max(1, args.steps)
+
+    ms8 = timed(fp8_half)
+    ms16 = timed(bf16_half)
+    N = model.wl.N
+    b8 = sum(4 * model.plans[i[0]].P + 5 * N * model.plans[i[0]].S + 2 * model.plans[i[0]].P
+             for i in model.instances)
+    b16 = sum(6 * N * model.plans[i[0]].S + 2 * N * model.plans[i[0]].S + 2 * model.plans[i[0]].P
+              for i in model.instances)
+    del ag8, ar8
+    return {"fp8_ms_per_step": round(ms8, 3), "fp8_bytes": b8,
+            "fp8_GBps": round(b8 / (ms8 * 1e-3) / 1e9, 1),
+            "bf16_ms_per_step": round(ms16, 3), "bf16_bytes": b16,
+            "bf16_GBps": round(b16 / (ms16 * 1e-3) / 1e9, 1),
+            "all_gather_payload_ratio": 0.5,
+            "launches_per_step": 2 * len(model.instances) + 3 * len(model.instances)}
 
 
 def run_latency(device, reps: int = 200):
@@ -758,6 +817,7 @@ def main(argv=None):
     ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--no-accumulate", action="store_true")
     ap.add_argument("--no-latency", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
