@@ -260,6 +260,8 @@ class Model:
                 self.stage_bytes[k] += b
         self.launches_per_step = 4 * len(self.instances)
         self.ag_groups = None
+        self._ag2 = None
+        self._arena2 = None
 
     def enable_fused(self):
         """Per-group bf16 all-gather buffers: the fused update writes the next
@@ -343,19 +345,57 @@ class Model:
         for idx in range(len(self.instances)):
             self.run_group(idx, stream, self.step_count, events=events)
 
+    def step_two_streams(self, s_gather, s_update):
+        """One full step on two streams, as FSDP2 splits communication from
+        compute: the all-gather half of each group (copy-in, copy-out, double
+        buffered) on `s_gather`, its reduce-scatter and AdamW on `s_update`
+        once its copy-in has read the pre-update master.  Group g+1's
+        all-gather overlaps group g's update.  The step ends with `s_gather`
+        waiting for `s_update`, so the next step's copy-ins see this step's
+        updates."""
+        import torch
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200 import workloads as W
+        if self._ag2 is None:
+            self._ag2 = [self.ag, torch.empty_like(self.ag)]
+            self._arena2 = [self.arena, torch.empty_like(self.arena)]
+        self.step_count += 1
+        hp = dict(W.ADAMW_DEFAULTS)
+        for idx, (gi, master, m, v, pj) in enumerate(self.instances):
+            g = self.plans[gi]
+            ag, arena = self._ag2[idx % 2], self._arena2[idx % 2]
+            abi.fsdp_copy_in(g, master, ag, s_gather)
+            read = torch.cuda.Event()
+            read.record(s_gather)
+            abi.fsdp_copy_out(g, ag, arena, s_gather)
+            s_update.wait_event(read)
+            abi.fsdp_rs_reduce(g, self.grads[gi][pj], self.wl.op, self.reduced, stream=s_update)
+            abi.fsdp_adamw_step(g, master, m, v, self.reduced, step=self.step_count,
+                                stream=s_update, **hp)
+        done = torch.cuda.Event()
+        done.record(s_update)
+        s_gather.wait_event(done)
+
 
 def run_ours(args, wl, device, rank, ws):
     import torch
     from fully_sharded_shard_b200 import workloads as W
     stream = torch.cuda.Stream(device)
+    s_update = torch.cuda.Stream(device)
     t_setup = time.time()
     model = Model(wl, device, args.grad_pool, rank)
     setup_s = time.time() - t_setup
 
+    def one_step():
+        if args.one_stream:
+            model.step(stream)
+        else:
+            model.step_two_streams(stream, s_update)
+
     # warm-up
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            model.step(stream)
+            one_step()
     torch.cuda.synchronize(device)
 
     # timed region: K whole steps between two events on the launching stream
@@ -367,7 +407,7 @@ def run_ours(args, wl, device, rank, ws):
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
     for _ in range(args.steps):
-        model.step(stream)
+        one_step()
     e_end.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -452,6 +492,8 @@ def run_ours(args, wl, device, rank, ws):
             "grad_pool_per_plan": args.grad_pool,
             "l2": "inputs larger than L2 (every group's state >> 126 MB)",
             "parallelism": f"{ws} GPU(s), each a full {wl.N}-virtual-rank replica",
+            "schedule": "one stream" if args.one_stream else
+                        "two streams: all-gather half / reduce-scatter + update half",
         },
         "stages": stages,
         "roofline": roofline,
@@ -818,6 +860,7 @@ def main(argv=None):
     ap.add_argument("--no-accumulate", action="store_true")
     ap.add_argument("--no-latency", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
+    ap.add_argument("--one-stream", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
