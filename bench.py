@@ -282,6 +282,31 @@ class Model:
             for k, b in fused_stage_bytes(N, g.S, g.P).items():
                 self.fused_bytes[k] += b
 
+    def fused_step_two_streams(self, s_gather, s_update):
+        """The fused step on two streams: each group's copy-out on
+        `s_gather`, its fused update on `s_update` once the copy-out has read
+        the group's all-gather buffer (the update rewrites it for the next
+        step); group g+1's copy-out overlaps group g's update."""
+        import torch
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200 import workloads as W
+        if self._arena2 is None:
+            self._arena2 = [self.arena, torch.empty_like(self.arena)]
+        self.step_count += 1
+        hp = dict(W.ADAMW_DEFAULTS)
+        for idx, (gi, master, m, v, pj) in enumerate(self.instances):
+            g = self.plans[gi]
+            ag = self.ag_groups[idx]
+            abi.fsdp_copy_out(g, ag, self._arena2[idx % 2], s_gather)
+            read = torch.cuda.Event()
+            read.record(s_gather)
+            s_update.wait_event(read)
+            abi.fsdp_rs_adamw_step(g, self.grads[gi][pj], self.wl.op, master, m, v,
+                                   step=self.step_count, ag_next=ag, stream=s_update, **hp)
+        done = torch.cuda.Event()
+        done.record(s_update)
+        s_gather.wait_event(done)
+
     def fused_step(self, stream, events=None):
         """One step with the reduce-scatter, AdamW and next copy-in fused."""
         import torch
@@ -515,16 +540,24 @@ def run_fused(args, model, device, stream, ws, ms_unfused, peak):
     model."""
     import torch
     model.enable_fused()
+    s_update = torch.cuda.Stream(device)
+
+    def one():
+        if args.one_stream:
+            model.fused_step(stream)
+        else:
+            model.fused_step_two_streams(stream, s_update)
+
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            model.fused_step(stream)
+            one()
     torch.cuda.synchronize(device)
     barrier(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        model.fused_step(stream)
+        one()
     e1.record(stream)
     torch.cuda.synchronize(device)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)

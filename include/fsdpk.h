@@ -64,6 +64,13 @@
 extern "C" {
 #endif
 
+/* Every entry point below is exported; the library hides everything else. */
+#if defined(FSDPK_BUILDING_LIBRARY)
+#define FSDP_API __attribute__((visibility("default")))
+#else
+#define FSDP_API
+#endif
+
 #define FSDP_MAX_NDIM 8
 #define FSDP_MAX_WORLD 1024
 #define FSDP_ABI_VERSION 1
@@ -120,22 +127,22 @@ typedef struct {
  * n_params >= 0; world_size in [1, FSDP_MAX_WORLD].  On success *out owns a
  * new plan.  Errors: EINVAL (bad descriptor, sizes overflow int64),
  * ENOMEM, ECUDA (device table upload). */
-int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params,
+FSDP_API int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params,
                     int32_t world_size, fsdp_group_t* out);
 
 /* S (per-rank padded shard elements), P (real elements), P_arena.
  * Any output pointer may be NULL. */
-int fsdp_group_sizes(fsdp_group_t group, int64_t* S, int64_t* P,
+FSDP_API int fsdp_group_sizes(fsdp_group_t group, int64_t* S, int64_t* P,
                      int64_t* P_arena);
 
 /* Per-parameter tables, each an int64 array of n_params entries supplied by
  * the caller (any may be NULL): off_i, u_i and c_i. */
-int fsdp_group_param_offsets(fsdp_group_t group, int64_t* shard_off,
+FSDP_API int fsdp_group_param_offsets(fsdp_group_t group, int64_t* shard_off,
                              int64_t* arena_off, int64_t* chunk_rows);
 
 /* Free a plan (NULL is ignored).  Work already enqueued that uses the plan
  * must have completed. */
-void fsdp_destroy_group(fsdp_group_t group);
+FSDP_API void fsdp_destroy_group(fsdp_group_t group);
 
 /* ------------------------------------------------------------------------ */
 /* Data path (asynchronous on `stream`)                                     */
@@ -144,14 +151,14 @@ void fsdp_destroy_group(fsdp_group_t group);
 /* Shard(0) placement: fp32 full parameters in arena layout [P_arena] ->
  * padded fp32 master [N][S] (pad rows written as +0).  This is fully_shard's
  * initial sharding ([ML] fully_shard paragraph). */
-int fsdp_shard_params(fsdp_group_t group, const float* full_arena,
+FSDP_API int fsdp_shard_params(fsdp_group_t group, const float* full_arena,
                       float* master, fsdp_stream_t stream);
 
 /* Stage 1, all-gather copy-in: ag[r][k] = bf16_rn(master[r][k]) for real
  * elements and +0 for pad elements ([ML] Mixed precision: bf16 copies are
  * all-gathered; [MS] Mixed Precision).  master: fp32 [N][S] (read);
  * ag: bf16 [N][S] (written). */
-int fsdp_copy_in(fsdp_group_t group, const float* master, uint16_t* ag,
+FSDP_API int fsdp_copy_in(fsdp_group_t group, const float* master, uint16_t* ag,
                  fsdp_stream_t stream);
 
 /* Stage 2, all-gather copy-out: the rank-major buffer is split into the
@@ -159,7 +166,7 @@ int fsdp_copy_in(fsdp_group_t group, const float* master, uint16_t* ag,
  * All-Gather state): arena[u_i + row*cols_i + col] =
  * ag[r*S + off_i + (row - r*c_i)*cols_i + col] with r = row / c_i.
  * ag: bf16 [N][S] (read); arena: bf16 [P_arena] (written, gaps untouched). */
-int fsdp_copy_out(fsdp_group_t group, const uint16_t* ag, uint16_t* arena,
+FSDP_API int fsdp_copy_out(fsdp_group_t group, const uint16_t* ag, uint16_t* arena,
                   fsdp_stream_t stream);
 
 /* Stages 3 + 4, reduce-scatter: each rank's bf16 full gradients are cast to
@@ -171,7 +178,7 @@ int fsdp_copy_out(fsdp_group_t group, const uint16_t* ag, uint16_t* arena,
  * reduce-scatter inputs and the reduction reads them back (staged path; for
  * FSDP_SUM_THEN_DIV the division is a separate pass).  Both paths give the
  * same bits. */
-int fsdp_rs_reduce(fsdp_group_t group, const uint16_t* grads, int32_t op,
+FSDP_API int fsdp_rs_reduce(fsdp_group_t group, const uint16_t* grads, int32_t op,
                    float* packed_or_null, float* reduced,
                    fsdp_stream_t stream);
 
@@ -183,7 +190,7 @@ int fsdp_rs_reduce(fsdp_group_t group, const uint16_t* grads, int32_t op,
  * master, m, v: fp32 [N][S] updated in place; grad: fp32 [N][S] (read).
  * A zero pad stays +0.  hparams: host pointer; step >= 1, lr >= 0,
  * 0 <= beta < 1, eps > 0.  Computed in binary32. */
-int fsdp_adamw_step(fsdp_group_t group, float* master, float* m, float* v,
+FSDP_API int fsdp_adamw_step(fsdp_group_t group, float* master, float* m, float* v,
                     const float* grad, const fsdp_adamw_hparams* hparams,
                     fsdp_stream_t stream);
 
@@ -204,7 +211,7 @@ int fsdp_adamw_step(fsdp_group_t group, float* master, float* m, float* v,
  *   reduced_or_null: fp32 [N][S] receiving the reduced gradient, or NULL.
  * Algorithmic bytes: 2N per real element + 24 (+2 with ag, +4 with reduced)
  * per padded element.  Errors as for fsdp_rs_reduce and fsdp_adamw_step. */
-int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32_t op,
+FSDP_API int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32_t op,
                        float* master, float* m, float* v,
                        const fsdp_adamw_hparams* hparams,
                        uint16_t* ag_next_or_null, float* reduced_or_null,
@@ -219,7 +226,7 @@ int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32_t op,
  * read by the reduce-scatter).  grads: bf16 [N][P_arena] (read); acc: fp32
  * [N][P_arena] (updated; not read when first != 0).  Algorithmic bytes per
  * element: 6 (first) or 10. */
-int fsdp_grad_accumulate(fsdp_group_t group, const uint16_t* grads, float* acc,
+FSDP_API int fsdp_grad_accumulate(fsdp_group_t group, const uint16_t* grads, float* acc,
                          int32_t first, fsdp_stream_t stream);
 
 /* The reduce-scatter of the last microbatch when gradients were accumulated:
@@ -230,7 +237,7 @@ int fsdp_grad_accumulate(fsdp_group_t group, const uint16_t* grads, float* acc,
  * writing acc back.  acc: fp32 [N][P_arena] (read); reduced: fp32 [N][S]
  * (written, pads +0).  Algorithmic bytes: 6N (4N without grads) per real
  * element + 4 per padded element. */
-int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grads_or_null,
+FSDP_API int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grads_or_null,
                                const float* acc, int32_t op, float* reduced,
                                fsdp_stream_t stream);
 
@@ -247,13 +254,13 @@ int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grads_or_null
  * master: fp32 [N][S] (read); ag8: uint8 [N][S] (written); scales: fp32
  * [n_params] (written; 4-byte aligned).  Algorithmic bytes: 4 (amax pass) +
  * 4 + 1 per padded element. */
-int fsdp_copy_in_fp8(fsdp_group_t group, const float* master, uint8_t* ag8,
+FSDP_API int fsdp_copy_in_fp8(fsdp_group_t group, const float* master, uint8_t* ag8,
                      float* scales, fsdp_stream_t stream);
 
 /* FP8 copy-out: the byte-for-byte counterpart of fsdp_copy_out.
  * ag8: uint8 [N][S] (read); arena8: uint8 [P_arena] (written, gaps
  * untouched).  Algorithmic bytes: 1 read + 1 written per real element. */
-int fsdp_copy_out_fp8(fsdp_group_t group, const uint8_t* ag8, uint8_t* arena8,
+FSDP_API int fsdp_copy_out_fp8(fsdp_group_t group, const uint8_t* ag8, uint8_t* arena8,
                       fsdp_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
@@ -293,7 +300,7 @@ int fsdp_copy_out_fp8(fsdp_group_t group, const uint8_t* ag8, uint8_t* arena8,
  * fsdp_rs_reduce, and for a group that needs more than
  * FSDP_NOALLOC_MAX_UNITS table entries (nothing is enqueued then);
  * FSDP_EALIGN; FSDP_ECUDA. */
-int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_params,
+FSDP_API int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_params,
                            int32_t world_size, const uint16_t* grads, int32_t op,
                            float* reduced, fsdp_stream_t stream);
 
@@ -302,13 +309,13 @@ int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_params,
 /* ------------------------------------------------------------------------ */
 
 /* Static description of a status code. */
-const char* fsdp_status_string(int status);
+FSDP_API const char* fsdp_status_string(int status);
 
 /* The cudaError_t of the most recent FSDP_ECUDA on this thread (0 if none). */
-int fsdp_last_cuda_error(void);
+FSDP_API int fsdp_last_cuda_error(void);
 
 /* FSDP_ABI_VERSION of the loaded library. */
-int fsdp_abi_version(void);
+FSDP_API int fsdp_abi_version(void);
 
 #ifdef __cplusplus
 }
