@@ -123,14 +123,7 @@ class Group:
     """A plan of one parameter group (one fully_shard call) over N ranks."""
 
     def __init__(self, shapes: Sequence[Sequence[int]], world_size: int):
-        shapes = [tuple(int(d) for d in s) for s in shapes]
-        arr = (ParamDesc * max(1, len(shapes)))()
-        for i, s in enumerate(shapes):
-            if len(s) > FSDP_MAX_NDIM:
-                raise ValueError(f"parameter {i}: more than {FSDP_MAX_NDIM} dims")
-            arr[i].ndim = len(s)
-            for k, d in enumerate(s):
-                arr[i].shape[k] = d
+        shapes, arr = _descs(shapes)
         h = ctypes.c_void_p()
         _check(_lib.fsdp_plan_group(arr, len(shapes), int(world_size), ctypes.byref(h)),
                "fsdp_plan_group")

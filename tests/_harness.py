@@ -23,8 +23,6 @@ ADAM_TOL = 1e-6
 class Guarded:
     """A device buffer with sentinel guard bands before and after it."""
 
-    SENT = {torch.float32: -12345.5, torch.bfloat16: None, torch.int16: 0x3BEF}
-
     def __init__(self, n: int, dtype, device="cuda", fill=None):
         self.n = n
         self.full = torch.empty(n + 2 * GUARD, dtype=dtype, device=device)
@@ -332,18 +330,19 @@ def run_group_fp8(wl: W.Workload, group: W.Group, tag=()) -> None:
     W.fill_master(full, wl, group.name, *tag)
     master = torch.empty(max(NS, 1), dtype=torch.float32, device="cuda")
     abi.fsdp_shard_params(g, full, master)
-    ag8 = torch.full((NS + 2 * GUARD * 2,), 0x5A, dtype=torch.uint8, device="cuda")
-    ag8_t = ag8[2 * GUARD:2 * GUARD + NS]
+    G8 = 4 * GUARD  # guard bytes on each side (a multiple of 16)
+    ag8 = torch.full((NS + 2 * G8,), 0x5A, dtype=torch.uint8, device="cuda")
+    ag8_t = ag8[G8:G8 + NS]
     scales = torch.full((max(g.n, 1) + 2,), -3.0, dtype=torch.float32, device="cuda")
     abi.fsdp_copy_in_fp8(g, master[:NS], ag8_t, scales[1:1 + g.n] if g.n else scales[1:1])
-    arena8 = torch.full((g.P_arena + 4 * GUARD,), 0xA5, dtype=torch.uint8, device="cuda")
-    arena8_t = arena8[2 * GUARD:2 * GUARD + g.P_arena]
+    arena8 = torch.full((g.P_arena + 2 * G8,), 0xA5, dtype=torch.uint8, device="cuda")
+    arena8_t = arena8[G8:G8 + g.P_arena]
     abi.fsdp_copy_out_fp8(g, ag8_t, arena8_t)
     torch.cuda.synchronize()
     host_ag8 = ag8.cpu().numpy()
-    assert np.all(host_ag8[:2 * GUARD] == 0x5A) and np.all(host_ag8[2 * GUARD + NS:] == 0x5A)
+    assert np.all(host_ag8[:G8] == 0x5A) and np.all(host_ag8[G8 + NS:] == 0x5A)
     host_ar = arena8.cpu().numpy()
-    assert np.all(host_ar[:2 * GUARD] == 0xA5) and np.all(host_ar[2 * GUARD + g.P_arena:] == 0xA5)
+    assert np.all(host_ar[:G8] == 0xA5) and np.all(host_ar[G8 + g.P_arena:] == 0xA5)
     sc = scales.cpu().numpy()
     assert sc[0] == -3.0 and sc[1 + g.n] == -3.0
     master_o = oracle.shard(p, f32(full)[:p.P_arena] if p.P_arena else np.zeros(0, np.float32))
@@ -351,9 +350,9 @@ def run_group_fp8(wl: W.Workload, group: W.Group, tag=()) -> None:
     scales_o = oracle.fp8_scales(p, master_o)
     assert bits_equal(sc[1:1 + g.n], scales_o), "fp8 scales: " + first_mismatch(sc[1:1 + g.n], scales_o)
     ag8_o = oracle.copy_in_fp8(p, master_o, scales_o)
-    got = host_ag8[2 * GUARD:2 * GUARD + NS]
+    got = host_ag8[G8:G8 + NS]
     assert np.array_equal(got, ag8_o), f"fp8 copy-in: {int(np.sum(got != ag8_o))} mismatches"
     arena_o = oracle.copy_out_fp8(p, ag8_o, np.full(p.P_arena, 0xA5, np.uint8))
-    got = host_ar[2 * GUARD:2 * GUARD + g.P_arena]
+    got = host_ar[G8:G8 + g.P_arena]
     assert np.array_equal(got, arena_o), f"fp8 copy-out: {int(np.sum(got != arena_o))} mismatches"
     g.destroy()
