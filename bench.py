@@ -680,10 +680,11 @@ def run_fp8(args, model, device, stream):
 
 def run_latency(device, reps: int = 200):
     """The tiny MLP group (4 parameters, N = 2) is launch-bound: report the
-    step latency in microseconds, eager and with the whole step captured in a
-    CUDA graph and replayed.  (A captured step replays the AdamW step count
-    it was captured with.)"""
+    step latency in microseconds, eager (host-side AdamW step count) and as a
+    replayed CUDA graph of the whole step, whose AdamW step count lives in
+    device memory so that every replay is the next training step."""
     import torch
+    from fully_sharded_shard_b200 import abi
     from fully_sharded_shard_b200 import workloads as W
     wl = W.tiny_mlp()
     model = Model(wl, device, 1, 0)
@@ -706,19 +707,31 @@ def run_latency(device, reps: int = 200):
     t0 = time.perf_counter()
     eager_us = timed(lambda: model.step(stream))
     host_us = (time.perf_counter() - t0) * 1e6 / reps
+
+    ds = abi.DeviceStep(device)
+    hp = dict(W.ADAMW_DEFAULTS)
+
+    def graphed_step():
+        abi.fsdp_adamw_prepare(ds, stream=stream, **hp)
+        for gi, master, m, v, pj in model.instances:
+            g = model.plans[gi]
+            abi.fsdp_copy_in(g, master, model.ag, stream)
+            abi.fsdp_copy_out(g, model.ag, model.arena, stream)
+            abi.fsdp_rs_reduce(g, model.grads[gi][pj], wl.op, model.reduced, stream=stream)
+            abi.fsdp_adamw_step_dev(g, master, m, v, model.reduced, ds, stream=stream)
+
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        model.step(stream)
+        graphed_step()
     torch.cuda.synchronize(device)
     with torch.cuda.stream(stream):
         graph.replay()
-    torch.cuda.synchronize(device)
-    with torch.cuda.stream(stream):
         graph_us = timed(graph.replay)
     del graph
     return {"workload": wl.name, "launches_per_step": model.launches_per_step,
             "eager_us_per_step": round(eager_us, 2), "eager_host_us_per_step": round(host_us, 2),
-            "graph_us_per_step": round(graph_us, 2)}
+            "graph_us_per_step": round(graph_us, 2),
+            "graph_launches_per_step": model.launches_per_step + 1}
 
 
 def run_e2e(args, model, device, stream, ws):

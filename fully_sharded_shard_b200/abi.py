@@ -84,6 +84,12 @@ def _load() -> ctypes.CDLL:
     L.fsdp_copy_in_fp8.restype = ctypes.c_int
     L.fsdp_copy_out_fp8.argtypes = [vp, vp, vp, vp]
     L.fsdp_copy_out_fp8.restype = ctypes.c_int
+    L.fsdp_adamw_prepare.argtypes = [ctypes.POINTER(AdamWHparams), vp, vp, vp]
+    L.fsdp_adamw_prepare.restype = ctypes.c_int
+    L.fsdp_adamw_step_dev.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+    L.fsdp_adamw_step_dev.restype = ctypes.c_int
+    L.fsdp_rs_adamw_step_dev.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
+    L.fsdp_rs_adamw_step_dev.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
     L.fsdp_status_string.argtypes = [ctypes.c_int]
@@ -279,6 +285,46 @@ def fsdp_copy_out_fp8(g: Group, ag8: torch.Tensor, arena8: torch.Tensor, stream=
     _check(_lib.fsdp_copy_out_fp8(g.handle, _ptr(ag8, _U8, g.N * g.S, "ag8"),
                                   _ptr(arena8, _U8, g.P_arena, "arena8"), _stream(stream, ag8)),
            "fsdp_copy_out_fp8")
+
+
+class DeviceStep:
+    """A device step counter and that step's AdamW scalars (for CUDA graphs)."""
+
+    def __init__(self, device=None):
+        self.step = torch.zeros(1, dtype=torch.int64, device=device or "cuda")
+        self.scalars = torch.zeros(8, dtype=torch.float32, device=device or "cuda")
+
+
+def fsdp_adamw_prepare(ds: DeviceStep, *, lr: float, beta1: float, beta2: float, eps: float,
+                       weight_decay: float, stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), 0)
+    _check(_lib.fsdp_adamw_prepare(ctypes.byref(hp), _ptr(ds.step, (torch.int64,), 1, "step"),
+                                   _ptr(ds.scalars, _F32, 8, "scalars"),
+                                   _stream(stream, ds.scalars)), "fsdp_adamw_prepare")
+
+
+def fsdp_adamw_step_dev(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                        grad: torch.Tensor, ds: DeviceStep, stream=None):
+    n = g.N * g.S
+    _check(_lib.fsdp_adamw_step_dev(g.handle, _ptr(master, _F32, n, "master"),
+                                    _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                    _ptr(grad, _F32, n, "grad"),
+                                    _ptr(ds.scalars, _F32, 8, "scalars"),
+                                    _stream(stream, master)), "fsdp_adamw_step_dev")
+
+
+def fsdp_rs_adamw_step_dev(g: Group, grads: torch.Tensor, op: int, master: torch.Tensor,
+                           m: torch.Tensor, v: torch.Tensor, ds: DeviceStep, *,
+                           ag_next: Optional[torch.Tensor] = None,
+                           reduced: Optional[torch.Tensor] = None, stream=None):
+    n = g.N * g.S
+    _check(_lib.fsdp_rs_adamw_step_dev(g.handle, _ptr(grads, _B16, g.N * g.P_arena, "grads"),
+                                       int(op), _ptr(master, _F32, n, "master"),
+                                       _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                       _ptr(ds.scalars, _F32, 8, "scalars"),
+                                       _ptr(ag_next, _B16, n, "ag_next"),
+                                       _ptr(reduced, _F32, n, "reduced"),
+                                       _stream(stream, master)), "fsdp_rs_adamw_step_dev")
 
 FSDP_NOALLOC_MAX_UNITS = 131072
 

@@ -441,4 +441,56 @@ int fsdp_copy_out_fp8(fsdp_group_t g, const uint8_t* ag8, uint8_t* arena8, fsdp_
     return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
 }
 
+int fsdp_adamw_prepare(const fsdp_adamw_hparams* hp, int64_t* step_dev,
+                       fsdp_adamw_dev_scalars* scalars_dev, fsdp_stream_t stream) {
+    if (hp == nullptr || step_dev == nullptr || scalars_dev == nullptr) return FSDP_EINVAL;
+    fsdp_adamw_hparams probe = *hp;
+    probe.step = 1;  // the step comes from step_dev; validate the rest
+    fsdpk::AdamScalars unused;
+    if (!adam_scalars(&probe, &unused)) return FSDP_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(step_dev) & 7u) || !aligned16(scalars_dev))
+        return FSDP_EALIGN;
+    cudaError_t e = fsdpk::launch_adamw_prepare(
+        hp->lr, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step_dev,
+        reinterpret_cast<fsdpk::AdamScalars*>(scalars_dev), (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_adamw_step_dev(fsdp_group_t g, float* master, float* m, float* v, const float* grad,
+                        const fsdp_adamw_dev_scalars* scalars_dev, fsdp_stream_t stream) {
+    if (g == nullptr || scalars_dev == nullptr) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr || grad == nullptr))
+        return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad) ||
+        !aligned16(scalars_dev))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    const fsdpk::AdamScalars none{};
+    cudaError_t e = fsdpk::launch_adamw(*g, master, m, v, grad, none, (cudaStream_t)stream,
+                                        reinterpret_cast<const fsdpk::AdamScalars*>(scalars_dev));
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_rs_adamw_step_dev(fsdp_group_t g, const uint16_t* grads, int32_t op, float* master,
+                           float* m, float* v, const fsdp_adamw_dev_scalars* scalars_dev,
+                           uint16_t* ag_next, float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr || scalars_dev == nullptr) return FSDP_EINVAL;
+    if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr)) return FSDP_EINVAL;
+    if (g->P > 0 && grads == nullptr) return FSDP_EINVAL;
+    if (!aligned16(grads) || !aligned16(master) || !aligned16(m) || !aligned16(v) ||
+        !aligned16(ag_next) || !aligned16(reduced) || !aligned16(scalars_dev))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    const fsdpk::AdamScalars none{};
+    cudaError_t e = fsdpk::launch_rs_adamw(*g, grads, op, master, m, v, none, ag_next, reduced,
+                                           (cudaStream_t)stream,
+                                           reinterpret_cast<const fsdpk::AdamScalars*>(scalars_dev));
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
 }  // extern "C"

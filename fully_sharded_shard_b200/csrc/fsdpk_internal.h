@@ -85,6 +85,7 @@ struct AdamScalars {
     float inv_bc2_sqrt;  // 1 / sqrt(1 - b2^t)
     float eps;
 };
+static_assert(sizeof(AdamScalars) == 32, "AdamScalars is the 32-byte fsdp_adamw_dev_scalars");
 
 // Kernel launchers (fsdpk_kernels.cu).  They enqueue work and return the
 // cudaError_t of the launch.
@@ -100,7 +101,11 @@ cudaError_t launch_rs_reduce_packed(const fsdp_group& g, const float* packed, in
                                     float* reduced, cudaStream_t st);
 cudaError_t launch_div_inplace(const fsdp_group& g, float* reduced, cudaStream_t st);
 cudaError_t launch_adamw(const fsdp_group& g, float* master, float* m, float* v,
-                         const float* grad, const AdamScalars& sc, cudaStream_t st);
+                         const float* grad, const AdamScalars& sc, cudaStream_t st,
+                         const AdamScalars* sc_dev = nullptr);
+// Advance *step on the device and write that step's scalars to *out.
+cudaError_t launch_adamw_prepare(double lr, double beta1, double beta2, double eps, double wd,
+                                 int64_t* step, AdamScalars* out, cudaStream_t st);
 cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
                          cudaStream_t st);
 // The fused reduce-scatter over a caller-supplied unit table (device memory)
@@ -113,7 +118,7 @@ cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Un
 // optional reduced-gradient output).
 cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, float* master,
                             float* m, float* v, const AdamScalars& sc, uint16_t* ag_next,
-                            float* reduced, cudaStream_t st);
+                            float* reduced, cudaStream_t st, const AdamScalars* sc_dev = nullptr);
 
 // Gradient accumulation without sync over [N][P_arena] in fp32, and the
 // reduce-scatter of the accumulated arenas (+ the last microbatch's bf16

@@ -477,7 +477,9 @@ constexpr int64_t kAdamChunk4 = (int64_t)kThreads * kAdamV;  // float4 per CTA c
 
 __global__ void __launch_bounds__(kThreads, 3)
 k_adamw(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v,
-        const float* __restrict__ g, int64_t count, AdamScalars sc) {
+        const float* __restrict__ g, int64_t count, AdamScalars sc,
+        const AdamScalars* __restrict__ sc_dev) {
+    if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
     const int64_t n4 = count >> 2;
     float4* p4 = reinterpret_cast<float4*>(p);
     float4* m4 = reinterpret_cast<float4*>(m);
@@ -689,7 +691,9 @@ __device__ __forceinline__ void fused_body(const uint16_t* __restrict__ src_al, 
 template <int NR>
 __global__ void __launch_bounds__(kThreads, 2)
 k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o,
-           const Unit* __restrict__ units, int64_t n_units, int op_avg, AdamScalars sc) {
+           const Unit* __restrict__ units, int64_t n_units, int op_avg, AdamScalars sc,
+           const AdamScalars* __restrict__ sc_dev) {
+    if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
     const bool avg = op_avg != 0;
     const float fN = (float)N;
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
@@ -1058,11 +1062,33 @@ cudaError_t launch_reduce_nr(const fsdp_group& g, const uint16_t* grads, int64_t
 
 template <int NR>
 cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const FusedOut& o,
-                               int avg, const AdamScalars& sc, cudaStream_t st) {
+                               int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
+                               cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
     k_rs_adamw<NR><<<grid_for(g, (const void*)k_rs_adamw<NR>, nu), kThreads, 0, st>>>(
-        grads, g.P_arena, g.N, o, g.d_units, nu, avg, sc);
+        grads, g.P_arena, g.N, o, g.d_units, nu, avg, sc, sc_dev);
     return cudaGetLastError();
+}
+
+// One thread: advance the device step counter and compute that step's AdamW
+// scalars in binary64, in the same operation order as the host path.
+__global__ void k_adamw_prepare(double lr, double beta1, double beta2, double eps, double wd,
+                                int64_t* __restrict__ step, AdamScalars* __restrict__ out) {
+    if (blockIdx.x != 0 || threadIdx.x != 0) return;
+    const int64_t t = *step + 1;
+    *step = t;
+    const double bc1 = 1.0 - pow(beta1, (double)t);
+    const double bc2 = 1.0 - pow(beta2, (double)t);
+    AdamScalars sc;
+    sc.decay = (float)(1.0 - lr * wd);
+    sc.beta1 = (float)beta1;
+    sc.omb1 = (float)(1.0 - beta1);
+    sc.beta2 = (float)beta2;
+    sc.omb2 = (float)(1.0 - beta2);
+    sc.step_size = (float)(lr / bc1);
+    sc.inv_bc2_sqrt = (float)(1.0 / sqrt(bc2));
+    sc.eps = (float)eps;
+    *out = sc;
 }
 
 }  // namespace
@@ -1165,12 +1191,19 @@ cudaError_t launch_div_inplace(const fsdp_group& g, float* reduced, cudaStream_t
 }
 
 cudaError_t launch_adamw(const fsdp_group& g, float* master, float* m, float* v,
-                         const float* grad, const AdamScalars& sc, cudaStream_t st) {
+                         const float* grad, const AdamScalars& sc, cudaStream_t st,
+                         const AdamScalars* sc_dev) {
     const int64_t count = (int64_t)g.N * g.S;
     if (count == 0) return cudaSuccess;
     const int64_t items = ((count >> 2) + kAdamChunk4 - 1) / kAdamChunk4;
     k_adamw<<<grid_for(g, (const void*)k_adamw, items), kThreads, 0, st>>>(master, m, v, grad,
-                                                                            count, sc);
+                                                                            count, sc, sc_dev);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_adamw_prepare(double lr, double beta1, double beta2, double eps, double wd,
+                                 int64_t* step, AdamScalars* out, cudaStream_t st) {
+    k_adamw_prepare<<<1, 32, 0, st>>>(lr, beta1, beta2, eps, wd, step, out);
     return cudaGetLastError();
 }
 
@@ -1189,18 +1222,18 @@ namespace fsdpk {
 
 cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, float* master,
                             float* m, float* v, const AdamScalars& sc, uint16_t* ag_next,
-                            float* reduced, cudaStream_t st) {
+                            float* reduced, cudaStream_t st, const AdamScalars* sc_dev) {
     if (g.units.empty()) return cudaSuccess;
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
     const FusedOut o{master, m, v, reduced, ag_next};
     switch (g.N) {
 #define FSDPK_CASE(K) \
-    case K: return launch_rs_adamw_nr<K>(g, grads, o, avg, sc, st);
+    case K: return launch_rs_adamw_nr<K>(g, grads, o, avg, sc, sc_dev, st);
         FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
         FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
 #undef FSDPK_CASE
         default:
-            return launch_rs_adamw_nr<0>(g, grads, o, avg, sc, st);
+            return launch_rs_adamw_nr<0>(g, grads, o, avg, sc, sc_dev, st);
     }
 }
 

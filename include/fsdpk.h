@@ -117,6 +117,14 @@ typedef struct {
     int64_t step;
 } fsdp_adamw_hparams;
 
+/* One step's AdamW scalars in device memory (opaque, 32 bytes, 16-byte
+ * aligned), written by fsdp_adamw_prepare and read by the *_dev entry
+ * points, so that a captured CUDA graph advances the step count each time it
+ * is replayed. */
+typedef struct {
+    float opaque[8];
+} fsdp_adamw_dev_scalars;
+
 /* ------------------------------------------------------------------------ */
 /* Plan                                                                     */
 /* ------------------------------------------------------------------------ */
@@ -262,6 +270,33 @@ FSDP_API int fsdp_copy_in_fp8(fsdp_group_t group, const float* master, uint8_t* 
  * untouched).  Algorithmic bytes: 1 read + 1 written per real element. */
 FSDP_API int fsdp_copy_out_fp8(fsdp_group_t group, const uint8_t* ag8, uint8_t* arena8,
                       fsdp_stream_t stream);
+
+/* Graph-replayable AdamW.  fsdp_adamw_step and fsdp_rs_adamw_step take the
+ * step count t from the host, so a captured CUDA graph would replay the same
+ * t; these entry points read it from device memory instead.
+ * fsdp_adamw_prepare enqueues one thread that sets *step_dev += 1 and writes
+ * the scalars of that step (decay 1 - lr*wd, lr / (1 - beta1^t),
+ * 1 / sqrt(1 - beta2^t), ...; computed in binary64 on the device, as the host
+ * path computes them) to *scalars_dev.  hparams->step is ignored; the other
+ * fields are validated as for fsdp_adamw_step.  step_dev: device int64,
+ * 8-byte aligned, set to 0 by the caller before the first step;
+ * scalars_dev: device memory, 16-byte aligned.  One prepare per step serves
+ * every group that shares the hyper-parameters.
+ * fsdp_adamw_step_dev and fsdp_rs_adamw_step_dev are fsdp_adamw_step and
+ * fsdp_rs_adamw_step with the scalars read from scalars_dev (written by a
+ * prepare earlier on the same stream). */
+FSDP_API int fsdp_adamw_prepare(const fsdp_adamw_hparams* hparams, int64_t* step_dev,
+                                fsdp_adamw_dev_scalars* scalars_dev, fsdp_stream_t stream);
+
+FSDP_API int fsdp_adamw_step_dev(fsdp_group_t group, float* master, float* m, float* v,
+                                 const float* grad, const fsdp_adamw_dev_scalars* scalars_dev,
+                                 fsdp_stream_t stream);
+
+FSDP_API int fsdp_rs_adamw_step_dev(fsdp_group_t group, const uint16_t* grads, int32_t op,
+                                    float* master, float* m, float* v,
+                                    const fsdp_adamw_dev_scalars* scalars_dev,
+                                    uint16_t* ag_next_or_null, float* reduced_or_null,
+                                    fsdp_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Reduce-scatter without any allocation                                    */

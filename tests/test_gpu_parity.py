@@ -175,3 +175,65 @@ def test_host_validation_rejects_before_launch(H):
         abi.fsdp_rs_reduce(g, grads[:5], W.AVG, buf)      # too small: caught in the binding
     torch.cuda.synchronize()
     assert torch.count_nonzero(buf) == 0 and torch.count_nonzero(ag.view(torch.int16)) == 0
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["stages", "fused"])
+def test_graph_replayed_steps_equal_eager_steps(H, fused):
+    """A captured CUDA graph of one step (device step counter + AdamW scalars),
+    replayed 3 times, gives the same state as 3 eager steps with host step
+    counts, and stays within the AdamW tolerance of the oracle."""
+    import numpy as np
+    import oracle
+    from fully_sharded_shard_b200 import abi
+    wl = W.uneven(8)
+    grp = wl.groups[0]
+    g = abi.fsdp_plan_group(grp.shapes, wl.N)
+    p = oracle.plan(grp.shapes, wl.N)
+    NS = wl.N * g.S
+    full = torch.empty(g.P_arena, device="cuda")
+    W.fill_master(full, wl, grp.name)
+    grads = H.make_grads(g, wl, grp, 1)
+    hp = dict(W.ADAMW_DEFAULTS)
+    states = []
+    for _ in range(2):
+        master = torch.empty(NS, device="cuda")
+        abi.fsdp_shard_params(g, full, master)
+        states.append((master, torch.zeros(NS, device="cuda"), torch.zeros(NS, device="cuda"),
+                       torch.empty(NS, device="cuda"), torch.empty(NS, dtype=torch.bfloat16, device="cuda")))
+    (pa, ma, va, ra, aga), (pb, mb, vb, rb, agb) = states
+    for step in (1, 2, 3):                                  # eager, host step counts
+        if fused:
+            abi.fsdp_rs_adamw_step(g, grads, wl.op, pa, ma, va, step=step, ag_next=aga, **hp)
+        else:
+            abi.fsdp_rs_reduce(g, grads, wl.op, ra)
+            abi.fsdp_adamw_step(g, pa, ma, va, ra, step=step, **hp)
+    ds = abi.DeviceStep()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        abi.fsdp_adamw_prepare(ds, **hp)
+        if fused:
+            abi.fsdp_rs_adamw_step_dev(g, grads, wl.op, pb, mb, vb, ds, ag_next=agb)
+        else:
+            abi.fsdp_rs_reduce(g, grads, wl.op, rb)
+            abi.fsdp_adamw_step_dev(g, pb, mb, vb, rb, ds)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert int(ds.step.item()) == 3
+    for a, b in ((pa, pb), (ma, mb), (va, vb)):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    if fused:
+        assert torch.equal(aga.view(torch.int16), agb.view(torch.int16))
+    # the oracle, three steps on the same reduced gradient
+    red_o = oracle.reduce_scatter_direct(p, H.u16(grads), wl.op)
+    mo = oracle.shard(p, H.f32(full))
+    m_o, v_o = np.zeros_like(mo), np.zeros_like(mo)
+    for step in (1, 2, 3):
+        oracle.adamw(mo, m_o, v_o, red_o, step=step, **hp)
+    for gbuf, obuf in ((pb, mo), (mb, m_o), (vb, v_o)):
+        ok, ratio = H.adam_close(H.f32(gbuf), obuf)
+        assert ok, ratio
+    del graph
+    g.destroy()
