@@ -505,7 +505,8 @@ def run_ours(args, wl, device, rank, ws):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32+bf16",
+        "dtype": "f32",
+        "storage_dtypes": "fp32 master/m/v/reduced grads; bf16 all-gather buffer, params, per-rank grads",
         "data": "synthetic: seeded N(0,0.02) fp32 master, N(0,1e-3) bf16 per-rank grads",
         "config": {
             "workload": wl.name,
@@ -882,7 +883,7 @@ def run_reference(args, wl):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s",
         "params_per_s": round(p.P / dt, 1), "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32+bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic: seeded N(0,0.02) fp32 master, N(0,1e-3) bf16 per-rank grads",
         "config": {"workload": wl.name, "N_virtual_ranks": wl.N,
                    "sample_group": grp.name, "params_per_sample": p.P},

@@ -237,3 +237,33 @@ def test_graph_replayed_steps_equal_eager_steps(H, fused):
         assert ok, ratio
     del graph
     g.destroy()
+
+
+def test_bench_two_stream_schedules_match_one_stream(H):
+    """bench.py's two-stream schedules (all-gather half on one stream, the
+    update half on another) leave exactly the state of the one-stream
+    schedules: the event dependencies order every buffer reuse."""
+    import bench
+    wl = W.llama7b(16, layers=3)
+    dev = torch.device("cuda", 0)
+    a = bench.Model(wl, dev, 2, 0)
+    b = bench.Model(wl, dev, 2, 0)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(3):
+        a.step(s1)
+        b.step_two_streams(s1, s2)
+    torch.cuda.synchronize()
+    for (_, pa, ma, va, _), (_, pb, mb, vb, _) in zip(a.instances, b.instances):
+        for x, y in ((pa, pb), (ma, mb), (va, vb)):
+            assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+    a.enable_fused()
+    b.enable_fused()
+    for _ in range(3):
+        a.fused_step(s1)
+        b.fused_step_two_streams(s1, s2)
+    torch.cuda.synchronize()
+    for (_, pa, ma, va, _), (_, pb, mb, vb, _) in zip(a.instances, b.instances):
+        for x, y in ((pa, pb), (ma, mb), (va, vb)):
+            assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+    for x, y in zip(a.ag_groups, b.ag_groups):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
