@@ -267,3 +267,18 @@ def test_bench_two_stream_schedules_match_one_stream(H):
             assert torch.equal(x.view(torch.int32), y.view(torch.int32))
     for x, y in zip(a.ag_groups, b.ag_groups):
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+EDGE = [
+    _wl("max_world_1024", [(2000, 3), (5,), (1030, 1)], 1024, op=W.SUM_THEN_DIV),
+    _wl("conv_like_4d", [(64, 3, 7, 7), (64,), (128, 64, 3, 3), (10, 2, 3, 1, 5)], 6),
+    _wl("scalars_0d", [(), (3,), (), (17, 4)], 3),
+    _wl("rows_on_rank0_only", [(1, 4096), (2, 513), (1,)], 8),
+]
+
+
+@pytest.mark.parametrize("wl", EDGE, ids=[w.name for w in EDGE])
+def test_edge_shapes_and_world_sizes(H, wl):
+    H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=wl.N <= 64)
+    H.run_group_fused(wl, wl.groups[0], steps=2)
+    H.run_group_fp8(wl, wl.groups[0])
