@@ -848,6 +848,9 @@ def oracle_setup(wl):
 
 
 def cpu_baseline(wl, min_seconds: float):
+    """The oracle on the host cores: all threads for >= min_seconds, then one
+    single-threaded pass; both over one group of the workload, the full-step
+    time extrapolated from the per-element rate."""
     O, grp, p, full, grads, state = oracle_setup(wl)
     cores = O.get_threads()
     t0 = time.time()
@@ -858,12 +861,22 @@ def cpu_baseline(wl, min_seconds: float):
         if time.time() - t0 >= min_seconds:
             break
     dt = (time.time() - t0) / passes
+    O.set_threads(1)
+    t1 = time.time()
+    oracle_pass(O, p, full, grads, wl, state, passes + 1)
+    dt1 = time.time() - t1
+    O.set_threads(cores)
     b = group_bytes(wl.N, p.S, p.P)
+    step_params = wl.total_params()
     return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "params_per_s": round(p.P / dt, 1),
+            "value_1core": round(b / dt1 / 1e9, 3),
+            "extrapolated_full_step_s": round(dt * step_params / p.P, 1),
+            "extrapolated_full_step_s_1core": round(dt1 * step_params / p.P, 1),
             "sample": f"{passes} oracle pass(es) over one '{grp.name}' group of {wl.name} "
                       f"({p.P} params, N={wl.N}): copy-in, copy-out, reduce-scatter, AdamW; "
-                      f"{dt:.2f} s per pass, OpenMP over {cores} threads"}
+                      f"{dt:.2f} s per pass on {cores} threads (OpenMP), {dt1:.2f} s on 1 thread; "
+                      f"full step extrapolated by parameter count"}
 
 
 def run_reference(args, wl):

@@ -616,13 +616,13 @@ __device__ __forceinline__ void load_pmv8(const FusedOut& o, int64_t k, float4 (
     V[1] = __ldcs(v4 + 1);
 }
 
-// Rank-ordered fold of 8 elements; NR = N at compile time (1..8) or 0 (any).
-// A misaligned run folds its ranks in batches of 4 (two 16-byte vectors per
-// rank would otherwise be live at once next to master/m/v).
+// Rank-ordered fold of 8 elements; NR = N at compile time (1..8): all NR
+// ranks' loads (two 16-byte vectors per rank on a misaligned run) are issued
+// before the fold.  NR = 0 (any N): ranks in batches of 4.
 template <int NR, bool SHIFTED>
 __device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64_t stride, int N,
                                       int q, int D, float (&acc)[8]) {
-    if constexpr (NR != 0 && !SHIFTED) {
+    if constexpr (NR != 0) {
         uint4 a[NR], b[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
