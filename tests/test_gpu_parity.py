@@ -11,6 +11,7 @@ real shapes, in the same launch configuration the benchmark times (the 7B
 model's 32 block groups share one plan, so one block group plus the root
 group covers every launch it makes).
 """
+import numpy as np
 import pytest
 import torch
 
@@ -282,3 +283,25 @@ def test_edge_shapes_and_world_sizes(H, wl):
     H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=wl.N <= 64)
     H.run_group_fused(wl, wl.groups[0], steps=2)
     H.run_group_fp8(wl, wl.groups[0])
+
+
+def _random_group(rng, k):
+    N = int(rng.integers(1, 17))
+    shapes = []
+    for _ in range(int(rng.integers(1, 7))):
+        nd = int(rng.integers(0, 5))
+        dims = [int(rng.integers(0, 40)) if rng.random() < 0.1 else int(rng.integers(1, 300))]
+        dims += [int(rng.integers(1, 9)) for _ in range(max(nd - 1, 0))]
+        shapes.append(tuple(dims[:nd]) if nd > 0 else ())
+    return _wl(f"rand{k}", shapes, N, op=[W.SUM, W.AVG, W.SUM_THEN_DIV][k % 3])
+
+
+RANDOM = [_random_group(np.random.default_rng(1000 + k), k) for k in range(40)]
+
+
+@pytest.mark.parametrize("wl", RANDOM, ids=[w.name for w in RANDOM])
+def test_random_groups_brute_force(H, wl):
+    grp = wl.groups[0]
+    H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
+    H.run_group_fused(wl, grp, steps=1)
+    H.run_group_fp8(wl, grp)
