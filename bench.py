@@ -39,7 +39,7 @@ if ROOT not in sys.path:
 METRIC = "FSDP2 step GB/s and params/s over N virtual ranks; % of HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
-KERNELS_SRC = os.path.join(ROOT, "fully_sharded_shard_b200", "csrc", "fsdpk_kernels.cu")
+KERNELS_DIR = os.path.join(ROOT, "fully_sharded_shard_b200", "csrc")
 TRAFFIC_JSON = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
@@ -178,8 +178,13 @@ class ClockSampler:
 
 
 def kernels_hash() -> str:
-    with open(KERNELS_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of every kernel source file (the .cu files and the device header)."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(KERNELS_DIR)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(KERNELS_DIR, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):

@@ -1,0 +1,141 @@
+// fsdpk_device.cuh -- device helpers and launch geometry shared by the kernel
+// files of libfsdpk.so (fsdpk_gather.cu, fsdpk_reduce.cu, fsdpk_update.cu).
+// Every stage is HBM-bound streaming (well under one flop per byte), so
+// nothing here uses tensor cores: 16-byte coalesced accesses, enough bytes in
+// flight per SM to cover HBM latency, streaming (evict-first) cache hints for
+// data touched once, one CTA per work item launched in order.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "fsdpk_internal.h"
+
+namespace fsdpk {
+namespace {
+
+constexpr int kThreads = 256;
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
+    return __uint_as_float(h << 16);
+}
+
+// 8 bf16 (one 16-byte vector) -> 8 fp32, exact widening.
+__device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
+    x[0] = __uint_as_float(w.x << 16);
+    x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(w.y << 16);
+    x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+    x[4] = __uint_as_float(w.z << 16);
+    x[5] = __uint_as_float(w.z & 0xFFFF0000u);
+    x[6] = __uint_as_float(w.w << 16);
+    x[7] = __uint_as_float(w.w & 0xFFFF0000u);
+}
+
+// Two fp32 -> one bf16x2 word (round to nearest even); lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The 8 bf16 elements that start D (1..7) elements into the 16 elements a:b
+// (a at the lower address): word j of the result is bits [16*D, 16*D + 32)
+// of the 64-bit pair (w[j + D/2 + 1] : w[j + D/2]).
+__device__ __forceinline__ uint4 shift_bf16x8(const uint4& a, const uint4& b, int D) {
+    const int s = D >> 1;
+    const uint32_t sh = (D & 1) ? 16u : 0u;
+    const uint32_t w0 = s == 0 ? a.x : s == 1 ? a.y : s == 2 ? a.z : a.w;
+    const uint32_t w1 = s == 0 ? a.y : s == 1 ? a.z : s == 2 ? a.w : b.x;
+    const uint32_t w2 = s == 0 ? a.z : s == 1 ? a.w : s == 2 ? b.x : b.y;
+    const uint32_t w3 = s == 0 ? a.w : s == 1 ? b.x : s == 2 ? b.y : b.z;
+    const uint32_t w4 = s == 0 ? b.x : s == 1 ? b.y : s == 2 ? b.z : b.w;
+    return make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh),
+                      __funnelshift_r(w2, w3, sh), __funnelshift_r(w3, w4, sh));
+}
+
+// Aligned source vector load.  Unshifted, every vector is read once, so it
+// streams past L1; shifted, the neighbouring thread reads the same vector as
+// its second operand, so it is kept in L1 (read-only path).
+template <bool SHIFTED>
+__device__ __forceinline__ uint4 ld_src(const uint4* p) {
+    if constexpr (SHIFTED) {
+        return __ldg(p);
+    } else {
+        return __ldcs(p);
+    }
+}
+
+// Elements to peel before `p` reaches a 16-byte boundary (capped at len).
+template <typename T>
+__device__ __forceinline__ int64_t head_to_16B(const T* p, int64_t len) {
+    const int64_t h = (int64_t)((16u - (reinterpret_cast<uintptr_t>(p) & 15u)) & 15u) / sizeof(T);
+    return h < len ? h : len;
+}
+
+// Position, in bf16 elements, of `p` inside its 16-byte vector.
+__device__ __forceinline__ int bf16_phase(const uint16_t* p) {
+    return (int)((reinterpret_cast<uintptr_t>(p) >> 1) & 7u);
+}
+
+// Zero-fill `len` fp32 elements at dst (any alignment).
+__device__ __forceinline__ void zero_f32_run(float* __restrict__ dst, int64_t len) {
+    int64_t head = (4 - (reinterpret_cast<uintptr_t>(dst) >> 2 & 3)) & 3;
+    if (head > len) head = len;
+    if (threadIdx.x < head) dst[threadIdx.x] = 0.0f;
+    const int64_t nv = (len - head) >> 2;
+    float4* d4 = reinterpret_cast<float4*>(dst + head);
+    for (int64_t q = threadIdx.x; q < nv; q += blockDim.x)
+        __stcs(d4 + q, make_float4(0.f, 0.f, 0.f, 0.f));
+    const int64_t done = head + 4 * nv;
+    if (threadIdx.x < len - done) dst[done + threadIdx.x] = 0.0f;
+}
+
+template <int NR>
+__device__ __forceinline__ float fold_scalar(const uint16_t* __restrict__ src, int64_t stride,
+                                             int N) {
+    const int n = NR ? NR : N;
+    float acc = bf16_bits_to_f32(src[0]);
+    for (int r = 1; r < n; ++r) acc = __fadd_rn(acc, bf16_bits_to_f32(src[r * stride]));
+    return acc;
+}
+
+__device__ __forceinline__ float finish(float acc, bool avg, float fN) {
+    return avg ? __fdiv_rn(acc, fN) : acc;
+}
+
+__device__ __forceinline__ void store8(float* __restrict__ dst, const float (&acc)[8]) {
+    float4* o = reinterpret_cast<float4*>(dst);
+    __stcs(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
+    __stcs(o + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
+}
+
+__device__ __forceinline__ void adamw1(float& p, float& m, float& v, float g,
+                                       const AdamScalars& sc) {
+    p = p * sc.decay;
+    m = fmaf(sc.beta1, m, sc.omb1 * g);
+    v = fmaf(sc.beta2, v, sc.omb2 * g * g);
+    const float denom = fmaf(__fsqrt_rn(v), sc.inv_bc2_sqrt, sc.eps);
+    p = fmaf(-sc.step_size, __fdiv_rn(m, denom), p);
+}
+
+// ---------------------------------------------------------------------------
+// launch geometry
+// ---------------------------------------------------------------------------
+// One CTA per work item (tile, unit or chunk), launched in order.  On B200 a
+// grid that covers the work once streams 12-17 % faster than a persistent
+// grid-stride loop with a static cyclic assignment: the hardware hands out
+// CTAs in index order as slots free up, so the addresses in flight stay a
+// compact window instead of drifting apart across the arrays.
+inline unsigned grid_for(const fsdp_group&, const void*, int64_t items) {
+    return (unsigned)std::min<int64_t>(std::max<int64_t>(items, 1), 0x7FFFFFFF);
+}
+
+}  // namespace
+}  // namespace fsdpk

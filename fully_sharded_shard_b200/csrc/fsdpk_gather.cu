@@ -1,0 +1,391 @@
+// fsdpk_gather.cu -- the all-gather half of the step and the set-up shard:
+// copy-in (fp32 shards -> bf16 slots of the rank-major all-gather buffer),
+// copy-out (the buffer -> unsharded per-parameter views), Shard(0)
+// placement, and the FP8 (E4M3) copy-in / copy-out.
+//   copy-in  -- "Sharded Training: FSDP2, DTensor, Tensor and Pipeline
+//               Parallelism", Mixed precision paragraph: bf16 copies of the fp32
+//               shards are all-gathered.
+//   copy-out -- "Introduction to PyTorch FSDP2 Backend Features", Working
+//               Principle (All-Gather state): shards become full parameters.
+//   FP8      -- "PyTorch FSDP2 Guide: Distributed LLM Training with DTensor",
+//               Deep Dive, 2. Native FP8 Training with Float8Tensor.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cuda_fp8.h>
+
+#include "fsdpk_device.cuh"
+
+namespace fsdpk {
+namespace {
+
+// ---------------------------------------------------------------------------
+// copy-in: ag[k] = bf16_rn(master[k]) for real elements, +0 in pad rows
+// ---------------------------------------------------------------------------
+
+// Bit i set when element k0+i lies in a pad interval.  Intervals in
+// [rb, re) are sorted and disjoint; at most 8 of them can meet [k0, k0+8).
+__device__ __forceinline__ uint32_t pad_mask8(int64_t k0, const Interval* __restrict__ iv,
+                                              int rb, int re) {
+    // first interval with hi > k0
+    int lo = rb, hi = re;
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (iv[mid].hi > k0) hi = mid; else lo = mid + 1;
+    }
+    uint32_t mask = 0;
+    for (int t = lo; t < re; ++t) {
+        int64_t a = iv[t].lo, b = iv[t].hi;
+        if (a >= k0 + 8) break;
+        int64_t s = a > k0 ? a - k0 : 0;
+        int64_t e = b < k0 + 8 ? b - k0 : 8;
+        mask |= ((1u << e) - 1u) & ~((1u << s) - 1u);
+    }
+    return mask;
+}
+
+constexpr int kCopyInV = 4;  // vectors of 8 per thread per tile
+static_assert(kCopyInTile == kThreads * 8 * kCopyInV, "copy-in tile shape");
+
+__global__ void __launch_bounds__(kThreads)
+k_copy_in(const float* __restrict__ master, uint16_t* __restrict__ ag, int64_t count,
+          int64_t n_tiles, const Interval* __restrict__ iv,
+          const TileRange* __restrict__ tr) {
+    for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+        const int64_t base = t * kCopyInTile;
+        const int64_t end = min(base + kCopyInTile, count);
+        TileRange rng{0, 0};
+        if (tr != nullptr) rng = tr[t];
+        float4 x[kCopyInV][2];
+#pragma unroll
+        for (int j = 0; j < kCopyInV; ++j) {
+            const int64_t k = base + 8 * (threadIdx.x + (int64_t)j * kThreads);
+            if (k + 8 <= end) {
+                const float4* src = reinterpret_cast<const float4*>(master + k);
+                x[j][0] = __ldcs(src);
+                x[j][1] = __ldcs(src + 1);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kCopyInV; ++j) {
+            const int64_t k = base + 8 * (threadIdx.x + (int64_t)j * kThreads);
+            if (k + 8 <= end) {
+                float f[8] = {x[j][0].x, x[j][0].y, x[j][0].z, x[j][0].w,
+                              x[j][1].x, x[j][1].y, x[j][1].z, x[j][1].w};
+                if (rng.begin < rng.end) {
+                    uint32_t mk = pad_mask8(k, iv, rng.begin, rng.end);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (mk & (1u << e)) f[e] = 0.0f;
+                }
+                uint4 o = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                __stcs(reinterpret_cast<uint4*>(ag + k), o);
+            } else if (k < end) {
+                // ragged tail of the whole buffer: element by element
+                for (int64_t q = k; q < end; ++q) {
+                    float f = master[q];
+                    if (rng.begin < rng.end && (pad_mask8(q, iv, rng.begin, rng.end) & 1u))
+                        f = 0.0f;
+                    __nv_bfloat16 h = __float2bfloat16_rn(f);
+                    ag[q] = *reinterpret_cast<uint16_t*>(&h);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// copy-out: arena[arena_pos + e] = ag[shard_pos + e] for each real unit
+// ---------------------------------------------------------------------------
+
+template <bool SHIFTED>
+__device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_al,
+                                              uint16_t* __restrict__ dst, int nvec, int D) {
+    constexpr int V = SHIFTED ? 2 : 4;
+    const uint4* s = reinterpret_cast<const uint4*>(src_al);
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll 1
+    for (int q0 = threadIdx.x; q0 < nvec; q0 += blockDim.x * V) {
+        uint4 a[V], b[V];
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int q = q0 + k * blockDim.x;
+            if (q < nvec) {
+                a[k] = ld_src<SHIFTED>(s + q);
+                if constexpr (SHIFTED) b[k] = ld_src<SHIFTED>(s + q + 1);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int q = q0 + k * blockDim.x;
+            if (q < nvec) {
+                uint4 o;
+                if constexpr (SHIFTED) o = shift_bf16x8(a[k], b[k], D);
+                else o = a[k];
+                __stcs(d + q, o);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 5)
+k_copy_out(const uint16_t* __restrict__ ag, uint16_t* __restrict__ arena,
+           const Unit* __restrict__ units, int64_t n_units) {
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        uint16_t* dst_run = arena + u.arena_pos;
+        const uint16_t* src_run = ag + u.shard_pos;
+        const int head = (int)head_to_16B(dst_run, len);
+        if ((int)threadIdx.x < head) dst_run[threadIdx.x] = src_run[threadIdx.x];
+        const int nvec = (len - head) >> 3;
+        const int D = bf16_phase(src_run + head);
+        const uint16_t* src_al = src_run + head - D;
+        uint16_t* dst = dst_run + head;
+        if (D == 0) copy_out_body<false>(src_al, dst, nvec, 0);
+        else copy_out_body<true>(src_al, dst, nvec, D);
+        const int done = head + 8 * nvec;
+        if ((int)threadIdx.x < len - done) dst_run[done + threadIdx.x] = src_run[done + threadIdx.x];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// shard: master[shard_pos + e] = full[arena_pos + e]; pads +0 (set-up path)
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kThreads)
+k_shard(const float* __restrict__ full, float* __restrict__ master,
+        const Unit* __restrict__ units, int64_t n_units) {
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        if (u.is_pad) {
+            zero_f32_run(master + u.shard_pos, u.len);
+            continue;
+        }
+        for (int64_t e = threadIdx.x; e < u.len; e += blockDim.x)
+            master[u.shard_pos + e] = full[u.arena_pos + e];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// FP8 (E4M3) all-gather copy-in and copy-out
+//   amax_i = max |x| over parameter i (NaN ignored), scale_i = 448 / max(amax_i,
+//   1e-12), ag8[k] = e4m3_rn(clamp(x * scale_i, -448, 448)), pads 0x00.
+// ---------------------------------------------------------------------------
+
+// Max |x| of each real unit, folded into its parameter's slot with an integer
+// atomicMax (non-negative floats order like their bit patterns).
+__global__ void __launch_bounds__(kThreads)
+k_fp8_amax(const float* __restrict__ master, unsigned* __restrict__ amax_bits,
+           const Unit* __restrict__ units, const int32_t* __restrict__ unit_param,
+           int64_t n_real) {
+    __shared__ float part[kThreads / 32];
+    for (int64_t ui = blockIdx.x; ui < n_real; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const float* src = master + u.shard_pos;
+        const int len = u.len;
+        const int head = (int)head_to_16B(src, len);
+        float mx = 0.0f;
+        for (int e = threadIdx.x; e < head; e += blockDim.x) mx = fmaxf(mx, fabsf(src[e]));
+        const int nv = (len - head) >> 2;
+        const float4* s4 = reinterpret_cast<const float4*>(src + head);
+#pragma unroll 4
+        for (int q = threadIdx.x; q < nv; q += blockDim.x) {
+            const float4 x = __ldcs(s4 + q);
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+        }
+        for (int e = head + 4 * nv + threadIdx.x; e < len; e += blockDim.x)
+            mx = fmaxf(mx, fabsf(src[e]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            mx = threadIdx.x < kThreads / 32 ? part[threadIdx.x] : 0.0f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (threadIdx.x == 0) atomicMax(amax_bits + unit_param[ui], __float_as_uint(mx));
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_fp8_scales(float* __restrict__ scales, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) scales[i] = __fdiv_rn(448.0f, fmaxf(scales[i], 1e-12f));
+}
+
+// x * scale clamped to the finite E4M3 range (NaN passes through).
+__device__ __forceinline__ float fp8_in(float x, float sc) {
+    float y = __fmul_rn(x, sc);
+    if (y > 448.0f) y = 448.0f;
+    if (y < -448.0f) y = -448.0f;
+    return y;
+}
+
+// Two floats -> two E4M3 bytes (lo in bits 0..7), round to nearest even.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ uint8_t e4m3(float x) {
+    return (uint8_t)(e4m3x2(x, 0.0f) & 0xFFu);
+}
+
+__device__ __forceinline__ void zero_u8_run(uint8_t* __restrict__ dst, int len) {
+    const int head = (int)head_to_16B(dst, len);
+    if ((int)threadIdx.x < head) dst[threadIdx.x] = 0;
+    const int nv = (len - head) >> 4;
+    uint4* d = reinterpret_cast<uint4*>(dst + head);
+    for (int q = threadIdx.x; q < nv; q += blockDim.x) __stcs(d + q, make_uint4(0u, 0u, 0u, 0u));
+    const int done = head + 16 * nv;
+    if ((int)threadIdx.x < len - done) dst[done + threadIdx.x] = 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
+k_fp8_copy_in(const float* __restrict__ master, uint8_t* __restrict__ ag8,
+              const float* __restrict__ scales, const Unit* __restrict__ units,
+              const int32_t* __restrict__ unit_param, int64_t n_units) {
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        uint8_t* dst = ag8 + u.shard_pos;
+        const int len = u.len;
+        if (u.is_pad) {
+            zero_u8_run(dst, len);
+            continue;
+        }
+        const float sc = scales[unit_param[ui]];
+        const float* src = master + u.shard_pos;
+        // 16-byte output vectors; the fp32 source of a vector is then 64-byte aligned
+        const int head = (int)head_to_16B(dst, len);
+        if ((int)threadIdx.x < head) dst[threadIdx.x] = e4m3(fp8_in(src[threadIdx.x], sc));
+        const int nv = (len - head) >> 4;
+        const float4* s4 = reinterpret_cast<const float4*>(src + head);
+        uint4* d = reinterpret_cast<uint4*>(dst + head);
+#pragma unroll 1
+        for (int q = threadIdx.x; q < nv; q += blockDim.x) {
+            float4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[k] = __ldcs(s4 + 4 * q + k);
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t lo = e4m3x2(fp8_in(x[k].x, sc), fp8_in(x[k].y, sc));
+                const uint32_t hi = e4m3x2(fp8_in(x[k].z, sc), fp8_in(x[k].w, sc));
+                w[k] = (lo & 0xFFFFu) | (hi << 16);
+            }
+            __stcs(d + q, make_uint4(w[0], w[1], w[2], w[3]));
+        }
+        const int done = head + 16 * nv;
+        if ((int)threadIdx.x < len - done)
+            dst[done + threadIdx.x] = e4m3(fp8_in(src[done + threadIdx.x], sc));
+    }
+}
+
+// The 16 bytes that start D (1..15) bytes into the 32 bytes a:b.
+__device__ __forceinline__ uint4 shift_bytes16(const uint4& a, const uint4& b, int D) {
+    const int s = D >> 2;
+    const uint32_t sh = 8u * (uint32_t)(D & 3);
+    const uint32_t w0 = s == 0 ? a.x : s == 1 ? a.y : s == 2 ? a.z : a.w;
+    const uint32_t w1 = s == 0 ? a.y : s == 1 ? a.z : s == 2 ? a.w : b.x;
+    const uint32_t w2 = s == 0 ? a.z : s == 1 ? a.w : s == 2 ? b.x : b.y;
+    const uint32_t w3 = s == 0 ? a.w : s == 1 ? b.x : s == 2 ? b.y : b.z;
+    const uint32_t w4 = s == 0 ? b.x : s == 1 ? b.y : s == 2 ? b.z : b.w;
+    return make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh),
+                      __funnelshift_r(w2, w3, sh), __funnelshift_r(w3, w4, sh));
+}
+
+__global__ void __launch_bounds__(kThreads, 5)
+k_fp8_copy_out(const uint8_t* __restrict__ ag8, uint8_t* __restrict__ arena8,
+               const Unit* __restrict__ units, int64_t n_units) {
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        uint8_t* dst = arena8 + u.arena_pos;
+        const uint8_t* src = ag8 + u.shard_pos;
+        const int head = (int)head_to_16B(dst, len);
+        if ((int)threadIdx.x < head) dst[threadIdx.x] = src[threadIdx.x];
+        const int nv = (len - head) >> 4;
+        const int D = (int)(reinterpret_cast<uintptr_t>(src + head) & 15u);
+        const uint4* sa = reinterpret_cast<const uint4*>(src + head - D);
+        uint4* d = reinterpret_cast<uint4*>(dst + head);
+        if (D == 0) {
+#pragma unroll 4
+            for (int q = threadIdx.x; q < nv; q += blockDim.x) __stcs(d + q, __ldcs(sa + q));
+        } else {
+#pragma unroll 2
+            for (int q = threadIdx.x; q < nv; q += blockDim.x)
+                __stcs(d + q, shift_bytes16(__ldg(sa + q), __ldg(sa + q + 1), D));
+        }
+        const int done = head + 16 * nv;
+        if ((int)threadIdx.x < len - done) dst[done + threadIdx.x] = src[done + threadIdx.x];
+    }
+}
+
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* ag,
+                           cudaStream_t st) {
+    const int64_t count = (int64_t)g.N * g.S;
+    if (count == 0) return cudaSuccess;
+    const bool pads = !g.tile_ranges.empty();
+    k_copy_in<<<grid_for(g, (const void*)k_copy_in, g.n_tiles), kThreads, 0, st>>>(
+        master, ag, count, g.n_tiles, pads ? g.d_intervals : nullptr,
+        pads ? g.d_tile_ranges : nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* arena,
+                            cudaStream_t st) {
+    if (g.n_real_units == 0) return cudaSuccess;
+    k_copy_out<<<grid_for(g, (const void*)k_copy_out, g.n_real_units), kThreads, 0, st>>>(
+        ag, arena, g.d_units, g.n_real_units);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
+                         cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu == 0) return cudaSuccess;
+    k_shard<<<grid_for(g, (const void*)k_shard, nu), kThreads, 0, st>>>(full, master, g.d_units,
+                                                                        nu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_in_fp8(const fsdp_group& g, const float* master, uint8_t* ag8,
+                               float* scales, cudaStream_t st) {
+    if (g.n > 0) {
+        cudaError_t e = cudaMemsetAsync(scales, 0, (size_t)g.n * sizeof(float), st);
+        if (e != cudaSuccess) return e;
+        if (g.n_real_units > 0)
+            k_fp8_amax<<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
+                master, reinterpret_cast<unsigned*>(scales), g.d_units, g.d_unit_param,
+                g.n_real_units);
+        k_fp8_scales<<<(unsigned)((g.n + kThreads - 1) / kThreads), kThreads, 0, st>>>(scales, g.n);
+    }
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu > 0)
+        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(master, ag8, scales,
+                                                                     g.d_units, g.d_unit_param, nu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t* arena8,
+                                cudaStream_t st) {
+    if (g.n_real_units == 0) return cudaSuccess;
+    k_fp8_copy_out<<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(ag8, arena8,
+                                                                              g.d_units,
+                                                                              g.n_real_units);
+    return cudaGetLastError();
+}
+
+}  // namespace fsdpk

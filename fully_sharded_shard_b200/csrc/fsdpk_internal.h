@@ -87,7 +87,7 @@ struct AdamScalars {
 };
 static_assert(sizeof(AdamScalars) == 32, "AdamScalars is the 32-byte fsdp_adamw_dev_scalars");
 
-// Kernel launchers (fsdpk_kernels.cu).  They enqueue work and return the
+// Kernel launchers (fsdpk_gather.cu, fsdpk_reduce.cu, fsdpk_update.cu).  They enqueue work and return the
 // cudaError_t of the launch.
 cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* ag,
                            cudaStream_t st);

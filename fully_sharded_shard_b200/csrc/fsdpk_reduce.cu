@@ -1,0 +1,477 @@
+// fsdpk_reduce.cu -- the reduce-scatter: per-rank bf16 gradients cast to
+// reduce_dtype fp32, packed per destination rank and folded in rank order (SUM,
+// AVG, or SUM then FSDP's own division), fused or through a materialised
+// packed buffer; and gradient accumulation without sync with the
+// reduce-scatter of the accumulated gradients.
+//   "Introduction to PyTorch FSDP2 Backend Features", Mixed Precision;
+//   "Sharded Training: FSDP2, DTensor, Tensor and Pipeline Parallelism",
+//   Mixed precision and Other controls paragraphs, The bug Adam hid.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "fsdpk_device.cuh"
+
+namespace fsdpk {
+namespace {
+
+// ---------------------------------------------------------------------------
+// reduce-scatter, fused pack + rank-ordered reduction
+// red[shard_pos + e] = ((g_0 + g_1) + ...) + g_{N-1}, g_r = fp32(grads[r][arena_pos + e])
+// NR = ranks known at compile time (1..8), 0 = any N (batches of 4).
+// ---------------------------------------------------------------------------
+
+// Compile-time rank count: all NR loads of a vector are issued before the fold.
+template <int NR, bool SHIFTED, int V>
+__device__ __forceinline__ void reduce_body(const uint16_t* __restrict__ src_al, int64_t stride,
+                                            float* __restrict__ dst, int nvec, int D, bool avg,
+                                            float fN) {
+#pragma unroll 1
+    for (int q0 = threadIdx.x; q0 < nvec; q0 += blockDim.x * V) {
+        uint4 a[V][NR];
+        uint4 b[V][NR];
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int q = q0 + k * blockDim.x;
+            if (q < nvec) {
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const uint4* s = reinterpret_cast<const uint4*>(src_al + r * stride) + q;
+                    a[k][r] = ld_src<SHIFTED>(s);
+                    if constexpr (SHIFTED) b[k][r] = ld_src<SHIFTED>(s + 1);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int q = q0 + k * blockDim.x;
+            if (q < nvec) {
+                float acc[8];
+                unpack8(SHIFTED ? shift_bf16x8(a[k][0], b[k][0], D) : a[k][0], acc);
+#pragma unroll
+                for (int r = 1; r < NR; ++r) {
+                    float x[8];
+                    unpack8(SHIFTED ? shift_bf16x8(a[k][r], b[k][r], D) : a[k][r], x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], x[e]);
+                }
+                if (avg) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[e] = __fdiv_rn(acc[e], fN);
+                }
+                store8(dst + 8 * q, acc);
+            }
+        }
+    }
+}
+
+// Any rank count: ranks in batches of 4, folded in rank order.
+template <bool SHIFTED>
+__device__ __forceinline__ void reduce_body_any(const uint16_t* __restrict__ src_al,
+                                                int64_t stride, int N,
+                                                float* __restrict__ dst, int nvec, int D,
+                                                bool avg, float fN) {
+#pragma unroll 1
+    for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+        float acc[8];
+#pragma unroll 1
+        for (int r0 = 0; r0 < N; r0 += 4) {
+            uint4 a[4], b[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r0 + r < N) {
+                    const uint4* s =
+                        reinterpret_cast<const uint4*>(src_al + (int64_t)(r0 + r) * stride) + q;
+                    a[r] = ld_src<SHIFTED>(s);
+                    if constexpr (SHIFTED) b[r] = ld_src<SHIFTED>(s + 1);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r0 + r < N) {
+                    float x[8];
+                    unpack8(SHIFTED ? shift_bf16x8(a[r], b[r], D) : a[r], x);
+                    if (r0 + r == 0) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] = x[e];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], x[e]);
+                    }
+                }
+            }
+        }
+        if (avg) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fdiv_rn(acc[e], fN);
+        }
+        store8(dst + 8 * q, acc);
+    }
+}
+
+template <int NR, bool SHIFTED>
+__device__ __forceinline__ void reduce_body_dispatch(const uint16_t* src_al, int64_t stride,
+                                                     int N, float* dst, int nvec, int D, bool avg,
+                                                     float fN) {
+    if constexpr (NR == 0) {
+        reduce_body_any<SHIFTED>(src_al, stride, N, dst, nvec, D, avg, fN);
+    } else {
+        // keep about 4-8 independent 16-byte loads in flight per thread
+        constexpr int V = NR >= 4 ? 1 : (4 / NR);
+        reduce_body<NR, SHIFTED, V>(src_al, stride, dst, nvec, D, avg, fN);
+    }
+}
+
+// One launch covers every unit of the group.  blockIdx.y selects a source
+// rank for the pack kernel (NR == 1, src/dst offset per y); the fused
+// reduction runs with gridDim.y == 1.
+template <int NR>
+__global__ void __launch_bounds__(kThreads, 3)
+k_reduce_units(const uint16_t* __restrict__ grads, int64_t stride, int N,
+               float* __restrict__ out, int64_t y_src_step, int64_t y_dst_step,
+               const Unit* __restrict__ units, int64_t n_units, int op_avg) {
+    const uint16_t* gsrc = grads + (int64_t)blockIdx.y * y_src_step;
+    float* gdst = out + (int64_t)blockIdx.y * y_dst_step;
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        float* dst_run = gdst + u.shard_pos;
+        if (u.is_pad) {
+            zero_f32_run(dst_run, len);
+            continue;
+        }
+        const uint16_t* src_run = gsrc + u.arena_pos;
+        const int head = (int)head_to_16B(dst_run, len);
+        if ((int)threadIdx.x < head)
+            dst_run[threadIdx.x] =
+                finish(fold_scalar<NR>(src_run + threadIdx.x, stride, N), avg, fN);
+        const int nvec = (len - head) >> 3;
+        // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0),
+        // so one phase D holds for all N source streams
+        const int D = bf16_phase(src_run + head);
+        const uint16_t* src_al = src_run + head - D;
+        float* dst = dst_run + head;
+        if (D == 0) reduce_body_dispatch<NR, false>(src_al, stride, N, dst, nvec, 0, avg, fN);
+        else reduce_body_dispatch<NR, true>(src_al, stride, N, dst, nvec, D, avg, fN);
+        const int done = head + 8 * nvec;
+        if ((int)threadIdx.x < len - done)
+            dst_run[done + threadIdx.x] =
+                finish(fold_scalar<NR>(src_run + done + threadIdx.x, stride, N), avg, fN);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// staged reduce-scatter: reduce the materialised packed buffer
+// red[k] = fold_r packed[r*NS + k]; then an optional separate division pass.
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kThreads)
+k_reduce_packed_v4(const float* __restrict__ packed, int64_t NS, int N,
+                   float* __restrict__ red, int64_t n4, int op_avg) {
+    const float fN = (float)N;
+    for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < n4;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        float4 acc = __ldcs(reinterpret_cast<const float4*>(packed) + q);
+        for (int r = 1; r < N; ++r) {
+            float4 x = __ldcs(reinterpret_cast<const float4*>(packed + (int64_t)r * NS) + q);
+            acc.x = __fadd_rn(acc.x, x.x);
+            acc.y = __fadd_rn(acc.y, x.y);
+            acc.z = __fadd_rn(acc.z, x.z);
+            acc.w = __fadd_rn(acc.w, x.w);
+        }
+        if (op_avg) {
+            acc.x = __fdiv_rn(acc.x, fN);
+            acc.y = __fdiv_rn(acc.y, fN);
+            acc.z = __fdiv_rn(acc.z, fN);
+            acc.w = __fdiv_rn(acc.w, fN);
+        }
+        __stcs(reinterpret_cast<float4*>(red) + q, acc);
+    }
+}
+
+// Scalar form for the elements not covered by 16-byte vectors (all of them
+// when NS is not a multiple of 4, since rank streams are then misaligned).
+__global__ void __launch_bounds__(kThreads)
+k_reduce_packed_scalar(const float* __restrict__ packed, int64_t NS, int N,
+                       float* __restrict__ red, int64_t begin, int op_avg) {
+    const float fN = (float)N;
+    for (int64_t k = begin + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < NS;
+         k += (int64_t)gridDim.x * blockDim.x) {
+        float acc = packed[k];
+        for (int r = 1; r < N; ++r) acc = __fadd_rn(acc, packed[(int64_t)r * NS + k]);
+        red[k] = op_avg ? __fdiv_rn(acc, fN) : acc;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_div_inplace(float* __restrict__ red, int64_t count, float fN) {
+    for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < count;
+         k += (int64_t)gridDim.x * blockDim.x)
+        red[k] = __fdiv_rn(red[k], fN);
+}
+
+// ---------------------------------------------------------------------------
+// gradient accumulation without sync, in reduce_dtype fp32
+//   first: acc[k] = fp32(g[k]);  later: acc[k] = acc[k] + fp32(g[k])
+// over the flat per-rank arenas [N][P_arena] (a multiple of 8 elements).
+// ---------------------------------------------------------------------------
+
+constexpr int kAccV = 2;  // 8-element vectors per thread per chunk
+constexpr int64_t kAccChunk8 = (int64_t)kThreads * kAccV;
+
+__global__ void __launch_bounds__(kThreads, 3)
+k_accumulate(const uint16_t* __restrict__ g, float* __restrict__ acc, int64_t n8, int first) {
+    const uint4* g8 = reinterpret_cast<const uint4*>(g);
+    float4* a4 = reinterpret_cast<float4*>(acc);
+    const int64_t n_chunks = (n8 + kAccChunk8 - 1) / kAccChunk8;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        const int64_t q0 = c * kAccChunk8 + threadIdx.x;
+        uint4 w[kAccV];
+        float4 A[kAccV][2];
+#pragma unroll
+        for (int k = 0; k < kAccV; ++k) {
+            const int64_t q = q0 + k * kThreads;
+            if (q < n8) {
+                w[k] = __ldcs(g8 + q);
+                if (!first) {
+                    A[k][0] = __ldcs(a4 + 2 * q);
+                    A[k][1] = __ldcs(a4 + 2 * q + 1);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kAccV; ++k) {
+            const int64_t q = q0 + k * kThreads;
+            if (q < n8) {
+                float x[8];
+                unpack8(w[k], x);
+                if (!first) {
+                    const float a[8] = {A[k][0].x, A[k][0].y, A[k][0].z, A[k][0].w,
+                                        A[k][1].x, A[k][1].y, A[k][1].z, A[k][1].w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = __fadd_rn(a[e], x[e]);
+                }
+                __stcs(a4 + 2 * q, make_float4(x[0], x[1], x[2], x[3]));
+                __stcs(a4 + 2 * q + 1, make_float4(x[4], x[5], x[6], x[7]));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// reduce-scatter of the accumulated gradients (the last microbatch)
+//   red[shard_pos + e] = fold over r of x_r, x_r = acc_r[k] (+ fp32(g_r[k]))
+// with k = arena_pos + e, the same rank-ordered fold and division as
+// k_reduce_units.  A run whose source and destination are congruent mod 8
+// moves 16-byte vectors; any other run goes element by element.
+// ---------------------------------------------------------------------------
+
+template <bool WITH_G>
+__device__ __forceinline__ float acc_src1(const float* __restrict__ acc,
+                                          const uint16_t* __restrict__ g, int64_t k) {
+    float x = acc[k];
+    if constexpr (WITH_G) x = __fadd_rn(x, bf16_bits_to_f32(g[k]));
+    return x;
+}
+
+template <bool WITH_G>
+__global__ void __launch_bounds__(kThreads, 2)
+k_reduce_acc(const float* __restrict__ acc, const uint16_t* __restrict__ g, int64_t stride, int N,
+             float* __restrict__ out, const Unit* __restrict__ units, int64_t n_units,
+             int op_avg) {
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        float* dst = out + u.shard_pos;
+        if (u.is_pad) {
+            zero_f32_run(dst, len);
+            continue;
+        }
+        const int64_t s0 = u.arena_pos;
+        const bool vec = ((s0 - u.shard_pos) & 7) == 0;
+        int head = vec ? (int)((8 - (s0 & 7)) & 7) : len;
+        if (head > len) head = len;
+        for (int e = threadIdx.x; e < head; e += blockDim.x) {
+            float a = acc_src1<WITH_G>(acc, g, s0 + e);
+            for (int r = 1; r < N; ++r)
+                a = __fadd_rn(a, acc_src1<WITH_G>(acc, g, (int64_t)r * stride + s0 + e));
+            dst[e] = finish(a, avg, fN);
+        }
+        const int nvec = (len - head) >> 3;
+#pragma unroll 1
+        for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+            const int64_t k = s0 + head + 8 * (int64_t)q;
+            float accv[8];
+#pragma unroll 1
+            for (int r0 = 0; r0 < N; r0 += 4) {
+                float4 A[4][2];
+                uint4 w[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r0 + r < N) {
+                        const int64_t kr = (int64_t)(r0 + r) * stride + k;
+                        A[r][0] = __ldcs(reinterpret_cast<const float4*>(acc + kr));
+                        A[r][1] = __ldcs(reinterpret_cast<const float4*>(acc + kr) + 1);
+                        if constexpr (WITH_G) w[r] = __ldcs(reinterpret_cast<const uint4*>(g + kr));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r0 + r < N) {
+                        float x[8] = {A[r][0].x, A[r][0].y, A[r][0].z, A[r][0].w,
+                                      A[r][1].x, A[r][1].y, A[r][1].z, A[r][1].w};
+                        if constexpr (WITH_G) {
+                            float y[8];
+                            unpack8(w[r], y);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = __fadd_rn(x[e], y[e]);
+                        }
+                        if (r0 + r == 0) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) accv[e] = x[e];
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) accv[e] = __fadd_rn(accv[e], x[e]);
+                        }
+                    }
+                }
+            }
+            if (avg) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) accv[e] = __fdiv_rn(accv[e], fN);
+            }
+            store8(dst + head + 8 * q, accv);
+        }
+        const int done = head + 8 * nvec;
+        for (int e = done + threadIdx.x; e < len; e += blockDim.x) {
+            float a = acc_src1<WITH_G>(acc, g, s0 + e);
+            for (int r = 1; r < N; ++r)
+                a = __fadd_rn(a, acc_src1<WITH_G>(acc, g, (int64_t)r * stride + s0 + e));
+            dst[e] = finish(a, avg, fN);
+        }
+    }
+}
+
+template <int NR>
+cudaError_t launch_reduce_nr(const fsdp_group& g, const uint16_t* grads, int64_t stride, int N,
+                             float* out, int64_t y_src_step, int64_t y_dst_step,
+                             unsigned ydim, const Unit* units, int64_t n_units, int avg,
+                             cudaStream_t st) {
+    const void* kfn = (const void*)k_reduce_units<NR>;
+    dim3 grid(grid_for(g, kfn, n_units), ydim);
+    k_reduce_units<NR><<<grid, kThreads, 0, st>>>(grads, stride, N, out, y_src_step,
+                                                  y_dst_step, units, n_units, avg);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_rs_fused(const fsdp_group& g, const uint16_t* grads, int op, float* reduced,
+                            cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu == 0) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    const int64_t stride = g.P_arena;
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_reduce_nr<K>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_reduce_nr<0>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg,
+                                       st);
+    }
+}
+
+cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Unit* units,
+                                  int64_t n_units, const uint16_t* grads, int op, float* reduced,
+                                  cudaStream_t st) {
+    if (n_units == 0) return cudaSuccess;
+    fsdp_group g;  // only the SM count is read when sizing the grid
+    g.sm_count = sm_count;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    switch (N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_reduce_nr<K>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_reduce_nr<0>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg,
+                                       st);
+    }
+}
+
+cudaError_t launch_rs_pack(const fsdp_group& g, const uint16_t* grads, float* packed,
+                           cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu == 0) return cudaSuccess;
+    // blockIdx.y = source rank r: reads rank r's arena, writes packed[r]
+    return launch_reduce_nr<1>(g, grads, 0, 1, packed, g.P_arena, (int64_t)g.N * g.S,
+                               (unsigned)g.N, g.d_units, nu, 0, st);
+}
+
+cudaError_t launch_rs_reduce_packed(const fsdp_group& g, const float* packed, int op,
+                                    float* reduced, cudaStream_t st) {
+    const int64_t NS = (int64_t)g.N * g.S;
+    if (NS == 0) return cudaSuccess;
+    const int avg = (op == FSDP_AVG) ? 1 : 0;
+    int64_t begin = 0;
+    if (NS % 4 == 0) {
+        const int64_t n4 = NS / 4;
+        k_reduce_packed_v4<<<grid_for(g, (const void*)k_reduce_packed_v4, (n4 + kThreads - 1) / kThreads),
+                             kThreads, 0, st>>>(packed, NS, g.N, reduced, n4, avg);
+        begin = NS;
+    }
+    if (begin < NS) {
+        k_reduce_packed_scalar<<<grid_for(g, (const void*)k_reduce_packed_scalar,
+                                          (NS - begin + kThreads - 1) / kThreads),
+                                 kThreads, 0, st>>>(packed, NS, g.N, reduced, begin, avg);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_div_inplace(const fsdp_group& g, float* reduced, cudaStream_t st) {
+    const int64_t NS = (int64_t)g.N * g.S;
+    if (NS == 0) return cudaSuccess;
+    k_div_inplace<<<grid_for(g, (const void*)k_div_inplace, (NS + kThreads - 1) / kThreads),
+                    kThreads, 0, st>>>(reduced, NS, (float)g.N);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_accumulate(const fsdp_group& g, const uint16_t* grads, float* acc, int first,
+                              cudaStream_t st) {
+    const int64_t n8 = (int64_t)g.N * g.P_arena / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int64_t chunks = (n8 + kAccChunk8 - 1) / kAccChunk8;
+    k_accumulate<<<grid_for(g, (const void*)k_accumulate, chunks), kThreads, 0, st>>>(grads, acc,
+                                                                                     n8, first);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rs_reduce_acc(const fsdp_group& g, const uint16_t* grads, const float* acc,
+                                 int op, float* reduced, cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu == 0) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    if (grads != nullptr)
+        k_reduce_acc<true><<<grid_for(g, (const void*)k_reduce_acc<true>, nu), kThreads, 0, st>>>(
+            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+    else
+        k_reduce_acc<false><<<grid_for(g, (const void*)k_reduce_acc<false>, nu), kThreads, 0, st>>>(
+            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+    return cudaGetLastError();
+}
+
+}  // namespace fsdpk

@@ -1,0 +1,340 @@
+// fsdpk_update.cu -- the sharded AdamW update, the fused reduce-scatter +
+// AdamW + next-step copy-in, and the device-side step scalars for CUDA-graph
+// replay.
+//   "Sharded Training: FSDP2, DTensor, Tensor and Pipeline Parallelism",
+//   Fence 4 (the optimizer steps the sharded fp32 parameters, its state
+//   sharded the same way) and the opening paragraph (12 bytes of fp32 state);
+//   "Introduction to PyTorch FSDP2 Backend Features", Working Principle
+//   (reduce-scatter, then the sharded update, then the next all-gather).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "fsdpk_device.cuh"
+
+namespace fsdpk {
+namespace {
+
+// ---------------------------------------------------------------------------
+// AdamW over the flat [N][S] buffers (pads are zero and stay zero)
+// ---------------------------------------------------------------------------
+
+constexpr int kAdamV = 2;  // float4 per array per thread
+constexpr int64_t kAdamChunk4 = (int64_t)kThreads * kAdamV;  // float4 per CTA chunk
+
+__global__ void __launch_bounds__(kThreads, 3)
+k_adamw(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v,
+        const float* __restrict__ g, int64_t count, AdamScalars sc,
+        const AdamScalars* __restrict__ sc_dev) {
+    if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
+    const int64_t n4 = count >> 2;
+    float4* p4 = reinterpret_cast<float4*>(p);
+    float4* m4 = reinterpret_cast<float4*>(m);
+    float4* v4 = reinterpret_cast<float4*>(v);
+    const float4* g4 = reinterpret_cast<const float4*>(g);
+    const int64_t n_chunks = (n4 + kAdamChunk4 - 1) / kAdamChunk4;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        const int64_t q0 = c * kAdamChunk4 + threadIdx.x;
+        float4 P[kAdamV], M[kAdamV], Vv[kAdamV], G[kAdamV];
+#pragma unroll
+        for (int k = 0; k < kAdamV; ++k) {
+            const int64_t q = q0 + k * kThreads;
+            if (q < n4) {
+                P[k] = __ldcs(p4 + q);
+                M[k] = __ldcs(m4 + q);
+                Vv[k] = __ldcs(v4 + q);
+                G[k] = __ldcs(g4 + q);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kAdamV; ++k) {
+            const int64_t q = q0 + k * kThreads;
+            if (q < n4) {
+                adamw1(P[k].x, M[k].x, Vv[k].x, G[k].x, sc);
+                adamw1(P[k].y, M[k].y, Vv[k].y, G[k].y, sc);
+                adamw1(P[k].z, M[k].z, Vv[k].z, G[k].z, sc);
+                adamw1(P[k].w, M[k].w, Vv[k].w, G[k].w, sc);
+                __stcs(p4 + q, P[k]);
+                __stcs(m4 + q, M[k]);
+                __stcs(v4 + q, Vv[k]);
+            }
+        }
+    }
+    // ragged tail (count % 4 elements)
+    if (blockIdx.x == 0 && threadIdx.x < (count & 3)) {
+        const int64_t k = 4 * n4 + threadIdx.x;
+        float pp = p[k], mm = m[k], vv = v[k];
+        adamw1(pp, mm, vv, g[k], sc);
+        p[k] = pp;
+        m[k] = mm;
+        v[k] = vv;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// fused reduce-scatter + AdamW + next-step copy-in
+// For each element k of [N][S]:  g = rank-ordered fold of the N ranks'
+// gradients (then / N for AVG and SUM_THEN_DIV; +0 in pad rows), AdamW on
+// master/m/v[k] with g, then ag[k] = bf16_rn(master[k]) (+0 in pad rows) and
+// optionally reduced[k] = g.  The fold, the division and the AdamW arithmetic
+// are the ones of k_reduce_units and k_adamw, so the results are the same bits
+// as the three separate stages.  The reduced gradient never goes to HBM.
+// ---------------------------------------------------------------------------
+
+struct FusedOut {
+    float* p;
+    float* m;
+    float* v;
+    float* red;    // may be null
+    uint16_t* ag;  // may be null
+};
+
+// One element: adamw with g, then the optional outputs.
+__device__ __forceinline__ void fused1(const FusedOut& o, int64_t k, float g, bool pad,
+                                       const AdamScalars& sc) {
+    float pp = o.p[k], mm = o.m[k], vv = o.v[k];
+    adamw1(pp, mm, vv, g, sc);
+    o.p[k] = pp;
+    o.m[k] = mm;
+    o.v[k] = vv;
+    if (o.red) o.red[k] = g;
+    if (o.ag) {
+        __nv_bfloat16 h = __float2bfloat16_rn(pad ? 0.0f : pp);
+        o.ag[k] = *reinterpret_cast<uint16_t*>(&h);
+    }
+}
+
+// Eight elements starting at an index that is a multiple of 8 (every fp32
+// pointer 32-byte aligned, the bf16 pointer 16-byte aligned).
+__device__ __forceinline__ void fused8(const FusedOut& o, int64_t k, const float (&g)[8],
+                                       const float4 (&P)[2], const float4 (&M)[2],
+                                       const float4 (&V)[2], bool pad, const AdamScalars& sc) {
+    float pp[8] = {P[0].x, P[0].y, P[0].z, P[0].w, P[1].x, P[1].y, P[1].z, P[1].w};
+    float mm[8] = {M[0].x, M[0].y, M[0].z, M[0].w, M[1].x, M[1].y, M[1].z, M[1].w};
+    float vv[8] = {V[0].x, V[0].y, V[0].z, V[0].w, V[1].x, V[1].y, V[1].z, V[1].w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) adamw1(pp[e], mm[e], vv[e], g[e], sc);
+    float4* p4 = reinterpret_cast<float4*>(o.p + k);
+    float4* m4 = reinterpret_cast<float4*>(o.m + k);
+    float4* v4 = reinterpret_cast<float4*>(o.v + k);
+    __stcs(p4, make_float4(pp[0], pp[1], pp[2], pp[3]));
+    __stcs(p4 + 1, make_float4(pp[4], pp[5], pp[6], pp[7]));
+    __stcs(m4, make_float4(mm[0], mm[1], mm[2], mm[3]));
+    __stcs(m4 + 1, make_float4(mm[4], mm[5], mm[6], mm[7]));
+    __stcs(v4, make_float4(vv[0], vv[1], vv[2], vv[3]));
+    __stcs(v4 + 1, make_float4(vv[4], vv[5], vv[6], vv[7]));
+    if (o.red) store8(o.red + k, g);
+    if (o.ag) {
+        uint4 w = pad ? make_uint4(0u, 0u, 0u, 0u)
+                      : make_uint4(pack_bf16x2(pp[0], pp[1]), pack_bf16x2(pp[2], pp[3]),
+                                   pack_bf16x2(pp[4], pp[5]), pack_bf16x2(pp[6], pp[7]));
+        __stcs(reinterpret_cast<uint4*>(o.ag + k), w);
+    }
+}
+
+__device__ __forceinline__ void load_pmv8(const FusedOut& o, int64_t k, float4 (&P)[2],
+                                          float4 (&M)[2], float4 (&V)[2]) {
+    const float4* p4 = reinterpret_cast<const float4*>(o.p + k);
+    const float4* m4 = reinterpret_cast<const float4*>(o.m + k);
+    const float4* v4 = reinterpret_cast<const float4*>(o.v + k);
+    P[0] = __ldcs(p4);
+    P[1] = __ldcs(p4 + 1);
+    M[0] = __ldcs(m4);
+    M[1] = __ldcs(m4 + 1);
+    V[0] = __ldcs(v4);
+    V[1] = __ldcs(v4 + 1);
+}
+
+// Rank-ordered fold of 8 elements; NR = N at compile time (1..8): all NR
+// ranks' loads (two 16-byte vectors per rank on a misaligned run) are issued
+// before the fold.  NR = 0 (any N): ranks in batches of 4.
+template <int NR, bool SHIFTED>
+__device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64_t stride, int N,
+                                      int q, int D, float (&acc)[8]) {
+    if constexpr (NR != 0) {
+        uint4 a[NR], b[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            const uint4* s = reinterpret_cast<const uint4*>(src_al + r * stride) + q;
+            a[r] = ld_src<SHIFTED>(s);
+            if constexpr (SHIFTED) b[r] = ld_src<SHIFTED>(s + 1);
+        }
+        unpack8(SHIFTED ? shift_bf16x8(a[0], b[0], D) : a[0], acc);
+#pragma unroll
+        for (int r = 1; r < NR; ++r) {
+            float x[8];
+            unpack8(SHIFTED ? shift_bf16x8(a[r], b[r], D) : a[r], x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], x[e]);
+        }
+    } else {
+#pragma unroll 1
+        for (int r0 = 0; r0 < N; r0 += 4) {
+            uint4 a[4], b[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r0 + r < N) {
+                    const uint4* s =
+                        reinterpret_cast<const uint4*>(src_al + (int64_t)(r0 + r) * stride) + q;
+                    a[r] = ld_src<SHIFTED>(s);
+                    if constexpr (SHIFTED) b[r] = ld_src<SHIFTED>(s + 1);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r0 + r < N) {
+                    float x[8];
+                    unpack8(SHIFTED ? shift_bf16x8(a[r], b[r], D) : a[r], x);
+                    if (r0 + r == 0) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] = x[e];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], x[e]);
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int NR, bool SHIFTED>
+__device__ __forceinline__ void fused_body(const uint16_t* __restrict__ src_al, int64_t stride,
+                                           int N, int D, const FusedOut& o, int64_t k0, int nvec,
+                                           bool avg, float fN, const AdamScalars& sc) {
+#pragma unroll 1
+    for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+        const int64_t k = k0 + 8 * (int64_t)q;
+        float4 P[2], M[2], V[2];
+        load_pmv8(o, k, P, M, V);
+        float g[8];
+        fold8<NR, SHIFTED>(src_al, stride, N, q, D, g);
+        if (avg) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = __fdiv_rn(g[e], fN);
+        }
+        fused8(o, k, g, P, M, V, false, sc);
+    }
+}
+
+template <int NR>
+__global__ void __launch_bounds__(kThreads, 2)
+k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o,
+           const Unit* __restrict__ units, int64_t n_units, int op_avg, AdamScalars sc,
+           const AdamScalars* __restrict__ sc_dev) {
+    if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        const int len = u.len;
+        const int64_t k0 = u.shard_pos;
+        // peel to an index that is a multiple of 8 (bf16 16-byte vectors)
+        int head = (int)((8 - (k0 & 7)) & 7);
+        if (head > len) head = len;
+        const int nvec = (len - head) >> 3;
+        const int done = head + 8 * nvec;
+        if (u.is_pad) {
+            const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if ((int)threadIdx.x < head) fused1(o, k0 + threadIdx.x, 0.0f, true, sc);
+#pragma unroll 1
+            for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+                const int64_t k = k0 + head + 8 * (int64_t)q;
+                float4 P[2], M[2], V[2];
+                load_pmv8(o, k, P, M, V);
+                fused8(o, k, zero8, P, M, V, true, sc);
+            }
+            if ((int)threadIdx.x < len - done) fused1(o, k0 + done + threadIdx.x, 0.0f, true, sc);
+            continue;
+        }
+        const uint16_t* src_run = grads + u.arena_pos;
+        if ((int)threadIdx.x < head)
+            fused1(o, k0 + threadIdx.x,
+                   finish(fold_scalar<NR>(src_run + threadIdx.x, stride, N), avg, fN), false, sc);
+        // every rank's arena starts on a 16-byte boundary, so one phase D
+        // holds for all N source streams
+        const int D = bf16_phase(src_run + head);
+        const uint16_t* src_al = src_run + head - D;
+        if (D == 0) fused_body<NR, false>(src_al, stride, N, 0, o, k0 + head, nvec, avg, fN, sc);
+        else fused_body<NR, true>(src_al, stride, N, D, o, k0 + head, nvec, avg, fN, sc);
+        if ((int)threadIdx.x < len - done)
+            fused1(o, k0 + done + threadIdx.x,
+                   finish(fold_scalar<NR>(src_run + done + threadIdx.x, stride, N), avg, fN),
+                   false, sc);
+    }
+}
+
+template <int NR>
+cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const FusedOut& o,
+                               int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
+                               cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    k_rs_adamw<NR><<<grid_for(g, (const void*)k_rs_adamw<NR>, nu), kThreads, 0, st>>>(
+        grads, g.P_arena, g.N, o, g.d_units, nu, avg, sc, sc_dev);
+    return cudaGetLastError();
+}
+
+// One thread: advance the device step counter and compute that step's AdamW
+// scalars in binary64, in the same operation order as the host path.
+__global__ void k_adamw_prepare(double lr, double beta1, double beta2, double eps, double wd,
+                                int64_t* __restrict__ step, AdamScalars* __restrict__ out) {
+    if (blockIdx.x != 0 || threadIdx.x != 0) return;
+    const int64_t t = *step + 1;
+    *step = t;
+    const double bc1 = 1.0 - pow(beta1, (double)t);
+    const double bc2 = 1.0 - pow(beta2, (double)t);
+    AdamScalars sc;
+    sc.decay = (float)(1.0 - lr * wd);
+    sc.beta1 = (float)beta1;
+    sc.omb1 = (float)(1.0 - beta1);
+    sc.beta2 = (float)beta2;
+    sc.omb2 = (float)(1.0 - beta2);
+    sc.step_size = (float)(lr / bc1);
+    sc.inv_bc2_sqrt = (float)(1.0 / sqrt(bc2));
+    sc.eps = (float)eps;
+    *out = sc;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_adamw(const fsdp_group& g, float* master, float* m, float* v,
+                         const float* grad, const AdamScalars& sc, cudaStream_t st,
+                         const AdamScalars* sc_dev) {
+    const int64_t count = (int64_t)g.N * g.S;
+    if (count == 0) return cudaSuccess;
+    const int64_t items = ((count >> 2) + kAdamChunk4 - 1) / kAdamChunk4;
+    k_adamw<<<grid_for(g, (const void*)k_adamw, items), kThreads, 0, st>>>(master, m, v, grad,
+                                                                            count, sc, sc_dev);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_adamw_prepare(double lr, double beta1, double beta2, double eps, double wd,
+                                 int64_t* step, AdamScalars* out, cudaStream_t st) {
+    k_adamw_prepare<<<1, 32, 0, st>>>(lr, beta1, beta2, eps, wd, step, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, float* master,
+                            float* m, float* v, const AdamScalars& sc, uint16_t* ag_next,
+                            float* reduced, cudaStream_t st, const AdamScalars* sc_dev) {
+    if (g.units.empty()) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    const FusedOut o{master, m, v, reduced, ag_next};
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_rs_adamw_nr<K>(g, grads, o, avg, sc, sc_dev, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_rs_adamw_nr<0>(g, grads, o, avg, sc, sc_dev, st);
+    }
+}
+
+}  // namespace fsdpk
