@@ -305,3 +305,57 @@ def test_random_groups_brute_force(H, wl):
     H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
     H.run_group_fused(wl, grp, steps=1)
     H.run_group_fp8(wl, grp)
+
+
+GRID = [_wl(f"grid_n{N}", [((d0, c) if c > 1 else (d0,)) for d0 in range(21) for c in (1, 3, 8)], N,
+            op=[W.SUM, W.AVG, W.SUM_THEN_DIV][N % 3]) for N in range(1, 10)]
+
+
+@pytest.mark.parametrize("wl", GRID, ids=[w.name for w in GRID])
+def test_brute_force_grid_d0_cols_world(H, wl):
+    """Every d0 in [0, 20] x cols in {1, 3, 8} as one 63-parameter group, for
+    every N in [1, 9]: all stages, all ops, the fused and FP8 paths."""
+    grp = wl.groups[0]
+    H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
+    H.run_group_fused(wl, grp, steps=1)
+    H.run_group_fp8(wl, grp)
+
+
+def test_checkpoint_resume_is_bit_exact(H, tmp_path):
+    """Two steps, save, restore into fresh buffers, one more step: the same
+    bits as three uninterrupted steps."""
+    from fully_sharded_shard_b200 import abi, checkpoint as C
+    wl = W.uneven(16)
+    grp = wl.groups[0]
+    g = abi.fsdp_plan_group(grp.shapes, wl.N)
+    NS = wl.N * g.S
+    full = torch.empty(g.P_arena, device="cuda")
+    W.fill_master(full, wl, grp.name)
+    hp = dict(W.ADAMW_DEFAULTS)
+    grads = [H.make_grads(g, wl, grp, s) for s in (1, 2, 3)]
+    red = torch.empty(NS, device="cuda")
+
+    def fresh():
+        p = torch.empty(NS, device="cuda")
+        abi.fsdp_shard_params(g, full, p)
+        return p, torch.zeros(NS, device="cuda"), torch.zeros(NS, device="cuda")
+
+    def step(state, t):
+        abi.fsdp_rs_reduce(g, grads[t - 1], wl.op, red)
+        abi.fsdp_adamw_step(g, *state, red, step=t, **hp)
+
+    a = fresh()
+    for t in (1, 2, 3):
+        step(a, t)
+    b = fresh()
+    for t in (1, 2):
+        step(b, t)
+    torch.cuda.synchronize()
+    C.save_group_state(str(tmp_path), grp.shapes, wl.N, g.S, 2, *b)
+    c = (torch.empty(NS, device="cuda"), torch.empty(NS, device="cuda"), torch.empty(NS, device="cuda"))
+    t0 = C.load_group_state(str(tmp_path), grp.shapes, wl.N, g.S, *c)
+    step(c, t0 + 1)
+    torch.cuda.synchronize()
+    for x, y in zip(a, c):
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+    g.destroy()
