@@ -72,6 +72,19 @@ def fused_stage_bytes(N: int, S: int, P: int) -> dict:
     }
 
 
+def fused_fp8_stage_bytes(N: int, S: int, P: int, n: int) -> dict:
+    """The fused step with an FP8 all-gather (delayed scaling): the byte
+    copy-out, then one kernel that reads the N ranks' gradients and
+    master/m/v and writes master/m/v and the E4M3 all-gather input of the next
+    step; the per-parameter scales (n of them, read and written) are
+    negligible but counted."""
+    Pp = N * S
+    return {
+        "copy_out": Pp + P,
+        "rs_adamw_copy_in_fp8": 2 * N * P + 24 * Pp + Pp + 12 * n,
+    }
+
+
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
@@ -484,6 +497,11 @@ def run_ours(args, wl, device, rank, ws):
     if not args.no_fused:
         fused = run_fused(args, model, device, stream, ws, ms_step, peak)
 
+    fused8 = None
+    if not args.no_fused and not args.no_fp8:
+        fused8 = run_fused_fp8(args, model, device, stream, ws,
+                               fused["ms_per_step"] if fused else None, peak)
+
     accum = None
     if not args.no_accumulate:
         accum = run_accumulate(args, model, device, stream)
@@ -532,6 +550,7 @@ def run_ours(args, wl, device, rank, ws):
         "clocks": clocks,
         "e2e": e2e,
         "fused_step": fused,
+        "fused_step_fp8_all_gather": fused8,
         "grad_accumulation": accum,
         "fp8_all_gather": fp8,
         "tiny_latency": latency,
@@ -585,6 +604,108 @@ def run_fused(args, model, device, stream, ws, ms_unfused, peak):
                        "GBps": round(model.fused_bytes[k] / (stage_ms[k] * 1e-3) / 1e9, 1)}
                    for k in stage_ms},
         "launches_per_step": 2 * len(model.instances),
+    }
+
+
+def run_fused_fp8(args, model, device, stream, ws, ms_fused, peak):
+    """Time the fused step with an FP8 all-gather (per-group byte copy-out,
+    then reduce-scatter + AdamW + E4M3 next copy-in with the previous step's
+    scales + next scales) on the same state, under its own byte model.  Each
+    group's FP8 all-gather input lives in the first half of its bf16 buffer;
+    each group keeps two scale buffers that swap every step."""
+    import torch
+    from fully_sharded_shard_b200 import abi
+    from fully_sharded_shard_b200 import workloads as W
+    if not hasattr(model, "ag_groups"):
+        model.enable_fused()
+    N = model.wl.N
+    ag8s, scales = [], []
+    for idx, (gi, master, m, v, pj) in enumerate(model.instances):
+        g = model.plans[gi]
+        ag8 = model.ag_groups[idx].view(torch.uint8)[:max(N * g.S, 1)]
+        sc = [torch.empty(max(g.n, 1), dtype=torch.float32, device=device) for _ in range(2)]
+        abi.fsdp_copy_in_fp8(g, master, ag8, sc[0])
+        ag8s.append(ag8)
+        scales.append(sc)
+    arena8 = [model.arena.view(torch.uint8), torch.empty_like(model.arena).view(torch.uint8)]
+    s_update = torch.cuda.Stream(device)
+    hp = dict(W.ADAMW_DEFAULTS)
+    state = {"t": 0}
+
+    def one(events=None):
+        state["t"] += 1
+        model.step_count += 1
+        t = state["t"]
+        for idx, (gi, master, m, v, pj) in enumerate(model.instances):
+            g = model.plans[gi]
+            prev, nxt = scales[idx][(t - 1) % 2], scales[idx][t % 2]
+            if events is not None or args.one_stream:
+                calls = (("copy_out", lambda: abi.fsdp_copy_out_fp8(g, ag8s[idx], arena8[0], stream)),
+                         ("rs_adamw_copy_in_fp8", lambda: abi.fsdp_rs_adamw_step_fp8(
+                             g, model.grads[gi][pj], model.wl.op, master, m, v,
+                             step=model.step_count, scales_prev=prev, ag8_next=ag8s[idx],
+                             scales_next=nxt, stream=stream, **hp)))
+                for name, fn in calls:
+                    if events is None:
+                        fn()
+                        continue
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                    events[name].append((e0, e1))
+                continue
+            abi.fsdp_copy_out_fp8(g, ag8s[idx], arena8[idx % 2], stream)
+            read = torch.cuda.Event()
+            read.record(stream)
+            s_update.wait_event(read)
+            abi.fsdp_rs_adamw_step_fp8(g, model.grads[gi][pj], model.wl.op, master, m, v,
+                                       step=model.step_count, scales_prev=prev,
+                                       ag8_next=ag8s[idx], scales_next=nxt, stream=s_update,
+                                       **hp)
+        if events is None and not args.one_stream:
+            done = torch.cuda.Event()
+            done.record(s_update)
+            stream.wait_event(done)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
+    events = {k: [] for k in ("copy_out", "rs_adamw_copy_in_fp8")}
+    one(events)
+    torch.cuda.synchronize(device)
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in events.items()}
+    sb = {k: 0 for k in stage_ms}
+    for i in model.instances:
+        g = model.plans[i[0]]
+        for k, b in fused_fp8_stage_bytes(N, g.S, g.P, g.n).items():
+            sb[k] += b
+    total = sum(sb.values())
+    del arena8
+    return {
+        "ms_per_step": round(ms, 3),
+        "bytes_per_step": total,
+        "bytes_per_param": round(total / model.P_total, 3),
+        "value": round(ws * total / (ms * 1e-3) / 1e9, 1),
+        "unit": "GB/s (own byte model)",
+        "frac_of_measured_peak": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+        "params_per_s": round(ws * model.P_total / (ms * 1e-3), 1),
+        "speedup_vs_bf16_fused_step": round(ms_fused / ms, 3) if ms_fused else None,
+        "stages": {k: {"ms_per_step": round(stage_ms[k], 3),
+                       "GBps": round(sb[k] / (stage_ms[k] * 1e-3) / 1e9, 1)}
+                   for k in stage_ms},
+        "launches_per_step": 3 * len(model.instances),
     }
 
 

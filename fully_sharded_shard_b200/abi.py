@@ -82,6 +82,11 @@ def _load() -> ctypes.CDLL:
     L.fsdp_rs_reduce_accumulated.restype = ctypes.c_int
     L.fsdp_copy_in_fp8.argtypes = [vp, vp, vp, vp, vp]
     L.fsdp_copy_in_fp8.restype = ctypes.c_int
+    L.fsdp_copy_in_fp8_scaled.argtypes = [vp, vp, vp, vp, vp]
+    L.fsdp_copy_in_fp8_scaled.restype = ctypes.c_int
+    L.fsdp_rs_adamw_step_fp8.argtypes = [vp, vp, i32, vp, vp, vp, ctypes.POINTER(AdamWHparams),
+                                         vp, vp, vp, vp, vp]
+    L.fsdp_rs_adamw_step_fp8.restype = ctypes.c_int
     L.fsdp_copy_out_fp8.argtypes = [vp, vp, vp, vp]
     L.fsdp_copy_out_fp8.restype = ctypes.c_int
     L.fsdp_adamw_prepare.argtypes = [ctypes.POINTER(AdamWHparams), vp, vp, vp]
@@ -279,6 +284,34 @@ def fsdp_copy_in_fp8(g: Group, master: torch.Tensor, ag8: torch.Tensor, scales: 
                                  _ptr(ag8, _U8, g.N * g.S, "ag8"),
                                  _ptr(scales, _F32, g.n, "scales"), _stream(stream, master)),
            "fsdp_copy_in_fp8")
+
+
+def fsdp_copy_in_fp8_scaled(g: Group, master: torch.Tensor, scales: torch.Tensor,
+                            ag8: torch.Tensor, stream=None):
+    _check(_lib.fsdp_copy_in_fp8_scaled(g.handle, _ptr(master, _F32, g.N * g.S, "master"),
+                                        _ptr(scales, _F32, g.n, "scales"),
+                                        _ptr(ag8, _U8, g.N * g.S, "ag8"),
+                                        _stream(stream, master)), "fsdp_copy_in_fp8_scaled")
+
+
+def fsdp_rs_adamw_step_fp8(g: Group, grads: torch.Tensor, op: int, master: torch.Tensor,
+                           m: torch.Tensor, v: torch.Tensor, *, lr: float, beta1: float,
+                           beta2: float, eps: float, weight_decay: float, step: int,
+                           scales_prev: torch.Tensor, ag8_next: torch.Tensor,
+                           scales_next: torch.Tensor, reduced: Optional[torch.Tensor] = None,
+                           stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = g.N * g.S
+    _check(_lib.fsdp_rs_adamw_step_fp8(g.handle, _ptr(grads, _B16, g.N * g.P_arena, "grads"),
+                                       int(op), _ptr(master, _F32, n, "master"),
+                                       _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                       ctypes.byref(hp),
+                                       _ptr(scales_prev, _F32, g.n, "scales_prev"),
+                                       _ptr(ag8_next, _U8, n, "ag8_next"),
+                                       _ptr(scales_next, _F32, g.n, "scales_next"),
+                                       _ptr(reduced, _F32, n, "reduced"),
+                                       _stream(stream, master)), "fsdp_rs_adamw_step_fp8")
 
 
 def fsdp_copy_out_fp8(g: Group, ag8: torch.Tensor, arena8: torch.Tensor, stream=None):

@@ -431,6 +431,52 @@ int fsdp_copy_in_fp8(fsdp_group_t g, const float* master, uint8_t* ag8, float* s
     return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
 }
 
+int fsdp_copy_in_fp8_scaled(fsdp_group_t g, const float* master, const float* scales,
+                            uint8_t* ag8, fsdp_stream_t stream) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if ((int64_t)g->N * g->S > 0 && (master == nullptr || ag8 == nullptr)) return FSDP_EINVAL;
+    if (g->n > 0 && scales == nullptr) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(ag8) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    cudaError_t e = fsdpk::launch_copy_in_fp8_scaled(*g, master, ag8, scales, (cudaStream_t)stream);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+int fsdp_rs_adamw_step_fp8(fsdp_group_t g, const uint16_t* grads, int32_t op, float* master,
+                           float* m, float* v, const fsdp_adamw_hparams* hp,
+                           const float* scales_prev, uint8_t* ag8_next, float* scales_next,
+                           float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr || hp == nullptr) return FSDP_EINVAL;
+    if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr || ag8_next == nullptr))
+        return FSDP_EINVAL;
+    if (g->P > 0 && grads == nullptr) return FSDP_EINVAL;
+    if (g->n > 0 && (scales_prev == nullptr || scales_next == nullptr)) return FSDP_EINVAL;
+    if (scales_prev != nullptr && scales_prev == scales_next) return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!adam_scalars(hp, &sc)) return FSDP_EINVAL;
+    if (!aligned16(grads) || !aligned16(master) || !aligned16(m) || !aligned16(v) ||
+        !aligned16(ag8_next) || !aligned16(reduced) ||
+        (reinterpret_cast<uintptr_t>(scales_prev) & 3u) ||
+        (reinterpret_cast<uintptr_t>(scales_next) & 3u))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (g->n > 0) e = cudaMemsetAsync(scales_next, 0, sizeof(float) * (size_t)g->n, s);
+    // scales_next holds the amax bits (non-negative floats order as integers)
+    // until the last launch turns them into scales
+    if (e == cudaSuccess)
+        e = fsdpk::launch_rs_adamw_fp8(*g, grads, op, master, m, v, sc, scales_prev, ag8_next,
+                                       reinterpret_cast<unsigned*>(scales_next), reduced, s);
+    if (e == cudaSuccess) e = fsdpk::launch_fp8_scales_from_amax(*g, scales_next, s);
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
 int fsdp_copy_out_fp8(fsdp_group_t g, const uint8_t* ag8, uint8_t* arena8, fsdp_stream_t stream) {
     if (g == nullptr) return FSDP_EINVAL;
     if (g->P > 0 && (ag8 == nullptr || arena8 == nullptr)) return FSDP_EINVAL;

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -123,6 +124,24 @@ __device__ __forceinline__ void adamw1(float& p, float& m, float& v, float g,
     v = fmaf(sc.beta2, v, sc.omb2 * g * g);
     const float denom = fmaf(__fsqrt_rn(v), sc.inv_bc2_sqrt, sc.eps);
     p = fmaf(-sc.step_size, __fdiv_rn(m, denom), p);
+}
+
+// FP8 (E4M3 "fn") helpers
+// x * scale clamped to the finite E4M3 range (NaN passes through).
+__device__ __forceinline__ float fp8_in(float x, float sc) {
+    float y = __fmul_rn(x, sc);
+    if (y > 448.0f) y = 448.0f;
+    if (y < -448.0f) y = -448.0f;
+    return y;
+}
+
+// Two floats -> two E4M3 bytes (lo in bits 0..7), round to nearest even.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ uint8_t e4m3(float x) {
+    return (uint8_t)(e4m3x2(x, 0.0f) & 0xFFu);
 }
 
 // ---------------------------------------------------------------------------

@@ -219,23 +219,6 @@ k_fp8_scales(float* __restrict__ scales, int n) {
     if (i < n) scales[i] = __fdiv_rn(448.0f, fmaxf(scales[i], 1e-12f));
 }
 
-// x * scale clamped to the finite E4M3 range (NaN passes through).
-__device__ __forceinline__ float fp8_in(float x, float sc) {
-    float y = __fmul_rn(x, sc);
-    if (y > 448.0f) y = 448.0f;
-    if (y < -448.0f) y = -448.0f;
-    return y;
-}
-
-// Two floats -> two E4M3 bytes (lo in bits 0..7), round to nearest even.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
-}
-
-__device__ __forceinline__ uint8_t e4m3(float x) {
-    return (uint8_t)(e4m3x2(x, 0.0f) & 0xFFu);
-}
-
 __device__ __forceinline__ void zero_u8_run(uint8_t* __restrict__ dst, int len) {
     const int head = (int)head_to_16B(dst, len);
     if ((int)threadIdx.x < head) dst[threadIdx.x] = 0;
@@ -372,6 +355,21 @@ cudaError_t launch_copy_in_fp8(const fsdp_group& g, const float* master, uint8_t
                 g.n_real_units);
         k_fp8_scales<<<(unsigned)((g.n + kThreads - 1) / kThreads), kThreads, 0, st>>>(scales, g.n);
     }
+    const int64_t nu = (int64_t)g.units.size();
+    if (nu > 0)
+        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(master, ag8, scales,
+                                                                     g.d_units, g.d_unit_param, nu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_scales_from_amax(const fsdp_group& g, float* scales, cudaStream_t st) {
+    if (g.n == 0) return cudaSuccess;
+    k_fp8_scales<<<(unsigned)((g.n + kThreads - 1) / kThreads), kThreads, 0, st>>>(scales, g.n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_in_fp8_scaled(const fsdp_group& g, const float* master, uint8_t* ag8,
+                                      const float* scales, cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
     if (nu > 0)
         k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(master, ag8, scales,

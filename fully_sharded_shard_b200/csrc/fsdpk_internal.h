@@ -135,4 +135,16 @@ cudaError_t launch_copy_in_fp8(const fsdp_group& g, const float* master, uint8_t
 cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t* arena8,
                                 cudaStream_t st);
 
+// FP8 with given scales: scales from amax in place, and the copy-in with
+// scales supplied by the caller (no amax pass).
+cudaError_t launch_fp8_scales_from_amax(const fsdp_group& g, float* scales, cudaStream_t st);
+cudaError_t launch_copy_in_fp8_scaled(const fsdp_group& g, const float* master, uint8_t* ag8,
+                                      const float* scales, cudaStream_t st);
+// The fused update writing the next all-gather input in FP8 with delayed
+// scales and folding max |updated master| per parameter into amax_bits.
+cudaError_t launch_rs_adamw_fp8(const fsdp_group& g, const uint16_t* grads, int op, float* master,
+                                float* m, float* v, const AdamScalars& sc, const float* scales_prev,
+                                uint8_t* ag8_next, unsigned* amax_bits, float* reduced,
+                                cudaStream_t st, const AdamScalars* sc_dev = nullptr);
+
 }  // namespace fsdpk

@@ -81,36 +81,51 @@ k_adamw(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v,
 // optionally reduced[k] = g.  The fold, the division and the AdamW arithmetic
 // are the ones of k_reduce_units and k_adamw, so the results are the same bits
 // as the three separate stages.  The reduced gradient never goes to HBM.
+// FP8 mode (delayed scaling): instead of the bf16 copy, ag8[k] =
+// e4m3_rn(clamp(master[k] * scale_i, -448, 448)) with the scale of the
+// previous step, and max |master| over each parameter (the next scale's amax)
+// folded into amax_bits[i].
 // ---------------------------------------------------------------------------
 
 struct FusedOut {
     float* p;
     float* m;
     float* v;
-    float* red;    // may be null
-    uint16_t* ag;  // may be null
+    float* red;                 // may be null
+    uint16_t* ag;               // bf16 next all-gather input; may be null
+    uint8_t* ag8;               // FP8 mode: next all-gather input
+    const float* scales;        // FP8 mode: per-parameter scale applied to ag8
+    unsigned* amax_bits;        // FP8 mode: per-parameter max |updated master|
+    const int32_t* unit_param;  // FP8 mode: parameter of every unit
 };
 
 // One element: adamw with g, then the optional outputs.
+template <bool FP8>
 __device__ __forceinline__ void fused1(const FusedOut& o, int64_t k, float g, bool pad,
-                                       const AdamScalars& sc) {
+                                       const AdamScalars& sc, float scale, float& mx) {
     float pp = o.p[k], mm = o.m[k], vv = o.v[k];
     adamw1(pp, mm, vv, g, sc);
     o.p[k] = pp;
     o.m[k] = mm;
     o.v[k] = vv;
     if (o.red) o.red[k] = g;
-    if (o.ag) {
+    if constexpr (FP8) {
+        o.ag8[k] = pad ? (uint8_t)0 : e4m3(fp8_in(pp, scale));
+        if (!pad) mx = fmaxf(mx, fabsf(pp));
+    } else if (o.ag) {
         __nv_bfloat16 h = __float2bfloat16_rn(pad ? 0.0f : pp);
         o.ag[k] = *reinterpret_cast<uint16_t*>(&h);
     }
 }
 
 // Eight elements starting at an index that is a multiple of 8 (every fp32
-// pointer 32-byte aligned, the bf16 pointer 16-byte aligned).
+// pointer 32-byte aligned, the bf16 pointer 16-byte and the FP8 pointer
+// 8-byte aligned).
+template <bool FP8>
 __device__ __forceinline__ void fused8(const FusedOut& o, int64_t k, const float (&g)[8],
                                        const float4 (&P)[2], const float4 (&M)[2],
-                                       const float4 (&V)[2], bool pad, const AdamScalars& sc) {
+                                       const float4 (&V)[2], bool pad, const AdamScalars& sc,
+                                       float scale, float& mx) {
     float pp[8] = {P[0].x, P[0].y, P[0].z, P[0].w, P[1].x, P[1].y, P[1].z, P[1].w};
     float mm[8] = {M[0].x, M[0].y, M[0].z, M[0].w, M[1].x, M[1].y, M[1].z, M[1].w};
     float vv[8] = {V[0].x, V[0].y, V[0].z, V[0].w, V[1].x, V[1].y, V[1].z, V[1].w};
@@ -126,7 +141,19 @@ __device__ __forceinline__ void fused8(const FusedOut& o, int64_t k, const float
     __stcs(v4, make_float4(vv[0], vv[1], vv[2], vv[3]));
     __stcs(v4 + 1, make_float4(vv[4], vv[5], vv[6], vv[7]));
     if (o.red) store8(o.red + k, g);
-    if (o.ag) {
+    if constexpr (FP8) {
+        uint2 w = make_uint2(0u, 0u);
+        if (!pad) {
+            uint32_t b[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                b[e] = e4m3x2(fp8_in(pp[2 * e], scale), fp8_in(pp[2 * e + 1], scale)) & 0xFFFFu;
+            w = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(pp[e]));
+        }
+        __stcs(reinterpret_cast<uint2*>(o.ag8 + k), w);
+    } else if (o.ag) {
         uint4 w = pad ? make_uint4(0u, 0u, 0u, 0u)
                       : make_uint4(pack_bf16x2(pp[0], pp[1]), pack_bf16x2(pp[2], pp[3]),
                                    pack_bf16x2(pp[4], pp[5]), pack_bf16x2(pp[6], pp[7]));
@@ -200,10 +227,11 @@ __device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64
     }
 }
 
-template <int NR, bool SHIFTED>
+template <int NR, bool SHIFTED, bool FP8>
 __device__ __forceinline__ void fused_body(const uint16_t* __restrict__ src_al, int64_t stride,
                                            int N, int D, const FusedOut& o, int64_t k0, int nvec,
-                                           bool avg, float fN, const AdamScalars& sc) {
+                                           bool avg, float fN, const AdamScalars& sc, float scale,
+                                           float& mx) {
 #pragma unroll 1
     for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
         const int64_t k = k0 + 8 * (int64_t)q;
@@ -215,15 +243,16 @@ __device__ __forceinline__ void fused_body(const uint16_t* __restrict__ src_al, 
 #pragma unroll
             for (int e = 0; e < 8; ++e) g[e] = __fdiv_rn(g[e], fN);
         }
-        fused8(o, k, g, P, M, V, false, sc);
+        fused8<FP8>(o, k, g, P, M, V, false, sc, scale, mx);
     }
 }
 
-template <int NR>
+template <int NR, bool FP8>
 __global__ void __launch_bounds__(kThreads, 2)
 k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o,
            const Unit* __restrict__ units, int64_t n_units, int op_avg, AdamScalars sc,
            const AdamScalars* __restrict__ sc_dev) {
+    __shared__ float part[kThreads / 32];
     if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
     const bool avg = op_avg != 0;
     const float fN = (float)N;
@@ -231,6 +260,10 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o
         const Unit u = units[ui];
         const int len = u.len;
         const int64_t k0 = u.shard_pos;
+        float scale = 0.0f, mx = 0.0f;
+        if constexpr (FP8) {
+            if (!u.is_pad) scale = o.scales[o.unit_param[ui]];
+        }
         // peel to an index that is a multiple of 8 (bf16 16-byte vectors)
         int head = (int)((8 - (k0 & 7)) & 7);
         if (head > len) head = len;
@@ -238,42 +271,76 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o
         const int done = head + 8 * nvec;
         if (u.is_pad) {
             const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if ((int)threadIdx.x < head) fused1(o, k0 + threadIdx.x, 0.0f, true, sc);
+            if ((int)threadIdx.x < head) fused1<FP8>(o, k0 + threadIdx.x, 0.0f, true, sc, scale, mx);
 #pragma unroll 1
             for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
                 const int64_t k = k0 + head + 8 * (int64_t)q;
                 float4 P[2], M[2], V[2];
                 load_pmv8(o, k, P, M, V);
-                fused8(o, k, zero8, P, M, V, true, sc);
+                fused8<FP8>(o, k, zero8, P, M, V, true, sc, scale, mx);
             }
-            if ((int)threadIdx.x < len - done) fused1(o, k0 + done + threadIdx.x, 0.0f, true, sc);
+            if ((int)threadIdx.x < len - done)
+                fused1<FP8>(o, k0 + done + threadIdx.x, 0.0f, true, sc, scale, mx);
             continue;
         }
         const uint16_t* src_run = grads + u.arena_pos;
         if ((int)threadIdx.x < head)
-            fused1(o, k0 + threadIdx.x,
-                   finish(fold_scalar<NR>(src_run + threadIdx.x, stride, N), avg, fN), false, sc);
+            fused1<FP8>(o, k0 + threadIdx.x,
+                        finish(fold_scalar<NR>(src_run + threadIdx.x, stride, N), avg, fN), false,
+                        sc, scale, mx);
         // every rank's arena starts on a 16-byte boundary, so one phase D
         // holds for all N source streams
         const int D = bf16_phase(src_run + head);
         const uint16_t* src_al = src_run + head - D;
-        if (D == 0) fused_body<NR, false>(src_al, stride, N, 0, o, k0 + head, nvec, avg, fN, sc);
-        else fused_body<NR, true>(src_al, stride, N, D, o, k0 + head, nvec, avg, fN, sc);
+        if (D == 0)
+            fused_body<NR, false, FP8>(src_al, stride, N, 0, o, k0 + head, nvec, avg, fN, sc, scale, mx);
+        else
+            fused_body<NR, true, FP8>(src_al, stride, N, D, o, k0 + head, nvec, avg, fN, sc, scale, mx);
         if ((int)threadIdx.x < len - done)
-            fused1(o, k0 + done + threadIdx.x,
-                   finish(fold_scalar<NR>(src_run + done + threadIdx.x, stride, N), avg, fN),
-                   false, sc);
+            fused1<FP8>(o, k0 + done + threadIdx.x,
+                        finish(fold_scalar<NR>(src_run + done + threadIdx.x, stride, N), avg, fN),
+                        false, sc, scale, mx);
+        if constexpr (FP8) {
+            // the unit's max |updated master| into its parameter's amax slot
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = mx;
+            __syncthreads();
+            if (threadIdx.x < 32) {
+                mx = threadIdx.x < kThreads / 32 ? part[threadIdx.x] : 0.0f;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                if (threadIdx.x == 0) atomicMax(o.amax_bits + o.unit_param[ui], __float_as_uint(mx));
+            }
+            __syncthreads();
+        }
     }
 }
 
-template <int NR>
+template <int NR, bool FP8>
 cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const FusedOut& o,
                                int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
                                cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
-    k_rs_adamw<NR><<<grid_for(g, (const void*)k_rs_adamw<NR>, nu), kThreads, 0, st>>>(
+    k_rs_adamw<NR, FP8><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
         grads, g.P_arena, g.N, o, g.d_units, nu, avg, sc, sc_dev);
     return cudaGetLastError();
+}
+
+template <bool FP8>
+cudaError_t launch_rs_adamw_any(const fsdp_group& g, const uint16_t* grads, const FusedOut& o,
+                                int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
+                                cudaStream_t st) {
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_rs_adamw_nr<K, FP8>(g, grads, o, avg, sc, sc_dev, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_rs_adamw_nr<0, FP8>(g, grads, o, avg, sc, sc_dev, st);
+    }
 }
 
 // One thread: advance the device step counter and compute that step's AdamW
@@ -325,16 +392,19 @@ cudaError_t launch_rs_adamw(const fsdp_group& g, const uint16_t* grads, int op, 
                             float* reduced, cudaStream_t st, const AdamScalars* sc_dev) {
     if (g.units.empty()) return cudaSuccess;
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
-    const FusedOut o{master, m, v, reduced, ag_next};
-    switch (g.N) {
-#define FSDPK_CASE(K) \
-    case K: return launch_rs_adamw_nr<K>(g, grads, o, avg, sc, sc_dev, st);
-        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
-        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
-#undef FSDPK_CASE
-        default:
-            return launch_rs_adamw_nr<0>(g, grads, o, avg, sc, sc_dev, st);
-    }
+    const FusedOut o{master, m, v, reduced, ag_next, nullptr, nullptr, nullptr, nullptr};
+    return launch_rs_adamw_any<false>(g, grads, o, avg, sc, sc_dev, st);
+}
+
+cudaError_t launch_rs_adamw_fp8(const fsdp_group& g, const uint16_t* grads, int op, float* master,
+                                float* m, float* v, const AdamScalars& sc, const float* scales_prev,
+                                uint8_t* ag8_next, unsigned* amax_bits, float* reduced,
+                                cudaStream_t st, const AdamScalars* sc_dev) {
+    if (g.units.empty()) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    const FusedOut o{master, m, v, reduced, nullptr, ag8_next, scales_prev, amax_bits,
+                     g.d_unit_param};
+    return launch_rs_adamw_any<true>(g, grads, o, avg, sc, sc_dev, st);
 }
 
 }  // namespace fsdpk

@@ -265,6 +265,42 @@ FSDP_API int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grad
 FSDP_API int fsdp_copy_in_fp8(fsdp_group_t group, const float* master, uint8_t* ag8,
                      float* scales, fsdp_stream_t stream);
 
+/* FP8 copy-in with given scales (no amax pass): ag8 as for fsdp_copy_in_fp8
+ * with scale_i = scales[i] supplied by the caller, e.g. the previous step's
+ * scales in delayed scaling.  master: fp32 [N][S] (read); scales: fp32
+ * [n_params] (read; 4-byte aligned); ag8: uint8 [N][S] (written, 0x00 in
+ * pad rows).  Algorithmic bytes: 4 + 1 per padded element. */
+FSDP_API int fsdp_copy_in_fp8_scaled(fsdp_group_t group, const float* master,
+                                     const float* scales, uint8_t* ag8,
+                                     fsdp_stream_t stream);
+
+/* fsdp_rs_adamw_step with an FP8 next all-gather input (delayed scaling):
+ * the reduce-scatter and AdamW update of fsdp_rs_adamw_step, then, while the
+ * updated master is in registers,
+ *   ag8_next[r][k] = e4m3_rn(clamp(master[r][k] * scales_prev[i], -448, 448))
+ * (0x00 in pad rows) and the next scales from the updated master,
+ *   scales_next[i] = 448 / max(max |master| over parameter i, 1e-12),
+ * the scale rule of fsdp_copy_in_fp8.  The scales lag one step behind the
+ * master they quantise: the amax is known only after the update has passed
+ * over the whole parameter, and reading the master again to apply it would
+ * cost the 4 bytes per element the fusion saves.  The result equals
+ * fsdp_rs_reduce + fsdp_adamw_step + fsdp_copy_in_fp8_scaled(scales_prev),
+ * and scales_next equals the scales fsdp_copy_in_fp8 computes from the
+ * updated master.
+ *   grads, op, master, m, v, hparams, reduced_or_null: as for
+ *   fsdp_rs_adamw_step;  scales_prev: fp32 [n_params] (read);
+ *   ag8_next: uint8 [N][S] (written); scales_next: fp32 [n_params] (written;
+ *   a different buffer from scales_prev).  Both scale buffers 4-byte aligned.
+ * Algorithmic bytes: 2N per real element + 25 (+4 with reduced) per padded
+ * element.  Three launches on `stream`: a memset of scales_next, the fused
+ * kernel and a per-parameter division. */
+FSDP_API int fsdp_rs_adamw_step_fp8(fsdp_group_t group, const uint16_t* grads, int32_t op,
+                                    float* master, float* m, float* v,
+                                    const fsdp_adamw_hparams* hparams,
+                                    const float* scales_prev, uint8_t* ag8_next,
+                                    float* scales_next, float* reduced_or_null,
+                                    fsdp_stream_t stream);
+
 /* FP8 copy-out: the byte-for-byte counterpart of fsdp_copy_out.
  * ag8: uint8 [N][S] (read); arena8: uint8 [P_arena] (written, gaps
  * untouched).  Algorithmic bytes: 1 read + 1 written per real element. */

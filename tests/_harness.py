@@ -28,6 +28,8 @@ class Guarded:
         self.full = torch.empty(n + 2 * GUARD, dtype=dtype, device=device)
         if dtype == torch.float32:
             self.full.fill_(-12345.5)
+        elif dtype == torch.uint8:
+            self.full.fill_(0x5A)
         else:
             self.full.view(torch.int16).fill_(0x3BEF)
         self.t = self.full[GUARD:GUARD + n]
@@ -39,6 +41,8 @@ class Guarded:
             s = torch.tensor(-12345.5, dtype=torch.float32, device=self.full.device)
             lo, hi = self.full[:GUARD], self.full[GUARD + self.n:]
             return bool((lo == s).all() and (hi == s).all())
+        if self.full.dtype == torch.uint8:
+            return bool((self.full[:GUARD] == 0x5A).all() and (self.full[GUARD + self.n:] == 0x5A).all())
         v = self.full.view(torch.int16)
         return bool((v[:GUARD] == 0x3BEF).all() and (v[GUARD + self.n:] == 0x3BEF).all())
 
@@ -275,6 +279,130 @@ def run_group_fused(wl: W.Workload, group: W.Group, *, steps: int = 1, op=None,
         assert not np.any(diff & (f32(master.t).view(np.uint32) == master_o.view(np.uint32)))
         assert bf16_within_adam_band(ag_h[diff], ag_o[diff])
         del grads, ag, red, redu, agu
+    g.destroy()
+    return report
+
+
+def e4m3_value(q: np.ndarray) -> np.ndarray:
+    """E4M3 ("fn") codes decoded by torch's float8_e4m3fn."""
+    return torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn).float().numpy()
+
+
+def e4m3_within_band(a: np.ndarray, b: np.ndarray, xa: np.ndarray, xb: np.ndarray) -> bool:
+    """Two E4M3 codes of the quantiser inputs xa, xb (already scaled and
+    clamped): each code is within half a step of its input, so the decoded
+    values differ by at most one step at their magnitude plus |xa - xb|."""
+    va = e4m3_value(a).astype(np.float64)
+    vb = e4m3_value(b).astype(np.float64)
+    mag = np.maximum(np.maximum(np.abs(va), np.abs(vb)), 2.0 ** -6)
+    step = 2.0 ** (np.floor(np.log2(mag)) - 3)  # 3 mantissa bits; subnormal step 2^-9
+    d_in = np.abs(xa.astype(np.float64) - xb.astype(np.float64))
+    return bool(np.all(np.abs(va - vb) <= step + d_in))
+
+
+def run_group_fused_fp8(wl: W.Workload, group: W.Group, *, steps: int = 2, op=None,
+                        tag=()) -> dict:
+    """The fused reduce-scatter + AdamW + FP8 next copy-in (delayed scaling)
+    against (a) the separate GPU stages rs_reduce -> adamw -> copy_in_fp8_scaled
+    with the previous scales, plus copy_in_fp8 for the next scales, on a copy of
+    the same state (bit for bit) and (b) the oracle's composition (reduced
+    gradient bit for bit; master within the AdamW tolerance; scales and codes
+    within the band that tolerance allows, exact where the inputs agree)."""
+    N = wl.N
+    op = wl.op if op is None else op
+    g = abi.fsdp_plan_group(group.shapes, N)
+    p = oracle.plan(group.shapes, N)
+    check_plan(g, p)
+    NS = N * g.S
+    n = max(g.n, 1)
+    full = torch.empty(max(g.P_arena, 1), dtype=torch.float32, device="cuda")
+    W.fill_master(full, wl, group.name, *tag)
+    master = Guarded(NS, torch.float32)
+    abi.fsdp_shard_params(g, full, master.t)
+    torch.cuda.synchronize()
+    master_o = oracle.shard(p, f32(full)[:p.P_arena] if p.P_arena else np.zeros(0, np.float32))
+    m = Guarded(NS, torch.float32, fill=torch.zeros(NS))
+    v = Guarded(NS, torch.float32, fill=torch.zeros(NS))
+    mu, vu = torch.zeros(NS, device="cuda"), torch.zeros(NS, device="cuda")
+    masteru = master.t.clone()
+    m_o = np.zeros(NS, np.float32)
+    v_o = np.zeros(NS, np.float32)
+    hp = dict(W.ADAMW_DEFAULTS)
+    # step 0: dynamic scales of the initial master start the delayed chain
+    scales_prev = torch.empty(n, device="cuda")
+    abi.fsdp_copy_in_fp8(g, master.t, torch.empty(max(NS, 1), dtype=torch.uint8, device="cuda"),
+                         scales_prev)
+    torch.cuda.synchronize()
+    scales_prev_o = oracle.fp8_scales(p, master_o)
+    assert bits_equal(f32(scales_prev)[:g.n], scales_prev_o)
+    report = {"adam_max_ratio": 0.0, "fp8_code_diffs": 0}
+    for step in range(1, steps + 1):
+        grads = make_grads(g, wl, group, step, tag)
+        grads_h = u16(grads)
+        ag8 = Guarded(NS, torch.uint8)
+        red = Guarded(NS, torch.float32)
+        scales_next = Guarded(g.n, torch.float32)
+        abi.fsdp_rs_adamw_step_fp8(g, grads, op, master.t, m.t, v.t, step=step,
+                                   scales_prev=scales_prev, ag8_next=ag8.t,
+                                   scales_next=scales_next.t, reduced=red.t, **hp)
+        # the separate GPU stages
+        redu = torch.empty(NS, device="cuda")
+        ag8u = torch.empty(NS, dtype=torch.uint8, device="cuda")
+        dyn = torch.empty(n, device="cuda")
+        abi.fsdp_rs_reduce(g, grads, op, redu)
+        abi.fsdp_adamw_step(g, masteru, mu, vu, redu, step=step, **hp)
+        abi.fsdp_copy_in_fp8_scaled(g, masteru, scales_prev, ag8u)
+        abi.fsdp_copy_in_fp8(g, masteru, torch.empty(max(NS, 1), dtype=torch.uint8,
+                                                      device="cuda"), dyn)
+        torch.cuda.synchronize()
+        for buf in (master, m, v, ag8, red, scales_next):
+            assert buf.guards_intact(), "fused FP8 kernel wrote outside a buffer"
+        for name, a, b in (("master", master.t, masteru), ("m", m.t, mu), ("v", v.t, vu),
+                           ("reduced", red.t, redu), ("scales", scales_next.t, dyn[:g.n])):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32)), f"fused != unfused {name}"
+        assert torch.equal(ag8.t, ag8u), "fused != unfused ag8"
+        # oracle composition
+        red_o = oracle.reduce_scatter(p, grads_h, op)
+        assert bits_equal(f32(red.t), red_o), "fused reduced: " + first_mismatch(f32(red.t), red_o)
+        oracle.adamw(master_o, m_o, v_o, red_o, step=step, **hp)
+        for name, gbuf, obuf in (("master", master, master_o), ("m", m, m_o), ("v", v, v_o)):
+            ok, ratio = adam_close(f32(gbuf.t), obuf)
+            report["adam_max_ratio"] = max(report["adam_max_ratio"], ratio)
+            assert ok, f"fused fp8 adamw {name} step {step}: max |d|/tol = {ratio}"
+        sp = f32(scales_prev)[:g.n]
+        ag8_o = oracle.copy_in_fp8(p, master_o, scales_prev_o)
+        got = ag8.t.cpu().numpy()
+        same_in = (f32(master.t).view(np.uint32) == master_o.view(np.uint32))
+        if g.n:
+            pid = np.full(NS, -1, np.int64)
+            for i in range(g.n):
+                for r in range(N):
+                    o0 = r * g.S + int(p.shard_off[i])
+                    pid[o0:o0 + int(p.valid_rows(i, r)) * int(p.cols[i])] = i
+            real = pid >= 0
+            same_in &= ~real | (sp[np.maximum(pid, 0)].view(np.uint32)
+                                == scales_prev_o[np.maximum(pid, 0)].view(np.uint32))
+        else:
+            real = np.zeros(NS, bool)
+        diff = got != ag8_o
+        assert not np.any(diff & same_in), "fp8 code differs where master and scale agree"
+        assert not np.any(diff & ~real), "fp8 pad byte differs"
+        if np.any(diff):
+            idx = np.nonzero(diff)[0]
+            xa = np.clip(f32(master.t)[idx] * sp[pid[idx]], -448, 448).astype(np.float32)
+            xb = np.clip(master_o[idx] * scales_prev_o[pid[idx]], -448, 448).astype(np.float32)
+            assert e4m3_within_band(got[idx], ag8_o[idx], xa, xb)
+        report["fp8_code_diffs"] += int(np.sum(diff))
+        # next scales: oracle's from its own master, within the AdamW band of amax
+        sn = f32(scales_next.t)
+        sn_o = oracle.fp8_scales(p, master_o)
+        amax_o = np.float64(448.0) / sn_o.astype(np.float64)
+        rel = np.abs(sn.astype(np.float64) - sn_o) / sn_o
+        assert np.all(rel <= ADAM_TOL * (1.0 + amax_o) / amax_o + 2.0 ** -22), \
+            f"fp8 next scales: max rel {rel.max() if rel.size else 0}"
+        scales_prev = scales_next.t.clone() if g.n else scales_prev
+        scales_prev_o = sn_o
+        del grads, ag8, red, redu, ag8u
     g.destroy()
     return report
 

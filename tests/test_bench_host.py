@@ -80,3 +80,11 @@ def test_reference_arm_prints_one_json_line():
 def test_fused_byte_model_is_30_plus_2n_per_unpadded_param():
     for N in (2, 6, 8):
         assert sum(bench.fused_stage_bytes(N, 1000, N * 1000).values()) == (30 + 2 * N) * N * 1000
+
+
+def test_fused_fp8_byte_model_is_27_plus_2n_per_unpadded_param():
+    for N in (1, 2, 8):
+        b = bench.fused_fp8_stage_bytes(N, 1000, N * 1000, 0)
+        assert sum(b.values()) == (27 + 2 * N) * N * 1000
+        assert bench.fused_fp8_stage_bytes(N, 1000, N * 1000, 5)["rs_adamw_copy_in_fp8"] \
+            == b["rs_adamw_copy_in_fp8"] + 60

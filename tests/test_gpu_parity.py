@@ -103,6 +103,18 @@ def test_fused_full_size_llama7b_block(H):
     H.run_group_fused(wl, wl.groups[0], steps=1, direct_oracle=True)
 
 
+@pytest.mark.parametrize("wl", FUSED + [W.tiny_mlp(), W.uneven(8), W.moe(8)],
+                         ids=[w.name for w in FUSED] + ["tiny_mlp", "uneven_div8", "moe_div8"])
+def test_fused_rs_adamw_fp8_delayed_scaling(H, wl):
+    for g in wl.groups:
+        H.run_group_fused_fp8(wl, g, steps=3)
+
+
+def test_fused_fp8_full_size_llama7b_block(H):
+    wl = W.llama7b()
+    H.run_group_fused_fp8(wl, wl.groups[0], steps=1)
+
+
 ACCUM = SMALL[:4] + [W.tiny_mlp(), W.uneven(8), W.moe(16), W.llama7b(16, layers=1)]
 
 
@@ -283,6 +295,7 @@ def test_edge_shapes_and_world_sizes(H, wl):
     H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=wl.N <= 64)
     H.run_group_fused(wl, wl.groups[0], steps=2)
     H.run_group_fp8(wl, wl.groups[0])
+    H.run_group_fused_fp8(wl, wl.groups[0], steps=2)
 
 
 def _random_group(rng, k):
@@ -305,6 +318,7 @@ def test_random_groups_brute_force(H, wl):
     H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
     H.run_group_fused(wl, grp, steps=1)
     H.run_group_fp8(wl, grp)
+    H.run_group_fused_fp8(wl, grp, steps=1)
 
 
 GRID = [_wl(f"grid_n{N}", [((d0, c) if c > 1 else (d0,)) for d0 in range(21) for c in (1, 3, 8)], N,
@@ -314,11 +328,12 @@ GRID = [_wl(f"grid_n{N}", [((d0, c) if c > 1 else (d0,)) for d0 in range(21) for
 @pytest.mark.parametrize("wl", GRID, ids=[w.name for w in GRID])
 def test_brute_force_grid_d0_cols_world(H, wl):
     """Every d0 in [0, 20] x cols in {1, 3, 8} as one 63-parameter group, for
-    every N in [1, 9]: all stages, all ops, the fused and FP8 paths."""
+    every N in [1, 9]: all stages, all ops, the fused, FP8 and fused FP8 paths."""
     grp = wl.groups[0]
     H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
     H.run_group_fused(wl, grp, steps=1)
     H.run_group_fp8(wl, grp)
+    H.run_group_fused_fp8(wl, grp, steps=1)
 
 
 def test_checkpoint_resume_is_bit_exact(H, tmp_path):
