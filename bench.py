@@ -109,15 +109,28 @@ def max_over_ranks(value: float, device=None) -> float:
     import torch.distributed as dist
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device=device)
+    on_dev = dist.get_backend() == "nccl"
+    t = torch.tensor([value], dtype=torch.float64, device=device if on_dev else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, device=None) -> float:
+    """Sum of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    on_dev = dist.get_backend() == "nccl"
+    t = torch.tensor([value], dtype=torch.float64, device=device if on_dev else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
 
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
-        if device is not None and device.type == "cuda":
+        if device is not None and device.type == "cuda" and dist.get_backend() == "nccl":
             dist.barrier(device_ids=[device.index])
         else:
             dist.barrier()
@@ -709,6 +722,174 @@ def run_fused_fp8(args, model, device, stream, ws, ms_fused, peak):
     }
 
 
+def peer_stage_bytes(N: int, S: int, P: int, L: int, P_local: int) -> dict:
+    """Per-device bytes of one group step when the N virtual ranks are spread
+    over devices, L per device (P_local real elements in the local shards):
+    the local copy-in, the copy-out of the whole group on every device (it
+    pulls every rank's rows), the reduce-scatter of the local destination
+    rows (N source arenas each) and the local AdamW."""
+    LS = L * S
+    return {"copy_in": 6 * LS, "copy_out": 2 * N * S + 2 * P,
+            "rs_reduce": 2 * N * P_local + 4 * LS, "adamw": 28 * LS}
+
+
+def peer_exchange_bytes(N: int, S: int, L: int, P_local: int, D: int) -> int:
+    """Bytes one device pulls from the other devices per group step: the
+    other ranks' slot rows (copy-out) and the other ranks' gradient rows of
+    the local shards (reduce-scatter)."""
+    if D == 1:
+        return 0
+    return 2 * (N - L) * S + 2 * (N - L) * P_local
+
+
+def run_peer(args, wl, device, rank, ws):
+    """The step with the N virtual ranks of every group spread over the ws
+    processes (L = N / ws per device; one model, so the total work is fixed
+    and the scaling is strong).  Each device copies its ranks in into a slot
+    that every device maps (CUDA IPC), then pulls every rank's rows in its
+    copy-out; its reduce-scatter pulls the N source arenas of its own rows;
+    AdamW is local.  Host barriers order the phases across devices: after the
+    copy-ins, and at the end of the step (no slot is rewritten while a peer
+    may still read it)."""
+    import torch
+    from fully_sharded_shard_b200 import abi
+    from fully_sharded_shard_b200 import peer
+    from fully_sharded_shard_b200 import workloads as W
+    N = wl.N
+    if N % ws:
+        raise SystemExit(f"--exchange peer needs N = {N} divisible by the {ws} processes")
+    stream = torch.cuda.Stream(device)
+    t_setup = time.time()
+    hp = dict(W.ADAMW_DEFAULTS)
+    shared, instances, plans = [], [], []
+    max_A, max_LS = 1, 1
+    for gi, grp in enumerate(wl.groups):
+        first = peer.PeerGroup(grp.shapes, N, device=device)
+        L, S, A, r0 = first.L, first.S, first.P_arena, first.r0
+        g = first.g
+        for r in range(r0, r0 + L):
+            W.fill_grads_bf16(first.grads[r - r0], wl, grp.name, "peer", "pool", 0, r)
+            if grp.zero_grad:
+                W.zero_param_ranges(first.grads[r - r0], g.arena_off, g.numel, grp.zero_grad)
+        P_local = 0
+        for i, shape in enumerate(grp.shapes):
+            d0 = shape[0] if len(shape) else 1
+            cols = g.numel[i] // d0 if d0 else 0
+            c = g.chunk_rows[i]
+            P_local += sum(max(0, min(c, d0 - j * c)) * cols for j in range(r0, r0 + L))
+        plans.append((g, L, S, A, P_local))
+        full = torch.empty(max(A, 1), dtype=torch.float32, device=device)
+        master_full = torch.empty(max(N * S, 1), dtype=torch.float32, device=device)
+        for rep_i in range(grp.repeat):
+            pg = first if rep_i == 0 else peer.PeerGroup(grp.shapes, N, device=device,
+                                                          grads=first.grad_buf)
+            W.fill_master(full[:A], wl, grp.name, "peer", "layer", rep_i)
+            abi.fsdp_shard_params(g, full, master_full)
+            master = master_full[r0 * S:(r0 + L) * S].clone()
+            m = torch.zeros(L * S, dtype=torch.float32, device=device)
+            v = torch.zeros(L * S, dtype=torch.float32, device=device)
+            instances.append((gi, pg, master, m, v))
+            shared.append(pg)
+        del full, master_full
+        max_A, max_LS = max(max_A, A), max(max_LS, L * S)
+    arenas = [torch.empty(max_A, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    reduced = torch.empty(max_LS, dtype=torch.float32, device=device)
+    torch.cuda.synchronize(device)
+    setup_s = time.time() - t_setup
+    state = {"t": 0}
+
+    def one_step(events=None):
+        state["t"] += 1
+
+        def timed(name, fn):
+            if events is None:
+                fn()
+                return
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            events[name].append((e0, e1))
+
+        for gi, pg, master, m, v in instances:
+            timed("copy_in", lambda: pg.copy_in(master, stream))
+        peer.barrier(device)
+        for idx, (gi, pg, master, m, v) in enumerate(instances):
+            timed("copy_out", lambda: pg.copy_out(arenas[idx % 2], stream))
+            timed("rs_reduce", lambda: pg.rs_reduce(wl.op, reduced, stream))
+            timed("adamw", lambda: pg.adamw_step(master, m, v, reduced, stream=stream,
+                                                 step=state["t"], **hp))
+        peer.barrier(device)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            one_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(e_start.elapsed_time(e_end), device) / args.steps
+    events = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
+    with torch.cuda.stream(stream):
+        one_step(events)
+    torch.cuda.synchronize(device)
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in events.items()}
+    sb = {k: 0 for k in stage_ms}
+    xbytes = 0
+    P_total = 0
+    for gi, pg, master, m, v in instances:
+        g, L, S, A, P_local = plans[gi]
+        for k, b in peer_stage_bytes(N, S, g.P, L, P_local).items():
+            sb[k] += b
+        xbytes += peer_exchange_bytes(N, S, L, P_local, ws)
+        P_total += g.P
+    dev_bytes = sum(sb.values())
+    job_bytes = sum_over_ranks(float(dev_bytes), device)
+    peak, peak_kind = hbm_peak()
+    dom = max(stage_ms, key=stage_ms.get)
+    dom_achieved = sb[dom] / (stage_ms[dom] * 1e-3) / 1e9
+    kernel_names = {"copy_in": "k_copy_in", "copy_out": "k_copy_out<TAB>",
+                    "rs_reduce": "k_reduce_units_tab", "adamw": "k_adamw"}
+    out = {
+        "metric": METRIC, "value": round(job_bytes / (ms_step * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "params_per_s": round(P_total / (ms_step * 1e-3), 1),
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: seeded N(0,0.02) fp32 master, N(0,1e-3) bf16 per-rank grads",
+        "config": {"workload": wl.name, "N_virtual_ranks": N, "ranks_per_gpu": N // ws,
+                   "groups_per_step": len(instances), "params": P_total,
+                   "exchange": "pulls over CUDA IPC peer memory (copy-out, reduce-scatter)",
+                   "barriers_per_step": 2,
+                   "bytes_per_step_per_gpu": dev_bytes,
+                   "exchange_bytes_per_step_per_gpu": xbytes,
+                   "l2": "inputs larger than L2",
+                   "parallelism": f"{ws} GPU(s), {N} virtual ranks, {N // ws} per GPU"},
+        "stages": {k: {"ms_per_step": round(stage_ms[k], 3),
+                       "GBps": round(sb[k] / (stage_ms[k] * 1e-3) / 1e9, 1)} for k in stage_ms},
+        "roofline": {"bound": "hbm", "kernel": kernel_names[dom],
+                     "achieved": round(dom_achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(dom_achieved / peak, 4),
+                     "avg_launch_ms": round(stage_ms[dom] / len(instances), 4),
+                     "traffic": None},
+        "gpu_launches": 4 * len(instances) * args.steps,
+        "clocks": clocks, "setup_s": round(setup_s, 1),
+    }
+    peer.release_all([b for pg in shared for b in pg.buffers()], device)
+    return out
+
+
 def run_accumulate(args, model, device, stream, micro: int = 4):
     """Gradient accumulation without sync on the largest repeated group:
     micro - 1 accumulations into fp32 per-rank arenas, then the reduce-scatter
@@ -1050,6 +1231,13 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--exchange", choices=["replicas", "peer"], default="replicas",
+                    help="replicas: one full N-rank replica per GPU (weak scaling); peer: one "
+                         "model whose N ranks are spread over the GPUs, exchanged as pulls "
+                         "over peer memory (strong scaling)")
+    ap.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
+                    help="process-group backend for N > 1 (gloo lets several processes share "
+                         "one GPU, to exercise --exchange peer without several GPUs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -1066,10 +1254,19 @@ def main(argv=None):
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
-    device = torch.device("cuda", local)
+    device = torch.device("cuda", local % torch.cuda.device_count())
     torch.cuda.set_device(device)
     if ws > 1:
-        init_dist("nccl")
+        init_dist(args.backend)
+    if args.exchange == "peer":
+        out = run_peer(args, wl, device, rank, ws)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if ws > 1:
+            import torch.distributed as dist
+            barrier(device)
+            dist.destroy_process_group()
+        return 0
     out, model = run_ours(args, wl, device, rank, ws)
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)

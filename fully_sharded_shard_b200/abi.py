@@ -28,6 +28,7 @@ FSDP_MAX_WORLD = 1024
 
 FSDP_OK, FSDP_EINVAL, FSDP_ENOMEM, FSDP_ECUDA, FSDP_EALIGN, FSDP_ESTATE = 0, -1, -2, -3, -4, -5
 FSDP_SUM, FSDP_AVG, FSDP_SUM_THEN_DIV = 0, 1, 2
+FSDP_PEER_MAX_RANKS = 64
 
 EXPORTED = (
     "fsdp_plan_group", "fsdp_group_sizes", "fsdp_group_param_offsets",
@@ -48,6 +49,10 @@ class FsdpError(RuntimeError):
 
 class ParamDesc(ctypes.Structure):
     _fields_ = [("ndim", ctypes.c_int32), ("shape", ctypes.c_int64 * FSDP_MAX_NDIM)]
+
+
+class IpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_uint8 * 64)]
 
 
 class AdamWHparams(ctypes.Structure):
@@ -97,6 +102,26 @@ def _load() -> ctypes.CDLL:
     L.fsdp_rs_adamw_step_dev.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
+    L.fsdp_peer_plan.argtypes = [vp, i32, i32, ctypes.POINTER(vp)]
+    L.fsdp_peer_local_ranks.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    L.fsdp_peer_set_sources.argtypes = [vp, vp, vp]
+    L.fsdp_destroy_peer_plan.argtypes = [vp]
+    L.fsdp_destroy_peer_plan.restype = None
+    L.fsdp_peer_copy_in.argtypes = [vp, vp, vp, vp]
+    L.fsdp_peer_copy_out.argtypes = [vp, vp, vp]
+    L.fsdp_peer_rs_reduce.argtypes = [vp, i32, vp, vp]
+    L.fsdp_peer_adamw_step.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp]
+    L.fsdp_peer_rs_adamw_step.argtypes = [vp, i32, vp, vp, vp, ctypes.POINTER(AdamWHparams),
+                                          vp, vp, vp]
+    L.fsdp_ipc_alloc.argtypes = [i64, ctypes.POINTER(vp), ctypes.POINTER(IpcHandle)]
+    L.fsdp_ipc_free.argtypes = [vp]
+    L.fsdp_ipc_open.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(vp)]
+    L.fsdp_ipc_close.argtypes = [vp]
+    for name in ("fsdp_peer_plan", "fsdp_peer_local_ranks", "fsdp_peer_set_sources",
+                 "fsdp_peer_copy_in", "fsdp_peer_copy_out", "fsdp_peer_rs_reduce",
+                 "fsdp_peer_adamw_step", "fsdp_peer_rs_adamw_step", "fsdp_ipc_alloc",
+                 "fsdp_ipc_free", "fsdp_ipc_open", "fsdp_ipc_close"):
+        getattr(L, name).restype = ctypes.c_int
     L.fsdp_status_string.argtypes = [ctypes.c_int]
     L.fsdp_status_string.restype = ctypes.c_char_p
     for name in ("fsdp_plan_group", "fsdp_group_sizes", "fsdp_group_param_offsets",
@@ -374,3 +399,145 @@ def fsdp_rs_reduce_noalloc(shapes: Sequence[Sequence[int]], world_size: int,
                                        _ptr(grads, _B16, N * P_arena, "grads"), int(op),
                                        _ptr(reduced, _F32, N * S, "reduced"),
                                        _stream(stream, reduced)), "fsdp_rs_reduce_noalloc")
+
+
+# ---------------------------------------------------------------------------
+# several devices: per-rank pointer tables and CUDA IPC
+# ---------------------------------------------------------------------------
+class PeerPlan:
+    """Device `index` of `n_devices` of a group: its local virtual ranks
+    [r0, r0 + L) and the per-rank pointer tables of the exchange steps."""
+
+    def __init__(self, group: Group, n_devices: int, index: int):
+        h = ctypes.c_void_p()
+        _check(_lib.fsdp_peer_plan(group.handle, int(n_devices), int(index), ctypes.byref(h)),
+               "fsdp_peer_plan")
+        self._h = h
+        self.group = group  # the group must outlive the peer plan
+        self.n_devices, self.index = int(n_devices), int(index)
+        L, r0 = ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.fsdp_peer_local_ranks(h, ctypes.byref(L), ctypes.byref(r0)),
+               "fsdp_peer_local_ranks")
+        self.L, self.r0 = L.value, r0.value
+        self.N, self.S, self.P, self.P_arena, self.n = (group.N, group.S, group.P,
+                                                        group.P_arena, group.n)
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise ValueError("peer plan destroyed")
+        return self._h
+
+    def destroy(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            _lib.fsdp_destroy_peer_plan(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def fsdp_peer_plan(group: Group, n_devices: int, index: int) -> PeerPlan:
+    return PeerPlan(group, n_devices, index)
+
+
+def fsdp_peer_set_sources(pp: PeerPlan, ag_rank_ptrs: Optional[Sequence[int]],
+                          grad_rank_ptrs: Optional[Sequence[int]]):
+    def table(ptrs):
+        if ptrs is None:
+            return None
+        if len(ptrs) != pp.N:
+            raise ValueError(f"{len(ptrs)} pointers for {pp.N} ranks")
+        return (ctypes.c_void_p * pp.N)(*[int(x) for x in ptrs])
+    _check(_lib.fsdp_peer_set_sources(pp.handle, table(ag_rank_ptrs), table(grad_rank_ptrs)),
+           "fsdp_peer_set_sources")
+
+
+def fsdp_peer_copy_in(pp: PeerPlan, master: torch.Tensor, ag_slot: torch.Tensor, stream=None):
+    n = pp.L * pp.S
+    _check(_lib.fsdp_peer_copy_in(pp.handle, _ptr(master, _F32, n, "master"),
+                                  _ptr(ag_slot, _B16, n, "ag_slot"), _stream(stream, master)),
+           "fsdp_peer_copy_in")
+
+
+def fsdp_peer_copy_out(pp: PeerPlan, arena: torch.Tensor, stream=None):
+    _check(_lib.fsdp_peer_copy_out(pp.handle, _ptr(arena, _B16, pp.P_arena, "arena"),
+                                   _stream(stream, arena)), "fsdp_peer_copy_out")
+
+
+def fsdp_peer_rs_reduce(pp: PeerPlan, op: int, reduced: torch.Tensor, stream=None):
+    _check(_lib.fsdp_peer_rs_reduce(pp.handle, int(op),
+                                    _ptr(reduced, _F32, pp.L * pp.S, "reduced"),
+                                    _stream(stream, reduced)), "fsdp_peer_rs_reduce")
+
+
+def fsdp_peer_adamw_step(pp: PeerPlan, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                         grad: torch.Tensor, *, lr: float, beta1: float, beta2: float,
+                         eps: float, weight_decay: float, step: int, stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = pp.L * pp.S
+    _check(_lib.fsdp_peer_adamw_step(pp.handle, _ptr(master, _F32, n, "master"),
+                                     _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                     _ptr(grad, _F32, n, "grad"), ctypes.byref(hp),
+                                     _stream(stream, master)), "fsdp_peer_adamw_step")
+
+
+def fsdp_peer_rs_adamw_step(pp: PeerPlan, op: int, master: torch.Tensor, m: torch.Tensor,
+                            v: torch.Tensor, *, lr: float, beta1: float, beta2: float,
+                            eps: float, weight_decay: float, step: int,
+                            ag_next: Optional[torch.Tensor] = None,
+                            reduced: Optional[torch.Tensor] = None, stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = pp.L * pp.S
+    _check(_lib.fsdp_peer_rs_adamw_step(pp.handle, int(op), _ptr(master, _F32, n, "master"),
+                                        _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                        ctypes.byref(hp), _ptr(ag_next, _B16, n, "ag_next"),
+                                        _ptr(reduced, _F32, n, "reduced"),
+                                        _stream(stream, master)), "fsdp_peer_rs_adamw_step")
+
+
+def fsdp_ipc_alloc(nbytes: int):
+    """Device memory another process can map: returns (pointer, 64-byte handle)."""
+    ptr, h = ctypes.c_void_p(), IpcHandle()
+    _check(_lib.fsdp_ipc_alloc(int(nbytes), ctypes.byref(ptr), ctypes.byref(h)),
+           "fsdp_ipc_alloc")
+    return int(ptr.value), bytes(h.bytes)
+
+
+def fsdp_ipc_free(ptr: int):
+    _check(_lib.fsdp_ipc_free(ctypes.c_void_p(int(ptr))), "fsdp_ipc_free")
+
+
+def fsdp_ipc_open(handle: bytes) -> int:
+    if len(handle) != 64:
+        raise ValueError("an IPC handle has 64 bytes")
+    h = IpcHandle()
+    ctypes.memmove(h.bytes, handle, 64)
+    ptr = ctypes.c_void_p()
+    _check(_lib.fsdp_ipc_open(ctypes.byref(h), ctypes.byref(ptr)), "fsdp_ipc_open")
+    return int(ptr.value)
+
+
+def fsdp_ipc_close(ptr: int):
+    _check(_lib.fsdp_ipc_close(ctypes.c_void_p(int(ptr))), "fsdp_ipc_close")
+
+
+class _DeviceSpan:
+    def __init__(self, ptr: int, nbytes: int):
+        self.__cuda_array_interface__ = {"shape": (int(nbytes),), "typestr": "|u1",
+                                         "data": (int(ptr), False), "version": 3}
+
+
+def device_tensor(ptr: int, numel: int, dtype: torch.dtype, device) -> torch.Tensor:
+    """A tensor view of `numel` elements of device memory this binding does
+    not own (e.g. from fsdp_ipc_alloc); the memory must outlive the tensor."""
+    esize = torch.empty(0, dtype=dtype).element_size()
+    if numel == 0:
+        return torch.empty(0, dtype=dtype, device=device)
+    raw = torch.as_tensor(_DeviceSpan(ptr, numel * esize), device=device)
+    return raw.view(dtype)

@@ -97,6 +97,124 @@ bool adam_scalars(const fsdp_adamw_hparams* hp, fsdpk::AdamScalars* sc) {
 
 }  // namespace
 
+namespace fsdpk {
+
+// The work tables of the virtual ranks [r0, r1), in the local index space
+// [(r1 - r0)][S] of buffers that hold only those ranks' shards: real units of
+// every (rank j, parameter i), then pad units, the merged pad intervals and
+// the copy-in tile ranges.  Reads the per-parameter tables of g.
+int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
+    const int64_t S = g->S;
+    const int32_t n_params = g->n;
+    g->units.clear();
+    g->unit_param.clear();
+    g->intervals.clear();
+    g->tile_ranges.clear();
+    try {
+        for (int64_t j = r0; j < r1; ++j)
+            for (int32_t i = 0; i < n_params; ++i) {
+                const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
+                push_units(g->units, g->unit_param, i, (j - r0) * S + g->off[i],
+                           g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);
+            }
+        g->n_real_units = (int64_t)g->units.size();
+        for (int64_t j = r0; j < r1; ++j)
+            for (int32_t i = 0; i < n_params; ++i) {
+                const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
+                const int64_t lo = (j - r0) * S + g->off[i] + v * g->cols[i];
+                const int64_t len = (g->c[i] - v) * g->cols[i];
+                push_units(g->units, g->unit_param, i, lo, 0, len, 1);
+                if (len > 0) {
+                    if (!g->intervals.empty() && g->intervals.back().hi == lo)
+                        g->intervals.back().hi = lo + len;  // merge adjacent pads
+                    else
+                        g->intervals.push_back(Interval{lo, lo + len});
+                }
+            }
+        if (g->intervals.size() > (size_t)std::numeric_limits<int32_t>::max()) return FSDP_EINVAL;
+        const int64_t NS = (r1 - r0) * S;
+        g->n_tiles = (NS + fsdpk::kCopyInTile - 1) / fsdpk::kCopyInTile;
+        if (!g->intervals.empty()) {
+            g->tile_ranges.resize((size_t)g->n_tiles);
+            size_t a = 0, b = 0;
+            for (int64_t t = 0; t < g->n_tiles; ++t) {
+                const int64_t lo = t * fsdpk::kCopyInTile;
+                const int64_t hi = lo + fsdpk::kCopyInTile;
+                while (a < g->intervals.size() && g->intervals[a].hi <= lo) ++a;
+                if (b < a) b = a;
+                while (b < g->intervals.size() && g->intervals[b].lo < hi) ++b;
+                g->tile_ranges[(size_t)t] = TileRange{(int32_t)a, (int32_t)b};
+            }
+        }
+    } catch (...) {
+        return FSDP_ENOMEM;
+    }
+    return FSDP_OK;
+}
+
+// One device allocation for the work tables of g, uploaded once; records the
+// current device and its SM count.
+int upload_tables(fsdp_group* g) {
+    cudaError_t e = cudaGetDevice(&g->device);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&g->sm_count, cudaDevAttrMultiProcessorCount, g->device);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const size_t b_units = g->units.size() * sizeof(Unit);
+    const size_t b_iv = g->intervals.size() * sizeof(Interval);
+    const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
+    const size_t b_up = g->unit_param.size() * sizeof(int32_t);
+    auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up);
+    if (total == 0) return FSDP_OK;
+    e = cudaMalloc(&g->dev_mem, total);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        g->dev_mem = nullptr;
+        return e == cudaErrorMemoryAllocation ? FSDP_ENOMEM : cuda_fail(e);
+    }
+    char* base = static_cast<char*>(g->dev_mem);
+    g->d_units = reinterpret_cast<const Unit*>(base);
+    g->d_intervals = reinterpret_cast<const Interval*>(base + up256(b_units));
+    g->d_tile_ranges = reinterpret_cast<const TileRange*>(base + up256(b_units) + up256(b_iv));
+    g->d_unit_param =
+        reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) + up256(b_tr));
+    if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && b_iv)
+        e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && b_tr)
+        e = cudaMemcpy((void*)g->d_tile_ranges, g->tile_ranges.data(), b_tr,
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && b_up)
+        e = cudaMemcpy((void*)g->d_unit_param, g->unit_param.data(), b_up, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(g->dev_mem);
+        g->dev_mem = nullptr;
+        return cuda_fail(e);
+    }
+    return FSDP_OK;
+}
+
+void free_tables(fsdp_group* g) {
+    if (g->dev_mem == nullptr) return;
+    int prev = -1;
+    bool switched = false;
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != g->device)
+        switched = cudaSetDevice(g->device) == cudaSuccess;
+    cudaFree(g->dev_mem);
+    g->dev_mem = nullptr;
+    if (switched) cudaSetDevice(prev);
+}
+
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
+int check_plan_device(const fsdp_group* g) { return check_device(g); }
+
+bool host_adam_scalars(const fsdp_adamw_hparams* hp, AdamScalars* sc) {
+    return adam_scalars(hp, sc);
+}
+
+}  // namespace fsdpk
+
 extern "C" {
 
 
@@ -183,85 +301,10 @@ int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t wor
     if (NS / fsdpk::kCopyInTile + 1 > std::numeric_limits<int32_t>::max()) return fail(FSDP_EINVAL);
     g->pad_elems = NS - P;
 
-    // work units: real runs for every (rank j, parameter i), then pad runs
-    try {
-        for (int64_t j = 0; j < N; ++j)
-            for (int32_t i = 0; i < n_params; ++i) {
-                const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
-                push_units(g->units, g->unit_param, i, j * S + g->off[i],
-                           g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);
-            }
-        g->n_real_units = (int64_t)g->units.size();
-        for (int64_t j = 0; j < N; ++j)
-            for (int32_t i = 0; i < n_params; ++i) {
-                const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
-                const int64_t lo = j * S + g->off[i] + v * g->cols[i];
-                const int64_t len = (g->c[i] - v) * g->cols[i];
-                push_units(g->units, g->unit_param, i, lo, 0, len, 1);
-                if (len > 0) {
-                    if (!g->intervals.empty() && g->intervals.back().hi == lo)
-                        g->intervals.back().hi = lo + len;  // merge adjacent pads
-                    else
-                        g->intervals.push_back(Interval{lo, lo + len});
-                }
-            }
-        if (g->intervals.size() > (size_t)std::numeric_limits<int32_t>::max())
-            return fail(FSDP_EINVAL);
-        g->n_tiles = (NS + fsdpk::kCopyInTile - 1) / fsdpk::kCopyInTile;
-        if (!g->intervals.empty()) {
-            g->tile_ranges.resize((size_t)g->n_tiles);
-            size_t a = 0, b = 0;
-            for (int64_t t = 0; t < g->n_tiles; ++t) {
-                const int64_t lo = t * fsdpk::kCopyInTile;
-                const int64_t hi = lo + fsdpk::kCopyInTile;
-                while (a < g->intervals.size() && g->intervals[a].hi <= lo) ++a;
-                if (b < a) b = a;
-                while (b < g->intervals.size() && g->intervals[b].lo < hi) ++b;
-                g->tile_ranges[(size_t)t] = TileRange{(int32_t)a, (int32_t)b};
-            }
-        }
-    } catch (...) {
-        return fail(FSDP_ENOMEM);
-    }
-
-    // device tables, one allocation, uploaded once
-    cudaError_t e = cudaGetDevice(&g->device);
-    if (e != cudaSuccess) return fail(cuda_fail(e));
-    e = cudaDeviceGetAttribute(&g->sm_count, cudaDevAttrMultiProcessorCount, g->device);
-    if (e != cudaSuccess) return fail(cuda_fail(e));
-    const size_t b_units = g->units.size() * sizeof(Unit);
-    const size_t b_iv = g->intervals.size() * sizeof(Interval);
-    const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
-    const size_t b_up = g->unit_param.size() * sizeof(int32_t);
-    auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up);
-    if (total > 0) {
-        e = cudaMalloc(&g->dev_mem, total);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            g->dev_mem = nullptr;
-            return fail(e == cudaErrorMemoryAllocation ? FSDP_ENOMEM : cuda_fail(e));
-        }
-        char* base = static_cast<char*>(g->dev_mem);
-        g->d_units = reinterpret_cast<const Unit*>(base);
-        g->d_intervals = reinterpret_cast<const Interval*>(base + up256(b_units));
-        g->d_tile_ranges = reinterpret_cast<const TileRange*>(base + up256(b_units) + up256(b_iv));
-        g->d_unit_param = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
-                                                           up256(b_tr));
-        if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
-        if (e == cudaSuccess && b_iv)
-            e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
-        if (e == cudaSuccess && b_tr)
-            e = cudaMemcpy((void*)g->d_tile_ranges, g->tile_ranges.data(), b_tr,
-                           cudaMemcpyHostToDevice);
-        if (e == cudaSuccess && b_up)
-            e = cudaMemcpy((void*)g->d_unit_param, g->unit_param.data(), b_up,
-                           cudaMemcpyHostToDevice);
-        if (e != cudaSuccess) {
-            cudaFree(g->dev_mem);
-            return fail(cuda_fail(e));
-        }
-    }
+    g->L = world_size;
+    int st = fsdpk::build_rank_tables(g, 0, N);
+    if (st == FSDP_OK) st = fsdpk::upload_tables(g);
+    if (st != FSDP_OK) return fail(st);
     *out = g;
     return FSDP_OK;
 }
@@ -287,14 +330,7 @@ int fsdp_group_param_offsets(fsdp_group_t g, int64_t* shard_off, int64_t* arena_
 
 void fsdp_destroy_group(fsdp_group_t g) {
     if (g == nullptr) return;
-    if (g->dev_mem) {
-        int prev = -1;
-        bool switched = false;
-        if (cudaGetDevice(&prev) == cudaSuccess && prev != g->device)
-            switched = cudaSetDevice(g->device) == cudaSuccess;
-        cudaFree(g->dev_mem);
-        if (switched) cudaSetDevice(prev);
-    }
+    fsdpk::free_tables(g);
     delete g;
 }
 

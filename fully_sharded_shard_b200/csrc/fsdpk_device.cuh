@@ -98,12 +98,42 @@ __device__ __forceinline__ void zero_f32_run(float* __restrict__ dst, int64_t le
     if (threadIdx.x < len - done) dst[done + threadIdx.x] = 0.0f;
 }
 
-template <int NR>
-__device__ __forceinline__ float fold_scalar(const uint16_t* __restrict__ src, int64_t stride,
-                                             int N) {
+// Where each source rank's gradient arena starts.
+//   StrideSrc: all N ranks in one buffer, rank r at base + r * stride.
+//   TableSrc:  one pointer per rank (arenas in separate allocations, such as
+//              peers' memory mapped into this process), held in shared memory.
+// at(off) moves every rank's pointer by off elements.
+struct StrideSrc {
+    const uint16_t* base;
+    int64_t stride;
+    __device__ __forceinline__ const uint16_t* rank(int r) const { return base + r * stride; }
+    __device__ __forceinline__ StrideSrc at(int64_t off) const {
+        return StrideSrc{base + off, stride};
+    }
+};
+
+struct TableSrc {
+    const uint16_t* const* tab;
+    int64_t off;
+    __device__ __forceinline__ const uint16_t* rank(int r) const { return tab[r] + off; }
+    __device__ __forceinline__ TableSrc at(int64_t o) const { return TableSrc{tab, off + o}; }
+};
+
+// Ranks a TableSrc kernel can address (its table lives in shared memory).
+constexpr int kPeerMaxRanks = FSDP_PEER_MAX_RANKS;
+
+// Copy an N-entry rank table into shared memory (every thread calls this).
+__device__ __forceinline__ void load_rank_table(const uint16_t* const* __restrict__ g_tab,
+                                                const uint16_t** s_tab, int N) {
+    for (int r = threadIdx.x; r < N; r += blockDim.x) s_tab[r] = g_tab[r];
+    __syncthreads();
+}
+
+template <int NR, class Src>
+__device__ __forceinline__ float fold_scalar(const Src& src, int N) {
     const int n = NR ? NR : N;
-    float acc = bf16_bits_to_f32(src[0]);
-    for (int r = 1; r < n; ++r) acc = __fadd_rn(acc, bf16_bits_to_f32(src[r * stride]));
+    float acc = bf16_bits_to_f32(src.rank(0)[0]);
+    for (int r = 1; r < n; ++r) acc = __fadd_rn(acc, bf16_bits_to_f32(src.rank(r)[0]));
     return acc;
 }
 

@@ -131,14 +131,23 @@ __device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_a
     }
 }
 
+// TAB: rank r's rows come from ag_tab[r], the start of rank r's [S] slot row
+// (a pull from wherever that rank's slot lives), instead of ag + r * S.
+template <bool TAB>
 __global__ void __launch_bounds__(kThreads, 5)
-k_copy_out(const uint16_t* __restrict__ ag, uint16_t* __restrict__ arena,
-           const Unit* __restrict__ units, int64_t n_units) {
+k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ ag_tab, int64_t S,
+           uint16_t* __restrict__ arena, const Unit* __restrict__ units, int64_t n_units) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
         const int len = u.len;
         uint16_t* dst_run = arena + u.arena_pos;
-        const uint16_t* src_run = ag + u.shard_pos;
+        const uint16_t* src_run;
+        if constexpr (TAB) {
+            const int64_t r = u.shard_pos / S;  // a unit never crosses a rank's row
+            src_run = ag_tab[r] + (u.shard_pos - r * S);
+        } else {
+            src_run = ag + u.shard_pos;
+        }
         const int head = (int)head_to_16B(dst_run, len);
         if ((int)threadIdx.x < head) dst_run[threadIdx.x] = src_run[threadIdx.x];
         const int nvec = (len - head) >> 3;
@@ -318,7 +327,7 @@ k_fp8_copy_out(const uint8_t* __restrict__ ag8, uint8_t* __restrict__ arena8,
 
 cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* ag,
                            cudaStream_t st) {
-    const int64_t count = (int64_t)g.N * g.S;
+    const int64_t count = (int64_t)g.L * g.S;
     if (count == 0) return cudaSuccess;
     const bool pads = !g.tile_ranges.empty();
     k_copy_in<<<grid_for(g, (const void*)k_copy_in, g.n_tiles), kThreads, 0, st>>>(
@@ -330,8 +339,16 @@ cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* a
 cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* arena,
                             cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
-    k_copy_out<<<grid_for(g, (const void*)k_copy_out, g.n_real_units), kThreads, 0, st>>>(
-        ag, arena, g.d_units, g.n_real_units);
+    k_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
+        ag, nullptr, g.S, arena, g.d_units, g.n_real_units);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* ag_tab,
+                                uint16_t* arena, cudaStream_t st) {
+    if (parent.n_real_units == 0) return cudaSuccess;
+    k_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
+        nullptr, ag_tab, parent.S, arena, parent.d_units, parent.n_real_units);
     return cudaGetLastError();
 }
 

@@ -52,19 +52,22 @@ struct TileRange {
 struct fsdp_group {
     int device = -1;
     int sm_count = 0;
-    int32_t N = 0;
+    int32_t N = 0;  // virtual ranks of the group (sources of every reduction)
+    int32_t L = 0;  // ranks whose shards this plan's [L][S] buffers hold: N, or
+                    // N / D for the local view of a device's D-way peer plan
     int32_t n = 0;
     std::vector<int64_t> d0, cols, c, s, off, u;
     int64_t S = 0, P = 0, P_arena = 0;
     int64_t pad_elems = 0;  // N*S - P
 
-    // host copies (kept for inspection and tests of the plan)
+    // host copies (kept for inspection and tests of the plan); shard
+    // positions index the [L][S] buffers
     std::vector<fsdpk::Unit> units;  // real units first, then pad units
     std::vector<int32_t> unit_param;  // parameter index of every unit
     int64_t n_real_units = 0;
     std::vector<fsdpk::Interval> intervals;
     std::vector<fsdpk::TileRange> tile_ranges;  // empty when no padding
-    int64_t n_tiles = 0;                        // copy-in tiles over N*S
+    int64_t n_tiles = 0;                        // copy-in tiles over L*S
 
     // one device allocation holding the three tables
     void* dev_mem = nullptr;
@@ -74,7 +77,32 @@ struct fsdp_group {
     const int32_t* d_unit_param = nullptr;
 };
 
+// The opaque peer plan behind fsdp_peer_t: device `index` of `n_devices` holds the
+// virtual ranks [r0, r0 + L) of `parent`'s group.
+struct fsdp_peer {
+    const fsdp_group* parent = nullptr;  // copy-out units of all N ranks; not owned
+    fsdp_group local;                    // tables of the local ranks, local coordinates
+    int32_t n_devices = 0;
+    int32_t index = 0;
+    int64_t r0 = 0;
+    // one device allocation: N all-gather slot row pointers, then N gradient
+    // arena pointers (set by fsdp_peer_set_sources)
+    void* dev_tab = nullptr;
+    bool have_ag = false;
+    bool have_grads = false;
+};
+
 namespace fsdpk {
+
+// Plan helpers (fsdpk_api.cu): the work tables of ranks [r0, r1) in local
+// coordinates, their upload, their release, and the recording of a CUDA
+// error for fsdp_last_cuda_error.  Return FSDP status codes.
+int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1);
+int upload_tables(fsdp_group* g);
+void free_tables(fsdp_group* g);
+int record_cuda_error(cudaError_t e);
+// FSDP_OK when the current device is g's, FSDP_ESTATE (or FSDP_ECUDA) otherwise.
+int check_plan_device(const fsdp_group* g);
 
 // Scalars of one AdamW step, precomputed on the host in binary64.
 struct AdamScalars {
@@ -86,6 +114,9 @@ struct AdamScalars {
     float eps;
 };
 static_assert(sizeof(AdamScalars) == 32, "AdamScalars is the 32-byte fsdp_adamw_dev_scalars");
+
+// Validate AdamW hyper-parameters and compute one step's scalars (binary64).
+bool host_adam_scalars(const fsdp_adamw_hparams* hp, AdamScalars* sc);
 
 // Kernel launchers (fsdpk_gather.cu, fsdpk_reduce.cu, fsdpk_update.cu).  They enqueue work and return the
 // cudaError_t of the launch.
@@ -113,6 +144,19 @@ cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
 cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Unit* units,
                                   int64_t n_units, const uint16_t* grads, int op, float* reduced,
                                   cudaStream_t st);
+
+// The exchange steps over per-rank pointer tables (device arrays of N
+// pointers): the copy-out pulling rank r's rows from ag_tab[r] (the start of
+// rank r's [S] slot row), and the reductions folding rank r's gradient arena
+// at grad_tab[r].  `parent` supplies the copy-out units, `local` the units of
+// the local destination ranks.
+cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* ag_tab,
+                                uint16_t* arena, cudaStream_t st);
+cudaError_t launch_rs_fused_tab(const fsdp_group& local, const uint16_t* const* grad_tab, int op,
+                                float* reduced, cudaStream_t st);
+cudaError_t launch_rs_adamw_tab(const fsdp_group& local, const uint16_t* const* grad_tab, int op,
+                                float* master, float* m, float* v, const AdamScalars& sc,
+                                uint16_t* ag_next, float* reduced, cudaStream_t st);
 
 // Fused reduce-scatter + AdamW (+ optional next-step copy-in into ag_next and
 // optional reduced-gradient output).

@@ -1,0 +1,250 @@
+// fsdpk_peer.cu -- host side of the multi-device exchange: the peer plan of
+// one device (the work tables of its local virtual ranks plus one pointer
+// per rank for the all-gather slots and the gradient arenas), its entry
+// points, and the CUDA IPC helpers that map other processes' buffers.
+//
+// The exchange steps of "Introduction to PyTorch FSDP2 Backend Features",
+// Working Principle (all-gather before use, reduce-scatter after backward)
+// run as pulls inside the copy-out and reduction kernels: each rank's data
+// is read where it lives, over NVLink when that is another GPU, and the
+// reduction keeps the rank order 0..N-1 of the single-device path.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "fsdpk.h"
+#include "fsdpk_internal.h"
+
+namespace {
+
+int cuda_status(cudaError_t e) {
+    return e == cudaSuccess ? FSDP_OK : fsdpk::record_cuda_error(e);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+const uint16_t* const* ag_table(const fsdp_peer* p) {
+    return static_cast<const uint16_t* const*>(p->dev_tab);
+}
+
+const uint16_t* const* grad_table(const fsdp_peer* p) {
+    return static_cast<const uint16_t* const*>(p->dev_tab) + p->parent->N;
+}
+
+int check_op(int32_t op) {
+    return (op == FSDP_SUM || op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? FSDP_OK : FSDP_EINVAL;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fsdp_peer_plan(fsdp_group_t g, int32_t n_devices, int32_t device_index, fsdp_peer_t* out) {
+    if (out == nullptr) return FSDP_EINVAL;
+    *out = nullptr;
+    if (g == nullptr || n_devices < 1 || device_index < 0 || device_index >= n_devices)
+        return FSDP_EINVAL;
+    if (g->L != g->N || g->N % n_devices != 0 || g->N > FSDP_PEER_MAX_RANKS) return FSDP_EINVAL;
+    int st = fsdpk::check_plan_device(g);
+    if (st != FSDP_OK) return st;
+    fsdp_peer* p = new (std::nothrow) fsdp_peer();
+    if (p == nullptr) return FSDP_ENOMEM;
+    p->parent = g;
+    p->n_devices = n_devices;
+    p->index = device_index;
+    const int32_t L = g->N / n_devices;
+    p->r0 = (int64_t)device_index * L;
+    fsdp_group& l = p->local;
+    try {
+        l.N = g->N;
+        l.L = L;
+        l.n = g->n;
+        l.d0 = g->d0;
+        l.cols = g->cols;
+        l.c = g->c;
+        l.s = g->s;
+        l.off = g->off;
+        l.u = g->u;
+        l.S = g->S;
+        l.P = g->P;
+        l.P_arena = g->P_arena;
+        l.pad_elems = g->pad_elems;
+    } catch (...) {
+        delete p;
+        return FSDP_ENOMEM;
+    }
+    st = fsdpk::build_rank_tables(&l, p->r0, p->r0 + L);
+    if (st == FSDP_OK) st = fsdpk::upload_tables(&l);
+    if (st == FSDP_OK) {
+        cudaError_t e = cudaMalloc(&p->dev_tab, 2 * (size_t)g->N * sizeof(void*));
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            p->dev_tab = nullptr;
+            st = e == cudaErrorMemoryAllocation ? FSDP_ENOMEM : cuda_status(e);
+        }
+    }
+    if (st != FSDP_OK) {
+        fsdpk::free_tables(&l);
+        delete p;
+        return st;
+    }
+    *out = p;
+    return FSDP_OK;
+}
+
+int fsdp_peer_local_ranks(fsdp_peer_t p, int32_t* L, int32_t* r0) {
+    if (p == nullptr) return FSDP_EINVAL;
+    if (L) *L = p->local.L;
+    if (r0) *r0 = (int32_t)p->r0;
+    return FSDP_OK;
+}
+
+int fsdp_peer_set_sources(fsdp_peer_t p, const uint16_t* const* ag_rank_ptrs,
+                          const uint16_t* const* grad_rank_ptrs) {
+    if (p == nullptr) return FSDP_EINVAL;
+    const int32_t N = p->parent->N;
+    for (int32_t r = 0; ag_rank_ptrs != nullptr && r < N; ++r) {
+        if (p->parent->S > 0 && ag_rank_ptrs[r] == nullptr) return FSDP_EINVAL;
+        if (reinterpret_cast<uintptr_t>(ag_rank_ptrs[r]) & 1u) return FSDP_EALIGN;
+    }
+    for (int32_t r = 0; grad_rank_ptrs != nullptr && r < N; ++r) {
+        if (p->parent->P_arena > 0 && grad_rank_ptrs[r] == nullptr) return FSDP_EINVAL;
+        if (!aligned16(grad_rank_ptrs[r])) return FSDP_EALIGN;
+    }
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    const size_t bytes = (size_t)N * sizeof(void*);
+    cudaError_t e = cudaSuccess;
+    if (ag_rank_ptrs != nullptr)
+        e = cudaMemcpy(p->dev_tab, ag_rank_ptrs, bytes, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && grad_rank_ptrs != nullptr)
+        e = cudaMemcpy(static_cast<char*>(p->dev_tab) + bytes, grad_rank_ptrs, bytes,
+                       cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (ag_rank_ptrs != nullptr) p->have_ag = true;
+    if (grad_rank_ptrs != nullptr) p->have_grads = true;
+    return FSDP_OK;
+}
+
+void fsdp_destroy_peer_plan(fsdp_peer_t p) {
+    if (p == nullptr) return;
+    int prev = -1;
+    bool switched = false;
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != p->local.device)
+        switched = cudaSetDevice(p->local.device) == cudaSuccess;
+    if (p->dev_tab) cudaFree(p->dev_tab);
+    if (switched) cudaSetDevice(prev);
+    fsdpk::free_tables(&p->local);
+    delete p;
+}
+
+int fsdp_peer_copy_in(fsdp_peer_t p, const float* master, uint16_t* ag_slot,
+                      fsdp_stream_t stream) {
+    if (p == nullptr) return FSDP_EINVAL;
+    const int64_t LS = (int64_t)p->local.L * p->local.S;
+    if (LS > 0 && (master == nullptr || ag_slot == nullptr)) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(ag_slot)) return FSDP_EALIGN;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(fsdpk::launch_copy_in(p->local, master, ag_slot, (cudaStream_t)stream));
+}
+
+int fsdp_peer_copy_out(fsdp_peer_t p, uint16_t* arena, fsdp_stream_t stream) {
+    if (p == nullptr) return FSDP_EINVAL;
+    if (p->parent->P > 0 && arena == nullptr) return FSDP_EINVAL;
+    if (!aligned16(arena)) return FSDP_EALIGN;
+    if (!p->have_ag) return FSDP_ESTATE;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(
+        fsdpk::launch_copy_out_tab(*p->parent, ag_table(p), arena, (cudaStream_t)stream));
+}
+
+int fsdp_peer_rs_reduce(fsdp_peer_t p, int32_t op, float* reduced, fsdp_stream_t stream) {
+    if (p == nullptr || check_op(op) != FSDP_OK) return FSDP_EINVAL;
+    if ((int64_t)p->local.L * p->local.S > 0 && reduced == nullptr) return FSDP_EINVAL;
+    if (!aligned16(reduced)) return FSDP_EALIGN;
+    if (!p->have_grads) return FSDP_ESTATE;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(
+        fsdpk::launch_rs_fused_tab(p->local, grad_table(p), op, reduced, (cudaStream_t)stream));
+}
+
+int fsdp_peer_adamw_step(fsdp_peer_t p, float* master, float* m, float* v, const float* grad,
+                         const fsdp_adamw_hparams* hp, fsdp_stream_t stream) {
+    if (p == nullptr || hp == nullptr) return FSDP_EINVAL;
+    const int64_t LS = (int64_t)p->local.L * p->local.S;
+    if (LS > 0 && (master == nullptr || m == nullptr || v == nullptr || grad == nullptr))
+        return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!fsdpk::host_adam_scalars(hp, &sc)) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad))
+        return FSDP_EALIGN;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(
+        fsdpk::launch_adamw(p->local, master, m, v, grad, sc, (cudaStream_t)stream));
+}
+
+int fsdp_peer_rs_adamw_step(fsdp_peer_t p, int32_t op, float* master, float* m, float* v,
+                            const fsdp_adamw_hparams* hp, uint16_t* ag_next, float* reduced,
+                            fsdp_stream_t stream) {
+    if (p == nullptr || hp == nullptr || check_op(op) != FSDP_OK) return FSDP_EINVAL;
+    const int64_t LS = (int64_t)p->local.L * p->local.S;
+    if (LS > 0 && (master == nullptr || m == nullptr || v == nullptr)) return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!fsdpk::host_adam_scalars(hp, &sc)) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(ag_next) ||
+        !aligned16(reduced))
+        return FSDP_EALIGN;
+    if (!p->have_grads) return FSDP_ESTATE;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(fsdpk::launch_rs_adamw_tab(p->local, grad_table(p), op, master, m, v, sc,
+                                                  ag_next, reduced, (cudaStream_t)stream));
+}
+
+int fsdp_ipc_alloc(int64_t bytes, void** ptr, fsdp_ipc_handle* handle) {
+    if (ptr == nullptr || handle == nullptr || bytes <= 0) return FSDP_EINVAL;
+    *ptr = nullptr;
+    static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(fsdp_ipc_handle), "IPC handle size");
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, (size_t)bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e == cudaErrorMemoryAllocation ? FSDP_ENOMEM : cuda_status(e);
+    }
+    cudaIpcMemHandle_t h;
+    e = cudaIpcGetMemHandle(&h, p);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return cuda_status(e);
+    }
+    std::memcpy(handle->bytes, &h, sizeof(h));
+    *ptr = p;
+    return FSDP_OK;
+}
+
+int fsdp_ipc_free(void* ptr) {
+    if (ptr == nullptr) return FSDP_EINVAL;
+    return cuda_status(cudaFree(ptr));
+}
+
+int fsdp_ipc_open(const fsdp_ipc_handle* handle, void** ptr) {
+    if (handle == nullptr || ptr == nullptr) return FSDP_EINVAL;
+    *ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle->bytes, sizeof(h));
+    return cuda_status(cudaIpcOpenMemHandle(ptr, h, cudaIpcMemLazyEnablePeerAccess));
+}
+
+int fsdp_ipc_close(void* ptr) {
+    if (ptr == nullptr) return FSDP_EINVAL;
+    return cuda_status(cudaIpcCloseMemHandle(ptr));
+}
+
+}  // extern "C"

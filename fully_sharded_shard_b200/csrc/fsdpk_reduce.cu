@@ -24,10 +24,9 @@ namespace {
 // ---------------------------------------------------------------------------
 
 // Compile-time rank count: all NR loads of a vector are issued before the fold.
-template <int NR, bool SHIFTED, int V>
-__device__ __forceinline__ void reduce_body(const uint16_t* __restrict__ src_al, int64_t stride,
-                                            float* __restrict__ dst, int nvec, int D, bool avg,
-                                            float fN) {
+template <int NR, bool SHIFTED, int V, class Src>
+__device__ __forceinline__ void reduce_body(const Src& src_al, float* __restrict__ dst, int nvec,
+                                            int D, bool avg, float fN) {
 #pragma unroll 1
     for (int q0 = threadIdx.x; q0 < nvec; q0 += blockDim.x * V) {
         uint4 a[V][NR];
@@ -38,7 +37,7 @@ __device__ __forceinline__ void reduce_body(const uint16_t* __restrict__ src_al,
             if (q < nvec) {
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
-                    const uint4* s = reinterpret_cast<const uint4*>(src_al + r * stride) + q;
+                    const uint4* s = reinterpret_cast<const uint4*>(src_al.rank(r)) + q;
                     a[k][r] = ld_src<SHIFTED>(s);
                     if constexpr (SHIFTED) b[k][r] = ld_src<SHIFTED>(s + 1);
                 }
@@ -68,9 +67,8 @@ __device__ __forceinline__ void reduce_body(const uint16_t* __restrict__ src_al,
 }
 
 // Any rank count: ranks in batches of 4, folded in rank order.
-template <bool SHIFTED>
-__device__ __forceinline__ void reduce_body_any(const uint16_t* __restrict__ src_al,
-                                                int64_t stride, int N,
+template <bool SHIFTED, class Src>
+__device__ __forceinline__ void reduce_body_any(const Src& src_al, int N,
                                                 float* __restrict__ dst, int nvec, int D,
                                                 bool avg, float fN) {
 #pragma unroll 1
@@ -82,8 +80,7 @@ __device__ __forceinline__ void reduce_body_any(const uint16_t* __restrict__ src
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 if (r0 + r < N) {
-                    const uint4* s =
-                        reinterpret_cast<const uint4*>(src_al + (int64_t)(r0 + r) * stride) + q;
+                    const uint4* s = reinterpret_cast<const uint4*>(src_al.rank(r0 + r)) + q;
                     a[r] = ld_src<SHIFTED>(s);
                     if constexpr (SHIFTED) b[r] = ld_src<SHIFTED>(s + 1);
                 }
@@ -111,17 +108,38 @@ __device__ __forceinline__ void reduce_body_any(const uint16_t* __restrict__ src
     }
 }
 
-template <int NR, bool SHIFTED>
-__device__ __forceinline__ void reduce_body_dispatch(const uint16_t* src_al, int64_t stride,
-                                                     int N, float* dst, int nvec, int D, bool avg,
-                                                     float fN) {
+template <int NR, bool SHIFTED, class Src>
+__device__ __forceinline__ void reduce_body_dispatch(const Src& src_al, int N, float* dst,
+                                                     int nvec, int D, bool avg, float fN) {
     if constexpr (NR == 0) {
-        reduce_body_any<SHIFTED>(src_al, stride, N, dst, nvec, D, avg, fN);
+        reduce_body_any<SHIFTED>(src_al, N, dst, nvec, D, avg, fN);
     } else {
         // keep about 4-8 independent 16-byte loads in flight per thread
         constexpr int V = NR >= 4 ? 1 : (4 / NR);
-        reduce_body<NR, SHIFTED, V>(src_al, stride, dst, nvec, D, avg, fN);
+        reduce_body<NR, SHIFTED, V>(src_al, dst, nvec, D, avg, fN);
     }
+}
+
+// One real unit: dst_run[e] = fold over ranks of src_run.rank(r)[e].
+template <int NR, class Src>
+__device__ __forceinline__ void reduce_unit(const Src& src_run, float* __restrict__ dst_run,
+                                            int len, int N, bool avg, float fN) {
+    const int head = (int)head_to_16B(dst_run, len);
+    if ((int)threadIdx.x < head)
+        dst_run[threadIdx.x] = finish(fold_scalar<NR>(src_run.at(threadIdx.x), N), avg, fN);
+    const int nvec = (len - head) >> 3;
+    // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0, and
+    // table pointers are checked on the host), so one phase D holds for all N
+    // source streams
+    const int D = bf16_phase(src_run.rank(0) + head);
+    const Src src_al = src_run.at(head - D);
+    float* dst = dst_run + head;
+    if (D == 0) reduce_body_dispatch<NR, false>(src_al, N, dst, nvec, 0, avg, fN);
+    else reduce_body_dispatch<NR, true>(src_al, N, dst, nvec, D, avg, fN);
+    const int done = head + 8 * nvec;
+    if ((int)threadIdx.x < len - done)
+        dst_run[done + threadIdx.x] =
+            finish(fold_scalar<NR>(src_run.at(done + threadIdx.x), N), avg, fN);
 }
 
 // One launch covers every unit of the group.  blockIdx.y selects a source
@@ -144,23 +162,28 @@ k_reduce_units(const uint16_t* __restrict__ grads, int64_t stride, int N,
             zero_f32_run(dst_run, len);
             continue;
         }
-        const uint16_t* src_run = gsrc + u.arena_pos;
-        const int head = (int)head_to_16B(dst_run, len);
-        if ((int)threadIdx.x < head)
-            dst_run[threadIdx.x] =
-                finish(fold_scalar<NR>(src_run + threadIdx.x, stride, N), avg, fN);
-        const int nvec = (len - head) >> 3;
-        // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0),
-        // so one phase D holds for all N source streams
-        const int D = bf16_phase(src_run + head);
-        const uint16_t* src_al = src_run + head - D;
-        float* dst = dst_run + head;
-        if (D == 0) reduce_body_dispatch<NR, false>(src_al, stride, N, dst, nvec, 0, avg, fN);
-        else reduce_body_dispatch<NR, true>(src_al, stride, N, dst, nvec, D, avg, fN);
-        const int done = head + 8 * nvec;
-        if ((int)threadIdx.x < len - done)
-            dst_run[done + threadIdx.x] =
-                finish(fold_scalar<NR>(src_run + done + threadIdx.x, stride, N), avg, fN);
+        reduce_unit<NR>(StrideSrc{gsrc + u.arena_pos, stride}, dst_run, len, N, avg, fN);
+    }
+}
+
+// The fused reduction with one source pointer per rank (a TableSrc):
+// red[shard_pos + e] = fold_r fp32(rank_tab[r][arena_pos + e]).
+template <int NR>
+__global__ void __launch_bounds__(kThreads, 3)
+k_reduce_units_tab(const uint16_t* const* __restrict__ rank_tab, int N, float* __restrict__ out,
+                   const Unit* __restrict__ units, int64_t n_units, int op_avg) {
+    __shared__ const uint16_t* s_tab[kPeerMaxRanks];
+    load_rank_table(rank_tab, s_tab, N);
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const Unit u = units[ui];
+        float* dst_run = out + u.shard_pos;
+        if (u.is_pad) {
+            zero_f32_run(dst_run, u.len);
+            continue;
+        }
+        reduce_unit<NR>(TableSrc{s_tab, u.arena_pos}, dst_run, u.len, N, avg, fN);
     }
 }
 
@@ -410,6 +433,30 @@ cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Un
         default:
             return launch_reduce_nr<0>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg,
                                        st);
+    }
+}
+
+template <int NR>
+cudaError_t launch_reduce_tab_nr(const fsdp_group& g, const uint16_t* const* tab, float* out,
+                                 int avg, cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    k_reduce_units_tab<NR><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(tab, g.N, out,
+                                                                          g.d_units, nu, avg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rs_fused_tab(const fsdp_group& g, const uint16_t* const* grad_tab, int op,
+                                float* reduced, cudaStream_t st) {
+    if (g.units.empty()) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_reduce_tab_nr<K>(g, grad_tab, reduced, avg, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_reduce_tab_nr<0>(g, grad_tab, reduced, avg, st);
     }
 }
 

@@ -177,14 +177,13 @@ __device__ __forceinline__ void load_pmv8(const FusedOut& o, int64_t k, float4 (
 // Rank-ordered fold of 8 elements; NR = N at compile time (1..8): all NR
 // ranks' loads (two 16-byte vectors per rank on a misaligned run) are issued
 // before the fold.  NR = 0 (any N): ranks in batches of 4.
-template <int NR, bool SHIFTED>
-__device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64_t stride, int N,
-                                      int q, int D, float (&acc)[8]) {
+template <int NR, bool SHIFTED, class Src>
+__device__ __forceinline__ void fold8(const Src& src_al, int N, int q, int D, float (&acc)[8]) {
     if constexpr (NR != 0) {
         uint4 a[NR], b[NR];
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-            const uint4* s = reinterpret_cast<const uint4*>(src_al + r * stride) + q;
+            const uint4* s = reinterpret_cast<const uint4*>(src_al.rank(r)) + q;
             a[r] = ld_src<SHIFTED>(s);
             if constexpr (SHIFTED) b[r] = ld_src<SHIFTED>(s + 1);
         }
@@ -203,8 +202,7 @@ __device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 if (r0 + r < N) {
-                    const uint4* s =
-                        reinterpret_cast<const uint4*>(src_al + (int64_t)(r0 + r) * stride) + q;
+                    const uint4* s = reinterpret_cast<const uint4*>(src_al.rank(r0 + r)) + q;
                     a[r] = ld_src<SHIFTED>(s);
                     if constexpr (SHIFTED) b[r] = ld_src<SHIFTED>(s + 1);
                 }
@@ -227,18 +225,17 @@ __device__ __forceinline__ void fold8(const uint16_t* __restrict__ src_al, int64
     }
 }
 
-template <int NR, bool SHIFTED, bool FP8>
-__device__ __forceinline__ void fused_body(const uint16_t* __restrict__ src_al, int64_t stride,
-                                           int N, int D, const FusedOut& o, int64_t k0, int nvec,
-                                           bool avg, float fN, const AdamScalars& sc, float scale,
-                                           float& mx) {
+template <int NR, bool SHIFTED, bool FP8, class Src>
+__device__ __forceinline__ void fused_body(const Src& src_al, int N, int D, const FusedOut& o,
+                                           int64_t k0, int nvec, bool avg, float fN,
+                                           const AdamScalars& sc, float scale, float& mx) {
 #pragma unroll 1
     for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
         const int64_t k = k0 + 8 * (int64_t)q;
         float4 P[2], M[2], V[2];
         load_pmv8(o, k, P, M, V);
         float g[8];
-        fold8<NR, SHIFTED>(src_al, stride, N, q, D, g);
+        fold8<NR, SHIFTED>(src_al, N, q, D, g);
         if (avg) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) g[e] = __fdiv_rn(g[e], fN);
@@ -247,12 +244,44 @@ __device__ __forceinline__ void fused_body(const uint16_t* __restrict__ src_al, 
     }
 }
 
-template <int NR, bool FP8>
+// One real unit: fold, AdamW and the outputs of every element, peeled to an
+// index that is a multiple of 8 (head / nvec vectors / tail).
+template <int NR, bool FP8, class Src>
+__device__ __forceinline__ void rs_adamw_real_unit(const Src& src_run, int N, const FusedOut& o,
+                                                   int64_t k0, int len, int head, int nvec,
+                                                   bool avg, float fN, const AdamScalars& sc,
+                                                   float scale, float& mx) {
+    const int done = head + 8 * nvec;
+    if ((int)threadIdx.x < head)
+        fused1<FP8>(o, k0 + threadIdx.x,
+                    finish(fold_scalar<NR>(src_run.at(threadIdx.x), N), avg, fN), false, sc,
+                    scale, mx);
+    // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0, and
+    // table pointers are checked on the host), so one phase D holds for all N
+    // source streams
+    const int D = bf16_phase(src_run.rank(0) + head);
+    const Src src_al = src_run.at(head - D);
+    if (D == 0)
+        fused_body<NR, false, FP8>(src_al, N, 0, o, k0 + head, nvec, avg, fN, sc, scale, mx);
+    else
+        fused_body<NR, true, FP8>(src_al, N, D, o, k0 + head, nvec, avg, fN, sc, scale, mx);
+    if ((int)threadIdx.x < len - done)
+        fused1<FP8>(o, k0 + done + threadIdx.x,
+                    finish(fold_scalar<NR>(src_run.at(done + threadIdx.x), N), avg, fN), false,
+                    sc, scale, mx);
+}
+
+// TAB: the N source arenas come from a table of per-rank pointers (rank_tab,
+// N <= kPeerMaxRanks) instead of grads + r * stride.
+template <int NR, bool FP8, bool TAB>
 __global__ void __launch_bounds__(kThreads, 2)
-k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o,
+k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride,
+           const uint16_t* const* __restrict__ rank_tab, int N, FusedOut o,
            const Unit* __restrict__ units, int64_t n_units, int op_avg, AdamScalars sc,
            const AdamScalars* __restrict__ sc_dev) {
     __shared__ float part[kThreads / 32];
+    __shared__ const uint16_t* s_tab[TAB ? kPeerMaxRanks : 1];
+    if constexpr (TAB) load_rank_table(rank_tab, s_tab, N);
     if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
     const bool avg = op_avg != 0;
     const float fN = (float)N;
@@ -268,8 +297,8 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o
         int head = (int)((8 - (k0 & 7)) & 7);
         if (head > len) head = len;
         const int nvec = (len - head) >> 3;
-        const int done = head + 8 * nvec;
         if (u.is_pad) {
+            const int done = head + 8 * nvec;
             const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if ((int)threadIdx.x < head) fused1<FP8>(o, k0 + threadIdx.x, 0.0f, true, sc, scale, mx);
 #pragma unroll 1
@@ -283,23 +312,12 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o
                 fused1<FP8>(o, k0 + done + threadIdx.x, 0.0f, true, sc, scale, mx);
             continue;
         }
-        const uint16_t* src_run = grads + u.arena_pos;
-        if ((int)threadIdx.x < head)
-            fused1<FP8>(o, k0 + threadIdx.x,
-                        finish(fold_scalar<NR>(src_run + threadIdx.x, stride, N), avg, fN), false,
-                        sc, scale, mx);
-        // every rank's arena starts on a 16-byte boundary, so one phase D
-        // holds for all N source streams
-        const int D = bf16_phase(src_run + head);
-        const uint16_t* src_al = src_run + head - D;
-        if (D == 0)
-            fused_body<NR, false, FP8>(src_al, stride, N, 0, o, k0 + head, nvec, avg, fN, sc, scale, mx);
+        if constexpr (TAB)
+            rs_adamw_real_unit<NR, FP8>(TableSrc{s_tab, u.arena_pos}, N, o, k0, len, head, nvec,
+                                        avg, fN, sc, scale, mx);
         else
-            fused_body<NR, true, FP8>(src_al, stride, N, D, o, k0 + head, nvec, avg, fN, sc, scale, mx);
-        if ((int)threadIdx.x < len - done)
-            fused1<FP8>(o, k0 + done + threadIdx.x,
-                        finish(fold_scalar<NR>(src_run + done + threadIdx.x, stride, N), avg, fN),
-                        false, sc, scale, mx);
+            rs_adamw_real_unit<NR, FP8>(StrideSrc{grads + u.arena_pos, stride}, N, o, k0, len,
+                                        head, nvec, avg, fN, sc, scale, mx);
         if constexpr (FP8) {
             // the unit's max |updated master| into its parameter's amax slot
 #pragma unroll
@@ -323,8 +341,8 @@ cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const
                                int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
                                cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
-    k_rs_adamw<NR, FP8><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
-        grads, g.P_arena, g.N, o, g.d_units, nu, avg, sc, sc_dev);
+    k_rs_adamw<NR, FP8, false><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
+        grads, g.P_arena, nullptr, g.N, o, g.d_units, nu, avg, sc, sc_dev);
     return cudaGetLastError();
 }
 
@@ -373,7 +391,7 @@ __global__ void k_adamw_prepare(double lr, double beta1, double beta2, double ep
 cudaError_t launch_adamw(const fsdp_group& g, float* master, float* m, float* v,
                          const float* grad, const AdamScalars& sc, cudaStream_t st,
                          const AdamScalars* sc_dev) {
-    const int64_t count = (int64_t)g.N * g.S;
+    const int64_t count = (int64_t)g.L * g.S;
     if (count == 0) return cudaSuccess;
     const int64_t items = ((count >> 2) + kAdamChunk4 - 1) / kAdamChunk4;
     k_adamw<<<grid_for(g, (const void*)k_adamw, items), kThreads, 0, st>>>(master, m, v, grad,
@@ -405,6 +423,33 @@ cudaError_t launch_rs_adamw_fp8(const fsdp_group& g, const uint16_t* grads, int 
     const FusedOut o{master, m, v, reduced, nullptr, ag8_next, scales_prev, amax_bits,
                      g.d_unit_param};
     return launch_rs_adamw_any<true>(g, grads, o, avg, sc, sc_dev, st);
+}
+
+template <int NR>
+cudaError_t launch_rs_adamw_tab_nr(const fsdp_group& g, const uint16_t* const* tab,
+                                   const FusedOut& o, int avg, const AdamScalars& sc,
+                                   cudaStream_t st) {
+    const int64_t nu = (int64_t)g.units.size();
+    k_rs_adamw<NR, false, true><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
+        nullptr, 0, tab, g.N, o, g.d_units, nu, avg, sc, nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rs_adamw_tab(const fsdp_group& g, const uint16_t* const* grad_tab, int op,
+                                float* master, float* m, float* v, const AdamScalars& sc,
+                                uint16_t* ag_next, float* reduced, cudaStream_t st) {
+    if (g.units.empty()) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    const FusedOut o{master, m, v, reduced, ag_next, nullptr, nullptr, nullptr, nullptr};
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_rs_adamw_tab_nr<K>(g, grad_tab, o, avg, sc, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_rs_adamw_tab_nr<0>(g, grad_tab, o, avg, sc, st);
+    }
 }
 
 }  // namespace fsdpk

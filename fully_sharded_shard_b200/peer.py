@@ -1,0 +1,176 @@
+"""One device's share of a parameter group whose N virtual ranks are spread
+over the D processes of a torch.distributed process group (one per GPU).
+
+Device d holds the L = N / D ranks [d*L, (d+1)*L): their fp32 master / m / v
+shards [L][S] (the caller's), their bf16 all-gather slot [L][S] and their bf16
+unsharded gradients [L][P_arena].  The slot and the gradients live in CUDA IPC
+memory that every other process maps (SharedBuffer), so the two exchange
+steps of the group ("Introduction to PyTorch FSDP2 Backend Features", Working
+Principle: the all-gather before use, the reduce-scatter after backward) are
+pulls inside the library's copy-out and reduction kernels, with the reduction
+folding ranks 0..N-1 in order exactly as on one device.
+
+torch.distributed is plumbing here: it swaps the 64-byte IPC handles once and
+provides the barrier that orders the devices between the phases of a step.
+Without an initialised process group everything runs as one device (D = 1).
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+import torch.distributed as dist
+
+from . import abi
+
+
+def _world(group=None) -> Tuple[int, int]:
+    if dist.is_available() and dist.is_initialized():
+        return dist.get_world_size(group), dist.get_rank(group)
+    return 1, 0
+
+
+def rank_pointer_tables(slot_bases: Sequence[int], grad_bases: Sequence[int], L: int, S: int,
+                        P_arena: int) -> Tuple[List[int], List[int]]:
+    """Per-rank pointers: rank r is row r % L of device r // L's slot
+    ([L][S] bf16) and gradient arenas ([L][P_arena] bf16)."""
+    if len(slot_bases) != len(grad_bases):
+        raise ValueError("one slot base and one gradient base per device")
+    N = L * len(slot_bases)
+    ag = [int(slot_bases[r // L]) + 2 * S * (r % L) for r in range(N)]
+    gr = [int(grad_bases[r // L]) + 2 * P_arena * (r % L) for r in range(N)]
+    return ag, gr
+
+
+def exchange(obj, group=None) -> list:
+    """Every process's `obj`, in rank order (one all_gather_object)."""
+    D, _ = _world(group)
+    if D == 1:
+        return [obj]
+    out = [None] * D
+    dist.all_gather_object(out, obj, group=group)
+    return out
+
+
+def barrier(device, group=None) -> None:
+    """Every device's queued work is complete before any device goes on."""
+    torch.cuda.synchronize(device)
+    if _world(group)[0] > 1:
+        dist.barrier(group=group)
+
+
+class SharedBuffer:
+    """`nbytes` of this device's memory, mapped into every process of the
+    group: `bases[j]` is device j's buffer as seen from this process."""
+
+    def __init__(self, nbytes: int, *, group=None, device=None):
+        self.D, self.d = _world(group)
+        self.device = device
+        self.nbytes = int(nbytes)
+        self.ptr, handle = abi.fsdp_ipc_alloc(max(self.nbytes, 16))
+        self._opened: List[int] = []
+        self.bases: List[int] = []
+        for j, h in enumerate(exchange(handle, group)):
+            if j == self.d:
+                self.bases.append(self.ptr)
+            else:
+                p = abi.fsdp_ipc_open(h)
+                self._opened.append(p)
+                self.bases.append(p)
+
+    def view(self, numel: int, dtype: torch.dtype) -> torch.Tensor:
+        """This device's buffer as a tensor (valid until release())."""
+        return abi.device_tensor(self.ptr, numel, dtype, self.device)
+
+    def unmap_peers(self) -> None:
+        for p in self._opened:
+            abi.fsdp_ipc_close(p)
+        self._opened = []
+
+    def release(self) -> None:
+        if self.ptr:
+            abi.fsdp_ipc_free(self.ptr)
+            self.ptr = 0
+
+
+def release_all(buffers: Sequence[SharedBuffer], device, group=None) -> None:
+    """Unmap every peer buffer, then free this device's, with a barrier
+    before each half so that no process still reads a buffer being freed."""
+    barrier(device, group)
+    for b in buffers:
+        b.unmap_peers()
+    barrier(device, group)
+    for b in buffers:
+        b.release()
+
+
+class PeerGroup:
+    """This process's device's part of one parameter group over N virtual
+    ranks on the D processes of `group` (default: the world).
+
+    Order of a step across devices (the caller's, via barrier()):
+      copy_in (own slot)            -> barrier -> copy_out (pulls every slot)
+      gradients into self.grads     -> barrier -> rs_adamw_step / rs_reduce
+    and no slot is rewritten before every device's copy-out of it is done
+    (the second barrier covers that when copy-outs precede it).
+    `grads` may be another PeerGroup's gradient buffer of the same group
+    shapes (several instances of one layer share one gradient buffer)."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], N: int, *, group=None, device=None,
+                 grads: Optional[SharedBuffer] = None):
+        self.pg = group
+        self.device = torch.device(device) if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
+        self.D, self.d = _world(group)
+        self.g = abi.fsdp_plan_group(shapes, N)
+        self.pp = abi.fsdp_peer_plan(self.g, self.D, self.d)
+        L, S, A = self.pp.L, self.g.S, self.g.P_arena
+        self.L, self.r0, self.S, self.P_arena, self.N = L, self.pp.r0, S, A, self.g.N
+        self.slot_buf = SharedBuffer(2 * L * S, group=group, device=self.device)
+        self._own_grads = grads is None
+        if grads is None:
+            grads = SharedBuffer(2 * L * A, group=group, device=self.device)
+        elif grads.nbytes < 2 * L * A:
+            raise ValueError("shared gradient buffer too small for this group")
+        self.grad_buf = grads
+        self.ag_slot = self.slot_buf.view(L * S, torch.bfloat16)
+        self.grads = self.grad_buf.view(L * A, torch.bfloat16).view(L, A)
+        ag, gr = rank_pointer_tables(self.slot_buf.bases, self.grad_buf.bases, L, S, A)
+        abi.fsdp_peer_set_sources(self.pp, ag, gr)
+        self.barrier()
+
+    def barrier(self) -> None:
+        barrier(self.device, self.pg)
+
+    # the stages of this device's ranks
+    def copy_in(self, master: torch.Tensor, stream=None) -> None:
+        abi.fsdp_peer_copy_in(self.pp, master, self.ag_slot, stream)
+
+    def copy_out(self, arena: torch.Tensor, stream=None) -> None:
+        abi.fsdp_peer_copy_out(self.pp, arena, stream)
+
+    def rs_reduce(self, op: int, reduced: torch.Tensor, stream=None) -> None:
+        abi.fsdp_peer_rs_reduce(self.pp, op, reduced, stream)
+
+    def adamw_step(self, master, m, v, grad, *, stream=None, **hp) -> None:
+        abi.fsdp_peer_adamw_step(self.pp, master, m, v, grad, stream=stream, **hp)
+
+    def rs_adamw_step(self, op: int, master, m, v, *, next_copy_in: bool = True,
+                      reduced: Optional[torch.Tensor] = None, stream=None, **hp) -> None:
+        abi.fsdp_peer_rs_adamw_step(self.pp, op, master, m, v,
+                                    ag_next=self.ag_slot if next_copy_in else None,
+                                    reduced=reduced, stream=stream, **hp)
+
+    def buffers(self) -> List[SharedBuffer]:
+        return [self.slot_buf] + ([self.grad_buf] if self._own_grads else [])
+
+    def close(self) -> None:
+        """Release the shared buffers (after barriers, so that no peer still
+        reads them) and the plans."""
+        if self.pp is None:
+            return
+        self.ag_slot = self.grads = None
+        release_all(self.buffers(), self.device, self.pg)
+        self.pp.destroy()
+        self.g.destroy()
+        self.pp = None

@@ -376,6 +376,110 @@ FSDP_API int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_par
                            float* reduced, fsdp_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Several devices: the exchange steps as pulls over peer memory            */
+/* ------------------------------------------------------------------------ */
+
+/* With D devices (one process per GPU), device d holds the L = N / D virtual
+ * ranks [d*L, (d+1)*L) of a group: their master, m, v shards and reduced
+ * gradients, fp32 [L][S]; their all-gather slot, bf16 [L][S] (the copy-in
+ * output, rank-major like the [N][S] buffer it is a slice of); and their
+ * unsharded gradients, bf16 [L][P_arena].  The group's two exchange steps
+ * ("Introduction to PyTorch FSDP2 Backend Features", Working Principle: the
+ * all-gather before the parameters are used, the reduce-scatter after the
+ * backward pass) become pulls inside the stage kernels, over NVLink when a
+ * source lives on another GPU:
+ *   copy-out  reads each rank's rows straight from that rank's slot row;
+ *   reduce    reads each source rank's gradient arena and folds the N ranks
+ *             in rank order 0..N-1, the same bits as on one device.
+ * The caller maps the other devices' buffers into its address space
+ * (fsdp_ipc_*) and passes one pointer per rank.  Ordering across devices is
+ * the caller's: a slot row must be complete before any copy-out reads it and
+ * must not be rewritten (by a copy-in or a fused update) while one still
+ * reads it; a gradient arena must be complete before any reduction reads it.
+ * Pulls are plain loads; no kernel waits on another device. */
+
+#define FSDP_PEER_MAX_RANKS 64
+
+typedef struct fsdp_peer* fsdp_peer_t;
+
+/* The plan of device `device_index` of `n_devices` for `group`: N must be a
+ * multiple of n_devices and N <= FSDP_PEER_MAX_RANKS.  `group` must outlive
+ * the peer plan (its copy-out table is shared).  n_devices == 1 is allowed
+ * (every rank local).  Allocates the local work tables and the two pointer
+ * tables on the current device, which must be the group's.
+ * Errors: FSDP_EINVAL, FSDP_ESTATE (other device), FSDP_ENOMEM, FSDP_ECUDA. */
+FSDP_API int fsdp_peer_plan(fsdp_group_t group, int32_t n_devices, int32_t device_index,
+                            fsdp_peer_t* out);
+
+/* Sizes of the local buffers: L ranks, first rank r0. */
+FSDP_API int fsdp_peer_local_ranks(fsdp_peer_t peer, int32_t* L, int32_t* r0);
+
+/* Where every rank's data lives.  ag_rank_ptrs: host array of N device
+ * pointers, entry r = the first element of rank r's bf16 slot row (S
+ * elements), 2-byte aligned; grad_rank_ptrs: host array of N device
+ * pointers, entry r = rank r's bf16 gradient arena (P_arena elements),
+ * 16-byte aligned.  Either array may be NULL to keep the previous table.
+ * Pointers may be this device's or mapped from peers; they are copied to the
+ * device synchronously.  Errors: FSDP_EINVAL (NULL entry where S or
+ * P_arena > 0), FSDP_EALIGN, FSDP_ECUDA. */
+FSDP_API int fsdp_peer_set_sources(fsdp_peer_t peer, const uint16_t* const* ag_rank_ptrs,
+                                   const uint16_t* const* grad_rank_ptrs);
+
+/* Release the peer plan's tables (not the group, not any data buffer). */
+FSDP_API void fsdp_destroy_peer_plan(fsdp_peer_t peer);
+
+/* Copy-in of the local ranks: master fp32 [L][S] -> ag_slot bf16 [L][S], as
+ * fsdp_copy_in for these ranks (pads +0). */
+FSDP_API int fsdp_peer_copy_in(fsdp_peer_t peer, const float* master, uint16_t* ag_slot,
+                               fsdp_stream_t stream);
+
+/* Copy-out of all N ranks into this device's unsharded arena (bf16
+ * [P_arena], gaps untouched), pulling rank r's rows from ag_rank_ptrs[r].
+ * Same bits as fsdp_copy_out of the gathered [N][S] buffer.  Needs the
+ * all-gather table (FSDP_ESTATE otherwise). */
+FSDP_API int fsdp_peer_copy_out(fsdp_peer_t peer, uint16_t* arena, fsdp_stream_t stream);
+
+/* The fused reduce-scatter for the local destination ranks: reduced fp32
+ * [L][S] (pads +0) from the N gradient arenas of grad_rank_ptrs, in rank
+ * order; same bits as the local rows of fsdp_rs_reduce.  Needs the gradient
+ * table (FSDP_ESTATE otherwise). */
+FSDP_API int fsdp_peer_rs_reduce(fsdp_peer_t peer, int32_t op, float* reduced,
+                                 fsdp_stream_t stream);
+
+/* AdamW on the local shards (fp32 [L][S]), as fsdp_adamw_step. */
+FSDP_API int fsdp_peer_adamw_step(fsdp_peer_t peer, float* master, float* m, float* v,
+                                  const float* grad, const fsdp_adamw_hparams* hparams,
+                                  fsdp_stream_t stream);
+
+/* fsdp_rs_adamw_step for the local ranks: the pull reduce-scatter, AdamW on
+ * master/m/v fp32 [L][S], and optionally the next copy-in into ag_next_or_null
+ * (bf16 [L][S], normally this device's slot) and the reduced gradient into
+ * reduced_or_null (fp32 [L][S]).  Same bits as the local rows of
+ * fsdp_rs_adamw_step. */
+FSDP_API int fsdp_peer_rs_adamw_step(fsdp_peer_t peer, int32_t op, float* master, float* m,
+                                     float* v, const fsdp_adamw_hparams* hparams,
+                                     uint16_t* ag_next_or_null, float* reduced_or_null,
+                                     fsdp_stream_t stream);
+
+/* Device memory other processes can map (CUDA IPC).  fsdp_ipc_alloc
+ * allocates `bytes` (> 0) on the current device with cudaMalloc and writes
+ * the handle another process passes to fsdp_ipc_open; free it with
+ * fsdp_ipc_free once no process has it open.  fsdp_ipc_open maps a handle
+ * from another process (any device of this node that can access the owner's
+ * memory) at *ptr, with peer access enabled lazily; fsdp_ipc_close unmaps
+ * it.  A handle cannot be opened in the process that allocated it.
+ * Errors: FSDP_EINVAL (null arguments, bytes <= 0), FSDP_ENOMEM,
+ * FSDP_ECUDA. */
+typedef struct {
+    uint8_t bytes[64];
+} fsdp_ipc_handle;
+
+FSDP_API int fsdp_ipc_alloc(int64_t bytes, void** ptr, fsdp_ipc_handle* handle);
+FSDP_API int fsdp_ipc_free(void* ptr);
+FSDP_API int fsdp_ipc_open(const fsdp_ipc_handle* handle, void** ptr);
+FSDP_API int fsdp_ipc_close(void* ptr);
+
+/* ------------------------------------------------------------------------ */
 /* Misc                                                                     */
 /* ------------------------------------------------------------------------ */
 

@@ -76,3 +76,28 @@ def test_data_calls_reject_null_group(abi):
     assert L.fsdp_shard_params(None, None, None, None) == abi.FSDP_EINVAL
     assert L.fsdp_group_sizes(None, None, None, None) == abi.FSDP_EINVAL
     L.fsdp_destroy_group(None)
+
+
+def test_peer_and_ipc_calls_reject_bad_arguments_on_host(abi):
+    L = abi.lib()
+    h = ctypes.c_void_p()
+    assert L.fsdp_peer_plan(None, 1, 0, ctypes.byref(h)) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_plan(None, 1, 0, None) == abi.FSDP_EINVAL
+    assert h.value is None
+    assert L.fsdp_peer_local_ranks(None, None, None) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_set_sources(None, None, None) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_copy_in(None, None, None, None) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_copy_out(None, None, None) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_rs_reduce(None, 0, None, None) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_adamw_step(None, None, None, None, None, None, None) == abi.FSDP_EINVAL
+    assert L.fsdp_peer_rs_adamw_step(None, 0, None, None, None, None, None, None,
+                                     None) == abi.FSDP_EINVAL
+    L.fsdp_destroy_peer_plan(None)
+    ptr, hd = ctypes.c_void_p(), abi.IpcHandle()
+    assert L.fsdp_ipc_alloc(0, ctypes.byref(ptr), ctypes.byref(hd)) == abi.FSDP_EINVAL
+    assert L.fsdp_ipc_alloc(-5, ctypes.byref(ptr), ctypes.byref(hd)) == abi.FSDP_EINVAL
+    assert L.fsdp_ipc_alloc(64, None, ctypes.byref(hd)) == abi.FSDP_EINVAL
+    assert L.fsdp_ipc_open(None, ctypes.byref(ptr)) == abi.FSDP_EINVAL
+    assert L.fsdp_ipc_free(None) == abi.FSDP_EINVAL
+    assert L.fsdp_ipc_close(None) == abi.FSDP_EINVAL
+    assert ctypes.sizeof(abi.IpcHandle) == 64

@@ -88,3 +88,18 @@ def test_fused_fp8_byte_model_is_27_plus_2n_per_unpadded_param():
         assert sum(b.values()) == (27 + 2 * N) * N * 1000
         assert bench.fused_fp8_stage_bytes(N, 1000, N * 1000, 5)["rs_adamw_copy_in_fp8"] \
             == b["rs_adamw_copy_in_fp8"] + 60
+
+
+def test_peer_byte_model_reduces_to_the_single_device_model():
+    N, S, P = 8, 1000, 7900
+    one = bench.peer_stage_bytes(N, S, P, N, P)
+    assert sum(one.values()) == bench.group_bytes(N, S, P)
+    assert bench.peer_exchange_bytes(N, S, N, P, 1) == 0
+    # spread over 4 devices: the local stages split, every device copies out all
+    P_local = [2000, 2000, 2000, 1900]
+    per = [bench.peer_stage_bytes(N, S, P, 2, pl) for pl in P_local]
+    assert sum(b["copy_in"] for b in per) == one["copy_in"]
+    assert sum(b["rs_reduce"] for b in per) == one["rs_reduce"]
+    assert sum(b["adamw"] for b in per) == one["adamw"]
+    assert all(b["copy_out"] == one["copy_out"] for b in per)
+    assert bench.peer_exchange_bytes(N, S, 2, 2000, 4) == 2 * 6 * S + 2 * 6 * 2000

@@ -1,0 +1,278 @@
+"""The several-device exchange on one GPU: per-rank pointer tables and CUDA
+IPC, against the single-device path bit for bit.
+
+* In one process, D "devices" are D disjoint sets of buffers (each with its
+  own slot and gradient arenas) and D peer plans; the pulls of the copy-out
+  and of the reductions read across those allocations exactly as they read
+  peers' memory, and every result equals the single-device group's rows.
+* Across processes, D processes on the one GPU map each other's buffers with
+  CUDA IPC (fully_sharded_shard_b200.peer.PeerGroup) and run two fused steps;
+  gloo barriers order the phases on the host (no kernel waits on another).
+
+The single-device path is itself pinned to the oracle elsewhere; the reduced
+gradient is also checked against the oracle here.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import fully_sharded_shard_b200.workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(name, shapes, N, op=W.AVG, zero=()):
+    g = W.Group(name, [tuple(s) for s in shapes], [f"p{i}" for i in range(len(shapes))],
+                zero_grad=list(zero))
+    return W.Workload(name, N, [g], op, 0, "normal", 0.02, 1e-3, steps=2)
+
+
+@pytest.fixture(scope="module")
+def H():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from tests import _harness
+    return _harness
+
+
+def run_group_peer(H, wl, grp, D, *, steps=2, oracle_check=True, tag=()):
+    """Every stage of D emulated devices against the single-device group."""
+    from fully_sharded_shard_b200 import abi
+    from fully_sharded_shard_b200.peer import rank_pointer_tables
+    import oracle
+    N, op = wl.N, wl.op
+    L = N // D
+    g = abi.fsdp_plan_group(grp.shapes, N)
+    S, A = g.S, g.P_arena
+    full = torch.empty(max(A, 1), device="cuda")
+    W.fill_master(full, wl, grp.name, *tag)
+    master = torch.empty(max(N * S, 1), device="cuda")
+    abi.fsdp_shard_params(g, full, master)
+    ref = {"p": master[:N * S].clone(), "m": torch.zeros(N * S, device="cuda"),
+           "v": torch.zeros(N * S, device="cuda")}
+    pps = [abi.fsdp_peer_plan(g, D, d) for d in range(D)]
+    assert [(pp.L, pp.r0) for pp in pps] == [(L, d * L) for d in range(D)]
+    slots = [H.Guarded(L * S, torch.bfloat16) for _ in range(D)]
+    gbufs = [H.Guarded(L * A, torch.bfloat16) for _ in range(D)]
+    ag_ptrs, gr_ptrs = rank_pointer_tables([s.t.data_ptr() for s in slots],
+                                           [b.t.data_ptr() for b in gbufs], L, S, A)
+    for pp in pps:
+        abi.fsdp_peer_set_sources(pp, ag_ptrs, gr_ptrs)
+    dev = [{"p": ref["p"][d * L * S:(d + 1) * L * S].clone(),
+            "m": torch.zeros(L * S, device="cuda"), "v": torch.zeros(L * S, device="cuda")}
+           for d in range(D)]
+    hp = dict(W.ADAMW_DEFAULTS)
+    sentinel = 0x3BEF
+
+    def gathered_and_copied_out(ag_ref):
+        """Copy-out on every device from the slots; the reference copy-out of
+        the single-device all-gather buffer; compare."""
+        arena_ref = torch.full((max(A, 1),), sentinel, dtype=torch.int16, device="cuda")
+        abi.fsdp_copy_out(g, ag_ref, arena_ref.view(torch.bfloat16)[:A] if A else arena_ref.view(torch.bfloat16))
+        got = torch.cat([s.t.view(torch.int16) for s in slots]) if S else None
+        if S:
+            assert torch.equal(got, ag_ref.view(torch.int16)[:N * S]), "slots != all-gather buffer"
+        for d in range(D):
+            arena = H.Guarded(A, torch.bfloat16)
+            arena.t.view(torch.int16).fill_(sentinel)
+            abi.fsdp_peer_copy_out(pps[d], arena.t)
+            torch.cuda.synchronize()
+            assert arena.guards_intact()
+            assert torch.equal(arena.t.view(torch.int16), arena_ref[:A]), f"device {d} copy-out"
+
+    # step 0: copy-in on every device, then the pulls of the copy-out
+    for d in range(D):
+        abi.fsdp_peer_copy_in(pps[d], dev[d]["p"], slots[d].t)
+    ag_ref = torch.empty(max(N * S, 1), dtype=torch.bfloat16, device="cuda")
+    abi.fsdp_copy_in(g, ref["p"], ag_ref)
+    torch.cuda.synchronize()
+    gathered_and_copied_out(ag_ref)
+    p = oracle.plan(grp.shapes, N) if oracle_check else None
+    for step in range(1, steps + 1):
+        grads = H.make_grads(g, wl, grp, step, tag)
+        for d in range(D):
+            gbufs[d].t.copy_(grads[d * L:(d + 1) * L].reshape(-1))
+        # the reduce-scatter pulls
+        red_ref = torch.empty(max(N * S, 1), device="cuda")
+        abi.fsdp_rs_reduce(g, grads, op, red_ref)
+        reds = [H.Guarded(L * S, torch.float32) for _ in range(D)]
+        for d in range(D):
+            abi.fsdp_peer_rs_reduce(pps[d], op, reds[d].t)
+        torch.cuda.synchronize()
+        for d in range(D):
+            assert reds[d].guards_intact()
+            assert torch.equal(reds[d].t.view(torch.int32),
+                               red_ref[d * L * S:(d + 1) * L * S].view(torch.int32)), \
+                f"device {d} reduce-scatter, step {step}"
+        if oracle_check:
+            red_o = oracle.reduce_scatter(p, H.u16(grads), op)
+            assert H.bits_equal(H.f32(red_ref[:N * S]), red_o)
+        # the unfused AdamW of the local shards, on copies of the state
+        full_cp = {k: t.clone() for k, t in ref.items()}
+        abi.fsdp_adamw_step(g, full_cp["p"], full_cp["m"], full_cp["v"], red_ref[:N * S],
+                            step=step, **hp)
+        for d in range(D):
+            cp = {k: t.clone() for k, t in dev[d].items()}
+            abi.fsdp_peer_adamw_step(pps[d], cp["p"], cp["m"], cp["v"], reds[d].t, step=step, **hp)
+            torch.cuda.synchronize()
+            for k in ("p", "m", "v"):
+                assert torch.equal(cp[k].view(torch.int32),
+                                   full_cp[k][d * L * S:(d + 1) * L * S].view(torch.int32)), \
+                    f"device {d} adamw {k}"
+        del full_cp
+        # the fused update with the next copy-in into each device's own slot
+        red2 = [H.Guarded(L * S, torch.float32) for _ in range(D)]
+        for d in range(D):
+            abi.fsdp_peer_rs_adamw_step(pps[d], op, dev[d]["p"], dev[d]["m"], dev[d]["v"],
+                                        step=step, ag_next=slots[d].t, reduced=red2[d].t, **hp)
+        red2_ref = torch.empty(max(N * S, 1), device="cuda")
+        abi.fsdp_rs_adamw_step(g, grads, op, ref["p"], ref["m"], ref["v"], step=step,
+                               ag_next=ag_ref, reduced=red2_ref, **hp)
+        torch.cuda.synchronize()
+        for d in range(D):
+            assert slots[d].guards_intact() and red2[d].guards_intact()
+            rows = slice(d * L * S, (d + 1) * L * S)
+            for k in ("p", "m", "v"):
+                assert torch.equal(dev[d][k].view(torch.int32), ref[k][rows].view(torch.int32)), \
+                    f"device {d} fused {k}, step {step}"
+            assert torch.equal(red2[d].t.view(torch.int32), red2_ref[rows].view(torch.int32))
+        # the next step's all-gather: pulls of the slots the fused update wrote
+        gathered_and_copied_out(ag_ref)
+        del grads
+    for pp in pps:
+        pp.destroy()
+    g.destroy()
+
+
+PEER = [
+    (_wl("peer_ragged_n4", [(7, 3), (5,), (1, 32), (1,), (0, 4), (13, 9), (2, 2)], 4, op=W.SUM), (1, 2, 4)),
+    (_wl("peer_n6_odd", [(1001, 3), (17,), (3, 4099), (8191, 1)], 6, op=W.SUM_THEN_DIV), (2, 3, 6)),
+    (_wl("peer_n12", [(37, 100), (6,), (1999, 31)], 12), (3, 4, 12)),
+    (_wl("peer_n2_shift", [(3,), (9001, 5), (7, 1), (16385,)], 2, zero=[1]), (1, 2)),
+    (_wl("peer_n64", [(129, 7), (64,), (1, 5), (300,)], 64), (8, 64)),
+    (W.tiny_mlp(), (2,)),
+    (W.uneven(8), (2, 3, 6)),
+    (W.moe(8), (2, 8)),
+]
+
+
+@pytest.mark.parametrize("case", PEER, ids=[c[0].name for c in PEER])
+def test_peer_pulls_equal_single_device(H, case):
+    wl, Ds = case
+    for grp in wl.groups:
+        for D in Ds:
+            run_group_peer(H, wl, grp, D, steps=2, oracle_check=(D == Ds[-1]))
+
+
+def test_peer_full_size_llama7b_block_eight_devices(H):
+    wl = W.llama7b()
+    run_group_peer(H, wl, wl.groups[0], 8, steps=1, oracle_check=False)
+
+
+def test_peer_plan_rejects_bad_splits(H):
+    from fully_sharded_shard_b200 import abi
+    g = abi.fsdp_plan_group([(10, 3)], 6)
+    for D, d in ((4, 0), (0, 0), (3, 3), (3, -1)):
+        with pytest.raises(abi.FsdpError) as e:
+            abi.fsdp_peer_plan(g, D, d)
+        assert e.value.status == abi.FSDP_EINVAL
+    big = abi.fsdp_plan_group([(10, 3)], 128)
+    with pytest.raises(abi.FsdpError):
+        abi.fsdp_peer_plan(big, 2, 0)  # more ranks than a table holds
+    pp = abi.fsdp_peer_plan(g, 3, 1)
+    arena = torch.empty(g.P_arena, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(abi.FsdpError) as e:
+        abi.fsdp_peer_copy_out(pp, arena)  # no tables yet
+    assert e.value.status == abi.FSDP_ESTATE
+    buf = torch.empty(64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(abi.FsdpError) as e:  # a gradient arena must be 16-byte aligned
+        abi.fsdp_peer_set_sources(pp, None, [buf.data_ptr() + 2] * 6)
+    assert e.value.status == abi.FSDP_EALIGN
+    pp.destroy()
+    g.destroy()
+    big.destroy()
+
+
+# ---------------------------------------------------------------------------
+# several processes on the one GPU, CUDA IPC between them
+# ---------------------------------------------------------------------------
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _ipc_worker(rank, port, D, case_name, result_dir):
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=D, timeout=datetime.timedelta(seconds=120))
+    msg = "ok"
+    try:
+        torch.cuda.set_device(0)
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200.peer import PeerGroup
+        from tests import _harness as H
+        wl = {"uneven": W.uneven(16), "tiny": W.tiny_mlp(), "moe": W.moe(16)}[case_name]
+        grp = wl.groups[0]
+        N, op = wl.N, wl.op
+        pgrp = PeerGroup(grp.shapes, N, device="cuda:0")
+        g, S, A, L, r0 = pgrp.g, pgrp.S, pgrp.P_arena, pgrp.L, pgrp.r0
+        rows = slice(r0 * S, (r0 + L) * S)
+        full = torch.empty(max(A, 1), device="cuda")
+        W.fill_master(full, wl, grp.name)
+        master = torch.empty(max(N * S, 1), device="cuda")
+        abi.fsdp_shard_params(g, full, master)
+        ref = {"p": master[:N * S].clone(), "m": torch.zeros(N * S, device="cuda"),
+               "v": torch.zeros(N * S, device="cuda")}
+        mine = {k: t[rows].clone() for k, t in ref.items()}
+        hp = dict(W.ADAMW_DEFAULTS)
+        ag_ref = torch.empty(max(N * S, 1), dtype=torch.bfloat16, device="cuda")
+        abi.fsdp_copy_in(g, ref["p"], ag_ref)
+        pgrp.copy_in(mine["p"])
+        for step in range(1, 3):
+            pgrp.barrier()                       # every slot written
+            arena = torch.full((max(A, 1),), 0x3BEF, dtype=torch.int16, device="cuda")
+            pgrp.copy_out(arena.view(torch.bfloat16)[:A])
+            arena_ref = torch.full((max(A, 1),), 0x3BEF, dtype=torch.int16, device="cuda")
+            abi.fsdp_copy_out(g, ag_ref, arena_ref.view(torch.bfloat16)[:A])
+            grads = H.make_grads(g, wl, grp, step)
+            pgrp.grads.copy_(grads[r0:r0 + L])
+            pgrp.barrier()                       # every copy-out done, every gradient written
+            red = torch.empty(max(L * S, 1), device="cuda")
+            pgrp.rs_adamw_step(op, mine["p"], mine["m"], mine["v"], reduced=red, step=step, **hp)
+            red_ref = torch.empty(max(N * S, 1), device="cuda")
+            abi.fsdp_rs_adamw_step(g, grads, op, ref["p"], ref["m"], ref["v"], step=step,
+                                   ag_next=ag_ref, reduced=red_ref, **hp)
+            torch.cuda.synchronize()
+            if not torch.equal(arena, arena_ref):
+                msg = f"copy-out differs at step {step}"
+                break
+            bad = [k for k in ("p", "m", "v")
+                   if not torch.equal(mine[k].view(torch.int32), ref[k][rows].view(torch.int32))]
+            if bad or not torch.equal(red[:L * S].view(torch.int32), red_ref[rows].view(torch.int32)):
+                msg = f"fused update differs at step {step}: {bad or 'reduced'}"
+                break
+            if not torch.equal(pgrp.ag_slot.view(torch.int16), ag_ref[rows].view(torch.int16)):
+                msg = f"next copy-in differs at step {step}"
+                break
+        pgrp.close()
+    except Exception as e:  # reported through the result file
+        msg = f"error: {type(e).__name__}: {e}"
+    finally:
+        with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+            f.write(msg + "\n")
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("D,case", [(2, "tiny"), (2, "uneven"), (3, "uneven"), (4, "moe")])
+def test_peer_group_over_cuda_ipc_processes(H, tmp_path, D, case):
+    import torch.multiprocessing as mp
+    mp.spawn(_ipc_worker, args=(_free_port(), D, case, str(tmp_path)), nprocs=D, join=True)
+    for r in range(D):
+        assert open(tmp_path / f"r{r}.txt").read().strip() == "ok", f"process {r}"
