@@ -203,25 +203,40 @@ class ClockSampler:
                 "power_w_max": maxp}
 
 
-def kernels_hash() -> str:
-    """Hash of every kernel source file (the .cu files and the device header)."""
+# The file each profiled kernel is compiled from (with the device header and
+# the internal header every kernel file includes).
+KERNEL_FILES = {
+    "k_copy_in": "fsdpk_gather.cu", "k_copy_out": "fsdpk_gather.cu",
+    "k_fp8_copy_in": "fsdpk_gather.cu", "k_fp8_amax": "fsdpk_gather.cu",
+    "k_copy_out_tab": "fsdpk_gather.cu",
+    "k_reduce_units": "fsdpk_reduce.cu", "k_accumulate": "fsdpk_reduce.cu",
+    "k_reduce_acc": "fsdpk_reduce.cu", "k_reduce_units_tab": "fsdpk_reduce.cu",
+    "k_adamw": "fsdpk_update.cu", "k_rs_adamw": "fsdpk_update.cu",
+    "k_rs_adamw_fp8": "fsdpk_update.cu",
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources `kernel` is compiled from: its .cu file, the device
+    header and the internal header."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(KERNELS_DIR)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(KERNELS_DIR, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in (KERNEL_FILES[kernel], "fsdpk_device.cuh", "fsdpk_internal.h"):
+        with open(os.path.join(KERNELS_DIR, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
-    when it is absent or the kernels changed since it was captured."""
+    when it is absent or the kernel's sources changed since it was captured."""
     try:
         with open(TRAFFIC_JSON) as f:
             rec = json.load(f)
+        if rec.get("workload") != workload:
+            return None
+        if rec["sources_sha256_16"][kernel] != kernel_source_hash(kernel):
+            return None
     except Exception:
-        return None
-    if rec.get("kernels_sha256_16") != kernels_hash() or rec.get("workload") != workload:
         return None
     k = rec.get("per_launch_bytes", {}).get(kernel)
     return float(k) if k is not None else None
@@ -1036,10 +1051,55 @@ def run_latency(device, reps: int = 200):
         graph.replay()
         graph_us = timed(graph.replay)
     del graph
+
+    # the same step through fsdp_group_step: one call per group, and one
+    # single-CTA launch for a group this small
+    state = {"t": 0}
+
+    def single_call_step():
+        state["t"] += 1
+        for gi, master, m, v, pj in model.instances:
+            g = model.plans[gi]
+            abi.fsdp_group_step(g, master, m, v, model.grads[gi][pj], wl.op, step=state["t"],
+                                ag=model.ag, arena=model.arena, reduced=model.reduced,
+                                stream=stream, **hp)
+
+    for _ in range(10):
+        single_call_step()
+    t0 = time.perf_counter()
+    single_us = timed(single_call_step)
+    single_host_us = (time.perf_counter() - t0) * 1e6 / reps
+
+    def graphed_single():
+        abi.fsdp_adamw_prepare(ds, stream=stream, **hp)
+        for gi, master, m, v, pj in model.instances:
+            g = model.plans[gi]
+            abi.fsdp_group_step_dev(g, master, m, v, model.grads[gi][pj], wl.op, ds,
+                                    ag=model.ag, arena=model.arena, reduced=model.reduced,
+                                    stream=stream)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        graphed_single()
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        graph.replay()
+        graph_single_us = timed(graph.replay)
+    del graph
+    n_small = sum(1 for gi, *_ in model.instances
+                  if wl.N * model.plans[gi].S <= abi.FSDP_SMALL_STEP_ELEMS)
+    single_launches = sum(1 if wl.N * model.plans[gi].S <= abi.FSDP_SMALL_STEP_ELEMS else 4
+                          for gi, *_ in model.instances)
     return {"workload": wl.name, "launches_per_step": model.launches_per_step,
             "eager_us_per_step": round(eager_us, 2), "eager_host_us_per_step": round(host_us, 2),
             "graph_us_per_step": round(graph_us, 2),
-            "graph_launches_per_step": model.launches_per_step + 1}
+            "graph_launches_per_step": model.launches_per_step + 1,
+            "group_step": {"groups_in_one_launch": n_small,
+                           "launches_per_step": single_launches,
+                           "eager_us_per_step": round(single_us, 2),
+                           "eager_host_us_per_step": round(single_host_us, 2),
+                           "graph_us_per_step": round(graph_single_us, 2),
+                           "graph_launches_per_step": single_launches + 1}}
 
 
 def run_e2e(args, model, device, stream, ws):

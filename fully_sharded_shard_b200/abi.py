@@ -102,6 +102,11 @@ def _load() -> ctypes.CDLL:
     L.fsdp_rs_adamw_step_dev.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
+    L.fsdp_group_step.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.POINTER(AdamWHparams), vp, vp,
+                                  vp, vp]
+    L.fsdp_group_step.restype = ctypes.c_int
+    L.fsdp_group_step_dev.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp]
+    L.fsdp_group_step_dev.restype = ctypes.c_int
     L.fsdp_peer_plan.argtypes = [vp, i32, i32, ctypes.POINTER(vp)]
     L.fsdp_peer_local_ranks.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fsdp_peer_set_sources.argtypes = [vp, vp, vp]
@@ -283,6 +288,41 @@ def fsdp_rs_adamw_step(g: Group, grads: torch.Tensor, op: int, master: torch.Ten
                                    ctypes.byref(hp), _ptr(ag_next, _B16, n, "ag_next"),
                                    _ptr(reduced, _F32, n, "reduced"),
                                    _stream(stream, master)), "fsdp_rs_adamw_step")
+
+
+FSDP_SMALL_STEP_ELEMS = 16384
+
+
+def fsdp_group_step(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                    grads: torch.Tensor, op: int, *, lr: float, beta1: float, beta2: float,
+                    eps: float, weight_decay: float, step: int, ag: torch.Tensor,
+                    arena: torch.Tensor, reduced: torch.Tensor, stream=None):
+    """The whole step of one group (copy-in, copy-out, reduce-scatter,
+    AdamW); one launch for groups of at most FSDP_SMALL_STEP_ELEMS padded
+    elements."""
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = g.N * g.S
+    _check(_lib.fsdp_group_step(g.handle, _ptr(master, _F32, n, "master"), _ptr(m, _F32, n, "m"),
+                                _ptr(v, _F32, n, "v"),
+                                _ptr(grads, _B16, g.N * g.P_arena, "grads"), int(op),
+                                ctypes.byref(hp), _ptr(ag, _B16, n, "ag"),
+                                _ptr(arena, _B16, g.P_arena, "arena"),
+                                _ptr(reduced, _F32, n, "reduced"), _stream(stream, master)),
+           "fsdp_group_step")
+
+
+def fsdp_group_step_dev(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                        grads: torch.Tensor, op: int, ds: "DeviceStep", *, ag: torch.Tensor,
+                        arena: torch.Tensor, reduced: torch.Tensor, stream=None):
+    n = g.N * g.S
+    _check(_lib.fsdp_group_step_dev(g.handle, _ptr(master, _F32, n, "master"),
+                                    _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                    _ptr(grads, _B16, g.N * g.P_arena, "grads"), int(op),
+                                    _ptr(ds.scalars, _F32, 8, "scalars"),
+                                    _ptr(ag, _B16, n, "ag"), _ptr(arena, _B16, g.P_arena, "arena"),
+                                    _ptr(reduced, _F32, n, "reduced"), _stream(stream, master)),
+           "fsdp_group_step_dev")
 
 
 def fsdp_grad_accumulate(g: Group, grads: torch.Tensor, acc: torch.Tensor, first: bool,

@@ -429,6 +429,58 @@ int fsdp_rs_adamw_step(fsdp_group_t g, const uint16_t* grads, int32_t op, float*
     return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
 }
 
+namespace {
+
+int group_step(fsdp_group_t g, float* master, float* m, float* v, const uint16_t* grads,
+               int32_t op, const fsdpk::AdamScalars& sc, const fsdpk::AdamScalars* sc_dev,
+               uint16_t* ag, uint16_t* arena, float* reduced, fsdp_stream_t stream) {
+    if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
+    const int64_t NS = (int64_t)g->N * g->S;
+    if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr || ag == nullptr ||
+                   reduced == nullptr))
+        return FSDP_EINVAL;
+    if (g->P > 0 && (grads == nullptr || arena == nullptr)) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grads) ||
+        !aligned16(ag) || !aligned16(arena) || !aligned16(reduced) || !aligned16(sc_dev))
+        return FSDP_EALIGN;
+    int st = check_device(g);
+    if (st != FSDP_OK) return st;
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (NS <= FSDP_SMALL_STEP_ELEMS) {
+        e = fsdpk::launch_small_step(*g, master, m, v, grads, op, ag, arena, reduced, sc, sc_dev,
+                                     s);
+    } else {
+        e = fsdpk::launch_copy_in(*g, master, ag, s);
+        if (e == cudaSuccess) e = fsdpk::launch_copy_out(*g, ag, arena, s);
+        if (e == cudaSuccess) e = fsdpk::launch_rs_fused(*g, grads, op, reduced, s);
+        if (e == cudaSuccess) e = fsdpk::launch_adamw(*g, master, m, v, reduced, sc, s, sc_dev);
+    }
+    return e == cudaSuccess ? FSDP_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+int fsdp_group_step(fsdp_group_t g, float* master, float* m, float* v, const uint16_t* grads,
+                    int32_t op, const fsdp_adamw_hparams* hp, uint16_t* ag, uint16_t* arena,
+                    float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr || hp == nullptr) return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!adam_scalars(hp, &sc)) return FSDP_EINVAL;
+    return group_step(g, master, m, v, grads, op, sc, nullptr, ag, arena, reduced, stream);
+}
+
+int fsdp_group_step_dev(fsdp_group_t g, float* master, float* m, float* v,
+                        const uint16_t* grads, int32_t op,
+                        const fsdp_adamw_dev_scalars* scalars_dev, uint16_t* ag,
+                        uint16_t* arena, float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr || scalars_dev == nullptr) return FSDP_EINVAL;
+    const fsdpk::AdamScalars none{};
+    return group_step(g, master, m, v, grads, op, none,
+                      reinterpret_cast<const fsdpk::AdamScalars*>(scalars_dev), ag, arena,
+                      reduced, stream);
+}
+
 int fsdp_grad_accumulate(fsdp_group_t g, const uint16_t* grads, float* acc, int32_t first,
                          fsdp_stream_t stream) {
     if (g == nullptr) return FSDP_EINVAL;

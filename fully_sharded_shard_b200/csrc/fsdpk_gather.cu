@@ -131,11 +131,11 @@ __device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_a
     }
 }
 
-// TAB: rank r's rows come from ag_tab[r], the start of rank r's [S] slot row
-// (a pull from wherever that rank's slot lives), instead of ag + r * S.
+// TAB: unit ui's rows come from unit_src[ui] (a pull from wherever that
+// rank's slot lives, resolved on the host), instead of ag + shard_pos.
 template <bool TAB>
 __global__ void __launch_bounds__(kThreads, 5)
-k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ ag_tab, int64_t S,
+k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ unit_src,
            uint16_t* __restrict__ arena, const Unit* __restrict__ units, int64_t n_units) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
@@ -143,8 +143,7 @@ k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ 
         uint16_t* dst_run = arena + u.arena_pos;
         const uint16_t* src_run;
         if constexpr (TAB) {
-            const int64_t r = u.shard_pos / S;  // a unit never crosses a rank's row
-            src_run = ag_tab[r] + (u.shard_pos - r * S);
+            src_run = unit_src[ui];
         } else {
             src_run = ag + u.shard_pos;
         }
@@ -340,15 +339,15 @@ cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* a
                             cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
     k_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
-        ag, nullptr, g.S, arena, g.d_units, g.n_real_units);
+        ag, nullptr, arena, g.d_units, g.n_real_units);
     return cudaGetLastError();
 }
 
-cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* ag_tab,
+cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* unit_src,
                                 uint16_t* arena, cudaStream_t st) {
     if (parent.n_real_units == 0) return cudaSuccess;
     k_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
-        nullptr, ag_tab, parent.S, arena, parent.d_units, parent.n_real_units);
+        nullptr, unit_src, arena, parent.d_units, parent.n_real_units);
     return cudaGetLastError();
 }
 

@@ -85,8 +85,8 @@ struct fsdp_peer {
     int32_t n_devices = 0;
     int32_t index = 0;
     int64_t r0 = 0;
-    // one device allocation: N all-gather slot row pointers, then N gradient
-    // arena pointers (set by fsdp_peer_set_sources)
+    // one device allocation (set by fsdp_peer_set_sources): N gradient arena
+    // pointers, then one source pointer per copy-out unit of the parent
     void* dev_tab = nullptr;
     bool have_ag = false;
     bool have_grads = false;
@@ -145,18 +145,25 @@ cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Un
                                   int64_t n_units, const uint16_t* grads, int op, float* reduced,
                                   cudaStream_t st);
 
-// The exchange steps over per-rank pointer tables (device arrays of N
-// pointers): the copy-out pulling rank r's rows from ag_tab[r] (the start of
-// rank r's [S] slot row), and the reductions folding rank r's gradient arena
-// at grad_tab[r].  `parent` supplies the copy-out units, `local` the units of
-// the local destination ranks.
-cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* ag_tab,
+// The exchange steps over pointer tables in device memory: the copy-out
+// pulling each of the parent's real units from unit_src[unit] (inside the
+// slot row of the unit's rank), and the reductions folding rank r's gradient
+// arena at grad_tab[r] (N pointers).  `parent` supplies the copy-out units,
+// `local` the units of the local destination ranks.
+cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* unit_src,
                                 uint16_t* arena, cudaStream_t st);
 cudaError_t launch_rs_fused_tab(const fsdp_group& local, const uint16_t* const* grad_tab, int op,
                                 float* reduced, cudaStream_t st);
 cudaError_t launch_rs_adamw_tab(const fsdp_group& local, const uint16_t* const* grad_tab, int op,
                                 float* master, float* m, float* v, const AdamScalars& sc,
                                 uint16_t* ag_next, float* reduced, cudaStream_t st);
+
+// The whole step of a small group (copy-in, copy-out, fused reduce-scatter,
+// AdamW) in one single-CTA launch (fsdpk_step.cu).
+cudaError_t launch_small_step(const fsdp_group& g, float* master, float* m, float* v,
+                              const uint16_t* grads, int op, uint16_t* ag, uint16_t* arena,
+                              float* reduced, const AdamScalars& sc, const AdamScalars* sc_dev,
+                              cudaStream_t st);
 
 // Fused reduce-scatter + AdamW (+ optional next-step copy-in into ag_next and
 // optional reduced-gradient output).

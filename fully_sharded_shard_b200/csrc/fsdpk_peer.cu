@@ -26,11 +26,11 @@ int cuda_status(cudaError_t e) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-const uint16_t* const* ag_table(const fsdp_peer* p) {
+const uint16_t* const* grad_table(const fsdp_peer* p) {
     return static_cast<const uint16_t* const*>(p->dev_tab);
 }
 
-const uint16_t* const* grad_table(const fsdp_peer* p) {
+const uint16_t* const* unit_src_table(const fsdp_peer* p) {
     return static_cast<const uint16_t* const*>(p->dev_tab) + p->parent->N;
 }
 
@@ -79,7 +79,8 @@ int fsdp_peer_plan(fsdp_group_t g, int32_t n_devices, int32_t device_index, fsdp
     st = fsdpk::build_rank_tables(&l, p->r0, p->r0 + L);
     if (st == FSDP_OK) st = fsdpk::upload_tables(&l);
     if (st == FSDP_OK) {
-        cudaError_t e = cudaMalloc(&p->dev_tab, 2 * (size_t)g->N * sizeof(void*));
+        cudaError_t e = cudaMalloc(
+            &p->dev_tab, ((size_t)g->N + (size_t)g->n_real_units) * sizeof(void*));
         if (e != cudaSuccess) {
             cudaGetLastError();
             p->dev_tab = nullptr;
@@ -118,11 +119,25 @@ int fsdp_peer_set_sources(fsdp_peer_t p, const uint16_t* const* ag_rank_ptrs,
     if (st != FSDP_OK) return st;
     const size_t bytes = (size_t)N * sizeof(void*);
     cudaError_t e = cudaSuccess;
-    if (ag_rank_ptrs != nullptr)
-        e = cudaMemcpy(p->dev_tab, ag_rank_ptrs, bytes, cudaMemcpyHostToDevice);
+    if (ag_rank_ptrs != nullptr && p->parent->n_real_units > 0) {
+        // each copy-out unit's source: its rank's slot row + its offset in it
+        std::vector<const uint16_t*> src;
+        try {
+            src.resize((size_t)p->parent->n_real_units);
+        } catch (...) {
+            return FSDP_ENOMEM;
+        }
+        const int64_t S = p->parent->S;
+        for (int64_t ui = 0; ui < p->parent->n_real_units; ++ui) {
+            const int64_t pos = p->parent->units[(size_t)ui].shard_pos;
+            const int64_t r = pos / S;  // a unit never crosses a rank's row
+            src[(size_t)ui] = ag_rank_ptrs[r] + (pos - r * S);
+        }
+        e = cudaMemcpy(static_cast<char*>(p->dev_tab) + bytes, src.data(),
+                       src.size() * sizeof(void*), cudaMemcpyHostToDevice);
+    }
     if (e == cudaSuccess && grad_rank_ptrs != nullptr)
-        e = cudaMemcpy(static_cast<char*>(p->dev_tab) + bytes, grad_rank_ptrs, bytes,
-                       cudaMemcpyHostToDevice);
+        e = cudaMemcpy(p->dev_tab, grad_rank_ptrs, bytes, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_status(e);
     if (ag_rank_ptrs != nullptr) p->have_ag = true;
     if (grad_rank_ptrs != nullptr) p->have_grads = true;
@@ -160,7 +175,7 @@ int fsdp_peer_copy_out(fsdp_peer_t p, uint16_t* arena, fsdp_stream_t stream) {
     int st = fsdpk::check_plan_device(&p->local);
     if (st != FSDP_OK) return st;
     return cuda_status(
-        fsdpk::launch_copy_out_tab(*p->parent, ag_table(p), arena, (cudaStream_t)stream));
+        fsdpk::launch_copy_out_tab(*p->parent, unit_src_table(p), arena, (cudaStream_t)stream));
 }
 
 int fsdp_peer_rs_reduce(fsdp_peer_t p, int32_t op, float* reduced, fsdp_stream_t stream) {

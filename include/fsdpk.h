@@ -225,6 +225,35 @@ FSDP_API int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32
                        uint16_t* ag_next_or_null, float* reduced_or_null,
                        fsdp_stream_t stream);
 
+/* Groups with N*S at most this many elements run fsdp_group_step as one
+ * single-CTA launch. */
+#define FSDP_SMALL_STEP_ELEMS 16384
+
+/* The whole step of one group, stages 1-5 in the order of [MS] Working
+ * Principle: fsdp_copy_in of the pre-update master into ag, fsdp_copy_out of
+ * ag into arena, the fused fsdp_rs_reduce of grads into reduced, and
+ * fsdp_adamw_step with reduced.  Same bits as those four calls in turn.
+ * Groups with N*S <= FSDP_SMALL_STEP_ELEMS run as ONE launch of a single CTA
+ * (for them the launches, not the bytes, are the cost; a block barrier
+ * separates dependent stages); larger groups as the four stage kernels on
+ * `stream`.
+ *   master, m, v: fp32 [N][S] (updated); grads: bf16 [N][P_arena] (read);
+ *   op: an fsdp_reduce_op; hparams as for fsdp_adamw_step; ag: bf16 [N][S]
+ *   (written); arena: bf16 [P_arena] (written, gaps untouched); reduced:
+ *   fp32 [N][S] (written).  All 16-byte aligned.
+ * fsdp_group_step_dev takes the AdamW scalars from device memory (written
+ * by fsdp_adamw_prepare), for a step captured in a CUDA graph.
+ * Errors as for the four stage calls. */
+FSDP_API int fsdp_group_step(fsdp_group_t group, float* master, float* m, float* v,
+                             const uint16_t* grads, int32_t op,
+                             const fsdp_adamw_hparams* hparams, uint16_t* ag,
+                             uint16_t* arena, float* reduced, fsdp_stream_t stream);
+
+FSDP_API int fsdp_group_step_dev(fsdp_group_t group, float* master, float* m, float* v,
+                                 const uint16_t* grads, int32_t op,
+                                 const fsdp_adamw_dev_scalars* scalars_dev, uint16_t* ag,
+                                 uint16_t* arena, float* reduced, fsdp_stream_t stream);
+
 /* Gradient accumulation without sync ([ML] Other controls:
  * set_requires_gradient_sync(False) accumulates the unsharded gradients and
  * skips the reduce-scatter).  Each rank's unsharded gradient is accumulated in
@@ -420,7 +449,8 @@ FSDP_API int fsdp_peer_local_ranks(fsdp_peer_t peer, int32_t* L, int32_t* r0);
  * pointers, entry r = rank r's bf16 gradient arena (P_arena elements),
  * 16-byte aligned.  Either array may be NULL to keep the previous table.
  * Pointers may be this device's or mapped from peers; they are copied to the
- * device synchronously.  Errors: FSDP_EINVAL (NULL entry where S or
+ * device synchronously (the slot rows as one source pointer per copy-out
+ * work unit, resolved here, so the copy-out kernel does no rank lookup).  Errors: FSDP_EINVAL (NULL entry where S or
  * P_arena > 0), FSDP_EALIGN, FSDP_ECUDA. */
 FSDP_API int fsdp_peer_set_sources(fsdp_peer_t peer, const uint16_t* const* ag_rank_ptrs,
                                    const uint16_t* const* grad_rank_ptrs);

@@ -374,3 +374,81 @@ def test_checkpoint_resume_is_bit_exact(H, tmp_path):
     for x, y in zip(a, c):
         assert torch.equal(x.view(torch.int32), y.view(torch.int32))
     g.destroy()
+
+
+def _group_step_case(H, wl, grp, steps, graph):
+    """fsdp_group_step (eager, or its _dev form replayed from a CUDA graph)
+    against the four stage calls on a copy of the same state, bit for bit,
+    and its exact stages against the oracle."""
+    import oracle
+    from fully_sharded_shard_b200 import abi
+    N, op = wl.N, wl.op
+    g = abi.fsdp_plan_group(grp.shapes, N)
+    p = oracle.plan(grp.shapes, N)
+    NS, A = N * g.S, g.P_arena
+    full = torch.empty(max(A, 1), device="cuda")
+    W.fill_master(full, wl, grp.name)
+    hp = dict(W.ADAMW_DEFAULTS)
+
+    def state():
+        master = torch.empty(max(NS, 1), device="cuda")
+        abi.fsdp_shard_params(g, full, master)
+        return {"p": master, "m": torch.zeros(max(NS, 1), device="cuda"),
+                "v": torch.zeros(max(NS, 1), device="cuda"),
+                "ag": torch.empty(max(NS, 1), dtype=torch.bfloat16, device="cuda"),
+                "arena": torch.full((max(A, 1),), 0x3BEF, dtype=torch.int16,
+                                    device="cuda").view(torch.bfloat16),
+                "red": torch.empty(max(NS, 1), device="cuda")}
+    a, b = state(), state()
+    grads = [H.make_grads(g, wl, grp, t) for t in range(1, steps + 1)]
+    gbuf = torch.empty_like(grads[0])
+    if graph:
+        ds = abi.DeviceStep()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=s):
+            abi.fsdp_adamw_prepare(ds, **hp)
+            abi.fsdp_group_step_dev(g, a["p"], a["m"], a["v"], gbuf, op, ds, ag=a["ag"],
+                                    arena=a["arena"], reduced=a["red"])
+    for t in range(1, steps + 1):
+        if graph:
+            gbuf.copy_(grads[t - 1])
+            cg.replay()
+        else:
+            abi.fsdp_group_step(g, a["p"], a["m"], a["v"], grads[t - 1], op, step=t, ag=a["ag"],
+                                arena=a["arena"], reduced=a["red"], **hp)
+        abi.fsdp_copy_in(g, b["p"], b["ag"])
+        abi.fsdp_copy_out(g, b["ag"], b["arena"])
+        abi.fsdp_rs_reduce(g, grads[t - 1], op, b["red"])
+        abi.fsdp_adamw_step(g, b["p"], b["m"], b["v"], b["red"], step=t, **hp)
+        torch.cuda.synchronize()
+        for k in ("p", "m", "v", "red"):
+            assert torch.equal(a[k].view(torch.int32), b[k].view(torch.int32)), f"{k} step {t}"
+        for k in ("ag", "arena"):
+            assert torch.equal(a[k].view(torch.int16), b[k].view(torch.int16)), f"{k} step {t}"
+        red_o = oracle.reduce_scatter(p, H.u16(grads[t - 1]), op)
+        assert H.bits_equal(H.f32(a["red"][:NS]), red_o)
+    if graph:
+        assert int(ds.step.item()) == steps
+        del cg
+    g.destroy()
+
+
+GROUP_STEP = SMALL + [W.tiny_mlp(), W.uneven(64), W.moe(64)]
+
+
+@pytest.mark.parametrize("wl", GROUP_STEP, ids=[w.name for w in GROUP_STEP])
+def test_group_step_equals_the_four_stage_calls(H, wl):
+    from fully_sharded_shard_b200 import abi
+    for grp in wl.groups:
+        _group_step_case(H, wl, grp, steps=3, graph=False)
+    small = [grp for grp in wl.groups
+             if wl.N * abi.fsdp_plan_group(grp.shapes, wl.N).S <= abi.FSDP_SMALL_STEP_ELEMS]
+    for grp in small[:1]:
+        _group_step_case(H, wl, grp, steps=3, graph=True)
+
+
+@pytest.mark.parametrize("wl", GRID[:3], ids=[w.name for w in GRID[:3]])
+def test_group_step_single_launch_on_the_brute_force_grid(H, wl):
+    _group_step_case(H, wl, wl.groups[0], steps=2, graph=False)
