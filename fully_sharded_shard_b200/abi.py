@@ -102,6 +102,10 @@ def _load() -> ctypes.CDLL:
     L.fsdp_rs_adamw_step_dev.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
+    L.fsdp_copy_in_f32.argtypes = [vp, vp, vp, vp]
+    L.fsdp_copy_in_f32.restype = ctypes.c_int
+    L.fsdp_copy_out_f32.argtypes = [vp, vp, vp, vp]
+    L.fsdp_copy_out_f32.restype = ctypes.c_int
     L.fsdp_group_step.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.POINTER(AdamWHparams), vp, vp,
                                   vp, vp]
     L.fsdp_group_step.restype = ctypes.c_int
@@ -341,6 +345,21 @@ def fsdp_rs_reduce_accumulated(g: Group, grads: Optional[torch.Tensor], acc: tor
                                            _ptr(reduced, _F32, g.N * g.S, "reduced"),
                                            _stream(stream, reduced)),
            "fsdp_rs_reduce_accumulated")
+
+
+def fsdp_copy_in_f32(g: Group, master: torch.Tensor, ag32: torch.Tensor, stream=None):
+    """Copy-in with param_dtype fp32 (test mode: no cast)."""
+    n = g.N * g.S
+    _check(_lib.fsdp_copy_in_f32(g.handle, _ptr(master, _F32, n, "master"),
+                                 _ptr(ag32, _F32, n, "ag32"), _stream(stream, master)),
+           "fsdp_copy_in_f32")
+
+
+def fsdp_copy_out_f32(g: Group, ag32: torch.Tensor, arena32: torch.Tensor, stream=None):
+    """Copy-out with param_dtype fp32 (test mode: no cast)."""
+    _check(_lib.fsdp_copy_out_f32(g.handle, _ptr(ag32, _F32, g.N * g.S, "ag32"),
+                                  _ptr(arena32, _F32, g.P_arena, "arena32"),
+                                  _stream(stream, ag32)), "fsdp_copy_out_f32")
 
 
 def fsdp_copy_in_fp8(g: Group, master: torch.Tensor, ag8: torch.Tensor, scales: torch.Tensor,

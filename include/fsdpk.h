@@ -278,6 +278,19 @@ FSDP_API int fsdp_rs_reduce_accumulated(fsdp_group_t group, const uint16_t* grad
                                const float* acc, int32_t op, float* reduced,
                                fsdp_stream_t stream);
 
+/* The all-gather copy-in and copy-out with param_dtype fp32 (no
+ * MixedPrecisionPolicy: [ML] Mixed precision), a test mode: nothing is cast,
+ * so fsdp_copy_out_f32(fsdp_copy_in_f32(shard(x))) == x bit for bit.
+ *   fsdp_copy_in_f32: master fp32 [N][S] (read) -> ag32 fp32 [N][S] (written,
+ *   +0 in pad rows).  fsdp_copy_out_f32: ag32 -> arena32 fp32 [P_arena]
+ *   (written on real elements, gaps untouched).  16-byte aligned pointers.
+ * Algorithmic bytes: 8 per padded element (copy-in), 8 per real element
+ * (copy-out). */
+FSDP_API int fsdp_copy_in_f32(fsdp_group_t group, const float* master, float* ag32,
+                              fsdp_stream_t stream);
+FSDP_API int fsdp_copy_out_f32(fsdp_group_t group, const float* ag32, float* arena32,
+                               fsdp_stream_t stream);
+
 /* FP8 all-gather copy-in ("PyTorch FSDP2 Guide: Distributed LLM Training
  * with DTensor", Deep Dive, "2. Native FP8 Training with Float8Tensor":
  * parameters in FP8 E4M3, the all-gather moves raw FP8 bytes).  The page

@@ -9,6 +9,9 @@ as a failure.
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -18,6 +21,19 @@ from fully_sharded_shard_b200 import workloads as W
 
 GUARD = 64  # elements on each side (a multiple of 16 bytes for every dtype here)
 ADAM_TOL = 1e-6
+
+
+def log_parity(path: str, wl: W.Workload, group: W.Group, g: abi.Group, **rec) -> None:
+    """One JSON line per passed parity case, appended to $FSDPK_PARITY_LOG
+    when it is set: the case, the stages compared bit for bit and the largest
+    AdamW difference as a fraction of the tolerance."""
+    out = os.environ.get("FSDPK_PARITY_LOG")
+    if not out:
+        return
+    rec = {"path": path, "workload": wl.name, "group": group.name, "N": wl.N, "n_params": g.n,
+           "S": g.S, "P": g.P, **rec}
+    with open(out, "a") as f:
+        f.write(json.dumps(rec) + "\n")
 
 
 class Guarded:
@@ -214,6 +230,9 @@ def run_group(wl: W.Workload, group: W.Group, *, steps: int = 1, ops=None, stage
             ok, ratio = adam_close(f32(gbuf.t), obuf)
             report["adam_max_ratio"] = max(report["adam_max_ratio"], ratio)
             assert ok, f"adamw {name} step {step}: max |d|/tol = {ratio}"
+    log_parity("stages", wl, group, g, steps=steps, ops=[W.OP_NAMES[o] for o in ops],
+               bit_exact=["shard", "copy_in", "copy_out", "rs_fused"] + (["pack", "rs_staged"] if staged else []),
+               adam_max_ratio=report["adam_max_ratio"])
     g.destroy()
     return report
 
@@ -279,6 +298,9 @@ def run_group_fused(wl: W.Workload, group: W.Group, *, steps: int = 1, op=None,
         assert not np.any(diff & (f32(master.t).view(np.uint32) == master_o.view(np.uint32)))
         assert bf16_within_adam_band(ag_h[diff], ag_o[diff])
         del grads, ag, red, redu, agu
+    log_parity("fused", wl, group, g, steps=steps, ops=[W.OP_NAMES[op]],
+               bit_exact=["fused_vs_stages", "rs_vs_oracle"],
+               adam_max_ratio=report["adam_max_ratio"])
     g.destroy()
     return report
 
@@ -403,6 +425,10 @@ def run_group_fused_fp8(wl: W.Workload, group: W.Group, *, steps: int = 2, op=No
         scales_prev = scales_next.t.clone() if g.n else scales_prev
         scales_prev_o = sn_o
         del grads, ag8, red, redu, ag8u
+    log_parity("fused_fp8", wl, group, g, steps=steps, ops=[W.OP_NAMES[op]],
+               bit_exact=["fused_vs_stages", "rs_vs_oracle"],
+               adam_max_ratio=report["adam_max_ratio"],
+               fp8_code_diffs_vs_oracle=report["fp8_code_diffs"])
     g.destroy()
     return report
 
@@ -443,6 +469,8 @@ def run_group_accumulate(wl: W.Workload, group: W.Group, *, micro: int = 3, op=N
     abi.fsdp_rs_reduce_accumulated(g, None, acc.t, op, red2)
     torch.cuda.synchronize()
     assert bits_equal(f32(red2), red_o)
+    log_parity("accumulate", wl, group, g, microbatches=micro, ops=[W.OP_NAMES[op]],
+               bit_exact=["accumulate", "rs_accumulated", "rs_accumulated_no_last"])
     g.destroy()
 
 
@@ -483,4 +511,5 @@ def run_group_fp8(wl: W.Workload, group: W.Group, tag=()) -> None:
     arena_o = oracle.copy_out_fp8(p, ag8_o, np.full(p.P_arena, 0xA5, np.uint8))
     got = host_ar[G8:G8 + g.P_arena]
     assert np.array_equal(got, arena_o), f"fp8 copy-out: {int(np.sum(got != arena_o))} mismatches"
+    log_parity("fp8", wl, group, g, bit_exact=["scales", "fp8_copy_in", "fp8_copy_out"])
     g.destroy()

@@ -452,3 +452,41 @@ def test_group_step_equals_the_four_stage_calls(H, wl):
 @pytest.mark.parametrize("wl", GRID[:3], ids=[w.name for w in GRID[:3]])
 def test_group_step_single_launch_on_the_brute_force_grid(H, wl):
     _group_step_case(H, wl, wl.groups[0], steps=2, graph=False)
+
+
+F32 = SMALL + [W.tiny_mlp(), W.uneven(16), W.moe(16)]
+
+
+@pytest.mark.parametrize("wl", F32, ids=[w.name for w in F32])
+def test_fp32_param_dtype_all_gather_is_the_identity(H, wl):
+    """param_dtype fp32 (test mode): the copy-in equals the oracle's padded
+    shards bit for bit, and the copy-out of it gives back every parameter
+    exactly (all-gather(shard(x)) == x), gaps untouched."""
+    import numpy as np
+    import oracle
+    from fully_sharded_shard_b200 import abi
+    for grp in wl.groups:
+        g = abi.fsdp_plan_group(grp.shapes, wl.N)
+        p = oracle.plan(grp.shapes, wl.N)
+        NS, A = wl.N * g.S, g.P_arena
+        full = torch.empty(max(A, 1), device="cuda")
+        W.fill_master(full, wl, grp.name)
+        master = torch.empty(max(NS, 1), device="cuda")
+        abi.fsdp_shard_params(g, full, master)
+        ag32 = H.Guarded(NS, torch.float32)
+        abi.fsdp_copy_in_f32(g, master[:NS], ag32.t)
+        arena = H.Guarded(A, torch.float32)
+        abi.fsdp_copy_out_f32(g, ag32.t, arena.t)
+        torch.cuda.synchronize()
+        assert ag32.guards_intact() and arena.guards_intact()
+        full_h = H.f32(full)[:A]
+        shard_o = oracle.shard(p, full_h) if A else np.zeros(0, np.float32)
+        assert H.bits_equal(H.f32(ag32.t), shard_o), "fp32 copy-in: " + H.first_mismatch(H.f32(ag32.t), shard_o)
+        got = H.f32(arena.t)
+        real = np.zeros(A, bool)
+        for i in range(g.n):
+            real[g.arena_off[i]:g.arena_off[i] + g.numel[i]] = True
+        assert np.array_equal(got[real].view(np.uint32), full_h[real].view(np.uint32)), \
+            "fp32 all-gather is not the identity"
+        assert np.all(got[~real] == np.float32(-12345.5)), "fp32 copy-out wrote a gap"
+        g.destroy()
