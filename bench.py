@@ -1001,11 +1001,13 @@ def run_fp8(args, model, device, stream):
             "launches_per_step": 2 * len(model.instances) + 3 * len(model.instances)}
 
 
-def run_latency(device, reps: int = 200):
+def run_latency(device, reps: int = 200, graph_steps: int = 20):
     """The tiny MLP group (4 parameters, N = 2) is launch-bound: report the
     step latency in microseconds, eager (host-side AdamW step count) and as a
-    replayed CUDA graph of the whole step, whose AdamW step count lives in
-    device memory so that every replay is the next training step."""
+    replayed CUDA graph of `graph_steps` whole steps, whose AdamW step count
+    lives in device memory so that every step in it is the next training
+    step.  One graph holds several steps so that the device time per step is
+    measured, not the host's graph-launch rate."""
     import torch
     from fully_sharded_shard_b200 import abi
     from fully_sharded_shard_b200 import workloads as W
@@ -1045,11 +1047,12 @@ def run_latency(device, reps: int = 200):
 
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        graphed_step()
+        for _ in range(graph_steps):
+            graphed_step()
     torch.cuda.synchronize(device)
     with torch.cuda.stream(stream):
         graph.replay()
-        graph_us = timed(graph.replay)
+        graph_us = timed(graph.replay) / graph_steps
     del graph
 
     # the same step through fsdp_group_step: one call per group, and one
@@ -1080,11 +1083,12 @@ def run_latency(device, reps: int = 200):
 
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        graphed_single()
+        for _ in range(graph_steps):
+            graphed_single()
     torch.cuda.synchronize(device)
     with torch.cuda.stream(stream):
         graph.replay()
-        graph_single_us = timed(graph.replay)
+        graph_single_us = timed(graph.replay) / graph_steps
     del graph
     n_small = sum(1 for gi, *_ in model.instances
                   if wl.N * model.plans[gi].S <= abi.FSDP_SMALL_STEP_ELEMS)
@@ -1093,6 +1097,7 @@ def run_latency(device, reps: int = 200):
     return {"workload": wl.name, "launches_per_step": model.launches_per_step,
             "eager_us_per_step": round(eager_us, 2), "eager_host_us_per_step": round(host_us, 2),
             "graph_us_per_step": round(graph_us, 2),
+            "graph_steps_per_replay": graph_steps,
             "graph_launches_per_step": model.launches_per_step + 1,
             "group_step": {"groups_in_one_launch": n_small,
                            "launches_per_step": single_launches,

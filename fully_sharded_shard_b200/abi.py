@@ -294,7 +294,7 @@ def fsdp_rs_adamw_step(g: Group, grads: torch.Tensor, op: int, master: torch.Ten
                                    _stream(stream, master)), "fsdp_rs_adamw_step")
 
 
-FSDP_SMALL_STEP_ELEMS = 16384
+FSDP_SMALL_STEP_ELEMS = 8192
 
 
 def fsdp_group_step(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,

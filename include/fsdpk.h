@@ -227,7 +227,7 @@ FSDP_API int fsdp_rs_adamw_step(fsdp_group_t group, const uint16_t* grads, int32
 
 /* Groups with N*S at most this many elements run fsdp_group_step as one
  * single-CTA launch. */
-#define FSDP_SMALL_STEP_ELEMS 16384
+#define FSDP_SMALL_STEP_ELEMS 8192
 
 /* The whole step of one group, stages 1-5 in the order of [MS] Working
  * Principle: fsdp_copy_in of the pre-update master into ag, fsdp_copy_out of
