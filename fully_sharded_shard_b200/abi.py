@@ -122,6 +122,15 @@ def _load() -> ctypes.CDLL:
     L.fsdp_peer_adamw_step.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(AdamWHparams), vp]
     L.fsdp_peer_rs_adamw_step.argtypes = [vp, i32, vp, vp, vp, ctypes.POINTER(AdamWHparams),
                                           vp, vp, vp]
+    L.fsdp_peer_set_fp8_sources.argtypes = [vp, vp, vp]
+    L.fsdp_peer_copy_in_fp8_scaled.argtypes = [vp, vp, vp, vp, vp]
+    L.fsdp_peer_copy_out_fp8.argtypes = [vp, vp, vp]
+    L.fsdp_peer_rs_adamw_step_fp8.argtypes = [vp, i32, vp, vp, vp, ctypes.POINTER(AdamWHparams),
+                                              vp, vp, vp, vp, vp]
+    L.fsdp_peer_fp8_scales.argtypes = [vp, vp, vp]
+    for name in ("fsdp_peer_set_fp8_sources", "fsdp_peer_copy_in_fp8_scaled",
+                 "fsdp_peer_copy_out_fp8", "fsdp_peer_rs_adamw_step_fp8", "fsdp_peer_fp8_scales"):
+        getattr(L, name).restype = ctypes.c_int
     L.fsdp_ipc_alloc.argtypes = [i64, ctypes.POINTER(vp), ctypes.POINTER(IpcHandle)]
     L.fsdp_ipc_free.argtypes = [vp]
     L.fsdp_ipc_open.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(vp)]
@@ -558,6 +567,57 @@ def fsdp_peer_rs_adamw_step(pp: PeerPlan, op: int, master: torch.Tensor, m: torc
                                         ctypes.byref(hp), _ptr(ag_next, _B16, n, "ag_next"),
                                         _ptr(reduced, _F32, n, "reduced"),
                                         _stream(stream, master)), "fsdp_peer_rs_adamw_step")
+
+
+def fsdp_peer_set_fp8_sources(pp: PeerPlan, ag8_rank_ptrs: Sequence[int],
+                              amax_device_ptrs: Sequence[int]):
+    if len(ag8_rank_ptrs) != pp.N or len(amax_device_ptrs) != pp.n_devices:
+        raise ValueError("one slot row per rank and one amax array per device")
+    ag = (ctypes.c_void_p * pp.N)(*[int(x) for x in ag8_rank_ptrs])
+    am = (ctypes.c_void_p * pp.n_devices)(*[int(x) for x in amax_device_ptrs])
+    _check(_lib.fsdp_peer_set_fp8_sources(pp.handle, ag, am), "fsdp_peer_set_fp8_sources")
+
+
+def fsdp_peer_copy_in_fp8_scaled(pp: PeerPlan, master: torch.Tensor, scales: torch.Tensor,
+                                 ag8_slot: torch.Tensor, stream=None):
+    n = pp.L * pp.S
+    _check(_lib.fsdp_peer_copy_in_fp8_scaled(pp.handle, _ptr(master, _F32, n, "master"),
+                                             _ptr(scales, _F32, pp.n, "scales"),
+                                             _ptr(ag8_slot, _U8, n, "ag8_slot"),
+                                             _stream(stream, master)),
+           "fsdp_peer_copy_in_fp8_scaled")
+
+
+def fsdp_peer_copy_out_fp8(pp: PeerPlan, arena8: torch.Tensor, stream=None):
+    _check(_lib.fsdp_peer_copy_out_fp8(pp.handle, _ptr(arena8, _U8, pp.P_arena, "arena8"),
+                                       _stream(stream, arena8)), "fsdp_peer_copy_out_fp8")
+
+
+_U32 = (torch.int32, torch.uint32)
+
+
+def fsdp_peer_rs_adamw_step_fp8(pp: PeerPlan, op: int, master: torch.Tensor, m: torch.Tensor,
+                                v: torch.Tensor, *, lr: float, beta1: float, beta2: float,
+                                eps: float, weight_decay: float, step: int,
+                                scales_prev: torch.Tensor, ag8_next: torch.Tensor,
+                                amax_local: torch.Tensor, reduced: Optional[torch.Tensor] = None,
+                                stream=None):
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                      int(step))
+    n = pp.L * pp.S
+    _check(_lib.fsdp_peer_rs_adamw_step_fp8(pp.handle, int(op), _ptr(master, _F32, n, "master"),
+                                            _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                            ctypes.byref(hp),
+                                            _ptr(scales_prev, _F32, pp.n, "scales_prev"),
+                                            _ptr(ag8_next, _U8, n, "ag8_next"),
+                                            _ptr(amax_local, _U32, pp.n, "amax_local"),
+                                            _ptr(reduced, _F32, n, "reduced"),
+                                            _stream(stream, master)), "fsdp_peer_rs_adamw_step_fp8")
+
+
+def fsdp_peer_fp8_scales(pp: PeerPlan, scales_next: torch.Tensor, stream=None):
+    _check(_lib.fsdp_peer_fp8_scales(pp.handle, _ptr(scales_next, _F32, pp.n, "scales_next"),
+                                     _stream(stream, scales_next)), "fsdp_peer_fp8_scales")
 
 
 def fsdp_ipc_alloc(nbytes: int):

@@ -290,14 +290,22 @@ __device__ __forceinline__ uint4 shift_bytes16(const uint4& a, const uint4& b, i
                       __funnelshift_r(w2, w3, sh), __funnelshift_r(w3, w4, sh));
 }
 
+// TAB: unit ui's bytes come from unit_src[ui] (resolved on the host) instead
+// of ag8 + shard_pos.
+template <bool TAB>
 __global__ void __launch_bounds__(kThreads, 5)
-k_fp8_copy_out(const uint8_t* __restrict__ ag8, uint8_t* __restrict__ arena8,
-               const Unit* __restrict__ units, int64_t n_units) {
+k_fp8_copy_out(const uint8_t* __restrict__ ag8, const uint8_t* const* __restrict__ unit_src,
+               uint8_t* __restrict__ arena8, const Unit* __restrict__ units, int64_t n_units) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
         const int len = u.len;
         uint8_t* dst = arena8 + u.arena_pos;
-        const uint8_t* src = ag8 + u.shard_pos;
+        const uint8_t* src;
+        if constexpr (TAB) {
+            src = unit_src[ui];
+        } else {
+            src = ag8 + u.shard_pos;
+        }
         const int head = (int)head_to_16B(dst, len);
         if ((int)threadIdx.x < head) dst[threadIdx.x] = src[threadIdx.x];
         const int nv = (len - head) >> 4;
@@ -317,6 +325,18 @@ k_fp8_copy_out(const uint8_t* __restrict__ ag8, uint8_t* __restrict__ arena8,
     }
 }
 
+// scales[i] = 448 / max(max over the D devices of amax_d[i], 1e-12): the
+// per-parameter amax is the maximum of the devices' partial maxima (each
+// device saw only its own ranks' rows).
+__global__ void __launch_bounds__(kThreads)
+k_fp8_scales_from_parts(const unsigned* const* __restrict__ amax_tab, int D,
+                        float* __restrict__ scales, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float mx = 0.0f;
+    for (int d = 0; d < D; ++d) mx = fmaxf(mx, __uint_as_float(amax_tab[d][i]));
+    scales[i] = __fdiv_rn(448.0f, fmaxf(mx, 1e-12f));
+}
 
 }  // namespace
 
@@ -396,9 +416,24 @@ cudaError_t launch_copy_in_fp8_scaled(const fsdp_group& g, const float* master, 
 cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t* arena8,
                                 cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
-    k_fp8_copy_out<<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(ag8, arena8,
-                                                                              g.d_units,
-                                                                              g.n_real_units);
+    k_fp8_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
+        ag8, nullptr, arena8, g.d_units, g.n_real_units);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_out_fp8_tab(const fsdp_group& parent, const uint8_t* const* unit_src,
+                                    uint8_t* arena8, cudaStream_t st) {
+    if (parent.n_real_units == 0) return cudaSuccess;
+    k_fp8_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
+        nullptr, unit_src, arena8, parent.d_units, parent.n_real_units);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_scales_from_parts(const unsigned* const* amax_tab, int D, float* scales,
+                                         int n, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    k_fp8_scales_from_parts<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, st>>>(
+        amax_tab, D, scales, n);
     return cudaGetLastError();
 }
 

@@ -85,11 +85,14 @@ struct fsdp_peer {
     int32_t n_devices = 0;
     int32_t index = 0;
     int64_t r0 = 0;
-    // one device allocation (set by fsdp_peer_set_sources): N gradient arena
-    // pointers, then one source pointer per copy-out unit of the parent
+    // one device allocation: N gradient arena pointers, one bf16 source
+    // pointer per copy-out unit of the parent, one FP8 source pointer per
+    // copy-out unit, then n_devices amax-array pointers (set by
+    // fsdp_peer_set_sources and fsdp_peer_set_fp8_sources)
     void* dev_tab = nullptr;
     bool have_ag = false;
     bool have_grads = false;
+    bool have_fp8 = false;
 };
 
 namespace fsdpk {
@@ -157,6 +160,19 @@ cudaError_t launch_rs_fused_tab(const fsdp_group& local, const uint16_t* const* 
 cudaError_t launch_rs_adamw_tab(const fsdp_group& local, const uint16_t* const* grad_tab, int op,
                                 float* master, float* m, float* v, const AdamScalars& sc,
                                 uint16_t* ag_next, float* reduced, cudaStream_t st);
+// The FP8 forms: the byte copy-out pulling each unit from unit_src8[unit],
+// the fused update writing the local E4M3 slot and the local partial amax
+// bits, and the scales from the devices' partial amax arrays (amax_tab: a
+// device array of D pointers).
+cudaError_t launch_copy_out_fp8_tab(const fsdp_group& parent, const uint8_t* const* unit_src8,
+                                    uint8_t* arena8, cudaStream_t st);
+cudaError_t launch_rs_adamw_tab_fp8(const fsdp_group& local, const uint16_t* const* grad_tab,
+                                    int op, float* master, float* m, float* v,
+                                    const AdamScalars& sc, const float* scales_prev,
+                                    uint8_t* ag8_next, unsigned* amax_bits, float* reduced,
+                                    cudaStream_t st);
+cudaError_t launch_fp8_scales_from_parts(const unsigned* const* amax_tab, int D, float* scales,
+                                         int n, cudaStream_t st);
 
 // The whole step of a small group (copy-in, copy-out, fused reduce-scatter,
 // AdamW) in one single-CTA launch (fsdpk_step.cu).

@@ -34,6 +34,18 @@ const uint16_t* const* unit_src_table(const fsdp_peer* p) {
     return static_cast<const uint16_t* const*>(p->dev_tab) + p->parent->N;
 }
 
+void* const* table_base(const fsdp_peer* p) { return static_cast<void* const*>(p->dev_tab); }
+
+const uint8_t* const* unit_src8_table(const fsdp_peer* p) {
+    return reinterpret_cast<const uint8_t* const*>(table_base(p) + p->parent->N +
+                                                   p->parent->n_real_units);
+}
+
+const unsigned* const* amax_table(const fsdp_peer* p) {
+    return reinterpret_cast<const unsigned* const*>(table_base(p) + p->parent->N +
+                                                    2 * p->parent->n_real_units);
+}
+
 int check_op(int32_t op) {
     return (op == FSDP_SUM || op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? FSDP_OK : FSDP_EINVAL;
 }
@@ -79,8 +91,9 @@ int fsdp_peer_plan(fsdp_group_t g, int32_t n_devices, int32_t device_index, fsdp
     st = fsdpk::build_rank_tables(&l, p->r0, p->r0 + L);
     if (st == FSDP_OK) st = fsdpk::upload_tables(&l);
     if (st == FSDP_OK) {
-        cudaError_t e = cudaMalloc(
-            &p->dev_tab, ((size_t)g->N + (size_t)g->n_real_units) * sizeof(void*));
+        cudaError_t e = cudaMalloc(&p->dev_tab, ((size_t)g->N + 2 * (size_t)g->n_real_units +
+                                                 (size_t)n_devices) *
+                                                    sizeof(void*));
         if (e != cudaSuccess) {
             cudaGetLastError();
             p->dev_tab = nullptr;
@@ -142,6 +155,104 @@ int fsdp_peer_set_sources(fsdp_peer_t p, const uint16_t* const* ag_rank_ptrs,
     if (ag_rank_ptrs != nullptr) p->have_ag = true;
     if (grad_rank_ptrs != nullptr) p->have_grads = true;
     return FSDP_OK;
+}
+
+int fsdp_peer_set_fp8_sources(fsdp_peer_t p, const uint8_t* const* ag8_rank_ptrs,
+                              const uint32_t* const* amax_device_ptrs) {
+    if (p == nullptr || ag8_rank_ptrs == nullptr || amax_device_ptrs == nullptr)
+        return FSDP_EINVAL;
+    const int32_t N = p->parent->N;
+    for (int32_t r = 0; r < N; ++r)
+        if (p->parent->S > 0 && ag8_rank_ptrs[r] == nullptr) return FSDP_EINVAL;
+    for (int32_t d = 0; d < p->n_devices; ++d) {
+        if (p->parent->n > 0 && amax_device_ptrs[d] == nullptr) return FSDP_EINVAL;
+        if (reinterpret_cast<uintptr_t>(amax_device_ptrs[d]) & 3u) return FSDP_EALIGN;
+    }
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    std::vector<const void*> tab;
+    try {
+        tab.resize((size_t)p->parent->n_real_units + (size_t)p->n_devices);
+    } catch (...) {
+        return FSDP_ENOMEM;
+    }
+    const int64_t S = p->parent->S;
+    for (int64_t ui = 0; ui < p->parent->n_real_units; ++ui) {
+        const int64_t pos = p->parent->units[(size_t)ui].shard_pos;
+        const int64_t r = pos / S;  // a unit never crosses a rank's row
+        tab[(size_t)ui] = ag8_rank_ptrs[r] + (pos - r * S);
+    }
+    for (int32_t d = 0; d < p->n_devices; ++d)
+        tab[(size_t)p->parent->n_real_units + (size_t)d] = amax_device_ptrs[d];
+    void* dst = const_cast<void**>(table_base(p) + N + p->parent->n_real_units);
+    cudaError_t e = cudaMemcpy(dst, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_status(e);
+    p->have_fp8 = true;
+    return FSDP_OK;
+}
+
+int fsdp_peer_copy_in_fp8_scaled(fsdp_peer_t p, const float* master, const float* scales,
+                                 uint8_t* ag8_slot, fsdp_stream_t stream) {
+    if (p == nullptr) return FSDP_EINVAL;
+    const int64_t LS = (int64_t)p->local.L * p->local.S;
+    if (LS > 0 && (master == nullptr || ag8_slot == nullptr)) return FSDP_EINVAL;
+    if (p->local.n > 0 && scales == nullptr) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(ag8_slot) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return FSDP_EALIGN;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(fsdpk::launch_copy_in_fp8_scaled(p->local, master, ag8_slot, scales,
+                                                        (cudaStream_t)stream));
+}
+
+int fsdp_peer_copy_out_fp8(fsdp_peer_t p, uint8_t* arena8, fsdp_stream_t stream) {
+    if (p == nullptr) return FSDP_EINVAL;
+    if (p->parent->P > 0 && arena8 == nullptr) return FSDP_EINVAL;
+    if (!aligned16(arena8)) return FSDP_EALIGN;
+    if (!p->have_fp8) return FSDP_ESTATE;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(fsdpk::launch_copy_out_fp8_tab(*p->parent, unit_src8_table(p), arena8,
+                                                      (cudaStream_t)stream));
+}
+
+int fsdp_peer_rs_adamw_step_fp8(fsdp_peer_t p, int32_t op, float* master, float* m, float* v,
+                                const fsdp_adamw_hparams* hp, const float* scales_prev,
+                                uint8_t* ag8_next, uint32_t* amax_local, float* reduced,
+                                fsdp_stream_t stream) {
+    if (p == nullptr || hp == nullptr || check_op(op) != FSDP_OK) return FSDP_EINVAL;
+    const int64_t LS = (int64_t)p->local.L * p->local.S;
+    if (LS > 0 && (master == nullptr || m == nullptr || v == nullptr || ag8_next == nullptr))
+        return FSDP_EINVAL;
+    if (p->local.n > 0 && (scales_prev == nullptr || amax_local == nullptr)) return FSDP_EINVAL;
+    fsdpk::AdamScalars sc;
+    if (!fsdpk::host_adam_scalars(hp, &sc)) return FSDP_EINVAL;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(ag8_next) ||
+        !aligned16(reduced) || (reinterpret_cast<uintptr_t>(scales_prev) & 3u) ||
+        (reinterpret_cast<uintptr_t>(amax_local) & 3u))
+        return FSDP_EALIGN;
+    if (!p->have_grads) return FSDP_ESTATE;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (p->local.n > 0) e = cudaMemsetAsync(amax_local, 0, sizeof(uint32_t) * (size_t)p->local.n, s);
+    if (e == cudaSuccess)
+        e = fsdpk::launch_rs_adamw_tab_fp8(p->local, grad_table(p), op, master, m, v, sc,
+                                           scales_prev, ag8_next, amax_local, reduced, s);
+    return cuda_status(e);
+}
+
+int fsdp_peer_fp8_scales(fsdp_peer_t p, float* scales_next, fsdp_stream_t stream) {
+    if (p == nullptr) return FSDP_EINVAL;
+    if (p->local.n > 0 && scales_next == nullptr) return FSDP_EINVAL;
+    if (reinterpret_cast<uintptr_t>(scales_next) & 3u) return FSDP_EALIGN;
+    if (!p->have_fp8) return FSDP_ESTATE;
+    int st = fsdpk::check_plan_device(&p->local);
+    if (st != FSDP_OK) return st;
+    return cuda_status(fsdpk::launch_fp8_scales_from_parts(amax_table(p), p->n_devices,
+                                                           scales_next, p->local.n,
+                                                           (cudaStream_t)stream));
 }
 
 void fsdp_destroy_peer_plan(fsdp_peer_t p) {

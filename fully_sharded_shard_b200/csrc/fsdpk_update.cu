@@ -428,14 +428,29 @@ cudaError_t launch_rs_adamw_fp8(const fsdp_group& g, const uint16_t* grads, int 
     return launch_rs_adamw_any<true>(g, grads, o, avg, sc, sc_dev, st);
 }
 
-template <int NR>
+template <int NR, bool FP8>
 cudaError_t launch_rs_adamw_tab_nr(const fsdp_group& g, const uint16_t* const* tab,
                                    const FusedOut& o, int avg, const AdamScalars& sc,
                                    cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
-    k_rs_adamw<NR, false, true><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
+    k_rs_adamw<NR, FP8, true><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
         nullptr, 0, tab, g.N, o, g.d_units, nu, avg, sc, nullptr);
     return cudaGetLastError();
+}
+
+template <bool FP8>
+cudaError_t launch_rs_adamw_tab_any(const fsdp_group& g, const uint16_t* const* grad_tab,
+                                    const FusedOut& o, int avg, const AdamScalars& sc,
+                                    cudaStream_t st) {
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_rs_adamw_tab_nr<K, FP8>(g, grad_tab, o, avg, sc, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_rs_adamw_tab_nr<0, FP8>(g, grad_tab, o, avg, sc, st);
+    }
 }
 
 cudaError_t launch_rs_adamw_tab(const fsdp_group& g, const uint16_t* const* grad_tab, int op,
@@ -444,15 +459,18 @@ cudaError_t launch_rs_adamw_tab(const fsdp_group& g, const uint16_t* const* grad
     if (g.units.empty()) return cudaSuccess;
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
     const FusedOut o{master, m, v, reduced, ag_next, nullptr, nullptr, nullptr, nullptr};
-    switch (g.N) {
-#define FSDPK_CASE(K) \
-    case K: return launch_rs_adamw_tab_nr<K>(g, grad_tab, o, avg, sc, st);
-        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
-        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
-#undef FSDPK_CASE
-        default:
-            return launch_rs_adamw_tab_nr<0>(g, grad_tab, o, avg, sc, st);
-    }
+    return launch_rs_adamw_tab_any<false>(g, grad_tab, o, avg, sc, st);
+}
+
+cudaError_t launch_rs_adamw_tab_fp8(const fsdp_group& g, const uint16_t* const* grad_tab, int op,
+                                    float* master, float* m, float* v, const AdamScalars& sc,
+                                    const float* scales_prev, uint8_t* ag8_next,
+                                    unsigned* amax_bits, float* reduced, cudaStream_t st) {
+    if (g.units.empty()) return cudaSuccess;
+    const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    const FusedOut o{master, m, v, reduced, nullptr, ag8_next, scales_prev, amax_bits,
+                     g.d_unit_param};
+    return launch_rs_adamw_tab_any<true>(g, grad_tab, o, avg, sc, st);
 }
 
 }  // namespace fsdpk

@@ -117,7 +117,7 @@ class PeerGroup:
     shapes (several instances of one layer share one gradient buffer)."""
 
     def __init__(self, shapes: Sequence[Sequence[int]], N: int, *, group=None, device=None,
-                 grads: Optional[SharedBuffer] = None):
+                 grads: Optional[SharedBuffer] = None, fp8: bool = False):
         self.pg = group
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
@@ -137,6 +137,16 @@ class PeerGroup:
         self.grads = self.grad_buf.view(L * A, torch.bfloat16).view(L, A)
         ag, gr = rank_pointer_tables(self.slot_buf.bases, self.grad_buf.bases, L, S, A)
         abi.fsdp_peer_set_sources(self.pp, ag, gr)
+        self.slot8_buf = self.amax_buf = None
+        if fp8:
+            # E4M3 slot rows (1 byte per element) and this device's partial
+            # per-parameter amax, both mapped by every device
+            self.slot8_buf = SharedBuffer(L * S, group=group, device=self.device)
+            self.amax_buf = SharedBuffer(4 * self.g.n, group=group, device=self.device)
+            self.ag8_slot = self.slot8_buf.view(L * S, torch.uint8)
+            self.amax = self.amax_buf.view(self.g.n, torch.int32)
+            ag8 = [int(self.slot8_buf.bases[r // L]) + S * (r % L) for r in range(self.N)]
+            abi.fsdp_peer_set_fp8_sources(self.pp, ag8, self.amax_buf.bases)
         self.barrier()
 
     def barrier(self) -> None:
@@ -161,8 +171,27 @@ class PeerGroup:
                                     ag_next=self.ag_slot if next_copy_in else None,
                                     reduced=reduced, stream=stream, **hp)
 
+    # the FP8 all-gather (delayed scaling): copy-in with given scales, the
+    # fused update writing the E4M3 slot and the partial amax, the scales
+    # from every device's partial amax (after a barrier), the byte copy-out
+    def copy_in_fp8(self, master: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+        abi.fsdp_peer_copy_in_fp8_scaled(self.pp, master, scales, self.ag8_slot, stream)
+
+    def rs_adamw_step_fp8(self, op: int, master, m, v, *, scales_prev: torch.Tensor,
+                          reduced: Optional[torch.Tensor] = None, stream=None, **hp) -> None:
+        abi.fsdp_peer_rs_adamw_step_fp8(self.pp, op, master, m, v, scales_prev=scales_prev,
+                                        ag8_next=self.ag8_slot, amax_local=self.amax,
+                                        reduced=reduced, stream=stream, **hp)
+
+    def fp8_scales(self, scales_next: torch.Tensor, stream=None) -> None:
+        abi.fsdp_peer_fp8_scales(self.pp, scales_next, stream)
+
+    def copy_out_fp8(self, arena8: torch.Tensor, stream=None) -> None:
+        abi.fsdp_peer_copy_out_fp8(self.pp, arena8, stream)
+
     def buffers(self) -> List[SharedBuffer]:
-        return [self.slot_buf] + ([self.grad_buf] if self._own_grads else [])
+        extra = [b for b in (self.slot8_buf, self.amax_buf) if b is not None]
+        return [self.slot_buf] + ([self.grad_buf] if self._own_grads else []) + extra
 
     def close(self) -> None:
         """Release the shared buffers (after barriers, so that no peer still
@@ -170,6 +199,7 @@ class PeerGroup:
         if self.pp is None:
             return
         self.ag_slot = self.grads = None
+        self.ag8_slot = self.amax = None
         release_all(self.buffers(), self.device, self.pg)
         self.pp.destroy()
         self.g.destroy()

@@ -504,6 +504,43 @@ FSDP_API int fsdp_peer_rs_adamw_step(fsdp_peer_t peer, int32_t op, float* master
                                      uint16_t* ag_next_or_null, float* reduced_or_null,
                                      fsdp_stream_t stream);
 
+/* The FP8 all-gather over several devices (delayed scaling, as
+ * fsdp_rs_adamw_step_fp8): each device's slot holds E4M3 bytes [L][S], so the
+ * copy-out pulls half the bytes.  The per-parameter amax spans every rank, so
+ * each device folds the maximum of its own rows into a partial amax array
+ * (uint32 [n_params], the bits of a non-negative float) and the scales are
+ * the maximum over the devices' partial arrays: one more exchange, of
+ * 4 * n_params bytes per device.
+ * fsdp_peer_set_fp8_sources: ag8_rank_ptrs, host array of N device pointers
+ * (entry r = rank r's E4M3 slot row, S bytes); amax_device_ptrs, host array
+ * of n_devices device pointers (device d's partial amax array, 4-byte
+ * aligned).  Resolved and copied to the device synchronously.
+ * fsdp_peer_copy_in_fp8_scaled: fsdp_copy_in_fp8_scaled for the local ranks
+ * (master fp32 [L][S] -> ag8_slot uint8 [L][S], scales fp32 [n_params]).
+ * fsdp_peer_copy_out_fp8: fsdp_copy_out_fp8 of all N ranks into arena8
+ * (uint8 [P_arena]), pulling each rank's bytes from its slot row.
+ * fsdp_peer_rs_adamw_step_fp8: fsdp_rs_adamw_step_fp8 for the local ranks,
+ * except that the amax of the updated local rows goes to amax_local (zeroed
+ * first) instead of the next scales; ag8_next is normally the device's own
+ * slot.  fsdp_peer_fp8_scales: scales_next[i] = 448 / max(max over devices
+ * of partial amax i, 1e-12), reading every device's array (after a barrier
+ * that follows every device's fused update).  The scales, slots and arena
+ * then equal those of fsdp_rs_adamw_step_fp8 and fsdp_copy_out_fp8 on one
+ * device.  Errors as for the single-device calls; FSDP_ESTATE before the
+ * tables are set. */
+FSDP_API int fsdp_peer_set_fp8_sources(fsdp_peer_t peer, const uint8_t* const* ag8_rank_ptrs,
+                                       const uint32_t* const* amax_device_ptrs);
+FSDP_API int fsdp_peer_copy_in_fp8_scaled(fsdp_peer_t peer, const float* master,
+                                          const float* scales, uint8_t* ag8_slot,
+                                          fsdp_stream_t stream);
+FSDP_API int fsdp_peer_copy_out_fp8(fsdp_peer_t peer, uint8_t* arena8, fsdp_stream_t stream);
+FSDP_API int fsdp_peer_rs_adamw_step_fp8(fsdp_peer_t peer, int32_t op, float* master, float* m,
+                                         float* v, const fsdp_adamw_hparams* hparams,
+                                         const float* scales_prev, uint8_t* ag8_next,
+                                         uint32_t* amax_local, float* reduced_or_null,
+                                         fsdp_stream_t stream);
+FSDP_API int fsdp_peer_fp8_scales(fsdp_peer_t peer, float* scales_next, fsdp_stream_t stream);
+
 /* Device memory other processes can map (CUDA IPC).  fsdp_ipc_alloc
  * allocates `bytes` (> 0) on the current device with cudaMalloc and writes
  * the handle another process passes to fsdp_ipc_open; free it with

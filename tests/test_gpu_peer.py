@@ -147,6 +147,90 @@ def run_group_peer(H, wl, grp, D, *, steps=2, oracle_check=True, tag=()):
     g.destroy()
 
 
+def run_group_peer_fp8(H, wl, grp, D, *, steps=2, tag=()):
+    """The FP8 all-gather over D emulated devices (delayed scaling): slots,
+    partial amax arrays, next scales, the byte copy-out pulls and the state
+    against fsdp_rs_adamw_step_fp8 / fsdp_copy_out_fp8 of the single-device
+    group, bit for bit."""
+    from fully_sharded_shard_b200 import abi
+    from fully_sharded_shard_b200.peer import rank_pointer_tables
+    N, op = wl.N, wl.op
+    L = N // D
+    g = abi.fsdp_plan_group(grp.shapes, N)
+    S, A, n = g.S, g.P_arena, g.n
+    full = torch.empty(max(A, 1), device="cuda")
+    W.fill_master(full, wl, grp.name, *tag)
+    master = torch.empty(max(N * S, 1), device="cuda")
+    abi.fsdp_shard_params(g, full, master)
+    ref = {"p": master[:N * S].clone(), "m": torch.zeros(N * S, device="cuda"),
+           "v": torch.zeros(N * S, device="cuda")}
+    pps = [abi.fsdp_peer_plan(g, D, d) for d in range(D)]
+    slots = [H.Guarded(L * S, torch.bfloat16) for _ in range(D)]
+    slots8 = [H.Guarded(L * S, torch.uint8) for _ in range(D)]
+    gbufs = [H.Guarded(L * A, torch.bfloat16) for _ in range(D)]
+    amax = [torch.empty(max(n, 1), dtype=torch.int32, device="cuda") for _ in range(D)]
+    ag_ptrs, gr_ptrs = rank_pointer_tables([s.t.data_ptr() for s in slots],
+                                           [b.t.data_ptr() for b in gbufs], L, S, A)
+    ag8_ptrs = [slots8[r // L].t.data_ptr() + S * (r % L) for r in range(N)]
+    for pp in pps:
+        abi.fsdp_peer_set_sources(pp, ag_ptrs, gr_ptrs)
+        abi.fsdp_peer_set_fp8_sources(pp, ag8_ptrs, [a.data_ptr() for a in amax])
+    dev = [{k: t[d * L * S:(d + 1) * L * S].clone() for k, t in ref.items()} for d in range(D)]
+    hp = dict(W.ADAMW_DEFAULTS)
+    # step 0: dynamic scales of the initial master, the scaled copy-in on every device
+    scales = torch.empty(max(n, 1), device="cuda")
+    ag8_ref = torch.empty(max(N * S, 1), dtype=torch.uint8, device="cuda")
+    abi.fsdp_copy_in_fp8(g, ref["p"], ag8_ref, scales)
+    for d in range(D):
+        abi.fsdp_peer_copy_in_fp8_scaled(pps[d], dev[d]["p"], scales, slots8[d].t)
+
+    def pulls_equal_reference():
+        torch.cuda.synchronize()
+        if S:
+            got = torch.cat([s.t for s in slots8])
+            assert torch.equal(got, ag8_ref[:N * S]), "E4M3 slots != single-device buffer"
+        ar_ref = torch.full((max(A, 1),), 0xA5, dtype=torch.uint8, device="cuda")
+        abi.fsdp_copy_out_fp8(g, ag8_ref, ar_ref)
+        for d in range(D):
+            ar = H.Guarded(A, torch.uint8)
+            ar.t.fill_(0xA5)
+            abi.fsdp_peer_copy_out_fp8(pps[d], ar.t)
+            torch.cuda.synchronize()
+            assert ar.guards_intact()
+            assert torch.equal(ar.t, ar_ref[:A]), f"device {d} FP8 copy-out"
+
+    pulls_equal_reference()
+    for step in range(1, steps + 1):
+        grads = H.make_grads(g, wl, grp, step, tag)
+        for d in range(D):
+            gbufs[d].t.copy_(grads[d * L:(d + 1) * L].reshape(-1))
+        nxt_ref = torch.empty(max(n, 1), device="cuda")
+        abi.fsdp_rs_adamw_step_fp8(g, grads, op, ref["p"], ref["m"], ref["v"], step=step,
+                                   scales_prev=scales, ag8_next=ag8_ref, scales_next=nxt_ref, **hp)
+        for d in range(D):
+            abi.fsdp_peer_rs_adamw_step_fp8(pps[d], op, dev[d]["p"], dev[d]["m"], dev[d]["v"],
+                                            step=step, scales_prev=scales, ag8_next=slots8[d].t,
+                                            amax_local=amax[d], **hp)
+        torch.cuda.synchronize()  # every device's partial amax is complete
+        nxt = [torch.empty(max(n, 1), device="cuda") for _ in range(D)]
+        for d in range(D):
+            abi.fsdp_peer_fp8_scales(pps[d], nxt[d])
+        torch.cuda.synchronize()
+        for d in range(D):
+            assert slots8[d].guards_intact()
+            assert torch.equal(nxt[d][:n].view(torch.int32), nxt_ref[:n].view(torch.int32)), \
+                f"device {d} next scales, step {step}"
+            rows = slice(d * L * S, (d + 1) * L * S)
+            for k in ("p", "m", "v"):
+                assert torch.equal(dev[d][k].view(torch.int32), ref[k][rows].view(torch.int32))
+        pulls_equal_reference()
+        scales = nxt_ref
+        del grads
+    for pp in pps:
+        pp.destroy()
+    g.destroy()
+
+
 PEER = [
     (_wl("peer_ragged_n4", [(7, 3), (5,), (1, 32), (1,), (0, 4), (13, 9), (2, 2)], 4, op=W.SUM), (1, 2, 4)),
     (_wl("peer_n6_odd", [(1001, 3), (17,), (3, 4099), (8191, 1)], 6, op=W.SUM_THEN_DIV), (2, 3, 6)),
@@ -165,6 +249,14 @@ def test_peer_pulls_equal_single_device(H, case):
     for grp in wl.groups:
         for D in Ds:
             run_group_peer(H, wl, grp, D, steps=2, oracle_check=(D == Ds[-1]))
+
+
+@pytest.mark.parametrize("case", PEER, ids=[c[0].name for c in PEER])
+def test_peer_fp8_all_gather_equals_single_device(H, case):
+    wl, Ds = case
+    for grp in wl.groups:
+        for D in Ds:
+            run_group_peer_fp8(H, wl, grp, D, steps=2)
 
 
 def test_peer_full_size_llama7b_block_eight_devices(H):
@@ -274,5 +366,85 @@ def _ipc_worker(rank, port, D, case_name, result_dir):
 def test_peer_group_over_cuda_ipc_processes(H, tmp_path, D, case):
     import torch.multiprocessing as mp
     mp.spawn(_ipc_worker, args=(_free_port(), D, case, str(tmp_path)), nprocs=D, join=True)
+    for r in range(D):
+        assert open(tmp_path / f"r{r}.txt").read().strip() == "ok", f"process {r}"
+
+
+def _ipc_fp8_worker(rank, port, D, case_name, result_dir):
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=D, timeout=datetime.timedelta(seconds=120))
+    msg = "ok"
+    try:
+        torch.cuda.set_device(0)
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200.peer import PeerGroup
+        from tests import _harness as H
+        wl = {"uneven": W.uneven(16), "moe": W.moe(16)}[case_name]
+        grp = wl.groups[0]
+        N, op = wl.N, wl.op
+        pgrp = PeerGroup(grp.shapes, N, device="cuda:0", fp8=True)
+        g, S, A, L, r0, n = pgrp.g, pgrp.S, pgrp.P_arena, pgrp.L, pgrp.r0, pgrp.g.n
+        rows = slice(r0 * S, (r0 + L) * S)
+        full = torch.empty(max(A, 1), device="cuda")
+        W.fill_master(full, wl, grp.name)
+        master = torch.empty(max(N * S, 1), device="cuda")
+        abi.fsdp_shard_params(g, full, master)
+        ref = {"p": master[:N * S].clone(), "m": torch.zeros(N * S, device="cuda"),
+               "v": torch.zeros(N * S, device="cuda")}
+        mine = {k: t[rows].clone() for k, t in ref.items()}
+        hp = dict(W.ADAMW_DEFAULTS)
+        scales = torch.empty(max(n, 1), device="cuda")
+        ag8_ref = torch.empty(max(N * S, 1), dtype=torch.uint8, device="cuda")
+        abi.fsdp_copy_in_fp8(g, ref["p"], ag8_ref, scales)
+        pgrp.copy_in_fp8(mine["p"], scales)
+        for step in range(1, 3):
+            pgrp.barrier()                       # every E4M3 slot written
+            ar = torch.full((max(A, 1),), 0xA5, dtype=torch.uint8, device="cuda")
+            pgrp.copy_out_fp8(ar[:A])
+            ar_ref = torch.full((max(A, 1),), 0xA5, dtype=torch.uint8, device="cuda")
+            abi.fsdp_copy_out_fp8(g, ag8_ref, ar_ref[:A])
+            grads = H.make_grads(g, wl, grp, step)
+            pgrp.grads.copy_(grads[r0:r0 + L])
+            pgrp.barrier()                       # copy-outs done, gradients written
+            pgrp.rs_adamw_step_fp8(op, mine["p"], mine["m"], mine["v"], scales_prev=scales,
+                                   step=step, **hp)
+            nxt_ref = torch.empty(max(n, 1), device="cuda")
+            abi.fsdp_rs_adamw_step_fp8(g, grads, op, ref["p"], ref["m"], ref["v"], step=step,
+                                       scales_prev=scales, ag8_next=ag8_ref,
+                                       scales_next=nxt_ref, **hp)
+            pgrp.barrier()                       # every partial amax complete
+            nxt = torch.empty(max(n, 1), device="cuda")
+            pgrp.fp8_scales(nxt)
+            torch.cuda.synchronize()
+            if not torch.equal(ar, ar_ref):
+                msg = f"FP8 copy-out differs at step {step}"
+                break
+            if not torch.equal(nxt[:n].view(torch.int32), nxt_ref[:n].view(torch.int32)):
+                msg = f"next scales differ at step {step}"
+                break
+            if not torch.equal(pgrp.ag8_slot, ag8_ref[rows]):
+                msg = f"E4M3 slot differs at step {step}"
+                break
+            bad = [k for k in ("p", "m", "v")
+                   if not torch.equal(mine[k].view(torch.int32), ref[k][rows].view(torch.int32))]
+            if bad:
+                msg = f"fused FP8 update differs at step {step}: {bad}"
+                break
+            scales = nxt_ref
+        pgrp.close()
+    except Exception as e:  # reported through the result file
+        msg = f"error: {type(e).__name__}: {e}"
+    finally:
+        with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+            f.write(msg + "\n")
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("D,case", [(2, "uneven"), (4, "moe")])
+def test_peer_fp8_group_over_cuda_ipc_processes(H, tmp_path, D, case):
+    import torch.multiprocessing as mp
+    mp.spawn(_ipc_fp8_worker, args=(_free_port(), D, case, str(tmp_path)), nprocs=D, join=True)
     for r in range(D):
         assert open(tmp_path / f"r{r}.txt").read().strip() == "ok", f"process {r}"
