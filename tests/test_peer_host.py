@@ -54,7 +54,8 @@ class _FakeLib:
         self.d, self.log = d, log
 
     def fsdp_plan_group(self, shapes, N):
-        return types.SimpleNamespace(N=N, S=10, P_arena=24, destroy=lambda: self.log.append("g.destroy"))
+        return types.SimpleNamespace(N=N, S=10, P_arena=24, n=len(shapes),
+                                     destroy=lambda: self.log.append("g.destroy"))
 
     def fsdp_peer_plan(self, g, D, d):
         L = g.N // D
@@ -82,6 +83,9 @@ class _FakeLib:
 
     def fsdp_peer_set_sources(self, pp, ag, gr):
         self.log.append(("tables", list(ag), list(gr)))
+
+    def fsdp_peer_set_fp8_sources(self, pp, ag8, amax):
+        self.log.append(("fp8_tables", list(ag8), list(amax)))
 
 
 def _protocol_worker(rank, port, D, N, result_dir):
@@ -133,5 +137,46 @@ def _protocol_worker(rank, port, D, N, result_dir):
 @pytest.mark.parametrize("D,N", [(2, 4), (3, 3)])
 def test_peer_group_protocol_gloo(tmp_path, D, N):
     mp.spawn(_protocol_worker, args=(_free_port(), D, N, str(tmp_path)), nprocs=D, join=True)
+    for r in range(D):
+        assert open(tmp_path / f"r{r}.txt").read().strip() == "ok"
+
+
+def _fp8_protocol_worker(rank, port, D, N, result_dir):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=D)
+    try:
+        import fully_sharded_shard_b200.peer as peer
+        log = []
+        peer.abi = _FakeLib(rank, log)
+        peer.torch.cuda.synchronize = lambda *a, **k: log.append("sync")
+        pg = peer.PeerGroup([(7, 3), (5,)], N, device="cpu", fp8=True)
+        L = N // D
+        allocs = [e for e in log if e[0] == "alloc"]
+        # bf16 slot, gradients, E4M3 slot (1 B per element), partial amax (4 B per
+        # parameter); every shared buffer is at least 16 bytes
+        assert [a[2] for a in allocs] == [2 * L * 10, 2 * L * 24, max(L * 10, 16), max(4 * 2, 16)]
+        fp8 = [e for e in log if e[0] == "fp8_tables"]
+        assert len(fp8) == 1
+        _, ag8, amax = fp8[0]
+        for r in range(N):
+            j, row = divmod(r, L)
+            base = (j + 1) * 0x1000000 + 2 * 0x100000 + (0 if j == rank else 0x10)
+            assert ag8[r] == base + 10 * row  # byte rows
+        assert amax == [(j + 1) * 0x1000000 + 3 * 0x100000 + (0 if j == rank else 0x10)
+                        for j in range(D)]
+        n_before = len(log)
+        pg.close()
+        tail = log[n_before:]
+        assert sorted(e[1] for e in tail if e[0] == "free") == sorted(a[1] for a in allocs)
+        assert len([e for e in tail if e[0] == "close"]) == 4 * (D - 1)
+        with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+            f.write("ok\n")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_group_fp8_protocol_gloo(tmp_path):
+    D, N = 2, 4
+    mp.spawn(_fp8_protocol_worker, args=(_free_port(), D, N, str(tmp_path)), nprocs=D, join=True)
     for r in range(D):
         assert open(tmp_path / f"r{r}.txt").read().strip() == "ok"
