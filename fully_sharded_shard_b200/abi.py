@@ -106,6 +106,10 @@ def _load() -> ctypes.CDLL:
     L.fsdp_copy_in_f32.restype = ctypes.c_int
     L.fsdp_copy_out_f32.argtypes = [vp, vp, vp, vp]
     L.fsdp_copy_out_f32.restype = ctypes.c_int
+    L.fsdp_plan_group_host.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, ctypes.POINTER(vp)]
+    L.fsdp_plan_group_host.restype = ctypes.c_int
+    L.fsdp_group_check.argtypes = [vp, ctypes.POINTER(i64)]
+    L.fsdp_group_check.restype = ctypes.c_int
     L.fsdp_group_step.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.POINTER(AdamWHparams), vp, vp,
                                   vp, vp]
     L.fsdp_group_step.restype = ctypes.c_int
@@ -176,11 +180,12 @@ def _descs(shapes):
 class Group:
     """A plan of one parameter group (one fully_shard call) over N ranks."""
 
-    def __init__(self, shapes: Sequence[Sequence[int]], world_size: int):
+    def __init__(self, shapes: Sequence[Sequence[int]], world_size: int, host_only: bool = False):
         shapes, arr = _descs(shapes)
         h = ctypes.c_void_p()
-        _check(_lib.fsdp_plan_group(arr, len(shapes), int(world_size), ctypes.byref(h)),
-               "fsdp_plan_group")
+        fn = _lib.fsdp_plan_group_host if host_only else _lib.fsdp_plan_group
+        _check(fn(arr, len(shapes), int(world_size), ctypes.byref(h)),
+               "fsdp_plan_group_host" if host_only else "fsdp_plan_group")
         self._h = h
         self.shapes = shapes
         self.N = int(world_size)
@@ -217,6 +222,19 @@ class Group:
 
 def fsdp_plan_group(shapes: Sequence[Sequence[int]], world_size: int) -> Group:
     return Group(shapes, world_size)
+
+
+def fsdp_plan_group_host(shapes: Sequence[Sequence[int]], world_size: int) -> Group:
+    """The same plan on the host only (no CUDA call): for inspection and
+    fsdp_group_check; data calls refuse it."""
+    return Group(shapes, world_size, host_only=True)
+
+
+def fsdp_group_check(g: Group) -> int:
+    """Number of failed consistency checks of the plan's work tables (0 expected)."""
+    v = ctypes.c_int64()
+    _check(_lib.fsdp_group_check(g.handle, ctypes.byref(v)), "fsdp_group_check")
+    return v.value
 
 
 def _stream(stream, t: torch.Tensor):

@@ -11,6 +11,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -19,8 +20,10 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfsdpk.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
-         "-shared", "--expt-relaxed-constexpr", "-DFSDPK_BUILDING_LIBRARY"]
+CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
+          "--expt-relaxed-constexpr", "-DFSDPK_BUILDING_LIBRARY"]
+LDFLAGS = ["-shared", "-Xcompiler", "-fPIC"]
+OBJDIR = os.path.join(PKG, "_build")
 
 
 def sources():
@@ -29,7 +32,8 @@ def sources():
 
 def _inputs():
     return sources() + glob.glob(os.path.join(CSRC, "*.h")) + \
-        glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
+        glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")) + \
+        [os.path.abspath(__file__)]
 
 
 def nvcc() -> str:
@@ -40,15 +44,27 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every kernel file to an object in parallel (one nvcc per file),
+    then link the shared library."""
     if (not force and os.path.exists(LIB)
             and os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in _inputs())):
         return LIB
+    os.makedirs(OBJDIR, exist_ok=True)
+    extra = ["-Xptxas=-v"] if verbose else []
+
+    def compile_one(src: str) -> str:
+        obj = os.path.join(OBJDIR, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc(), *ARCH, *CFLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd))
+        subprocess.run(cmd, check=True)
+        return obj
+
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(compile_one, srcs))
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
+    subprocess.run([nvcc(), *ARCH, *LDFLAGS, "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
     return LIB
 

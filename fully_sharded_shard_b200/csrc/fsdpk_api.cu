@@ -234,8 +234,11 @@ const char* fsdp_status_string(int status) {
     }
 }
 
-int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t world_size,
-                    fsdp_group_t* out) {
+namespace {
+
+// The per-parameter tables and the work tables of all N ranks, on the host.
+int plan_on_host(const fsdp_param_desc* params, int32_t n_params, int32_t world_size,
+                 fsdp_group_t* out) {
     if (out == nullptr) return FSDP_EINVAL;
     *out = nullptr;
     if (n_params < 0 || (n_params > 0 && params == nullptr)) return FSDP_EINVAL;
@@ -303,9 +306,104 @@ int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t wor
 
     g->L = world_size;
     int st = fsdpk::build_rank_tables(g, 0, N);
-    if (st == FSDP_OK) st = fsdpk::upload_tables(g);
     if (st != FSDP_OK) return fail(st);
     *out = g;
+    return FSDP_OK;
+}
+
+// Every check the data calls rely on, over the host copies of the work
+// tables: the extents of every unit, exact coverage of [L][S] by the units,
+// each real unit's arena position recomputed from its shard position (the
+// Shard(0) placement), the pad intervals against the pad units, and each
+// copy-in tile's interval range.  Returns the number of violations.
+int64_t check_tables(const fsdp_group& g) {
+    int64_t bad = 0;
+    const int64_t LS = (int64_t)g.L * g.S;
+    const int64_t r0 = 0;  // a group plan holds the ranks [0, N)
+    std::vector<std::pair<int64_t, int64_t>> spans;  // (shard_pos, len)
+    int64_t pad_elems = 0;
+    if (g.unit_param.size() != g.units.size()) ++bad;
+    for (size_t k = 0; k < g.units.size(); ++k) {
+        const Unit& u = g.units[k];
+        const int32_t i = k < g.unit_param.size() ? g.unit_param[k] : -1;
+        if (u.len < 1 || u.len > fsdpk::kUnitElems || u.shard_pos < 0 || u.shard_pos + u.len > LS ||
+            i < 0 || i >= g.n) {
+            ++bad;
+            continue;
+        }
+        if ((k < (size_t)g.n_real_units) == (u.is_pad != 0)) ++bad;  // real units first
+        spans.emplace_back(u.shard_pos, u.len);
+        // the unit lies inside parameter i's padded shard of its rank
+        const int64_t j = u.shard_pos / g.S + r0;
+        const int64_t e0 = u.shard_pos - (j - r0) * g.S - g.off[i];
+        const int64_t valid = std::clamp<int64_t>(g.d0[i] - j * g.c[i], 0, g.c[i]) * g.cols[i];
+        if (e0 < 0 || e0 + u.len > g.s[i]) {
+            ++bad;
+            continue;
+        }
+        if (u.is_pad) {
+            pad_elems += u.len;
+            if (u.arena_pos != 0 || e0 < valid) ++bad;  // pad rows follow the valid rows
+        } else {
+            if (e0 + u.len > valid) ++bad;
+            // rank j's rows of parameter i start at u_i + j * c_i * cols_i in the arena
+            if (u.arena_pos != g.u[i] + j * g.c[i] * g.cols[i] + e0) ++bad;
+            if (u.arena_pos < 0 || u.arena_pos + u.len > g.P_arena) ++bad;
+        }
+    }
+    std::sort(spans.begin(), spans.end());
+    int64_t at = 0;
+    for (const auto& sp : spans) {
+        if (sp.first != at) ++bad;  // a gap or an overlap in the coverage of [L][S]
+        at = sp.first + sp.second;
+    }
+    if (at != LS) ++bad;
+    // pad intervals: sorted, disjoint, inside [L][S], as many elements as the pad units
+    int64_t iv_elems = 0, prev_hi = -1;
+    for (const Interval& iv : g.intervals) {
+        if (iv.lo < 0 || iv.hi > LS || iv.lo >= iv.hi || iv.lo <= prev_hi) ++bad;
+        iv_elems += iv.hi - iv.lo;
+        prev_hi = iv.hi;
+    }
+    if (iv_elems != pad_elems || (g.L == g.N && pad_elems != LS - g.P)) ++bad;
+    // copy-in tiles: each tile's range holds exactly the intervals that meet it
+    if (!g.intervals.empty()) {
+        if ((int64_t)g.tile_ranges.size() != g.n_tiles) ++bad;
+        for (int64_t t = 0; t < (int64_t)g.tile_ranges.size(); ++t) {
+            const int64_t lo = t * fsdpk::kCopyInTile, hi = lo + fsdpk::kCopyInTile;
+            const TileRange& tr = g.tile_ranges[(size_t)t];
+            for (int32_t q = 0; q < (int32_t)g.intervals.size(); ++q) {
+                const bool meets = g.intervals[(size_t)q].lo < hi && g.intervals[(size_t)q].hi > lo;
+                const bool inside = q >= tr.begin && q < tr.end;
+                if (meets != inside) ++bad;
+            }
+        }
+    }
+    return bad;
+}
+
+}  // namespace
+
+int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params, int32_t world_size,
+                    fsdp_group_t* out) {
+    int st = plan_on_host(params, n_params, world_size, out);
+    if (st != FSDP_OK) return st;
+    st = fsdpk::upload_tables(*out);
+    if (st != FSDP_OK) {
+        delete *out;
+        *out = nullptr;
+    }
+    return st;
+}
+
+int fsdp_plan_group_host(const fsdp_param_desc* params, int32_t n_params, int32_t world_size,
+                         fsdp_group_t* out) {
+    return plan_on_host(params, n_params, world_size, out);
+}
+
+int fsdp_group_check(fsdp_group_t g, int64_t* violations) {
+    if (g == nullptr || violations == nullptr) return FSDP_EINVAL;
+    *violations = check_tables(*g);
     return FSDP_OK;
 }
 

@@ -138,6 +138,23 @@ typedef struct {
 FSDP_API int fsdp_plan_group(const fsdp_param_desc* params, int32_t n_params,
                     int32_t world_size, fsdp_group_t* out);
 
+/* A plan built on the host only: the same layout and work tables as
+ * fsdp_plan_group, with no CUDA call and no device memory, for inspecting and
+ * checking a layout on a machine without a GPU.  Every data call refuses it
+ * (FSDP_ESTATE, or FSDP_ECUDA where no device is present); destroy it with
+ * fsdp_destroy_group. */
+FSDP_API int fsdp_plan_group_host(const fsdp_param_desc* params, int32_t n_params,
+                                  int32_t world_size, fsdp_group_t* out);
+
+/* Checks the host copies of a plan's work tables against everything the data
+ * calls assume: each unit inside [N][S] and inside its parameter's padded
+ * shard, the units covering [N][S] exactly once, each real unit's arena
+ * position recomputed from its shard position (the Shard(0) placement), pad
+ * units on the pad rows, the pad intervals matching the pad units, and each
+ * copy-in tile's interval range.  *violations receives the number of failed
+ * checks (0 for every plan this library builds).  Host only. */
+FSDP_API int fsdp_group_check(fsdp_group_t group, int64_t* violations);
+
 /* S (per-rank padded shard elements), P (real elements), P_arena.
  * Any output pointer may be NULL. */
 FSDP_API int fsdp_group_sizes(fsdp_group_t group, int64_t* S, int64_t* P,

@@ -1,0 +1,126 @@
+"""The C++ plan builder on the host (no GPU): every layout table against the
+oracle's plan, and the library's own consistency check of its work tables
+(extents, exact coverage, Shard(0) arena positions, pad intervals, copy-in
+tile ranges), over the workloads, random groups and the brute-force grid
+d0 in [0, 20] x cols in {1, 3, 8} x N in [1, 9]."""
+import ctypes
+
+import numpy as np
+import pytest
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from fully_sharded_shard_b200 import build
+    build.build()
+    from fully_sharded_shard_b200 import abi as _abi
+    return _abi
+
+
+def _compare(abi, oracle, shapes, N):
+    g = abi.fsdp_plan_group_host(shapes, N)
+    p = oracle.plan(shapes, N)
+    assert (g.S, g.P, g.P_arena) == (p.S, p.P, p.P_arena)
+    assert list(g.shard_off) == [int(x) for x in p.shard_off]
+    assert list(g.arena_off) == [int(x) for x in p.arena_off]
+    assert list(g.chunk_rows) == [int(x) for x in p.chunk_rows]
+    assert abi.fsdp_group_check(g) == 0, (shapes, N)
+    g.destroy()
+
+
+def test_workload_plans_on_host(abi, oracle):
+    from fully_sharded_shard_b200 import workloads as W
+    for wl in (W.tiny_mlp(), W.llama_block(), W.uneven(), W.moe(), W.llama7b()):
+        for grp in wl.groups:
+            _compare(abi, oracle, grp.shapes, wl.N)
+
+
+def test_random_and_extreme_plans_on_host(abi, oracle):
+    rng = np.random.default_rng(7)
+    for k in range(200):
+        N = int(rng.integers(1, 65))
+        shapes = []
+        for _ in range(int(rng.integers(0, 8))):
+            nd = int(rng.integers(0, 4))
+            dims = [int(rng.integers(0, 3000))] + [int(rng.integers(1, 9)) for _ in range(max(nd - 1, 0))]
+            shapes.append(tuple(dims[:nd]) if nd else ())
+        _compare(abi, oracle, shapes, N)
+    _compare(abi, oracle, [(5, 3), (1,), (2, 2)], 1024)        # most ranks empty
+    _compare(abi, oracle, [(20000, 1)], 3)                     # units split at 8192
+    _compare(abi, oracle, [], 4)                               # no parameters
+
+
+def test_brute_force_grid_plans_on_host(abi, oracle):
+    shapes = [((d0, c) if c > 1 else (d0,)) for d0 in range(21) for c in (1, 3, 8)]
+    for N in range(1, 10):
+        _compare(abi, oracle, shapes, N)
+
+
+def test_data_calls_refuse_a_host_plan(abi):
+    L = abi.lib()
+    g = abi.fsdp_plan_group_host([(7, 3), (5,)], 2)
+    fake = ctypes.c_void_p(1 << 20)  # aligned and non-null; never dereferenced
+    st = L.fsdp_copy_in(g.handle, fake, fake, None)
+    assert st in (abi.FSDP_ESTATE, abi.FSDP_ECUDA)
+    st = L.fsdp_rs_reduce(g.handle, fake, abi.FSDP_AVG, None, fake, None)
+    assert st in (abi.FSDP_ESTATE, abi.FSDP_ECUDA)
+    g.destroy()
+
+
+# Mistakes planted in a copy of the host plan builder (compiled on the CPU,
+# never run on a GPU): the consistency check must report each of them.
+MUTANTS = [
+    ("arena one row off",
+     "g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);",
+     "g->u[i] + (j + 1) * g->c[i] * g->cols[i], v * g->cols[i], 0);"),
+    ("pad run one element short",
+     "const int64_t len = (g->c[i] - v) * g->cols[i];",
+     "const int64_t len = (g->c[i] - v) * g->cols[i] - (v < g->c[i] ? 1 : 0);"),
+    ("valid rows not clamped to the chunk",
+     "const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);\n                push_units(",
+     "const int64_t v = std::max<int64_t>(g->d0[i] - j * g->c[i], 0);\n                push_units("),
+    ("adjacent pads not merged",
+     "if (!g->intervals.empty() && g->intervals.back().hi == lo)",
+     "if (false)"),
+    ("tile range one interval short",
+     "g->tile_ranges[(size_t)t] = TileRange{(int32_t)a, (int32_t)b};",
+     "g->tile_ranges[(size_t)t] = TileRange{(int32_t)a, (int32_t)(b > a ? b - 1 : b)};"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
+    import glob
+    import os
+    import subprocess
+    from fully_sharded_shard_b200 import build as B
+    src = open(os.path.join(B.CSRC, "fsdpk_api.cu")).read()
+    assert src.count(old) == 1, name
+    mut = tmp_path / "fsdpk_api.cu"
+    mut.write_text(src.replace(old, new))
+    obj = tmp_path / "fsdpk_api.o"
+    subprocess.run([B.nvcc(), *B.ARCH, *B.CFLAGS, "-I", B.INCLUDE, "-I", B.CSRC, "-c", "-o",
+                    str(obj), str(mut)], check=True)
+    others = [o for o in glob.glob(os.path.join(B.OBJDIR, "*.o"))
+              if os.path.basename(o) != "fsdpk_api.o"]
+    lib = tmp_path / "libmut.so"
+    subprocess.run([B.nvcc(), *B.ARCH, *B.LDFLAGS, "-o", str(lib), str(obj), *others], check=True)
+    L = ctypes.CDLL(str(lib))
+    L.fsdp_plan_group_host.argtypes = [ctypes.POINTER(abi.ParamDesc), ctypes.c_int32,
+                                       ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p)]
+    L.fsdp_group_check.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)]
+    L.fsdp_destroy_group.argtypes = [ctypes.c_void_p]
+    L.fsdp_destroy_group.restype = None
+    # ragged rows on several ranks, pads that meet across parameters, a tile
+    # boundary inside a pad run
+    shapes = [(7, 3), (5,), (1, 32), (13, 9), (2, 2), (9001, 1), (3,)]
+    found = 0
+    for N in (2, 3, 4, 6):
+        _, arr = abi._descs(shapes)
+        h = ctypes.c_void_p()
+        assert L.fsdp_plan_group_host(arr, len(shapes), N, ctypes.byref(h)) == 0
+        v = ctypes.c_int64()
+        assert L.fsdp_group_check(h, ctypes.byref(v)) == 0
+        found += v.value
+        L.fsdp_destroy_group(h)
+    assert found > 0, f"planted mistake not reported: {name}"
