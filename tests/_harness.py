@@ -112,6 +112,7 @@ def adam_close(gpu: np.ndarray, ref: np.ndarray, tol: float = ADAM_TOL):
 
 
 def check_plan(g: abi.Group, p: oracle.Plan) -> None:
+    assert abi.fsdp_group_check(g) == 0, "the plan's work tables are inconsistent"
     assert (g.S, g.P, g.P_arena) == (p.S, p.P, p.P_arena)
     assert list(g.shard_off) == [int(x) for x in p.shard_off]
     assert list(g.arena_off) == [int(x) for x in p.arena_off]
