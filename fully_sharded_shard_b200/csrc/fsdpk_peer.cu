@@ -1,7 +1,9 @@
 // fsdpk_peer.cu -- host side of the multi-device exchange: the peer plan of
-// one device (the work tables of its local virtual ranks plus one pointer
-// per rank for the all-gather slots and the gradient arenas), its entry
-// points, and the CUDA IPC helpers that map other processes' buffers.
+// one device (the work tables of its local virtual ranks; one gradient-arena
+// pointer per rank; one source pointer per copy-out work unit into the bf16
+// and the FP8 slot rows, resolved here; one partial-amax pointer per device),
+// its entry points, and the CUDA IPC helpers that map other processes'
+// buffers.
 //
 // The exchange steps of "Introduction to PyTorch FSDP2 Backend Features",
 // Working Principle (all-gather before use, reduce-scatter after backward)
