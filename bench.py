@@ -534,6 +534,10 @@ def run_ours(args, wl, device, rank, ws):
     if not args.no_accumulate:
         accum = run_accumulate(args, model, device, stream)
 
+    staged = None
+    if not args.no_staged:
+        staged = run_staged(args, model, device, stream)
+
     fp8 = None
     if not args.no_fp8:
         fp8 = run_fp8(args, model, device, stream)
@@ -580,6 +584,7 @@ def run_ours(args, wl, device, rank, ws):
         "fused_step": fused,
         "fused_step_fp8_all_gather": fused8,
         "grad_accumulation": accum,
+        "staged_reduce_scatter": staged,
         "fp8_all_gather": fp8,
         "tiny_latency": latency,
         "setup_s": round(setup_s, 1),
@@ -903,6 +908,57 @@ def run_peer(args, wl, device, rank, ws):
     }
     peer.release_all([b for pg in shared for b in pg.buffers()], device)
     return out
+
+
+def staged_rs_bytes(N: int, S: int, P: int) -> int:
+    """The reduce-scatter with the packed buffer materialised: the pack reads
+    every rank's gradients (2 B per real element per rank) and writes the
+    fp32 packed buffer [N][N][S]; the reduction reads it back and writes
+    [N][S]: (2N + 8N + 4) B per unpadded parameter, the fused path + 8N."""
+    Pp = N * S
+    return 2 * N * P + 4 * N * Pp + 4 * N * Pp + 4 * Pp
+
+
+def run_staged(args, model, device, stream):
+    """The reduce-scatter of the largest repeated group through the staged
+    path (materialised fp32 packed buffer, pack then rank-ordered reduction)
+    against the fused path on the same gradients, each under its own byte
+    model."""
+    import torch
+    from fully_sharded_shard_b200 import abi
+    gi = max(range(len(model.plans)), key=lambda i: model.wl.groups[i].repeat)
+    g = model.plans[gi]
+    grads = model.grads[gi][0]
+    N = g.N
+    packed = torch.empty(N * N * g.S, dtype=torch.float32, device=device)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, args.warmup)):
+                fn()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(max(1, args.steps)):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / max(1, args.steps)
+
+    ms_staged = timed(lambda: abi.fsdp_rs_reduce(g, grads, model.wl.op, model.reduced,
+                                                 packed=packed, stream=stream))
+    ms_fused = timed(lambda: abi.fsdp_rs_reduce(g, grads, model.wl.op, model.reduced,
+                                                stream=stream))
+    b_staged = staged_rs_bytes(N, g.S, g.P)
+    b_fused = 2 * N * g.P + 4 * N * g.S
+    del packed
+    return {"group": model.wl.groups[gi].name, "params": g.P,
+            "staged_ms": round(ms_staged, 3), "staged_bytes": b_staged,
+            "staged_GBps": round(b_staged / (ms_staged * 1e-3) / 1e9, 1),
+            "fused_ms": round(ms_fused, 3), "fused_bytes": b_fused,
+            "fused_GBps": round(b_fused / (ms_fused * 1e-3) / 1e9, 1),
+            "speedup_fused_over_staged": round(ms_staged / ms_fused, 3)}
 
 
 def run_accumulate(args, model, device, stream, micro: int = 4):
@@ -1292,6 +1348,7 @@ def main(argv=None):
     ap.add_argument("--no-accumulate", action="store_true")
     ap.add_argument("--no-latency", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
+    ap.add_argument("--no-staged", action="store_true")
     ap.add_argument("--one-stream", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -103,3 +103,9 @@ def test_peer_byte_model_reduces_to_the_single_device_model():
     assert sum(b["adamw"] for b in per) == one["adamw"]
     assert all(b["copy_out"] == one["copy_out"] for b in per)
     assert bench.peer_exchange_bytes(N, S, 2, 2000, 4) == 2 * 6 * S + 2 * 6 * 2000
+
+
+def test_staged_byte_model_is_the_fused_one_plus_8n_per_param():
+    for N in (2, 6, 8):
+        fused = 2 * N * N * 1000 + 4 * N * 1000
+        assert bench.staged_rs_bytes(N, 1000, N * 1000) == fused + 8 * N * N * 1000
