@@ -753,6 +753,19 @@ def peer_stage_bytes(N: int, S: int, P: int, L: int, P_local: int) -> dict:
             "rs_reduce": 2 * N * P_local + 4 * LS, "adamw": 28 * LS}
 
 
+def local_real_elems(shapes, chunk_rows, r0: int, L: int) -> int:
+    """Real (unpadded) elements in the shards of ranks [r0, r0 + L): rank j
+    holds clamp(d0 - j * c, 0, c) rows of each parameter."""
+    total = 0
+    for shape, c in zip(shapes, chunk_rows):
+        d0 = shape[0] if len(shape) else 1
+        cols = 1
+        for d in shape[1:]:
+            cols *= d
+        total += sum(max(0, min(c, d0 - j * c)) * cols for j in range(r0, r0 + L))
+    return total
+
+
 def peer_exchange_bytes(N: int, S: int, L: int, P_local: int, D: int) -> int:
     """Bytes one device pulls from the other devices per group step: the
     other ranks' slot rows (copy-out) and the other ranks' gradient rows of
@@ -791,12 +804,7 @@ def run_peer(args, wl, device, rank, ws):
             W.fill_grads_bf16(first.grads[r - r0], wl, grp.name, "peer", "pool", 0, r)
             if grp.zero_grad:
                 W.zero_param_ranges(first.grads[r - r0], g.arena_off, g.numel, grp.zero_grad)
-        P_local = 0
-        for i, shape in enumerate(grp.shapes):
-            d0 = shape[0] if len(shape) else 1
-            cols = g.numel[i] // d0 if d0 else 0
-            c = g.chunk_rows[i]
-            P_local += sum(max(0, min(c, d0 - j * c)) * cols for j in range(r0, r0 + L))
+        P_local = local_real_elems(grp.shapes, g.chunk_rows, r0, L)
         plans.append((g, L, S, A, P_local))
         full = torch.empty(max(A, 1), dtype=torch.float32, device=device)
         master_full = torch.empty(max(N * S, 1), dtype=torch.float32, device=device)

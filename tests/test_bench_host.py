@@ -109,3 +109,19 @@ def test_staged_byte_model_is_the_fused_one_plus_8n_per_param():
     for N in (2, 6, 8):
         fused = 2 * N * N * 1000 + 4 * N * 1000
         assert bench.staged_rs_bytes(N, 1000, N * 1000) == fused + 8 * N * N * 1000
+
+
+def test_local_real_elems_split_the_group_across_devices(oracle):
+    from fully_sharded_shard_b200 import workloads as W
+    for wl in (W.uneven(), W.moe(), W.llama7b(), W.tiny_mlp()):
+        for grp in wl.groups:
+            p = oracle.plan(grp.shapes, wl.N)
+            rows = [int(x) for x in p.chunk_rows]
+            for D in [d for d in range(1, wl.N + 1) if wl.N % d == 0]:
+                L = wl.N // D
+                parts = [bench.local_real_elems(grp.shapes, rows, d * L, L) for d in range(D)]
+                assert sum(parts) == p.P
+                for d in range(D):  # against the oracle's valid rows, rank by rank
+                    want = sum(p.valid_rows(i, j) * int(p.cols[i])
+                               for i in range(p.n) for j in range(d * L, (d + 1) * L))
+                    assert parts[d] == want
