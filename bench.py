@@ -416,17 +416,30 @@ class Model:
         for idx in range(len(self.instances)):
             self.run_group(idx, stream, self.step_count, events=events)
 
-    def step_two_streams(self, s_gather, s_update):
+    def step_two_streams(self, s_gather, s_update, events=None):
         """One full step on two streams, as FSDP2 splits communication from
         compute: the all-gather half of each group (copy-in, copy-out, double
         buffered) on `s_gather`, its reduce-scatter and AdamW on `s_update`
         once its copy-in has read the pre-update master.  Group g+1's
         all-gather overlaps group g's update.  The step ends with `s_gather`
         waiting for `s_update`, so the next step's copy-ins see this step's
-        updates."""
+        updates.  events: optional dict stage -> list receiving (start, end)
+        events recorded around each launch on the stream it runs on."""
         import torch
         from fully_sharded_shard_b200 import abi
         from fully_sharded_shard_b200 import workloads as W
+
+        def timed(name, st, fn):
+            if events is None:
+                fn()
+                return
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn()
+            e1.record(st)
+            events[name].append((e0, e1))
+
         if self._ag2 is None:
             self._ag2 = [self.ag, torch.empty_like(self.ag)]
             self._arena2 = [self.arena, torch.empty_like(self.arena)]
@@ -435,14 +448,15 @@ class Model:
         for idx, (gi, master, m, v, pj) in enumerate(self.instances):
             g = self.plans[gi]
             ag, arena = self._ag2[idx % 2], self._arena2[idx % 2]
-            abi.fsdp_copy_in(g, master, ag, s_gather)
+            timed("copy_in", s_gather, lambda: abi.fsdp_copy_in(g, master, ag, s_gather))
             read = torch.cuda.Event()
             read.record(s_gather)
-            abi.fsdp_copy_out(g, ag, arena, s_gather)
+            timed("copy_out", s_gather, lambda: abi.fsdp_copy_out(g, ag, arena, s_gather))
             s_update.wait_event(read)
-            abi.fsdp_rs_reduce(g, self.grads[gi][pj], self.wl.op, self.reduced, stream=s_update)
-            abi.fsdp_adamw_step(g, master, m, v, self.reduced, step=self.step_count,
-                                stream=s_update, **hp)
+            timed("rs_reduce", s_update, lambda: abi.fsdp_rs_reduce(
+                g, self.grads[gi][pj], self.wl.op, self.reduced, stream=s_update))
+            timed("adamw", s_update, lambda: abi.fsdp_adamw_step(
+                g, master, m, v, self.reduced, step=self.step_count, stream=s_update, **hp))
         done = torch.cuda.Event()
         done.record(s_update)
         s_gather.wait_event(done)
@@ -457,11 +471,11 @@ def run_ours(args, wl, device, rank, ws):
     model = Model(wl, device, args.grad_pool, rank)
     setup_s = time.time() - t_setup
 
-    def one_step():
+    def one_step(events=None):
         if args.one_stream:
-            model.step(stream)
+            model.step(stream, events=events)
         else:
-            model.step_two_streams(stream, s_update)
+            model.step_two_streams(stream, s_update, events=events)
 
     # warm-up
     with torch.cuda.stream(stream):
@@ -476,9 +490,12 @@ def run_ours(args, wl, device, rank, ws):
     sampler.start()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
+    # events around every launch, on its own stream, give the per-kernel
+    # launch durations inside the timed region (the roofline's `achieved`)
+    live = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
     e_start.record(stream)
     for _ in range(args.steps):
-        one_step()
+        one_step(live)
     e_end.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -498,9 +515,11 @@ def run_ours(args, wl, device, rank, ws):
     peak, peak_kind = hbm_peak()
     gbs = ws * model.bytes_per_step / (ms_step * 1e-3) / 1e9
     params_s = ws * model.P_total / (ms_step * 1e-3)
-    dom = max(stage_ms, key=stage_ms.get)
-    dom_launch_ms = stage_ms[dom] / len(model.instances)
-    dom_achieved = model.stage_bytes[dom] / (stage_ms[dom] * 1e-3) / 1e9
+    live_ms = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in live.items()}
+    dom = max(live_ms, key=live_ms.get)
+    dom_launch_ms = live_ms[dom] / len(model.instances)
+    dom_achieved = model.stage_bytes[dom] / (live_ms[dom] * 1e-3) / 1e9
+    iso_achieved = model.stage_bytes[dom] / (stage_ms[dom] * 1e-3) / 1e9
     kernel_names = {"copy_in": "k_copy_in", "copy_out": "k_copy_out",
                     "rs_reduce": "k_reduce_units", "adamw": "k_adamw"}
     traffic = recorded_traffic(kernel_names[dom], wl.name)
@@ -510,6 +529,9 @@ def run_ours(args, wl, device, rank, ws):
         "frac": round(dom_achieved / peak, 4),
         "algorithmic_bytes_per_launch": int(model.stage_bytes[dom] / len(model.instances)),
         "avg_launch_ms": round(dom_launch_ms, 4),
+        "launch_timing": "CUDA events around every launch of the kernel inside the timed steps, "
+                         "on its own stream",
+        "achieved_serial_pass": round(iso_achieved, 1),
         "traffic": traffic,
     }
     stages = {k: {"ms_per_step": round(stage_ms[k], 3),
