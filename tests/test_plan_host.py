@@ -101,6 +101,8 @@ def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
     obj = tmp_path / "fsdpk_api.o"
     subprocess.run([B.nvcc(), *B.ARCH, *B.CFLAGS, "-I", B.INCLUDE, "-I", B.CSRC, "-c", "-o",
                     str(obj), str(mut)], check=True)
+    if len(glob.glob(os.path.join(B.OBJDIR, "*.o"))) < len(B.sources()):
+        B.build(force=True)  # the per-file objects the mutant links against
     others = [o for o in glob.glob(os.path.join(B.OBJDIR, "*.o"))
               if os.path.basename(o) != "fsdpk_api.o"]
     lib = tmp_path / "libmut.so"
