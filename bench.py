@@ -493,9 +493,13 @@ def run_ours(args, wl, device, rank, ws):
     # events around every launch, on its own stream, give the per-kernel
     # launch durations inside the timed region (the roofline's `achieved`)
     live = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
+    marks = []   # the end of every step on the launching stream
     e_start.record(stream)
     for _ in range(args.steps):
         one_step(live)
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        marks.append(ev)
     e_end.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -503,6 +507,8 @@ def run_ours(args, wl, device, rank, ws):
     ms_total = e_start.elapsed_time(e_end)
     ms_total = max_over_ranks(ms_total, device)
     ms_step = ms_total / args.steps
+    per_step = [a.elapsed_time(b) for a, b in zip([e_start] + marks[:-1], marks)]
+    ms_median = max_over_ranks(float(statistics.median(per_step)), device)
 
     # per-stage times: the same steps again with events around every launch
     events = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
@@ -579,6 +585,8 @@ def run_ours(args, wl, device, rank, ws):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 3),
+        "ms_per_step_median": round(ms_median, 3),
+        "ms_per_step_min_max": [round(min(per_step), 3), round(max(per_step), 3)],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -940,6 +948,175 @@ def run_peer(args, wl, device, rank, ws):
     return out
 
 
+def run_peer_pipelined(args, wl, device, rank, ws):
+    """The step of run_peer with the devices ordered by CUDA IPC events
+    instead of device-draining barriers: one host barrier per step (it waits
+    for no device), slots and gradient arenas double buffered by step
+    parity, and two streams per device -- the copy-ins and copy-out pulls on
+    one, each group's reduce-scatter pulls and AdamW on the other once its
+    copy-in has read the master -- so one group's exchange overlaps another
+    group's update, and one step's tail overlaps the next step's head (each
+    copy-in waits only for its own group's last update)."""
+    import torch
+    from fully_sharded_shard_b200 import abi
+    from fully_sharded_shard_b200 import peer
+    from fully_sharded_shard_b200 import workloads as W
+    N = wl.N
+    if N % ws:
+        raise SystemExit(f"--exchange peer needs N = {N} divisible by the {ws} processes")
+    s_gather = torch.cuda.Stream(device)
+    s_update = torch.cuda.Stream(device)
+    t_setup = time.time()
+    hp = dict(W.ADAMW_DEFAULTS)
+    groups, instances, plans = [], [], []
+    max_A, max_LS = 1, 1
+    for gi, grp in enumerate(wl.groups):
+        first = peer.PipelinedPeerGroup(grp.shapes, N, device=device)
+        L, S, A, r0 = first.L, first.S, first.P_arena, first.r0
+        g = first.g
+        for par in range(2):   # written once: both parities hold the same gradients
+            for r in range(r0, r0 + L):
+                W.fill_grads_bf16(first.grads[par][r - r0], wl, grp.name, "peer", "pool", 0, r)
+                if grp.zero_grad:
+                    W.zero_param_ranges(first.grads[par][r - r0], g.arena_off, g.numel,
+                                        grp.zero_grad)
+        P_local = local_real_elems(grp.shapes, g.chunk_rows, r0, L)
+        plans.append((g, L, S, A, P_local))
+        full = torch.empty(max(A, 1), dtype=torch.float32, device=device)
+        master_full = torch.empty(max(N * S, 1), dtype=torch.float32, device=device)
+        for rep_i in range(grp.repeat):
+            pg = first if rep_i == 0 else peer.PipelinedPeerGroup(grp.shapes, N, device=device,
+                                                                  grads=first)
+            W.fill_master(full[:A], wl, grp.name, "peer", "layer", rep_i)
+            abi.fsdp_shard_params(g, full, master_full)
+            master = master_full[r0 * S:(r0 + L) * S].clone()
+            m = torch.zeros(L * S, dtype=torch.float32, device=device)
+            v = torch.zeros(L * S, dtype=torch.float32, device=device)
+            instances.append((gi, pg, master, m, v))
+            if rep_i:
+                groups.append(pg)
+        groups.append(first)   # closed after the instances sharing its gradients
+        del full, master_full
+        max_A, max_LS = max(max_A, A), max(max_LS, L * S)
+    arenas = [torch.empty(max_A, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    reduced = torch.empty(max_LS, dtype=torch.float32, device=device)
+    for _, pg, *_ in instances:   # every device's grads are written: record it once
+        for par in range(2):
+            pg.grads_end(par, s_update)
+    torch.cuda.synchronize(device)
+    peer.host_barrier()
+    setup_s = time.time() - t_setup
+    state = {"t": 0}
+    n = len(instances)
+
+    def one_step(events=None):
+        state["t"] += 1
+        t = state["t"]
+        par = t % 2
+
+        def timed(name, st, fn):
+            if events is None:
+                fn()
+                return
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn()
+            e1.record(st)
+            events[name].append((e0, e1))
+
+        # phase A: every group's copy-in, each once its last update is done
+        read = []
+        for idx, (gi, pg, master, m, v) in enumerate(instances):
+            if "updated" in state:
+                s_gather.wait_event(state["updated"][idx])
+            timed("copy_in", s_gather, lambda: pg.copy_in(par, master, s_gather))
+            ev = torch.cuda.Event()
+            ev.record(s_gather)
+            read.append(ev)
+        peer.host_barrier()
+        # phase B: the copy-out pulls on one stream, the reduce-scatter pulls
+        # and AdamW on the other
+        updated = []
+        for idx, (gi, pg, master, m, v) in enumerate(instances):
+            timed("copy_out", s_gather, lambda: pg.copy_out(par, arenas[idx % 2], s_gather))
+            s_update.wait_event(read[idx])
+            timed("rs_reduce", s_update, lambda: pg.rs_reduce(par, wl.op, reduced, s_update))
+            timed("adamw", s_update, lambda: abi.fsdp_peer_adamw_step(
+                pg.pps[par], master, m, v, reduced, step=t, stream=s_update, **hp))
+            ev = torch.cuda.Event()
+            ev.record(s_update)
+            updated.append(ev)
+        state["updated"] = updated
+
+    def join():
+        """Both streams done: the launching stream waits for the last update."""
+        s_gather.wait_event(state["updated"][-1])
+
+    for _ in range(args.warmup):
+        one_step()
+    join()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(s_gather)
+    for _ in range(args.steps):
+        one_step()
+    join()
+    e_end.record(s_gather)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(e_start.elapsed_time(e_end), device) / args.steps
+    events = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
+    one_step(events)
+    join()
+    torch.cuda.synchronize(device)
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in events.items()}
+    sb = {k: 0 for k in stage_ms}
+    xbytes = 0
+    P_total = 0
+    for gi, pg, master, m, v in instances:
+        g, L, S, A, P_local = plans[gi]
+        for k, b in peer_stage_bytes(N, S, g.P, L, P_local).items():
+            sb[k] += b
+        xbytes += peer_exchange_bytes(N, S, L, P_local, ws)
+        P_total += g.P
+    dev_bytes = sum(sb.values())
+    job_bytes = sum_over_ranks(float(dev_bytes), device)
+    peak, peak_kind = hbm_peak()
+    out = {
+        "metric": METRIC, "value": round(job_bytes / (ms_step * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "params_per_s": round(P_total / (ms_step * 1e-3), 1),
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: seeded N(0,0.02) fp32 master, N(0,1e-3) bf16 per-rank grads",
+        "config": {"workload": wl.name, "N_virtual_ranks": N, "ranks_per_gpu": N // ws,
+                   "groups_per_step": n, "params": P_total,
+                   "exchange": "pulls over CUDA IPC peer memory (copy-out, reduce-scatter)",
+                   "ordering": "CUDA IPC events; one host barrier per step, no device sync; "
+                               "slots and gradient arenas double buffered by step parity",
+                   "bytes_per_step_per_gpu": dev_bytes,
+                   "exchange_bytes_per_step_per_gpu": xbytes,
+                   "l2": "inputs larger than L2",
+                   "parallelism": f"{ws} GPU(s), {N} virtual ranks, {N // ws} per GPU"},
+        "stages_in_overlapped_step": {
+            k: {"ms_per_step": round(stage_ms[k], 3),
+                "GBps": round(sb[k] / (stage_ms[k] * 1e-3) / 1e9, 1)} for k in stage_ms},
+        "peak": peak, "peak_kind": peak_kind,
+        "gpu_launches": 4 * n * args.steps,
+        "clocks": clocks, "setup_s": round(setup_s, 1),
+    }
+    torch.cuda.synchronize(device)
+    for pg in groups:
+        pg.close()
+    return out
+
+
 def staged_rs_bytes(N: int, S: int, P: int) -> int:
     """The reduce-scatter with the packed buffer materialised: the pack reads
     every rank's gradients (2 B per real element per rank) and writes the
@@ -1268,6 +1445,47 @@ def run_e2e(args, model, device, stream, ws):
             "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": 4}
 
 
+def workload_summary(args, name, device, rank, ws):
+    """Another workload after the headline one (its state freed first): the
+    five-stage step on two streams, each stage timed alone (events around
+    every launch, one stream), and the fused step, as GB/s and fractions of
+    the HBM peak under the same byte models."""
+    import argparse as _ap
+    import gc
+    import torch
+    from fully_sharded_shard_b200 import workloads as W
+    gc.collect()
+    torch.cuda.empty_cache()
+    sub = _ap.Namespace(**vars(args))
+    for flag in ("no_e2e", "no_accumulate", "no_latency", "no_fp8", "no_staged"):
+        setattr(sub, flag, True)
+    sub.no_fused = False
+    wl = W.by_name(name)
+    out, model = run_ours(sub, wl, device, rank, ws)
+    del model
+    gc.collect()
+    torch.cuda.empty_cache()
+    peak = out["roofline"]["peak"]
+    fused = out["fused_step"]
+    return {
+        "N_virtual_ranks": wl.N, "reduce_op": W.OP_NAMES[wl.op], "params": out["config"]["params"],
+        "groups_per_step": out["config"]["groups_per_step"],
+        "value": out["value"], "unit": "GB/s", "ms_per_step": out["ms_per_step"],
+        "ms_per_step_median": out["ms_per_step_median"],
+        "frac_of_peak": round(out["value"] / ws / peak, 4),
+        "stages": out["stages"],
+        "fused_step": {
+            "ms_per_step": fused["ms_per_step"], "value": fused["value"],
+            "frac_of_peak": fused["frac_of_measured_peak"],
+            "stages": {k: dict(v, frac_of_peak=round(v["GBps"] / peak, 4))
+                       for k, v in fused["stages"].items()},
+        },
+        "peak": peak, "peak_kind": out["roofline"]["peak_kind"],
+        "clocks": out["clocks"],
+        "gpu_launches": out["gpu_launches"],
+    }
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
@@ -1305,6 +1523,20 @@ def oracle_setup(wl):
     return O, grp, p, full, grads, state
 
 
+def cpu_model() -> str:
+    """The host CPU's model name and logical core count."""
+    name = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return f"{name} ({os.cpu_count()} logical cores)"
+
+
 def cpu_baseline(wl, min_seconds: float):
     """The oracle on the host cores: all threads for >= min_seconds, then one
     single-threaded pass; both over one group of the workload, the full-step
@@ -1327,6 +1559,7 @@ def cpu_baseline(wl, min_seconds: float):
     b = group_bytes(wl.N, p.S, p.P)
     step_params = wl.total_params()
     return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu": cpu_model(),
             "params_per_s": round(p.P / dt, 1),
             "value_1core": round(b / dt1 / 1e9, 3),
             "extrapolated_full_step_s": round(dt * step_params / p.P, 1),
@@ -1359,7 +1592,7 @@ def run_reference(args, wl):
         "config": {"workload": wl.name, "N_virtual_ranks": wl.N,
                    "sample_group": grp.name, "params_per_sample": p.P},
         "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "cpu": cpu_model(), "sample": sample},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -1380,13 +1613,20 @@ def main(argv=None):
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-staged", action="store_true")
     ap.add_argument("--one-stream", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--extra-workloads", default="uneven,moe",
+                    help="comma-separated workloads timed after the headline one (per-stage "
+                         "GB/s of the five-stage and the fused step); empty for none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--exchange", choices=["replicas", "peer"], default="replicas",
                     help="replicas: one full N-rank replica per GPU (weak scaling); peer: one "
                          "model whose N ranks are spread over the GPUs, exchanged as pulls "
                          "over peer memory (strong scaling)")
+    ap.add_argument("--peer-sync", choices=["barriers", "events"], default="events",
+                    help="--exchange peer: order the devices by CUDA IPC events with one host "
+                         "barrier per step (events), or by two device-draining barriers per "
+                         "step (barriers)")
     ap.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
                     help="process-group backend for N > 1 (gloo lets several processes share "
                          "one GPU, to exercise --exchange peer without several GPUs)")
@@ -1411,7 +1651,10 @@ def main(argv=None):
     if ws > 1:
         init_dist(args.backend)
     if args.exchange == "peer":
-        out = run_peer(args, wl, device, rank, ws)
+        if args.peer_sync == "events":
+            out = run_peer_pipelined(args, wl, device, rank, ws)
+        else:
+            out = run_peer(args, wl, device, rank, ws)
         if rank == 0:
             print(json.dumps(out), flush=True)
         if ws > 1:
@@ -1420,6 +1663,12 @@ def main(argv=None):
             dist.destroy_process_group()
         return 0
     out, model = run_ours(args, wl, device, rank, ws)
+    del model
+    extra = [w for w in args.extra_workloads.split(",") if w and w != wl.name]
+    if extra:
+        out["workloads"] = {}
+        for name in extra:
+            out["workloads"][name] = workload_summary(args, name, device, rank, ws)
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     if rank == 0:

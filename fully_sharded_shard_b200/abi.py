@@ -21,7 +21,10 @@ from typing import Optional, Sequence
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfsdpk.so")
+# FSDPK_DEBUG=1 loads the debug build (kernels check every work unit against
+# the extents of their buffers; see fsdp_debug_set_error_words)
+DEBUG = os.environ.get("FSDPK_DEBUG", "") == "1"
+LIB_PATH = os.path.join(_PKG, "libfsdpk_debug.so" if DEBUG else "libfsdpk.so")
 
 FSDP_MAX_NDIM = 8
 FSDP_MAX_WORLD = 1024
@@ -64,8 +67,9 @@ class AdamWHparams(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"libfsdpk.so is not built ({LIB_PATH}); run "
-            "`python -m fully_sharded_shard_b200.build` (needs nvcc)")
+            f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
+            "`python -m fully_sharded_shard_b200.build" + (" --debug" if DEBUG else "") +
+            "` (needs nvcc)")
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     L.fsdp_plan_group.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, ctypes.POINTER(vp)]
@@ -100,6 +104,9 @@ def _load() -> ctypes.CDLL:
     L.fsdp_adamw_step_dev.restype = ctypes.c_int
     L.fsdp_rs_adamw_step_dev.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
     L.fsdp_rs_adamw_step_dev.restype = ctypes.c_int
+    L.fsdp_debug_build.restype = ctypes.c_int
+    L.fsdp_debug_set_error_words.argtypes = [vp, i64]
+    L.fsdp_debug_set_error_words.restype = ctypes.c_int
     L.fsdp_rs_reduce_noalloc.argtypes = [ctypes.POINTER(ParamDesc), i32, i32, vp, i32, vp, vp]
     L.fsdp_rs_reduce_noalloc.restype = ctypes.c_int
     L.fsdp_copy_in_f32.argtypes = [vp, vp, vp, vp]
@@ -470,20 +477,63 @@ def fsdp_rs_adamw_step_dev(g: Group, grads: torch.Tensor, op: int, master: torch
                                        _ptr(reduced, _F32, n, "reduced"),
                                        _stream(stream, master)), "fsdp_rs_adamw_step_dev")
 
+def fsdp_debug_build() -> bool:
+    return bool(_lib.fsdp_debug_build())
+
+
+def fsdp_debug_set_error_words(words: Optional[torch.Tensor], shrink: int = 0) -> None:
+    """Debug build: record violations in `words` (int32 [4] on the device of
+    the launches that follow; None stops recording)."""
+    ptr = None if words is None else _ptr(words, (torch.int32,), 4, "words")
+    _check(_lib.fsdp_debug_set_error_words(ptr, int(shrink)), "fsdp_debug_set_error_words")
+
+
 FSDP_NOALLOC_MAX_UNITS = 131072
+
+
+def group_layout(shapes: Sequence[Sequence[int]], world_size: int) -> tuple:
+    """(S, P, P_arena) of a group from its shapes alone, by the layout rules
+    of include/fsdpk.h: c_i = ceil(d0_i / N) chunk rows (torch.chunk along
+    dim 0), S = sum c_i * cols_i, and each parameter's arena start rounded up
+    to 8 elements.  Size checks only; the library derives the same values."""
+    N = int(world_size)
+    if N < 1:
+        raise ValueError("world_size must be >= 1")
+    S = P = A = 0
+    for s in shapes:
+        s = tuple(int(d) for d in s)
+        if any(d < 0 for d in s):
+            raise ValueError(f"negative dimension in {s}")
+        d0 = s[0] if s else 1
+        cols = 1
+        for d in s[1:]:
+            cols *= d
+        c = -(-d0 // N)
+        S += c * cols
+        P += d0 * cols
+        A = (A + 7) // 8 * 8 + d0 * cols
+    return S, P, (A + 7) // 8 * 8
 
 
 def fsdp_rs_reduce_noalloc(shapes: Sequence[Sequence[int]], world_size: int,
                            grads: torch.Tensor, op: int, reduced: torch.Tensor,
-                           *, P_arena: int, S: int, stream=None):
+                           *, P_arena: Optional[int] = None, S: Optional[int] = None,
+                           stream=None):
     """The fused reduce-scatter without any allocation (no plan object): for
-    callers that cannot allocate device memory.  P_arena and S size-check the
-    tensors here; the library derives them again from the shapes."""
-    shapes, arr = _descs(shapes)
+    callers that cannot allocate device memory.  The tensors are size-checked
+    against S and P_arena worked out here from the shapes (the C call cannot
+    see buffer sizes); P_arena / S, when given, must agree with them."""
     N = int(world_size)
+    shapes = [tuple(int(d) for d in s) for s in shapes]
+    S_, _, A_ = group_layout(shapes, N)
+    if S is not None and int(S) != S_:
+        raise ValueError(f"S={S} does not match the shapes' layout (S={S_})")
+    if P_arena is not None and int(P_arena) != A_:
+        raise ValueError(f"P_arena={P_arena} does not match the shapes' layout (P_arena={A_})")
+    shapes, arr = _descs(shapes)
     _check(_lib.fsdp_rs_reduce_noalloc(arr, len(shapes), N,
-                                       _ptr(grads, _B16, N * P_arena, "grads"), int(op),
-                                       _ptr(reduced, _F32, N * S, "reduced"),
+                                       _ptr(grads, _B16, N * A_, "grads"), int(op),
+                                       _ptr(reduced, _F32, N * S_, "reduced"),
                                        _stream(stream, reduced)), "fsdp_rs_reduce_noalloc")
 
 

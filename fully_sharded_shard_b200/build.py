@@ -1,8 +1,11 @@
 """Build libfsdpk.so in-tree with nvcc for sm_100a (B200).
 
-Usage: ``python -m fully_sharded_shard_b200.build [--force] [--verbose]``.
+Usage: ``python -m fully_sharded_shard_b200.build [--force] [--verbose] [--debug]``.
 The library links the CUDA runtime statically, so it does not depend on the
-runtime version torch ships with.
+runtime version torch ships with.  ``--debug`` builds libfsdpk_debug.so, the
+same sources with -DFSDPK_DEBUG (every table-driven kernel checks its work
+units against the extents of its buffers); ``FSDPK_DEBUG=1`` makes the
+binding load it.
 """
 from __future__ import annotations
 
@@ -18,12 +21,14 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfsdpk.so")
+LIB_DEBUG = os.path.join(PKG, "libfsdpk_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
           "--expt-relaxed-constexpr", "-DFSDPK_BUILDING_LIBRARY"]
 LDFLAGS = ["-shared", "-Xcompiler", "-fPIC"]
 OBJDIR = os.path.join(PKG, "_build")
+OBJDIR_DEBUG = os.path.join(PKG, "_build_debug")
 
 
 def sources():
@@ -43,17 +48,19 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: cannot build libfsdpk.so")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
     """Compile every kernel file to an object in parallel (one nvcc per file),
-    then link the shared library."""
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in _inputs())):
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
-    extra = ["-Xptxas=-v"] if verbose else []
+    then link the shared library (the debug library with debug=True)."""
+    lib = LIB_DEBUG if debug else LIB
+    objdir = OBJDIR_DEBUG if debug else OBJDIR
+    if (not force and os.path.exists(lib)
+            and os.path.getmtime(lib) >= max(os.path.getmtime(p) for p in _inputs())):
+        return lib
+    os.makedirs(objdir, exist_ok=True)
+    extra = (["-Xptxas=-v"] if verbose else []) + (["-DFSDPK_DEBUG"] if debug else [])
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(OBJDIR, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         cmd = [nvcc(), *ARCH, *CFLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
         if verbose:
             print(" ".join(cmd))
@@ -63,12 +70,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
     srcs = sources()
     with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     subprocess.run([nvcc(), *ARCH, *LDFLAGS, "-o", tmp, *objs], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                debug="--debug" in sys.argv))

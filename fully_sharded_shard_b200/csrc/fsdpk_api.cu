@@ -213,12 +213,55 @@ bool host_adam_scalars(const fsdp_adamw_hparams* hp, AdamScalars* sc) {
     return adam_scalars(hp, sc);
 }
 
+// Debug build: the caller's error words and the test-only narrowing of every
+// launch's extents (so that a check can be seen to fire on valid tables).
+namespace {
+uint32_t* g_debug_words = nullptr;
+int64_t g_debug_shrink = 0;
+}  // namespace
+
+DebugBounds debug_bounds_raw(int64_t ns, int64_t arena, int32_t kernel, int64_t n_aux) {
+    DebugBounds b;
+    b.ns = ns - g_debug_shrink;
+    b.arena = arena - g_debug_shrink;
+    b.n_aux = n_aux;
+    b.words = g_debug_words;
+    b.kernel = kernel;
+    return b;
+}
+
+DebugBounds debug_bounds(const fsdp_group& g, int32_t kernel, int64_t n_aux) {
+    return debug_bounds_raw((int64_t)g.L * g.S, g.P_arena, kernel, n_aux);
+}
+
 }  // namespace fsdpk
 
 extern "C" {
 
 
 int fsdp_abi_version(void) { return FSDP_ABI_VERSION; }
+
+int fsdp_debug_build(void) {
+#ifdef FSDPK_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int fsdp_debug_set_error_words(uint32_t* words, int64_t shrink) {
+#ifdef FSDPK_DEBUG
+    if (shrink < 0) return FSDP_EINVAL;
+    if (words != nullptr && (reinterpret_cast<uintptr_t>(words) & 3u) != 0) return FSDP_EALIGN;
+    fsdpk::g_debug_words = words;
+    fsdpk::g_debug_shrink = shrink;
+    return FSDP_OK;
+#else
+    (void)words;
+    (void)shrink;
+    return FSDP_ESTATE;
+#endif
+}
 
 int fsdp_last_cuda_error(void) { return g_last_cuda_error; }
 
@@ -229,7 +272,7 @@ const char* fsdp_status_string(int status) {
         case FSDP_ENOMEM: return "out of memory";
         case FSDP_ECUDA: return "CUDA error";
         case FSDP_EALIGN: return "pointer not 16-byte aligned";
-        case FSDP_ESTATE: return "plan used on a different device";
+        case FSDP_ESTATE: return "call not valid in this state (plan of another device, host-only plan, or a capturing stream)";
         default: return "unknown status";
     }
 }

@@ -147,12 +147,24 @@ __device__ __forceinline__ void store8(float* __restrict__ dst, const float (&ac
     __stcs(o + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
 }
 
+// One AdamW step of one element in binary32.  Where (1 - b2) * g^2 overflows
+// binary32 (|g| above about 5.8e20) the stored second moment is +Inf, as the
+// exact value rounds to; the update then takes sqrt(v) as
+// |g| * sqrt(b2 * (v_old / g^2) + (1 - b2)), which stays finite, so the
+// parameter still moves by about lr * sign(g) as AdamW's definition gives
+// (rather than by 0 through m / Inf).
 __device__ __forceinline__ void adamw1(float& p, float& m, float& v, float g,
                                        const AdamScalars& sc) {
+    const float v_old = v;
     p = p * sc.decay;
     m = fmaf(sc.beta1, m, sc.omb1 * g);
     v = fmaf(sc.beta2, v, sc.omb2 * g * g);
-    const float denom = fmaf(__fsqrt_rn(v), sc.inv_bc2_sqrt, sc.eps);
+    float sqrt_v = __fsqrt_rn(v);
+    if (v > 3.40282347e38f && fabsf(g) <= 3.40282347e38f && v_old <= 3.40282347e38f) {
+        const float a = fabsf(g);
+        sqrt_v = a * __fsqrt_rn(fmaf(sc.beta2, __fdiv_rn(__fdiv_rn(v_old, a), a), sc.omb2));
+    }
+    const float denom = fmaf(sqrt_v, sc.inv_bc2_sqrt, sc.eps);
     p = fmaf(-sc.step_size, __fdiv_rn(m, denom), p);
 }
 
@@ -172,6 +184,48 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 
 __device__ __forceinline__ uint8_t e4m3(float x) {
     return (uint8_t)(e4m3x2(x, 0.0f) & 0xFFu);
+}
+
+// ---------------------------------------------------------------------------
+// debug build: unit and tile checks against the extents a launch was given
+// ---------------------------------------------------------------------------
+#ifdef FSDPK_DEBUG
+#define FSDPK_DBG_PARAM , DebugBounds dbg
+#define FSDPK_DBG_ARG(x) , x
+#define FSDPK_UNIT_GUARD(u, ui, what) \
+    if (!unit_in_bounds(dbg, (u), (ui), (what))) continue
+#define FSDPK_GUARD(ok, where) \
+    if (!debug_ok(dbg, (ok), (where))) continue
+#else
+#define FSDPK_DBG_PARAM
+#define FSDPK_DBG_ARG(x)
+#define FSDPK_UNIT_GUARD(u, ui, what) ((void)0)
+#define FSDPK_GUARD(ok, where) ((void)0)
+#endif
+
+constexpr int kChkShard = 1;  // shard_pos + len within [0, ns)
+constexpr int kChkArena = 2;  // a real unit's arena_pos + len within [0, arena)
+
+// Every thread evaluates the same condition for a unit, so a skip is uniform
+// across the block; lane 0 of each warp that sees a violation records it.
+__device__ __forceinline__ bool debug_ok(const DebugBounds& b, bool ok, int64_t where) {
+    if (!ok && (threadIdx.x & 31) == 0 && b.words != nullptr) {
+        if (atomicAdd(b.words, 1u) == 0u) {
+            b.words[1] = (uint32_t)b.kernel;
+            b.words[2] = (uint32_t)where;
+            b.words[3] = blockIdx.x;
+        }
+    }
+    return ok;
+}
+
+__device__ __forceinline__ bool unit_in_bounds(const DebugBounds& b, const Unit& u, int64_t ui,
+                                               int what) {
+    bool ok = u.len >= 0;
+    if (what & kChkShard) ok = ok && u.shard_pos >= 0 && u.shard_pos + u.len <= b.ns;
+    if ((what & kChkArena) && !u.is_pad)
+        ok = ok && u.arena_pos >= 0 && u.arena_pos + u.len <= b.arena;
+    return debug_ok(b, ok, ui);
 }
 
 // ---------------------------------------------------------------------------

@@ -40,9 +40,10 @@ __device__ __forceinline__ void copy_f32_run(const float* __restrict__ src, floa
 // ag32[shard_pos + e] = master[shard_pos + e] on real units, +0 on pad units.
 __global__ void __launch_bounds__(kThreads)
 k_copy_in_f32(const float* __restrict__ master, float* __restrict__ ag32,
-              const Unit* __restrict__ units, int64_t n_units) {
+              const Unit* __restrict__ units, int64_t n_units FSDPK_DBG_PARAM) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard);
         copy_f32_run(u.is_pad ? nullptr : master + u.shard_pos, ag32 + u.shard_pos, u.len);
     }
 }
@@ -50,9 +51,10 @@ k_copy_in_f32(const float* __restrict__ master, float* __restrict__ ag32,
 // arena32[arena_pos + e] = ag32[shard_pos + e] on real units.
 __global__ void __launch_bounds__(kThreads)
 k_copy_out_f32(const float* __restrict__ ag32, float* __restrict__ arena32,
-               const Unit* __restrict__ units, int64_t n_real) {
+               const Unit* __restrict__ units, int64_t n_real FSDPK_DBG_PARAM) {
     for (int64_t ui = blockIdx.x; ui < n_real; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
         copy_f32_run(ag32 + u.shard_pos, arena32 + u.arena_pos, u.len);
     }
 }
@@ -75,7 +77,8 @@ int fsdp_copy_in_f32(fsdp_group_t g, const float* master, float* ag32, fsdp_stre
     const int64_t nu = (int64_t)g->units.size();
     if (nu == 0) return FSDP_OK;
     fsdpk::k_copy_in_f32<<<fsdpk::grid_for(*g, nullptr, nu), fsdpk::kThreads, 0,
-                           (cudaStream_t)stream>>>(master, ag32, g->d_units, nu);
+                           (cudaStream_t)stream>>>(master, ag32, g->d_units, nu
+                           FSDPK_DBG_ARG(fsdpk::debug_bounds(*g, fsdpk::kDbgCopyInF32)));
     return fsdpk::status_of(cudaGetLastError());
 }
 
@@ -87,7 +90,8 @@ int fsdp_copy_out_f32(fsdp_group_t g, const float* ag32, float* arena32, fsdp_st
     if (st != FSDP_OK) return st;
     if (g->n_real_units == 0) return FSDP_OK;
     fsdpk::k_copy_out_f32<<<fsdpk::grid_for(*g, nullptr, g->n_real_units), fsdpk::kThreads, 0,
-                            (cudaStream_t)stream>>>(ag32, arena32, g->d_units, g->n_real_units);
+                            (cudaStream_t)stream>>>(ag32, arena32, g->d_units, g->n_real_units
+                            FSDPK_DBG_ARG(fsdpk::debug_bounds(*g, fsdpk::kDbgCopyOutF32)));
     return fsdpk::status_of(cudaGetLastError());
 }
 

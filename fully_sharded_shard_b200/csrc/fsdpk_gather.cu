@@ -52,12 +52,14 @@ static_assert(kCopyInTile == kThreads * 8 * kCopyInV, "copy-in tile shape");
 __global__ void __launch_bounds__(kThreads)
 k_copy_in(const float* __restrict__ master, uint16_t* __restrict__ ag, int64_t count,
           int64_t n_tiles, const Interval* __restrict__ iv,
-          const TileRange* __restrict__ tr) {
+          const TileRange* __restrict__ tr FSDPK_DBG_PARAM) {
     for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
         const int64_t base = t * kCopyInTile;
         const int64_t end = min(base + kCopyInTile, count);
         TileRange rng{0, 0};
         if (tr != nullptr) rng = tr[t];
+        FSDPK_GUARD(end <= dbg.ns && rng.begin >= 0 && rng.begin <= rng.end &&
+                        rng.end <= dbg.n_aux, t);
         float4 x[kCopyInV][2];
 #pragma unroll
         for (int j = 0; j < kCopyInV; ++j) {
@@ -136,9 +138,12 @@ __device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_a
 template <bool TAB>
 __global__ void __launch_bounds__(kThreads, 5)
 k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ unit_src,
-           uint16_t* __restrict__ arena, const Unit* __restrict__ units, int64_t n_units) {
+           uint16_t* __restrict__ arena, const Unit* __restrict__ units,
+           int64_t n_units FSDPK_DBG_PARAM) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        // a pulled unit's source is a pointer of the table, not a shard position
+        FSDPK_UNIT_GUARD(u, ui, TAB ? kChkArena : (kChkShard | kChkArena));
         const int len = u.len;
         uint16_t* dst_run = arena + u.arena_pos;
         const uint16_t* src_run;
@@ -166,9 +171,10 @@ k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ 
 
 __global__ void __launch_bounds__(kThreads)
 k_shard(const float* __restrict__ full, float* __restrict__ master,
-        const Unit* __restrict__ units, int64_t n_units) {
+        const Unit* __restrict__ units, int64_t n_units FSDPK_DBG_PARAM) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
         if (u.is_pad) {
             zero_f32_run(master + u.shard_pos, u.len);
             continue;
@@ -189,10 +195,12 @@ k_shard(const float* __restrict__ full, float* __restrict__ master,
 __global__ void __launch_bounds__(kThreads)
 k_fp8_amax(const float* __restrict__ master, unsigned* __restrict__ amax_bits,
            const Unit* __restrict__ units, const int32_t* __restrict__ unit_param,
-           int64_t n_real) {
+           int64_t n_real FSDPK_DBG_PARAM) {
     __shared__ float part[kThreads / 32];
     for (int64_t ui = blockIdx.x; ui < n_real; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard);
+        FSDPK_GUARD(unit_param[ui] >= 0 && unit_param[ui] < dbg.n_aux, ui);
         const float* src = master + u.shard_pos;
         const int len = u.len;
         const int head = (int)head_to_16B(src, len);
@@ -240,9 +248,11 @@ __device__ __forceinline__ void zero_u8_run(uint8_t* __restrict__ dst, int len) 
 __global__ void __launch_bounds__(kThreads, 4)
 k_fp8_copy_in(const float* __restrict__ master, uint8_t* __restrict__ ag8,
               const float* __restrict__ scales, const Unit* __restrict__ units,
-              const int32_t* __restrict__ unit_param, int64_t n_units) {
+              const int32_t* __restrict__ unit_param, int64_t n_units FSDPK_DBG_PARAM) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard);
+        FSDPK_GUARD(u.is_pad || (unit_param[ui] >= 0 && unit_param[ui] < dbg.n_aux), ui);
         uint8_t* dst = ag8 + u.shard_pos;
         const int len = u.len;
         if (u.is_pad) {
@@ -295,9 +305,11 @@ __device__ __forceinline__ uint4 shift_bytes16(const uint4& a, const uint4& b, i
 template <bool TAB>
 __global__ void __launch_bounds__(kThreads, 5)
 k_fp8_copy_out(const uint8_t* __restrict__ ag8, const uint8_t* const* __restrict__ unit_src,
-               uint8_t* __restrict__ arena8, const Unit* __restrict__ units, int64_t n_units) {
+               uint8_t* __restrict__ arena8, const Unit* __restrict__ units,
+               int64_t n_units FSDPK_DBG_PARAM) {
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, TAB ? kChkArena : (kChkShard | kChkArena));
         const int len = u.len;
         uint8_t* dst = arena8 + u.arena_pos;
         const uint8_t* src;
@@ -351,7 +363,8 @@ cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* a
     const bool pads = !g.tile_ranges.empty();
     k_copy_in<<<grid_for(g, (const void*)k_copy_in, g.n_tiles), kThreads, 0, st>>>(
         master, ag, count, g.n_tiles, pads ? g.d_intervals : nullptr,
-        pads ? g.d_tile_ranges : nullptr);
+        pads ? g.d_tile_ranges : nullptr
+        FSDPK_DBG_ARG(debug_bounds(g, kDbgCopyIn, (int64_t)g.intervals.size())));
     return cudaGetLastError();
 }
 
@@ -359,7 +372,7 @@ cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* a
                             cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
     k_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
-        ag, nullptr, arena, g.d_units, g.n_real_units);
+        ag, nullptr, arena, g.d_units, g.n_real_units FSDPK_DBG_ARG(debug_bounds(g, kDbgCopyOut)));
     return cudaGetLastError();
 }
 
@@ -367,7 +380,8 @@ cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const*
                                 uint16_t* arena, cudaStream_t st) {
     if (parent.n_real_units == 0) return cudaSuccess;
     k_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
-        nullptr, unit_src, arena, parent.d_units, parent.n_real_units);
+        nullptr, unit_src, arena, parent.d_units, parent.n_real_units
+        FSDPK_DBG_ARG(debug_bounds(parent, kDbgCopyOutTab)));
     return cudaGetLastError();
 }
 
@@ -375,8 +389,8 @@ cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
                          cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
     if (nu == 0) return cudaSuccess;
-    k_shard<<<grid_for(g, (const void*)k_shard, nu), kThreads, 0, st>>>(full, master, g.d_units,
-                                                                        nu);
+    k_shard<<<grid_for(g, (const void*)k_shard, nu), kThreads, 0, st>>>(
+        full, master, g.d_units, nu FSDPK_DBG_ARG(debug_bounds(g, kDbgShard)));
     return cudaGetLastError();
 }
 
@@ -388,13 +402,14 @@ cudaError_t launch_copy_in_fp8(const fsdp_group& g, const float* master, uint8_t
         if (g.n_real_units > 0)
             k_fp8_amax<<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
                 master, reinterpret_cast<unsigned*>(scales), g.d_units, g.d_unit_param,
-                g.n_real_units);
+                g.n_real_units FSDPK_DBG_ARG(debug_bounds(g, kDbgFp8Amax, g.n)));
         k_fp8_scales<<<(unsigned)((g.n + kThreads - 1) / kThreads), kThreads, 0, st>>>(scales, g.n);
     }
     const int64_t nu = (int64_t)g.units.size();
     if (nu > 0)
-        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(master, ag8, scales,
-                                                                     g.d_units, g.d_unit_param, nu);
+        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
+            master, ag8, scales, g.d_units, g.d_unit_param, nu
+            FSDPK_DBG_ARG(debug_bounds(g, kDbgFp8CopyIn, g.n)));
     return cudaGetLastError();
 }
 
@@ -408,8 +423,9 @@ cudaError_t launch_copy_in_fp8_scaled(const fsdp_group& g, const float* master, 
                                       const float* scales, cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
     if (nu > 0)
-        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(master, ag8, scales,
-                                                                     g.d_units, g.d_unit_param, nu);
+        k_fp8_copy_in<<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
+            master, ag8, scales, g.d_units, g.d_unit_param, nu
+            FSDPK_DBG_ARG(debug_bounds(g, kDbgFp8CopyIn, g.n)));
     return cudaGetLastError();
 }
 
@@ -417,7 +433,8 @@ cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t
                                 cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
     k_fp8_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
-        ag8, nullptr, arena8, g.d_units, g.n_real_units);
+        ag8, nullptr, arena8, g.d_units, g.n_real_units
+        FSDPK_DBG_ARG(debug_bounds(g, kDbgFp8CopyOut)));
     return cudaGetLastError();
 }
 
@@ -425,7 +442,8 @@ cudaError_t launch_copy_out_fp8_tab(const fsdp_group& parent, const uint8_t* con
                                     uint8_t* arena8, cudaStream_t st) {
     if (parent.n_real_units == 0) return cudaSuccess;
     k_fp8_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
-        nullptr, unit_src, arena8, parent.d_units, parent.n_real_units);
+        nullptr, unit_src, arena8, parent.d_units, parent.n_real_units
+        FSDPK_DBG_ARG(debug_bounds(parent, kDbgFp8CopyOutTab)));
     return cudaGetLastError();
 }
 

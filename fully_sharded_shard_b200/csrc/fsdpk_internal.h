@@ -46,6 +46,26 @@ struct TileRange {
     int32_t end;
 };
 
+// Debug build (-DFSDPK_DEBUG): the extents a table-driven kernel checks every
+// work unit (or tile) against before touching memory through it.  A unit that
+// would reach outside is skipped and counted in the caller's error words
+// (fsdp_debug_set_error_words); nothing traps and nothing waits.
+struct DebugBounds {
+    int64_t ns;       // elements of the [L][S] buffers that shard positions index
+    int64_t arena;    // elements of one unsharded arena that arena positions index
+    int64_t n_aux;    // entries of the side table the kernel indexes (pad
+                      // intervals, or parameters for the FP8 kernels)
+    uint32_t* words;  // [count, kernel id, unit or tile index, block], or null
+    int32_t kernel;   // DebugKernel of the launch
+};
+
+// Kernel ids recorded with the first violation.
+enum DebugKernel : int32_t {
+    kDbgCopyIn = 1, kDbgCopyOut, kDbgCopyOutTab, kDbgShard, kDbgReduce, kDbgReduceTab,
+    kDbgRsAdamw, kDbgRsAdamwTab, kDbgReduceAcc, kDbgFp8Amax, kDbgFp8CopyIn, kDbgFp8CopyOut,
+    kDbgFp8CopyOutTab, kDbgSmallStep, kDbgCopyInF32, kDbgCopyOutF32
+};
+
 }  // namespace fsdpk
 
 // The opaque plan behind fsdp_group_t.
@@ -107,6 +127,11 @@ int record_cuda_error(cudaError_t e);
 // FSDP_OK when the current device is g's, FSDP_ESTATE (or FSDP_ECUDA) otherwise.
 int check_plan_device(const fsdp_group* g);
 
+// The bounds of a launch over g's tables (debug build; the words and the
+// test-only shrink come from fsdp_debug_set_error_words).
+DebugBounds debug_bounds(const fsdp_group& g, int32_t kernel, int64_t n_aux = 0);
+DebugBounds debug_bounds_raw(int64_t ns, int64_t arena, int32_t kernel, int64_t n_aux = 0);
+
 // Scalars of one AdamW step, precomputed on the host in binary64.
 struct AdamScalars {
     float decay;         // 1 - lr*wd
@@ -146,7 +171,7 @@ cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
 // instead of a plan's own table.
 cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Unit* units,
                                   int64_t n_units, const uint16_t* grads, int op, float* reduced,
-                                  cudaStream_t st);
+                                  cudaStream_t st, int64_t NS);
 
 // The exchange steps over pointer tables in device memory: the copy-out
 // pulling each of the parent's real units from unit_src[unit] (inside the

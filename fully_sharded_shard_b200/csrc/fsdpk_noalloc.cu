@@ -4,8 +4,10 @@
 // The work table that fsdp_plan_group would upload into a cudaMalloc'd
 // buffer lives here in a fixed array in the library's own device memory.
 // Host code never uses the array's name as a pointer (in host code it is
-// only a stand-in for the device symbol); it looks the device address up
-// once per device with cudaGetSymbolAddress and passes that address on.
+// only a stand-in for the device symbol); every call looks the device
+// address up with cudaGetSymbolAddress on the current device and passes
+// that address on, so a device reset or another context never leaves a
+// stale address behind.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -18,7 +20,6 @@
 namespace {
 
 constexpr int64_t kMaxUnits = FSDP_NOALLOC_MAX_UNITS;
-constexpr int kMaxDevices = 64;
 
 // The shared work table: FSDP_NOALLOC_MAX_UNITS x 24 bytes on every device
 // that loads the library.  Only the first n_units entries of the current
@@ -26,12 +27,13 @@ constexpr int kMaxDevices = 64;
 // has to start at zero.
 static __device__ __align__(256) fsdpk::Unit g_noalloc_units[kMaxUnits];
 
-// Host staging copy of the table (static storage, not allocated per call)
-// and the per-device set-up results.  One mutex serialises host threads.
+// Host staging copy of the table (static storage, not allocated per call).
+// One mutex serialises host threads.  The copy to the device reads this
+// array when the call enqueues it, so a call is refused while its stream is
+// being captured: a captured copy would read whatever table a later call
+// left here each time the graph is replayed.
 std::mutex g_mu;
 fsdpk::Unit g_host_units[kMaxUnits];
-fsdpk::Unit* g_dev_units[kMaxDevices] = {};
-int g_dev_sms[kMaxDevices] = {};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -105,23 +107,23 @@ extern "C" int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_p
     if (NS > 0 && reduced == nullptr) return FSDP_EINVAL;
     if (P > 0 && grads == nullptr) return FSDP_EINVAL;
 
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    const cudaError_t qe = cudaStreamIsCapturing(st, &cap);
+    if (qe == cudaErrorStreamCaptureImplicit) {  // the legacy stream while another captures
+        (void)cudaGetLastError();
+        return FSDP_ESTATE;
+    }
+    if (qe != cudaSuccess) return FSDP_ECUDA;
+    if (cap != cudaStreamCaptureStatusNone) return FSDP_ESTATE;
+
     std::lock_guard<std::mutex> lock(g_mu);
 
-    // once per device: the device address of the table and the SM count
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return FSDP_ECUDA;
-    if (dev < 0 || dev >= kMaxDevices) return FSDP_ECUDA;
-    if (g_dev_units[dev] == nullptr) {
-        void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_noalloc_units);
-        if (e != cudaSuccess || ptr == nullptr) return FSDP_ECUDA;
-        int sms = 0;
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return FSDP_ECUDA;
-        g_dev_sms[dev] = sms;
-        g_dev_units[dev] = static_cast<fsdpk::Unit*>(ptr);
-    }
+    // the array's address on the current device (the first call on a device
+    // loads the library's device code and this array there)
+    void* dev_units = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&dev_units, g_noalloc_units);
+    if (e != cudaSuccess || dev_units == nullptr) return FSDP_ECUDA;
 
     // pass 2: the table -- real runs for every (rank j, parameter i), then pads
     int64_t n_units = 0;
@@ -147,11 +149,12 @@ extern "C" int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_p
     }
     if (n_units == 0) return FSDP_OK;
 
-    cudaStream_t st = (cudaStream_t)stream;
-    e = cudaMemcpyAsync(g_dev_units[dev], g_host_units, (size_t)n_units * sizeof(fsdpk::Unit),
+    e = cudaMemcpyAsync(dev_units, g_host_units, (size_t)n_units * sizeof(fsdpk::Unit),
                         cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return FSDP_ECUDA;
-    e = fsdpk::launch_rs_fused_units(g_dev_sms[dev], world_size, P_arena, g_dev_units[dev],
-                                     n_units, grads, op, reduced, st);
+    // the grid covers the units once and does not depend on the SM count
+    e = fsdpk::launch_rs_fused_units(0, world_size, P_arena,
+                                     static_cast<const fsdpk::Unit*>(dev_units), n_units, grads,
+                                     op, reduced, st, NS);
     return e == cudaSuccess ? FSDP_OK : FSDP_ECUDA;
 }

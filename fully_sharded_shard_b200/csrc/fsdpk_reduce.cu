@@ -153,13 +153,14 @@ template <int NR>
 __global__ void __launch_bounds__(kThreads, (NR >= 3 && NR <= 8) ? 4 : 3)
 k_reduce_units(const uint16_t* __restrict__ grads, int64_t stride, int N,
                float* __restrict__ out, int64_t y_src_step, int64_t y_dst_step,
-               const Unit* __restrict__ units, int64_t n_units, int op_avg) {
+               const Unit* __restrict__ units, int64_t n_units, int op_avg FSDPK_DBG_PARAM) {
     const uint16_t* gsrc = grads + (int64_t)blockIdx.y * y_src_step;
     float* gdst = out + (int64_t)blockIdx.y * y_dst_step;
     const bool avg = op_avg != 0;
     const float fN = (float)N;
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
         const int len = u.len;
         float* dst_run = gdst + u.shard_pos;
         if (u.is_pad) {
@@ -175,13 +176,14 @@ k_reduce_units(const uint16_t* __restrict__ grads, int64_t stride, int N,
 template <int NR>
 __global__ void __launch_bounds__(kThreads, (NR >= 3 && NR <= 8) ? 4 : 3)
 k_reduce_units_tab(const uint16_t* const* __restrict__ rank_tab, int N, float* __restrict__ out,
-                   const Unit* __restrict__ units, int64_t n_units, int op_avg) {
+                   const Unit* __restrict__ units, int64_t n_units, int op_avg FSDPK_DBG_PARAM) {
     __shared__ const uint16_t* s_tab[kPeerMaxRanks];
     load_rank_table(rank_tab, s_tab, N);
     const bool avg = op_avg != 0;
     const float fN = (float)N;
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
         float* dst_run = out + u.shard_pos;
         if (u.is_pad) {
             zero_f32_run(dst_run, u.len);
@@ -309,11 +311,12 @@ template <bool WITH_G>
 __global__ void __launch_bounds__(kThreads, 2)
 k_reduce_acc(const float* __restrict__ acc, const uint16_t* __restrict__ g, int64_t stride, int N,
              float* __restrict__ out, const Unit* __restrict__ units, int64_t n_units,
-             int op_avg) {
+             int op_avg FSDPK_DBG_PARAM) {
     const bool avg = op_avg != 0;
     const float fN = (float)N;
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
         const int len = u.len;
         float* dst = out + u.shard_pos;
         if (u.is_pad) {
@@ -389,11 +392,13 @@ template <int NR>
 cudaError_t launch_reduce_nr(const fsdp_group& g, const uint16_t* grads, int64_t stride, int N,
                              float* out, int64_t y_src_step, int64_t y_dst_step,
                              unsigned ydim, const Unit* units, int64_t n_units, int avg,
-                             cudaStream_t st) {
+                             cudaStream_t st, const DebugBounds& dbg) {
+    (void)dbg;
     const void* kfn = (const void*)k_reduce_units<NR>;
     dim3 grid(grid_for(g, kfn, n_units), ydim);
     k_reduce_units<NR><<<grid, kThreads, 0, st>>>(grads, stride, N, out, y_src_step,
-                                                  y_dst_step, units, n_units, avg);
+                                                  y_dst_step, units, n_units, avg
+                                                  FSDPK_DBG_ARG(dbg));
     return cudaGetLastError();
 }
 
@@ -409,34 +414,36 @@ cudaError_t launch_rs_fused(const fsdp_group& g, const uint16_t* grads, int op, 
     if (nu == 0) return cudaSuccess;
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
     const int64_t stride = g.P_arena;
+    const DebugBounds dbg = debug_bounds(g, kDbgReduce);
     switch (g.N) {
 #define FSDPK_CASE(K) \
-    case K: return launch_reduce_nr<K>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg, st);
+    case K: return launch_reduce_nr<K>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg, st, dbg);
         FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
         FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
 #undef FSDPK_CASE
         default:
             return launch_reduce_nr<0>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg,
-                                       st);
+                                       st, dbg);
     }
 }
 
 cudaError_t launch_rs_fused_units(int sm_count, int N, int64_t P_arena, const Unit* units,
                                   int64_t n_units, const uint16_t* grads, int op, float* reduced,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, int64_t NS) {
     if (n_units == 0) return cudaSuccess;
     fsdp_group g;  // only the SM count is read when sizing the grid
     g.sm_count = sm_count;
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
+    const DebugBounds dbg = debug_bounds_raw(NS, P_arena, kDbgReduce);
     switch (N) {
 #define FSDPK_CASE(K) \
-    case K: return launch_reduce_nr<K>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg, st);
+    case K: return launch_reduce_nr<K>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg, st, dbg);
         FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
         FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
 #undef FSDPK_CASE
         default:
             return launch_reduce_nr<0>(g, grads, P_arena, N, reduced, 0, 0, 1, units, n_units, avg,
-                                       st);
+                                       st, dbg);
     }
 }
 
@@ -444,8 +451,8 @@ template <int NR>
 cudaError_t launch_reduce_tab_nr(const fsdp_group& g, const uint16_t* const* tab, float* out,
                                  int avg, cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
-    k_reduce_units_tab<NR><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(tab, g.N, out,
-                                                                          g.d_units, nu, avg);
+    k_reduce_units_tab<NR><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
+        tab, g.N, out, g.d_units, nu, avg FSDPK_DBG_ARG(debug_bounds(g, kDbgReduceTab)));
     return cudaGetLastError();
 }
 
@@ -470,7 +477,7 @@ cudaError_t launch_rs_pack(const fsdp_group& g, const uint16_t* grads, float* pa
     if (nu == 0) return cudaSuccess;
     // blockIdx.y = source rank r: reads rank r's arena, writes packed[r]
     return launch_reduce_nr<1>(g, grads, 0, 1, packed, g.P_arena, (int64_t)g.N * g.S,
-                               (unsigned)g.N, g.d_units, nu, 0, st);
+                               (unsigned)g.N, g.d_units, nu, 0, st, debug_bounds(g, kDbgReduce));
 }
 
 cudaError_t launch_rs_reduce_packed(const fsdp_group& g, const float* packed, int op,
@@ -518,10 +525,12 @@ cudaError_t launch_rs_reduce_acc(const fsdp_group& g, const uint16_t* grads, con
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
     if (grads != nullptr)
         k_reduce_acc<true><<<grid_for(g, (const void*)k_reduce_acc<true>, nu), kThreads, 0, st>>>(
-            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg
+            FSDPK_DBG_ARG(debug_bounds(g, kDbgReduceAcc)));
     else
         k_reduce_acc<false><<<grid_for(g, (const void*)k_reduce_acc<false>, nu), kThreads, 0, st>>>(
-            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg);
+            acc, grads, g.P_arena, g.N, reduced, g.d_units, nu, avg
+            FSDPK_DBG_ARG(debug_bounds(g, kDbgReduceAcc)));
     return cudaGetLastError();
 }
 

@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, (NR >= 1 && NR <= 8) ? 3 : 2)
 k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride,
            const uint16_t* const* __restrict__ rank_tab, int N, FusedOut o,
            const Unit* __restrict__ units, int64_t n_units, int op_avg, AdamScalars sc,
-           const AdamScalars* __restrict__ sc_dev) {
+           const AdamScalars* __restrict__ sc_dev FSDPK_DBG_PARAM) {
     __shared__ float part[kThreads / 32];
     __shared__ const uint16_t* s_tab[TAB ? kPeerMaxRanks : 1];
     if constexpr (TAB) load_rank_table(rank_tab, s_tab, N);
@@ -290,6 +290,9 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride,
     const float fN = (float)N;
     for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
         const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
+        if constexpr (FP8)
+            FSDPK_GUARD(u.is_pad || (o.unit_param[ui] >= 0 && o.unit_param[ui] < dbg.n_aux), ui);
         const int len = u.len;
         const int64_t k0 = u.shard_pos;
         float scale = 0.0f, mx = 0.0f;
@@ -345,7 +348,8 @@ cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const
                                cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
     k_rs_adamw<NR, FP8, false><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
-        grads, g.P_arena, nullptr, g.N, o, g.d_units, nu, avg, sc, sc_dev);
+        grads, g.P_arena, nullptr, g.N, o, g.d_units, nu, avg, sc, sc_dev
+        FSDPK_DBG_ARG(debug_bounds(g, kDbgRsAdamw, g.n)));
     return cudaGetLastError();
 }
 
@@ -434,7 +438,8 @@ cudaError_t launch_rs_adamw_tab_nr(const fsdp_group& g, const uint16_t* const* t
                                    cudaStream_t st) {
     const int64_t nu = (int64_t)g.units.size();
     k_rs_adamw<NR, FP8, true><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
-        nullptr, 0, tab, g.N, o, g.d_units, nu, avg, sc, nullptr);
+        nullptr, 0, tab, g.N, o, g.d_units, nu, avg, sc, nullptr
+        FSDPK_DBG_ARG(debug_bounds(g, kDbgRsAdamwTab, g.n)));
     return cudaGetLastError();
 }
 

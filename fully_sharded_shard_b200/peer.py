@@ -13,6 +13,16 @@ folding ranks 0..N-1 in order exactly as on one device.
 torch.distributed is plumbing here: it swaps the 64-byte IPC handles once and
 provides the barrier that orders the devices between the phases of a step.
 Without an initialised process group everything runs as one device (D = 1).
+
+Two orderings across devices:
+  PeerGroup           -- two host barriers per step, each after a device
+                         synchronisation (the phases of every device drain);
+  PipelinedPeerGroup  -- one host barrier per step and no device
+                         synchronisation: every cross-device dependency is a
+                         stream wait on another process's CUDA event (CUDA IPC
+                         events), with the slots and gradient arenas double
+                         buffered by step parity, so one group's exchange
+                         overlaps another group's update on the GPU.
 """
 from __future__ import annotations
 
@@ -55,6 +65,15 @@ def exchange(obj, group=None) -> list:
 def barrier(device, group=None) -> None:
     """Every device's queued work is complete before any device goes on."""
     torch.cuda.synchronize(device)
+    if _world(group)[0] > 1:
+        dist.barrier(group=group)
+
+
+def host_barrier(group=None) -> None:
+    """Every process of the group has reached this point of its program (what
+    it enqueued before is enqueued; nothing is waited for on a device).  A
+    process that has left raises here in the others within the process
+    group's timeout."""
     if _world(group)[0] > 1:
         dist.barrier(group=group)
 
@@ -204,3 +223,158 @@ class PeerGroup:
         self.pp.destroy()
         self.g.destroy()
         self.pp = None
+
+
+class PeerEvents:
+    """Named interprocess CUDA events of this process, opened by every other
+    process of the group: record(name) marks a point on one of this process's
+    streams; wait_all(name) makes a stream wait for that point on every
+    device (this one included).  A wait on an event never recorded is a
+    no-op, so the first step waits for nothing."""
+
+    def __init__(self, names: Sequence[str], *, group=None, device=None):
+        self.D, self.d = _world(group)
+        with torch.cuda.device(device):
+            self.own = {n: torch.cuda.Event(interprocess=True) for n in names}
+            handles = {n: e.ipc_handle() for n, e in self.own.items()}
+        self.peers = []
+        for j, h in enumerate(exchange(handles, group)):
+            if j == self.d:
+                self.peers.append(self.own)
+            else:
+                self.peers.append({n: torch.cuda.Event.from_ipc_handle(device, h[n])
+                                   for n in names})
+
+    def record(self, name: str, stream) -> None:
+        self.own[name].record(stream)
+
+    def wait_all(self, name: str, stream) -> None:
+        for ev in self.peers:
+            stream.wait_event(ev[name])
+
+
+def _round_up(x: int, k: int) -> int:
+    return (x + k - 1) // k * k
+
+
+class PipelinedPeerGroup:
+    """This device's part of one parameter group, ordered across devices by
+    CUDA IPC events instead of device-draining barriers.
+
+    Buffers come in two copies, selected by the parity of the step
+    (par = step % 2): the all-gather slot rows [L][S] and the gradient arenas
+    [L][P_arena].  Each call waits, on the stream it is given, for the events
+    of every device that the data it touches depends on, and records its own:
+      copy_in(par)       waits: every device done reading slot[par] (the
+                         copy-outs two steps back); writes slot[par];
+                         records "in{par}"
+      copy_out(par)      waits: every device's "in{par}"; pulls every rank's
+                         slot[par] rows; records "out{par}"
+      grads_begin(par)   waits: every device done reading grads[par]
+      grads_end(par)     records "gw{par}" (the caller wrote grads[par])
+      rs_reduce(par)     waits: every device's "gw{par}"; pulls; records "gr{par}"
+      rs_adamw_step(par) as rs_reduce, and with the next copy-in it also waits
+                         for every device done reading slot[1 - par] and
+                         records "in{1 - par}" after writing it
+    The caller runs each step in two phases with ONE host barrier between
+    them (host_barrier(), which waits for no device): phase A enqueues the
+    step's copy-ins and gradient writes, phase B its copy-outs and
+    reductions.  That barrier is what makes every wait see the record it
+    needs: a wait of phase B sees the records of phase A of the same step,
+    and a wait of phase A sees the records of phase B two steps back (the
+    buffers of the other parity serve the step in between).  Ordering inside
+    this process (for example an update before the next copy-in of the same
+    master) is the caller's, as with any two streams."""
+
+    EVENTS = tuple(f"{k}{p}" for k in ("in", "out", "gw", "gr") for p in (0, 1))
+
+    def __init__(self, shapes: Sequence[Sequence[int]], N: int, *, group=None, device=None,
+                 grads: Optional["PipelinedPeerGroup"] = None):
+        self.pg = group
+        self.device = torch.device(device) if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
+        self.D, self.d = _world(group)
+        self.g = abi.fsdp_plan_group(shapes, N)
+        self.pps = [abi.fsdp_peer_plan(self.g, self.D, self.d) for _ in range(2)]
+        L, S, A = self.pps[0].L, self.g.S, self.g.P_arena
+        self.L, self.r0, self.S, self.P_arena, self.N = L, self.pps[0].r0, S, A, self.g.N
+        self._slot_half = _round_up(2 * L * S, 256)
+        self._grad_half = _round_up(2 * L * A, 256)
+        self.slot_buf = SharedBuffer(2 * self._slot_half, group=group, device=self.device)
+        # `grads`: share another instance's gradient arenas (same shapes), for
+        # gradients that are written once and only read afterwards
+        self._own_grads = grads is None
+        if grads is None:
+            self.grad_buf = SharedBuffer(2 * self._grad_half, group=group, device=self.device)
+        elif grads.P_arena != A or grads.L != L:
+            raise ValueError("shared gradient arenas of another layout")
+        else:
+            self.grad_buf = grads.grad_buf
+        self.ag_slots, self.grads = [], []
+        for par in range(2):
+            so, go = par * self._slot_half, par * self._grad_half
+            self.ag_slots.append(abi.device_tensor(self.slot_buf.ptr + so, L * S, torch.bfloat16,
+                                                   self.device))
+            self.grads.append(abi.device_tensor(self.grad_buf.ptr + go, L * A, torch.bfloat16,
+                                                self.device).view(L, A))
+            ag, gr = rank_pointer_tables([b + so for b in self.slot_buf.bases],
+                                         [b + go for b in self.grad_buf.bases], L, S, A)
+            abi.fsdp_peer_set_sources(self.pps[par], ag, gr)
+        self.ev = PeerEvents(self.EVENTS, group=group, device=self.device)
+        barrier(self.device, group)
+
+    # phase A
+    def copy_in(self, par: int, master: torch.Tensor, stream) -> None:
+        self.ev.wait_all(f"out{par}", stream)
+        abi.fsdp_peer_copy_in(self.pps[par], master, self.ag_slots[par], stream)
+        self.ev.record(f"in{par}", stream)
+
+    def grads_begin(self, par: int, stream) -> torch.Tensor:
+        """Wait until no device still reads grads[par]; returns the buffer to
+        write on `stream` (call grads_end after the write)."""
+        self.ev.wait_all(f"gr{par}", stream)
+        return self.grads[par]
+
+    def grads_end(self, par: int, stream) -> None:
+        self.ev.record(f"gw{par}", stream)
+
+    # phase B
+    def copy_out(self, par: int, arena: torch.Tensor, stream) -> None:
+        self.ev.wait_all(f"in{par}", stream)
+        abi.fsdp_peer_copy_out(self.pps[par], arena, stream)
+        self.ev.record(f"out{par}", stream)
+
+    def rs_reduce(self, par: int, op: int, reduced: torch.Tensor, stream) -> None:
+        self.ev.wait_all(f"gw{par}", stream)
+        abi.fsdp_peer_rs_reduce(self.pps[par], op, reduced, stream)
+        self.ev.record(f"gr{par}", stream)
+
+    def rs_adamw_step(self, par: int, op: int, master, m, v, *, stream, next_copy_in: bool = True,
+                      reduced: Optional[torch.Tensor] = None, **hp) -> None:
+        nxt = 1 - par
+        self.ev.wait_all(f"gw{par}", stream)
+        if next_copy_in:
+            self.ev.wait_all(f"out{nxt}", stream)
+        abi.fsdp_peer_rs_adamw_step(self.pps[par], op, master, m, v,
+                                    ag_next=self.ag_slots[nxt] if next_copy_in else None,
+                                    reduced=reduced, stream=stream, **hp)
+        self.ev.record(f"gr{par}", stream)
+        if next_copy_in:
+            self.ev.record(f"in{nxt}", stream)
+
+    def buffers(self) -> List[SharedBuffer]:
+        return [self.slot_buf] + ([self.grad_buf] if self._own_grads else [])
+
+    def close(self) -> None:
+        """Release the shared buffers (after barriers that drain every device,
+        so that no peer still reads them), the events and the plans.  An
+        instance that shares another's gradient arenas closes first."""
+        if self.pps is None:
+            return
+        self.ag_slots = self.grads = None
+        release_all(self.buffers(), self.device, self.pg)
+        self.ev = None
+        for pp in self.pps:
+            pp.destroy()
+        self.g.destroy()
+        self.pps = None

@@ -95,7 +95,10 @@ typedef enum {
     FSDP_ENOMEM = -2, /* host or device allocation of the plan failed      */
     FSDP_ECUDA = -3,  /* a CUDA runtime call or kernel launch failed       */
     FSDP_EALIGN = -4, /* a data pointer is not 16-byte aligned             */
-    FSDP_ESTATE = -5  /* plan used on a device other than its own          */
+    FSDP_ESTATE = -5  /* call not valid now: plan used on a device other
+                         than its own, a host-only plan given to a data
+                         call, or (fsdp_rs_reduce_noalloc) a capturing
+                         stream                                            */
 } fsdp_status;
 
 /* Reduce-scatter reduction ([ML] Other controls; The bug Adam hid). */
@@ -155,18 +158,30 @@ FSDP_API int fsdp_plan_group_host(const fsdp_param_desc* params, int32_t n_param
  * checks (0 for every plan this library builds).  Host only. */
 FSDP_API int fsdp_group_check(fsdp_group_t group, int64_t* violations);
 
-/* S (per-rank padded shard elements), P (real elements), P_arena.
- * Any output pointer may be NULL. */
+/* S (per-rank padded shard elements), P (real elements), P_arena of a plan:
+ * the sizes of one rank's padded shard of the group and of the unsharded
+ * group ("Sharded Training: FSDP2, DTensor, Tensor and Pipeline
+ * Parallelism", fully_shard paragraph: each rank keeps chunk r of
+ * torch.chunk along dim 0, padded when the rows do not divide).  Host only;
+ * any output pointer may be NULL.  Errors: FSDP_EINVAL (NULL group). */
 FSDP_API int fsdp_group_sizes(fsdp_group_t group, int64_t* S, int64_t* P,
                      int64_t* P_arena);
 
 /* Per-parameter tables, each an int64 array of n_params entries supplied by
- * the caller (any may be NULL): off_i, u_i and c_i. */
+ * the caller (any may be NULL): off_i (where parameter i's padded shard
+ * starts inside a rank's [S] slot), u_i (its start in the unsharded arena)
+ * and c_i (the torch.chunk chunk rows, ceil(d0_i / N)) -- the per-parameter
+ * placement of the same fully_shard paragraph.  Host only.
+ * Errors: FSDP_EINVAL (NULL group). */
 FSDP_API int fsdp_group_param_offsets(fsdp_group_t group, int64_t* shard_off,
                              int64_t* arena_off, int64_t* chunk_rows);
 
-/* Free a plan (NULL is ignored).  Work already enqueued that uses the plan
- * must have completed. */
+/* Free a plan (NULL is ignored): its host tables and its device table.  The
+ * plan is one fully_shard group's pre-computed layout, which FSDP2 keeps for
+ * the life of the module ("PyTorch FSDP2 Guide: Distributed LLM Training with
+ * DTensor", The Architecture, section 2: buffers are planned once and
+ * reused), so this is called once, at tear-down.  Work already enqueued that
+ * uses the plan must have completed. */
 FSDP_API void fsdp_destroy_group(fsdp_group_t group);
 
 /* ------------------------------------------------------------------------ */
@@ -406,22 +421,31 @@ FSDP_API int fsdp_rs_adamw_step_dev(fsdp_group_t group, const uint16_t* grads, i
 /* The fused reduce-scatter of fsdp_rs_reduce (packed_or_null == NULL), for
  * callers that cannot allocate device memory: a custom allocator or memory
  * pool that owns every byte of the device, code running where cudaMalloc is
- * forbidden or would synchronise (inside another library's critical
- * section, a signal-free runtime, a process whose memory budget is fixed up
- * front).  There is no plan object: the group is described by params /
- * n_params / world_size exactly as for fsdp_plan_group, and the work table
- * the kernel needs is written into a fixed array in the library's own
- * device memory (FSDP_NOALLOC_MAX_UNITS entries of 24 bytes, 3 MiB on every
- * GPU that loads the library, held until the process exits).  Nothing is
- * allocated on the device or the host, by this library or any library it
- * calls.  (The pages describe no counterpart of this entry point.)
+ * forbidden (inside another library's critical section, a process whose
+ * memory budget is fixed up front).  There is no plan object: the group is
+ * described by params / n_params / world_size exactly as for
+ * fsdp_plan_group, and the work table the kernel needs is written into a
+ * fixed array in the library's own device memory (FSDP_NOALLOC_MAX_UNITS
+ * entries of 24 bytes, 3 MiB on every GPU that loads the library, held until
+ * the process exits).  The call itself makes no cudaMalloc, cudaFree or
+ * other allocating call.  (The pages describe no counterpart of this entry
+ * point.)
  *   grads: bf16 [N][P_arena] (read); reduced: fp32 [N][S] (written, pads
  *   +0); op: an fsdp_reduce_op; results are bit-identical to fsdp_rs_reduce.
- *   P_arena and S follow the layout rules at the top of this file.
- * The first call on each device looks up the array's device address on the
- * device current at that time; make that first call before any stream
- * capture.  The table is copied from host memory with cudaMemcpyAsync on
- * `stream` before the kernel, so the call returns once the copy is staged.
+ *   P_arena and S follow the layout rules at the top of this file; the
+ *   library cannot see the sizes of the caller's buffers, so they must hold
+ *   at least N*P_arena and N*S elements.
+ * Set-up: the CUDA runtime loads the library's device code, and with it the
+ * 3 MiB array, on the first call on each device (lazy module loading).  Make
+ * that first call at set-up time, before the device's memory is handed to a
+ * pool.  Every call looks the array's address up on the current device.
+ * Ordering: the table is built on the host and copied into the array with
+ * cudaMemcpyAsync on `stream` from pageable host memory, so each call waits
+ * for the work already queued on `stream` before it returns (the copy from
+ * pageable memory synchronises with the stream), and the driver stages the
+ * copy through its own buffers.  That copy reads a host array that the next
+ * call overwrites, so while `stream` is being captured into a CUDA graph the
+ * call returns FSDP_ESTATE and enqueues nothing.
  * Every call shares the one array and leaves its last table there: calls on
  * the same device that overlap on the GPU (different streams without
  * ordering between them) race; serialise them on one stream.  Host threads
@@ -429,7 +453,7 @@ FSDP_API int fsdp_rs_adamw_step_dev(fsdp_group_t group, const uint16_t* grads, i
  * Errors: FSDP_EINVAL for the same argument errors as fsdp_plan_group and
  * fsdp_rs_reduce, and for a group that needs more than
  * FSDP_NOALLOC_MAX_UNITS table entries (nothing is enqueued then);
- * FSDP_EALIGN; FSDP_ECUDA. */
+ * FSDP_EALIGN; FSDP_ESTATE (stream capture, see above); FSDP_ECUDA. */
 FSDP_API int fsdp_rs_reduce_noalloc(const fsdp_param_desc* params, int32_t n_params,
                            int32_t world_size, const uint16_t* grads, int32_t op,
                            float* reduced, fsdp_stream_t stream);
@@ -580,11 +604,35 @@ FSDP_API int fsdp_ipc_close(void* ptr);
 /* Misc                                                                     */
 /* ------------------------------------------------------------------------ */
 
-/* Static description of a status code. */
+/* Static description of a status code (never NULL; unknown codes get a
+ * generic text).  The pages define no error model; the codes are this
+ * library's, so that nothing throws across the C ABI. */
 FSDP_API const char* fsdp_status_string(int status);
 
 /* The cudaError_t of the most recent FSDP_ECUDA on this thread (0 if none). */
 FSDP_API int fsdp_last_cuda_error(void);
+
+/* Debug build.  libfsdpk_debug.so is the same library compiled with
+ * -DFSDPK_DEBUG: every kernel that indexes memory through a plan's work
+ * tables checks each work unit (and each copy-in tile's pad-interval range)
+ * against the extents of the buffers the launch was given -- the [L][S]
+ * buffers, one unsharded arena, the pad-interval or parameter table -- before
+ * touching memory through it.  A unit that would reach outside is skipped and
+ * counted; nothing traps and nothing waits.  The pages describe no
+ * counterpart (their lab guards runs only with a wall-clock limit).
+ * fsdp_debug_build: 1 in the debug library, 0 otherwise.
+ * fsdp_debug_set_error_words: `words` is a caller-owned device buffer of 4
+ * uint32 (4-byte aligned; NULL to stop recording) on the device of the
+ * launches that follow: words[0] counts violations (one per warp that sees
+ * one), words[1..3] hold the first one's kernel id, unit or tile index and
+ * block index.  The caller zeroes it and reads it.  `shrink` (>= 0, tests
+ * only) narrows every launch's extents by that many elements, so that valid
+ * tables trip the checks without any access leaving the real buffers.  The
+ * setting is process-wide and read at each launch.
+ * Errors: FSDP_ESTATE in a release library; FSDP_EINVAL (shrink < 0);
+ * FSDP_EALIGN. */
+FSDP_API int fsdp_debug_build(void);
+FSDP_API int fsdp_debug_set_error_words(uint32_t* words, int64_t shrink);
 
 /* FSDP_ABI_VERSION of the loaded library. */
 FSDP_API int fsdp_abi_version(void);

@@ -101,3 +101,45 @@ def test_peer_and_ipc_calls_reject_bad_arguments_on_host(abi):
     assert L.fsdp_ipc_free(None) == abi.FSDP_EINVAL
     assert L.fsdp_ipc_close(None) == abi.FSDP_EINVAL
     assert ctypes.sizeof(abi.IpcHandle) == 64
+
+
+def test_noalloc_wrapper_derives_sizes_from_the_shapes(abi, oracle):
+    """The binding of fsdp_rs_reduce_noalloc works S and P_arena out of the
+    shapes (the C call cannot see buffer sizes) and refuses caller-supplied
+    values that disagree, before touching the tensors or the library."""
+    import torch
+    cases = [([(7, 3), (5,), (1, 32), (1,), (0, 4), (13, 9), (2, 2)], 4),
+             ([(32003, 64), (4096,), (17, 5)], 6), ([], 3), ([()], 2), ([(9, 5), (3,)], 12)]
+    for shapes, N in cases:
+        p = oracle.plan(shapes, N)
+        assert abi.group_layout(shapes, N) == (p.S, p.P, p.P_arena)
+    shapes, N = cases[0]
+    p = oracle.plan(shapes, N)
+    g = torch.zeros(4, dtype=torch.bfloat16)
+    r = torch.zeros(4)
+    for kw in ({"S": p.S - 1}, {"S": p.S + 8}, {"P_arena": p.P_arena - 8},
+               {"P_arena": p.P_arena + 1}):
+        with pytest.raises(ValueError, match="does not match"):
+            abi.fsdp_rs_reduce_noalloc(shapes, N, g, 1, r, **kw)
+    # right sizes: the next check (CUDA tensors of at least that size) is reached
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        abi.fsdp_rs_reduce_noalloc(shapes, N, g, 1, r, S=p.S, P_arena=p.P_arena)
+
+
+def test_debug_library_loads_and_exports_every_symbol(abi):
+    """libfsdpk_debug.so (-DFSDPK_DEBUG) exports the same C API; only it
+    accepts error words, and it validates them on the host."""
+    from fully_sharded_shard_b200 import build
+    path = build.build(debug=True)
+    D = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(D, n), f"{n} not exported by the debug library"
+    D.fsdp_debug_set_error_words.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+    assert D.fsdp_debug_build() == 1
+    assert D.fsdp_debug_set_error_words(None, -1) == abi.FSDP_EINVAL
+    assert D.fsdp_debug_set_error_words(ctypes.c_void_p(6), 0) == abi.FSDP_EALIGN
+    assert D.fsdp_debug_set_error_words(None, 0) == abi.FSDP_OK
+    R = abi.lib()
+    R.fsdp_debug_set_error_words.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+    assert R.fsdp_debug_build() == 0
+    assert R.fsdp_debug_set_error_words(None, 0) == abi.FSDP_ESTATE

@@ -376,10 +376,12 @@ def test_checkpoint_resume_is_bit_exact(H, tmp_path):
     g.destroy()
 
 
-def _group_step_case(H, wl, grp, steps, graph):
+def _group_step_case(H, wl, grp, steps, graph, full_init=None, grads_init=None):
     """fsdp_group_step (eager, or its _dev form replayed from a CUDA graph)
-    against the four stage calls on a copy of the same state, bit for bit,
-    and its exact stages against the oracle."""
+    against the four stage calls on a copy of the same state, bit for bit
+    (NaN as a class), and against the oracle applied to the step's own
+    inputs: copy-in of the pre-step master, copy-out of that all-gather
+    buffer, the reduce-scatter, and AdamW from the pre-step state."""
     import oracle
     from fully_sharded_shard_b200 import abi
     N, op = wl.N, wl.op
@@ -387,7 +389,11 @@ def _group_step_case(H, wl, grp, steps, graph):
     p = oracle.plan(grp.shapes, N)
     NS, A = N * g.S, g.P_arena
     full = torch.empty(max(A, 1), device="cuda")
-    W.fill_master(full, wl, grp.name)
+    if full_init is None:
+        W.fill_master(full, wl, grp.name)
+    else:
+        full.zero_()
+        full[:A].copy_(torch.from_numpy(np.ascontiguousarray(full_init, np.float32)))
     hp = dict(W.ADAMW_DEFAULTS)
 
     def state():
@@ -400,7 +406,7 @@ def _group_step_case(H, wl, grp, steps, graph):
                                     device="cuda").view(torch.bfloat16),
                 "red": torch.empty(max(NS, 1), device="cuda")}
     a, b = state(), state()
-    grads = [H.make_grads(g, wl, grp, t) for t in range(1, steps + 1)]
+    grads = [H._grads_for(g, wl, grp, t, (), grads_init) for t in range(1, steps + 1)]
     gbuf = torch.empty_like(grads[0])
     if graph:
         ds = abi.DeviceStep()
@@ -412,6 +418,8 @@ def _group_step_case(H, wl, grp, steps, graph):
             abi.fsdp_group_step_dev(g, a["p"], a["m"], a["v"], gbuf, op, ds, ag=a["ag"],
                                     arena=a["arena"], reduced=a["red"])
     for t in range(1, steps + 1):
+        torch.cuda.synchronize()
+        pre = tuple(H.f32(a[k][:NS]) for k in ("p", "m", "v"))
         if graph:
             gbuf.copy_(grads[t - 1])
             cg.replay()
@@ -424,11 +432,20 @@ def _group_step_case(H, wl, grp, steps, graph):
         abi.fsdp_adamw_step(g, b["p"], b["m"], b["v"], b["red"], step=t, **hp)
         torch.cuda.synchronize()
         for k in ("p", "m", "v", "red"):
-            assert torch.equal(a[k].view(torch.int32), b[k].view(torch.int32)), f"{k} step {t}"
+            assert H.equal_nan_class(H.f32(a[k]), H.f32(b[k]), "f32"), f"{k} step {t}"
         for k in ("ag", "arena"):
-            assert torch.equal(a[k].view(torch.int16), b[k].view(torch.int16)), f"{k} step {t}"
+            assert H.equal_nan_class(H.u16(a[k]), H.u16(b[k]), "bf16"), f"{k} step {t}"
+        ag_h = H.u16(a["ag"][:NS])
+        assert H.equal_nan_class(ag_h, oracle.copy_in(p, pre[0]), "bf16"), f"copy-in step {t}"
+        arena_o = oracle.copy_out(p, ag_h, np.full(A, 0x3BEF, np.uint16))
+        assert H.bits_equal(H.u16(a["arena"][:A]), arena_o), f"copy-out step {t}"
         red_o = oracle.reduce_scatter(p, H.u16(grads[t - 1]), op)
-        assert H.bits_equal(H.f32(a["red"][:NS]), red_o)
+        red_h = H.f32(a["red"][:NS])
+        assert H.equal_nan_class(red_h, red_o, "f32"), f"reduce-scatter step {t}"
+        want = H.adamw_from_state(*pre, red_h, t, hp)
+        for k, w in zip(("p", "m", "v"), want):
+            ok, ratio = H.adam_close_special(H.f32(a[k][:NS]), w)
+            assert ok, f"adamw {k} step {t}: {ratio}"
     if graph:
         assert int(ds.step.item()) == steps
         del cg
