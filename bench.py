@@ -1353,6 +1353,26 @@ def run_latency(device, reps: int = 200, graph_steps: int = 20):
         graph.replay()
         graph_single_us = timed(graph.replay) / graph_steps
     del graph
+    # one call per group that also advances the step counter: one launch per
+    # step for a small group, no separate prepare kernel
+    ds2 = abi.DeviceStep(device)
+
+    def graphed_one_call():
+        for gi, master, m, v, pj in model.instances:
+            g = model.plans[gi]
+            abi.fsdp_group_step_graph(g, master, m, v, model.grads[gi][pj], wl.op, ds2,
+                                      ag=model.ag, arena=model.arena, reduced=model.reduced,
+                                      stream=stream, **hp)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(graph_steps):
+            graphed_one_call()
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        graph.replay()
+        graph_one_call_us = timed(graph.replay) / graph_steps
+    del graph
     n_small = sum(1 for gi, *_ in model.instances
                   if wl.N * model.plans[gi].S <= abi.FSDP_SMALL_STEP_ELEMS)
     single_launches = sum(1 if wl.N * model.plans[gi].S <= abi.FSDP_SMALL_STEP_ELEMS else 4
@@ -1367,7 +1387,11 @@ def run_latency(device, reps: int = 200, graph_steps: int = 20):
                            "eager_us_per_step": round(single_us, 2),
                            "eager_host_us_per_step": round(single_host_us, 2),
                            "graph_us_per_step": round(graph_single_us, 2),
-                           "graph_launches_per_step": single_launches + 1}}
+                           "graph_launches_per_step": single_launches + 1},
+            "group_step_graph": {"graph_us_per_step": round(graph_one_call_us, 2),
+                                 "graph_launches_per_step": sum(
+                                     1 if wl.N * model.plans[gi].S <= abi.FSDP_SMALL_STEP_ELEMS
+                                     else 5 for gi, *_ in model.instances)}}
 
 
 def run_e2e(args, model, device, stream, ws):

@@ -122,6 +122,9 @@ def _load() -> ctypes.CDLL:
     L.fsdp_group_step.restype = ctypes.c_int
     L.fsdp_group_step_dev.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp]
     L.fsdp_group_step_dev.restype = ctypes.c_int
+    L.fsdp_group_step_graph.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.POINTER(AdamWHparams),
+                                        vp, vp, vp, vp, vp, vp]
+    L.fsdp_group_step_graph.restype = ctypes.c_int
     L.fsdp_peer_plan.argtypes = [vp, i32, i32, ctypes.POINTER(vp)]
     L.fsdp_peer_local_ranks.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fsdp_peer_set_sources.argtypes = [vp, vp, vp]
@@ -361,6 +364,24 @@ def fsdp_group_step_dev(g: Group, master: torch.Tensor, m: torch.Tensor, v: torc
                                     _ptr(ag, _B16, n, "ag"), _ptr(arena, _B16, g.P_arena, "arena"),
                                     _ptr(reduced, _F32, n, "reduced"), _stream(stream, master)),
            "fsdp_group_step_dev")
+
+
+def fsdp_group_step_graph(g: Group, master: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                          grads: torch.Tensor, op: int, ds: "DeviceStep", *, lr: float,
+                          beta1: float, beta2: float, eps: float, weight_decay: float,
+                          ag: torch.Tensor, arena: torch.Tensor, reduced: torch.Tensor,
+                          stream=None):
+    n = g.N * g.S
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), 0)
+    _check(_lib.fsdp_group_step_graph(g.handle, _ptr(master, _F32, n, "master"),
+                                      _ptr(m, _F32, n, "m"), _ptr(v, _F32, n, "v"),
+                                      _ptr(grads, _B16, g.N * g.P_arena, "grads"), int(op),
+                                      ctypes.byref(hp), _ptr(ds.step, (torch.int64,), 1, "step"),
+                                      _ptr(ds.scalars, _F32, 8, "scalars"),
+                                      _ptr(ag, _B16, n, "ag"),
+                                      _ptr(arena, _B16, g.P_arena, "arena"),
+                                      _ptr(reduced, _F32, n, "reduced"), _stream(stream, master)),
+           "fsdp_group_step_graph")
 
 
 def fsdp_grad_accumulate(g: Group, grads: torch.Tensor, acc: torch.Tensor, first: bool,

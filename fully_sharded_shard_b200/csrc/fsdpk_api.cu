@@ -118,6 +118,37 @@ int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
                            g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);
             }
         g->n_real_units = (int64_t)g->units.size();
+        // long real units first (a CTA each in the copy-outs), then the short
+        // ones, in packs
+        std::vector<size_t> order((size_t)g->n_real_units);
+        for (size_t k = 0; k < order.size(); ++k) order[k] = k;
+        std::stable_partition(order.begin(), order.end(), [&](size_t k) {
+            return g->units[k].len >= fsdpk::kShortRun;
+        });
+        std::vector<Unit> ru(order.size());
+        std::vector<int32_t> rp(order.size());
+        for (size_t k = 0; k < order.size(); ++k) {
+            ru[k] = g->units[order[k]];
+            rp[k] = g->unit_param[order[k]];
+        }
+        std::copy(ru.begin(), ru.end(), g->units.begin());
+        std::copy(rp.begin(), rp.end(), g->unit_param.begin());
+        g->n_long_units = 0;
+        while (g->n_long_units < g->n_real_units &&
+               g->units[(size_t)g->n_long_units].len >= fsdpk::kShortRun)
+            ++g->n_long_units;
+        g->packs.clear();
+        for (int64_t k = g->n_long_units; k < g->n_real_units;) {
+            g->packs.push_back((int32_t)k);
+            int64_t elems = 0, cnt = 0;
+            while (k < g->n_real_units && cnt < fsdpk::kPackUnits &&
+                   (cnt == 0 || elems + g->units[(size_t)k].len <= fsdpk::kPackElems)) {
+                elems += g->units[(size_t)k].len;
+                ++cnt;
+                ++k;
+            }
+        }
+        g->packs.push_back((int32_t)g->n_real_units);
         for (int64_t j = r0; j < r1; ++j)
             for (int32_t i = 0; i < n_params; ++i) {
                 const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
@@ -163,8 +194,9 @@ int upload_tables(fsdp_group* g) {
     const size_t b_iv = g->intervals.size() * sizeof(Interval);
     const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
     const size_t b_up = g->unit_param.size() * sizeof(int32_t);
+    const size_t b_pk = g->packs.size() * sizeof(int32_t);
     auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up);
+    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up) + up256(b_pk);
     if (total == 0) return FSDP_OK;
     e = cudaMalloc(&g->dev_mem, total);
     if (e != cudaSuccess) {
@@ -178,6 +210,8 @@ int upload_tables(fsdp_group* g) {
     g->d_tile_ranges = reinterpret_cast<const TileRange*>(base + up256(b_units) + up256(b_iv));
     g->d_unit_param =
         reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) + up256(b_tr));
+    g->d_packs = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
+                                                  up256(b_tr) + up256(b_up));
     if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && b_iv)
         e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
@@ -186,6 +220,8 @@ int upload_tables(fsdp_group* g) {
                        cudaMemcpyHostToDevice);
     if (e == cudaSuccess && b_up)
         e = cudaMemcpy((void*)g->d_unit_param, g->unit_param.data(), b_up, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && b_pk)
+        e = cudaMemcpy((void*)g->d_packs, g->packs.data(), b_pk, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
         cudaFree(g->dev_mem);
         g->dev_mem = nullptr;
@@ -394,6 +430,16 @@ int64_t check_tables(const fsdp_group& g) {
             if (u.arena_pos < 0 || u.arena_pos + u.len > g.P_arena) ++bad;
         }
     }
+    // long real units first, then the short ones in packs that cover them
+    if (g.n_long_units < 0 || g.n_long_units > g.n_real_units) ++bad;
+    for (int64_t k = 0; k < g.n_real_units && k < (int64_t)g.units.size(); ++k)
+        if ((g.units[(size_t)k].len >= fsdpk::kShortRun) != (k < g.n_long_units)) ++bad;
+    if (g.packs.empty() || g.packs.front() != g.n_long_units || g.packs.back() != g.n_real_units)
+        ++bad;
+    for (size_t p = 0; p + 1 < g.packs.size(); ++p) {
+        const int64_t cnt = (int64_t)g.packs[p + 1] - g.packs[p];
+        if (cnt < 1 || cnt > fsdpk::kPackUnits) ++bad;
+    }
     std::sort(spans.begin(), spans.end());
     int64_t at = 0;
     for (const auto& sp : spans) {
@@ -574,7 +620,8 @@ namespace {
 
 int group_step(fsdp_group_t g, float* master, float* m, float* v, const uint16_t* grads,
                int32_t op, const fsdpk::AdamScalars& sc, const fsdpk::AdamScalars* sc_dev,
-               uint16_t* ag, uint16_t* arena, float* reduced, fsdp_stream_t stream) {
+               uint16_t* ag, uint16_t* arena, float* reduced, fsdp_stream_t stream,
+               const fsdpk::StepCounter& ctr = fsdpk::StepCounter{}) {
     if (op != FSDP_SUM && op != FSDP_AVG && op != FSDP_SUM_THEN_DIV) return FSDP_EINVAL;
     const int64_t NS = (int64_t)g->N * g->S;
     if (NS > 0 && (master == nullptr || m == nullptr || v == nullptr || ag == nullptr ||
@@ -588,11 +635,19 @@ int group_step(fsdp_group_t g, float* master, float* m, float* v, const uint16_t
     if (st != FSDP_OK) return st;
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (NS <= FSDP_SMALL_STEP_ELEMS) {
+    if (NS == 0 && ctr.step != nullptr) {
+        // nothing to update, but the step still counts
+        e = fsdpk::launch_adamw_prepare(ctr.lr, ctr.beta1, ctr.beta2, ctr.eps, ctr.wd, ctr.step,
+                                        ctr.out, s);
+    } else if (NS <= FSDP_SMALL_STEP_ELEMS) {
         e = fsdpk::launch_small_step(*g, master, m, v, grads, op, ag, arena, reduced, sc, sc_dev,
-                                     s);
+                                     s, ctr);
     } else {
-        e = fsdpk::launch_copy_in(*g, master, ag, s);
+        e = cudaSuccess;
+        if (ctr.step != nullptr)  // the counter and the scalars first, for the stage kernels
+            e = fsdpk::launch_adamw_prepare(ctr.lr, ctr.beta1, ctr.beta2, ctr.eps, ctr.wd,
+                                            ctr.step, ctr.out, s);
+        if (e == cudaSuccess) e = fsdpk::launch_copy_in(*g, master, ag, s);
         if (e == cudaSuccess) e = fsdpk::launch_copy_out(*g, ag, arena, s);
         if (e == cudaSuccess) e = fsdpk::launch_rs_fused(*g, grads, op, reduced, s);
         if (e == cudaSuccess) e = fsdpk::launch_adamw(*g, master, m, v, reduced, sc, s, sc_dev);
@@ -620,6 +675,34 @@ int fsdp_group_step_dev(fsdp_group_t g, float* master, float* m, float* v,
     return group_step(g, master, m, v, grads, op, none,
                       reinterpret_cast<const fsdpk::AdamScalars*>(scalars_dev), ag, arena,
                       reduced, stream);
+}
+
+int fsdp_group_step_graph(fsdp_group_t g, float* master, float* m, float* v,
+                          const uint16_t* grads, int32_t op, const fsdp_adamw_hparams* hp,
+                          int64_t* step_dev, fsdp_adamw_dev_scalars* scalars_dev, uint16_t* ag,
+                          uint16_t* arena, float* reduced, fsdp_stream_t stream) {
+    if (g == nullptr || hp == nullptr || step_dev == nullptr || scalars_dev == nullptr)
+        return FSDP_EINVAL;
+    fsdp_adamw_hparams probe = *hp;
+    probe.step = 1;  // the step comes from step_dev; validate the rest
+    fsdpk::AdamScalars unused;
+    if (!adam_scalars(&probe, &unused)) return FSDP_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(step_dev) & 7u) || !aligned16(scalars_dev))
+        return FSDP_EALIGN;
+    fsdpk::StepCounter ctr;
+    ctr.step = step_dev;
+    ctr.out = reinterpret_cast<fsdpk::AdamScalars*>(scalars_dev);
+    ctr.lr = hp->lr;
+    ctr.beta1 = hp->beta1;
+    ctr.beta2 = hp->beta2;
+    ctr.eps = hp->eps;
+    ctr.wd = hp->weight_decay;
+    const int64_t NS = (int64_t)g->N * g->S;
+    // the stage kernels of a large group read the scalars the prepare wrote
+    const fsdpk::AdamScalars* sc_dev =
+        NS <= FSDP_SMALL_STEP_ELEMS ? nullptr : ctr.out;
+    return group_step(g, master, m, v, grads, op, fsdpk::AdamScalars{}, sc_dev, ag, arena,
+                      reduced, stream, ctr);
 }
 
 int fsdp_grad_accumulate(fsdp_group_t g, const uint16_t* grads, float* acc, int32_t first,

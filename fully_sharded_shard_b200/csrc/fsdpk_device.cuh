@@ -168,6 +168,24 @@ __device__ __forceinline__ void adamw1(float& p, float& m, float& v, float g,
     p = fmaf(-sc.step_size, __fdiv_rn(m, denom), p);
 }
 
+// The AdamW scalars of step t, in binary64 on the device, in the same
+// operation order as the host path.
+__device__ __forceinline__ AdamScalars adam_scalars_dev(double lr, double beta1, double beta2,
+                                                        double eps, double wd, int64_t t) {
+    const double bc1 = 1.0 - pow(beta1, (double)t);
+    const double bc2 = 1.0 - pow(beta2, (double)t);
+    AdamScalars sc;
+    sc.decay = (float)(1.0 - lr * wd);
+    sc.beta1 = (float)beta1;
+    sc.omb1 = (float)(1.0 - beta1);
+    sc.beta2 = (float)beta2;
+    sc.omb2 = (float)(1.0 - beta2);
+    sc.step_size = (float)(lr / bc1);
+    sc.inv_bc2_sqrt = (float)(1.0 / sqrt(bc2));
+    sc.eps = (float)eps;
+    return sc;
+}
+
 // FP8 (E4M3 "fn") helpers
 // x * scale clamped to the finite E4M3 range (NaN passes through).
 __device__ __forceinline__ float fp8_in(float x, float sc) {

@@ -102,67 +102,138 @@ k_copy_in(const float* __restrict__ master, uint16_t* __restrict__ ag, int64_t c
 // ---------------------------------------------------------------------------
 // copy-out: arena[arena_pos + e] = ag[shard_pos + e] for each real unit
 // ---------------------------------------------------------------------------
+// The destination of a unit is peeled to a 16-byte boundary; its source then
+// sits at a phase D (in elements) inside its 16-byte vectors, the same for
+// the whole unit.  A misaligned source is read once, in aligned 16-byte
+// vectors: a team of NW warps covers NW x 128 consecutive vectors per pass,
+// warp w's lanes holding vectors w*128 + 32k + lane (k = 0..3), and each
+// output vector takes its upper half from the next source vector, which the
+// next lane holds (one shuffle per 32-bit word); the last lane takes it from
+// lane 0's next slot, or from one extra load after the last slot.
+// Long units get a CTA (a team of 8 warps) each; short units are packed, a
+// warp per unit, so that a group of many small parameters does not pay a
+// CTA launch per run.
 
-template <bool SHIFTED>
-__device__ __forceinline__ void copy_out_body(const uint16_t* __restrict__ src_al,
-                                              uint16_t* __restrict__ dst, int nvec, int D) {
-    constexpr int V = SHIFTED ? 2 : 4;
-    const uint4* s = reinterpret_cast<const uint4*>(src_al);
-    uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll 1
-    for (int q0 = threadIdx.x; q0 < nvec; q0 += blockDim.x * V) {
-        uint4 a[V], b[V];
+__device__ __forceinline__ uint4 shfl_next(const uint4& v, int src) {
+    uint4 r;
+    r.x = __shfl_sync(0xffffffffu, v.x, src);
+    r.y = __shfl_sync(0xffffffffu, v.y, src);
+    r.z = __shfl_sync(0xffffffffu, v.z, src);
+    r.w = __shfl_sync(0xffffffffu, v.w, src);
+    return r;
+}
+
+// The 16 bytes that start D (1..15) bytes into the 32 bytes a:b.
+__device__ __forceinline__ uint4 shift_bytes16(const uint4& a, const uint4& b, int D) {
+    const int s = D >> 2;
+    const uint32_t sh = 8u * (uint32_t)(D & 3);
+    const uint32_t w0 = s == 0 ? a.x : s == 1 ? a.y : s == 2 ? a.z : a.w;
+    const uint32_t w1 = s == 0 ? a.y : s == 1 ? a.z : s == 2 ? a.w : b.x;
+    const uint32_t w2 = s == 0 ? a.z : s == 1 ? a.w : s == 2 ? b.x : b.y;
+    const uint32_t w3 = s == 0 ? a.w : s == 1 ? b.x : s == 2 ? b.y : b.z;
+    const uint32_t w4 = s == 0 ? b.x : s == 1 ? b.y : s == 2 ? b.z : b.w;
+    return make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh),
+                      __funnelshift_r(w2, w3, sh), __funnelshift_r(w3, w4, sh));
+}
+
+// One unit by a team of NW warps (this thread is lane `lane` of warp w of
+// the team, index t = 32 w + lane), in one pass: the team's 4 x 32 x NW
+// slots cover every 16-byte vector of the unit after the destination's head
+// peel (a long unit has at most kUnitElems elements, a short one fewer than
+// kShortRun).  T = uint16_t (bf16) or uint8_t.
+template <int NW, typename T>
+__device__ __forceinline__ void copy_unit(const T* src_run, T* dst_run, int len, int w, int lane,
+                                          int t) {
+    constexpr int kVec = 16 / (int)sizeof(T);
+    static_assert(kUnitElems <= 8 * 128 * 8 && kShortRun <= 128 * 8, "one pass per unit");
+    const int head = (int)head_to_16B(dst_run, len);
+    if (t < head) dst_run[t] = src_run[t];
+    const int nvec = (len - head) / kVec;
+    const int D = (int)((reinterpret_cast<uintptr_t>(src_run + head) / sizeof(T)) & (kVec - 1));
+    const uint4* s = reinterpret_cast<const uint4*>(src_run + head - D);
+    uint4* d = reinterpret_cast<uint4*>(dst_run + head);
+    const int q0 = w * 128;
+    // a misaligned run also reads vector nvec, which holds its last elements
+    const int lim = D ? nvec : nvec - 1;
+    uint4 a[4];
 #pragma unroll
-        for (int k = 0; k < V; ++k) {
-            const int q = q0 + k * blockDim.x;
-            if (q < nvec) {
-                a[k] = ld_src<SHIFTED>(s + q);
-                if constexpr (SHIFTED) b[k] = ld_src<SHIFTED>(s + q + 1);
-            }
-        }
+    for (int k = 0; k < 4; ++k) {
+        const int q = q0 + 32 * k + lane;
+        if (nvec > 0 && q <= lim) a[k] = __ldcs(s + q);
+    }
+    uint4 e = a[0];
+    if (NW > 1 && D != 0 && lane == 0 && q0 + 128 <= nvec) e = __ldcs(s + q0 + 128);
+    const int nxt = (lane + 1) & 31;
 #pragma unroll
-        for (int k = 0; k < V; ++k) {
-            const int q = q0 + k * blockDim.x;
-            if (q < nvec) {
-                uint4 o;
-                if constexpr (SHIFTED) o = shift_bf16x8(a[k], b[k], D);
-                else o = a[k];
-                __stcs(d + q, o);
-            }
+    for (int k = 0; k < 4; ++k) {
+        const int q = q0 + 32 * k + lane;
+        uint4 o = a[k];
+        if (D != 0) {  // uniform across the team
+            // lane l takes lane l+1's vector; lane 31 takes the first vector of
+            // the next 32, which lane 0 holds (its next slot, or e after the last)
+            const uint4 b = shfl_next(lane == 0 ? (k < 3 ? a[k < 3 ? k + 1 : 0] : e) : a[k], nxt);
+            if constexpr (sizeof(T) == 2) o = shift_bf16x8(a[k], b, D);
+            else o = shift_bytes16(a[k], b, D);
         }
+        if (q < nvec) __stcs(d + q, o);
+    }
+    const int done = head + kVec * nvec;
+    if (t < len - done) dst_run[done + t] = src_run[done + t];
+}
+
+// CTAs [0, n_long) copy one long unit each (a team of 8 warps); the others
+// one pack of short units each, a warp per unit.  One launch: the packs'
+// CTAs are the last of the grid, so they are not a second, small grid that
+// waits for SM slots behind another stream's kernel.
+// TAB: unit ui's rows come from unit_src[ui] (a pull from wherever that
+// rank's slot lives, resolved on the host), instead of ag + shard_pos.
+// A pack of short units, a warp per unit: not inlined into k_copy_out, so
+// that its registers do not add to those of the long-unit path.
+template <bool TAB, typename T>
+__device__ __noinline__ void copy_out_pack(const T* __restrict__ ag,
+                                           const T* const* __restrict__ unit_src,
+                                           T* __restrict__ arena, const Unit* __restrict__ units,
+                                           int b, int e FSDPK_DBG_PARAM) {
+    const int lane = threadIdx.x & 31;
+    for (int ui = b + (int)(threadIdx.x >> 5); ui < e; ui += kThreads / 32) {
+        const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, TAB ? kChkArena : (kChkShard | kChkArena));
+        const T* src = TAB ? unit_src[ui] : ag + u.shard_pos;
+        copy_unit<1>(src, arena + u.arena_pos, u.len, 0, lane, lane);
     }
 }
 
-// TAB: unit ui's rows come from unit_src[ui] (a pull from wherever that
-// rank's slot lives, resolved on the host), instead of ag + shard_pos.
-template <bool TAB>
+template <bool TAB, typename T>
 __global__ void __launch_bounds__(kThreads, 5)
-k_copy_out(const uint16_t* __restrict__ ag, const uint16_t* const* __restrict__ unit_src,
-           uint16_t* __restrict__ arena, const Unit* __restrict__ units,
-           int64_t n_units FSDPK_DBG_PARAM) {
-    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+k_copy_out(const T* __restrict__ ag, const T* const* __restrict__ unit_src,
+           T* __restrict__ arena, const Unit* __restrict__ units, int64_t n_long,
+           const int32_t* __restrict__ packs FSDPK_DBG_PARAM) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if ((int64_t)blockIdx.x < n_long) {
+        const int64_t ui = blockIdx.x;
         const Unit u = units[ui];
+#ifdef FSDPK_DEBUG
         // a pulled unit's source is a pointer of the table, not a shard position
-        FSDPK_UNIT_GUARD(u, ui, TAB ? kChkArena : (kChkShard | kChkArena));
-        const int len = u.len;
-        uint16_t* dst_run = arena + u.arena_pos;
-        const uint16_t* src_run;
-        if constexpr (TAB) {
-            src_run = unit_src[ui];
-        } else {
-            src_run = ag + u.shard_pos;
-        }
-        const int head = (int)head_to_16B(dst_run, len);
-        if ((int)threadIdx.x < head) dst_run[threadIdx.x] = src_run[threadIdx.x];
-        const int nvec = (len - head) >> 3;
-        const int D = bf16_phase(src_run + head);
-        const uint16_t* src_al = src_run + head - D;
-        uint16_t* dst = dst_run + head;
-        if (D == 0) copy_out_body<false>(src_al, dst, nvec, 0);
-        else copy_out_body<true>(src_al, dst, nvec, D);
-        const int done = head + 8 * nvec;
-        if ((int)threadIdx.x < len - done) dst_run[done + threadIdx.x] = src_run[done + threadIdx.x];
+        if (!unit_in_bounds(dbg, u, ui, TAB ? kChkArena : (kChkShard | kChkArena))) return;
+#endif
+        const T* src = TAB ? unit_src[ui] : ag + u.shard_pos;
+        copy_unit<kThreads / 32>(src, arena + u.arena_pos, u.len, warp, lane, threadIdx.x);
+        return;
     }
+    const int p = (int)((int64_t)blockIdx.x - n_long);
+    copy_out_pack<TAB>(ag, unit_src, arena, units, packs[p], packs[p + 1] FSDPK_DBG_ARG(dbg));
+}
+
+// The copy-out of a plan's real units: the long ones and the packs.
+template <bool TAB, typename T>
+cudaError_t launch_copy_out_units(const fsdp_group& g, const T* ag, const T* const* unit_src,
+                                  T* arena, int32_t dbg_kernel, cudaStream_t st) {
+    (void)dbg_kernel;
+    const int64_t n_packs = (int64_t)g.packs.size() - 1;
+    k_copy_out<TAB, T><<<grid_for(g, nullptr, g.n_long_units + n_packs), kThreads, 0, st>>>(
+        ag, unit_src, arena, g.d_units, g.n_long_units, g.d_packs
+        FSDPK_DBG_ARG(debug_bounds(g, dbg_kernel)));
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -287,56 +358,6 @@ k_fp8_copy_in(const float* __restrict__ master, uint8_t* __restrict__ ag8,
     }
 }
 
-// The 16 bytes that start D (1..15) bytes into the 32 bytes a:b.
-__device__ __forceinline__ uint4 shift_bytes16(const uint4& a, const uint4& b, int D) {
-    const int s = D >> 2;
-    const uint32_t sh = 8u * (uint32_t)(D & 3);
-    const uint32_t w0 = s == 0 ? a.x : s == 1 ? a.y : s == 2 ? a.z : a.w;
-    const uint32_t w1 = s == 0 ? a.y : s == 1 ? a.z : s == 2 ? a.w : b.x;
-    const uint32_t w2 = s == 0 ? a.z : s == 1 ? a.w : s == 2 ? b.x : b.y;
-    const uint32_t w3 = s == 0 ? a.w : s == 1 ? b.x : s == 2 ? b.y : b.z;
-    const uint32_t w4 = s == 0 ? b.x : s == 1 ? b.y : s == 2 ? b.z : b.w;
-    return make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh),
-                      __funnelshift_r(w2, w3, sh), __funnelshift_r(w3, w4, sh));
-}
-
-// TAB: unit ui's bytes come from unit_src[ui] (resolved on the host) instead
-// of ag8 + shard_pos.
-template <bool TAB>
-__global__ void __launch_bounds__(kThreads, 5)
-k_fp8_copy_out(const uint8_t* __restrict__ ag8, const uint8_t* const* __restrict__ unit_src,
-               uint8_t* __restrict__ arena8, const Unit* __restrict__ units,
-               int64_t n_units FSDPK_DBG_PARAM) {
-    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
-        const Unit u = units[ui];
-        FSDPK_UNIT_GUARD(u, ui, TAB ? kChkArena : (kChkShard | kChkArena));
-        const int len = u.len;
-        uint8_t* dst = arena8 + u.arena_pos;
-        const uint8_t* src;
-        if constexpr (TAB) {
-            src = unit_src[ui];
-        } else {
-            src = ag8 + u.shard_pos;
-        }
-        const int head = (int)head_to_16B(dst, len);
-        if ((int)threadIdx.x < head) dst[threadIdx.x] = src[threadIdx.x];
-        const int nv = (len - head) >> 4;
-        const int D = (int)(reinterpret_cast<uintptr_t>(src + head) & 15u);
-        const uint4* sa = reinterpret_cast<const uint4*>(src + head - D);
-        uint4* d = reinterpret_cast<uint4*>(dst + head);
-        if (D == 0) {
-#pragma unroll 4
-            for (int q = threadIdx.x; q < nv; q += blockDim.x) __stcs(d + q, __ldcs(sa + q));
-        } else {
-#pragma unroll 2
-            for (int q = threadIdx.x; q < nv; q += blockDim.x)
-                __stcs(d + q, shift_bytes16(__ldg(sa + q), __ldg(sa + q + 1), D));
-        }
-        const int done = head + 16 * nv;
-        if ((int)threadIdx.x < len - done) dst[done + threadIdx.x] = src[done + threadIdx.x];
-    }
-}
-
 // scales[i] = 448 / max(max over the D devices of amax_d[i], 1e-12): the
 // per-parameter amax is the maximum of the devices' partial maxima (each
 // device saw only its own ranks' rows).
@@ -371,18 +392,14 @@ cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* a
 cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* arena,
                             cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
-    k_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
-        ag, nullptr, arena, g.d_units, g.n_real_units FSDPK_DBG_ARG(debug_bounds(g, kDbgCopyOut)));
-    return cudaGetLastError();
+    return launch_copy_out_units<false, uint16_t>(g, ag, nullptr, arena, kDbgCopyOut, st);
 }
 
 cudaError_t launch_copy_out_tab(const fsdp_group& parent, const uint16_t* const* unit_src,
                                 uint16_t* arena, cudaStream_t st) {
     if (parent.n_real_units == 0) return cudaSuccess;
-    k_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
-        nullptr, unit_src, arena, parent.d_units, parent.n_real_units
-        FSDPK_DBG_ARG(debug_bounds(parent, kDbgCopyOutTab)));
-    return cudaGetLastError();
+    return launch_copy_out_units<true, uint16_t>(parent, nullptr, unit_src, arena,
+                                                 kDbgCopyOutTab, st);
 }
 
 cudaError_t launch_shard(const fsdp_group& g, const float* full, float* master,
@@ -432,19 +449,14 @@ cudaError_t launch_copy_in_fp8_scaled(const fsdp_group& g, const float* master, 
 cudaError_t launch_copy_out_fp8(const fsdp_group& g, const uint8_t* ag8, uint8_t* arena8,
                                 cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
-    k_fp8_copy_out<false><<<grid_for(g, nullptr, g.n_real_units), kThreads, 0, st>>>(
-        ag8, nullptr, arena8, g.d_units, g.n_real_units
-        FSDPK_DBG_ARG(debug_bounds(g, kDbgFp8CopyOut)));
-    return cudaGetLastError();
+    return launch_copy_out_units<false, uint8_t>(g, ag8, nullptr, arena8, kDbgFp8CopyOut, st);
 }
 
 cudaError_t launch_copy_out_fp8_tab(const fsdp_group& parent, const uint8_t* const* unit_src,
                                     uint8_t* arena8, cudaStream_t st) {
     if (parent.n_real_units == 0) return cudaSuccess;
-    k_fp8_copy_out<true><<<grid_for(parent, nullptr, parent.n_real_units), kThreads, 0, st>>>(
-        nullptr, unit_src, arena8, parent.d_units, parent.n_real_units
-        FSDPK_DBG_ARG(debug_bounds(parent, kDbgFp8CopyOutTab)));
-    return cudaGetLastError();
+    return launch_copy_out_units<true, uint8_t>(parent, nullptr, unit_src, arena8,
+                                                kDbgFp8CopyOutTab, st);
 }
 
 cudaError_t launch_fp8_scales_from_parts(const unsigned* const* amax_tab, int D, float* scales,

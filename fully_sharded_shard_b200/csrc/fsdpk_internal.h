@@ -19,6 +19,14 @@ constexpr int64_t kUnitElems = 8192;
 // Elements per tile of the flat copy-in kernel (256 threads x 8 x 4).
 constexpr int64_t kCopyInTile = 8192;
 
+// The copy-outs give each real unit of at least kShortRun elements a CTA of
+// its own; shorter units (small parameters, the last piece of a split run)
+// are packed, up to kPackUnits units and kPackElems elements per CTA, one
+// warp per unit.
+constexpr int64_t kShortRun = 1024;
+constexpr int64_t kPackUnits = 64;
+constexpr int64_t kPackElems = 16384;
+
 // One contiguous run of a (rank j, parameter i) shard segment.
 //   shard_pos: first element in the rank-major [N][S] index space
 //   arena_pos: first element of the matching rows in an unsharded arena
@@ -82,9 +90,13 @@ struct fsdp_group {
 
     // host copies (kept for inspection and tests of the plan); shard
     // positions index the [L][S] buffers
-    std::vector<fsdpk::Unit> units;  // real units first, then pad units
+    std::vector<fsdpk::Unit> units;  // real units first, then pad units; the real
+                                     // units of kShortRun elements or more first
     std::vector<int32_t> unit_param;  // parameter index of every unit
     int64_t n_real_units = 0;
+    int64_t n_long_units = 0;        // real units [0, n_long_units) are long
+    std::vector<int32_t> packs;      // pack p = units [packs[p], packs[p + 1]),
+                                     // packs[0] = n_long_units, back = n_real_units
     std::vector<fsdpk::Interval> intervals;
     std::vector<fsdpk::TileRange> tile_ranges;  // empty when no padding
     int64_t n_tiles = 0;                        // copy-in tiles over L*S
@@ -95,6 +107,7 @@ struct fsdp_group {
     const fsdpk::Interval* d_intervals = nullptr;
     const fsdpk::TileRange* d_tile_ranges = nullptr;
     const int32_t* d_unit_param = nullptr;
+    const int32_t* d_packs = nullptr;
 };
 
 // The opaque peer plan behind fsdp_peer_t: device `index` of `n_devices` holds the
@@ -142,6 +155,15 @@ struct AdamScalars {
     float eps;
 };
 static_assert(sizeof(AdamScalars) == 32, "AdamScalars is the 32-byte fsdp_adamw_dev_scalars");
+
+// A device step counter that a kernel advances itself (a graph-replayed
+// step), with the hyper-parameters of the scalars it then computes and where
+// to leave them (out may be null).  step == nullptr: no counter.
+struct StepCounter {
+    int64_t* step = nullptr;
+    AdamScalars* out = nullptr;
+    double lr = 0, beta1 = 0, beta2 = 0, eps = 0, wd = 0;
+};
 
 // Validate AdamW hyper-parameters and compute one step's scalars (binary64).
 bool host_adam_scalars(const fsdp_adamw_hparams* hp, AdamScalars* sc);
@@ -204,7 +226,7 @@ cudaError_t launch_fp8_scales_from_parts(const unsigned* const* amax_tab, int D,
 cudaError_t launch_small_step(const fsdp_group& g, float* master, float* m, float* v,
                               const uint16_t* grads, int op, uint16_t* ag, uint16_t* arena,
                               float* reduced, const AdamScalars& sc, const AdamScalars* sc_dev,
-                              cudaStream_t st);
+                              cudaStream_t st, const StepCounter& ctr = StepCounter{});
 
 // Fused reduce-scatter + AdamW (+ optional next-step copy-in into ag_next and
 // optional reduced-gradient output).

@@ -44,8 +44,10 @@ k_small_step(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v
              const uint16_t* __restrict__ grads, int64_t P_arena, int N,
              uint16_t* __restrict__ ag, uint16_t* __restrict__ arena, float* __restrict__ red,
              const Unit* __restrict__ units, int64_t n_units, int64_t count, int op_avg,
-             AdamScalars sc, const AdamScalars* __restrict__ sc_dev FSDPK_DBG_PARAM) {
+             AdamScalars sc, const AdamScalars* __restrict__ sc_dev, StepCounter ctr
+             FSDPK_DBG_PARAM) {
     extern __shared__ float smem[];  // [count]: master, then the reduced gradient
+    __shared__ AdamScalars s_sc;
     const bool avg = op_avg != 0;
     const float fN = (float)N;
     const int lane = threadIdx.x & 31;
@@ -55,6 +57,14 @@ k_small_step(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v
     Unit first{};
     if (warp < n_units) first = units[warp];
     if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
+    if (ctr.step != nullptr && threadIdx.x == 0) {
+        // the step of a graph-replayed call: advance the device counter and
+        // compute its scalars here (read after the block barrier below)
+        const int64_t t = *ctr.step + 1;
+        *ctr.step = t;
+        s_sc = adam_scalars_dev(ctr.lr, ctr.beta1, ctr.beta2, ctr.eps, ctr.wd, t);
+        if (ctr.out != nullptr) *ctr.out = s_sc;
+    }
     float pp[kStepPerThread], mm[kStepPerThread], vv[kStepPerThread];
 #pragma unroll
     for (int j = 0; j < kStepPerThread; ++j) {
@@ -71,6 +81,7 @@ k_small_step(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v
         if (k < count) smem[k] = pp[j];
     }
     __syncthreads();
+    if (ctr.step != nullptr) sc = s_sc;
     // step 2: per unit, the gradients first, then cast, copy out, fold
     for (int64_t ui = warp; ui < n_units; ui += n_warps) {
         const Unit u = ui == warp ? first : units[ui];
@@ -123,7 +134,7 @@ k_small_step(float* __restrict__ p, float* __restrict__ m, float* __restrict__ v
 cudaError_t launch_small_step(const fsdp_group& g, float* master, float* m, float* v,
                               const uint16_t* grads, int op, uint16_t* ag, uint16_t* arena,
                               float* reduced, const AdamScalars& sc, const AdamScalars* sc_dev,
-                              cudaStream_t st) {
+                              cudaStream_t st, const StepCounter& ctr) {
     const int64_t count = (int64_t)g.L * g.S;
     if (count == 0) return cudaSuccess;
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
@@ -132,7 +143,7 @@ cudaError_t launch_small_step(const fsdp_group& g, float* master, float* m, floa
     const size_t smem = (size_t)count * sizeof(float);
     k_small_step<<<1, kStepThreads, smem, st>>>(master, m, v, grads, g.P_arena, g.N, ag, arena,
                                                 reduced, g.d_units, (int64_t)g.units.size(),
-                                                count, avg, sc, sc_dev
+                                                count, avg, sc, sc_dev, ctr
                                                 FSDPK_DBG_ARG(debug_bounds(g, kDbgSmallStep)));
     return cudaGetLastError();
 }

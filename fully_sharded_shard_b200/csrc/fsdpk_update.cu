@@ -375,18 +375,7 @@ __global__ void k_adamw_prepare(double lr, double beta1, double beta2, double ep
     if (blockIdx.x != 0 || threadIdx.x != 0) return;
     const int64_t t = *step + 1;
     *step = t;
-    const double bc1 = 1.0 - pow(beta1, (double)t);
-    const double bc2 = 1.0 - pow(beta2, (double)t);
-    AdamScalars sc;
-    sc.decay = (float)(1.0 - lr * wd);
-    sc.beta1 = (float)beta1;
-    sc.omb1 = (float)(1.0 - beta1);
-    sc.beta2 = (float)beta2;
-    sc.omb2 = (float)(1.0 - beta2);
-    sc.step_size = (float)(lr / bc1);
-    sc.inv_bc2_sqrt = (float)(1.0 / sqrt(bc2));
-    sc.eps = (float)eps;
-    *out = sc;
+    *out = adam_scalars_dev(lr, beta1, beta2, eps, wd, t);
 }
 
 }  // namespace

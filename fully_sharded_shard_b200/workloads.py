@@ -137,6 +137,17 @@ def moe(scale: int = 1, experts: int = 64, zero_experts: int = 16) -> Workload:
                     "normal", 0.02, 1e-3)
 
 
+def small_params(count: int = 3000, seed: int = 5) -> Workload:
+    """A group of many small parameters (biases, norms, small tables): not one
+    of the pages' configurations -- a measurement of the copy-outs' packed
+    path, where every (rank, parameter) run is a few hundred elements.
+    d0 ~ U{1..299}, width from {1, 3, 17, 64} (1 = a 1-D parameter), N = 8."""
+    rng = np.random.default_rng(seed)
+    shapes = _random_shapes(rng, count, 299, (1, 3, 17, 64))
+    g = Group("small", shapes, [f"p{k}" for k in range(count)])
+    return Workload("small_params", 8, [g], AVG, seed, "normal", 0.02, 1e-3)
+
+
 def llama7b(scale: int = 1, layers: int = 32) -> Workload:
     d, ffn, vocab = 4096 // scale, 11008 // scale, 32000 // scale
     blk = _block(d, ffn, d)
@@ -157,6 +168,7 @@ def by_name(name: str) -> Workload:
         "uneven": uneven,
         "moe": moe,
         "llama7b": llama7b,
+        "small_params": small_params,
     }
     if name in table:
         return table[name]()

@@ -286,6 +286,27 @@ FSDP_API int fsdp_group_step_dev(fsdp_group_t group, float* master, float* m, fl
                                  const fsdp_adamw_dev_scalars* scalars_dev, uint16_t* ag,
                                  uint16_t* arena, float* reduced, fsdp_stream_t stream);
 
+/* The whole step of one group as ONE call that a CUDA graph can replay as
+ * successive training steps ("Introduction to PyTorch FSDP2 Backend
+ * Features", Working Principle: all-gather, reduce-scatter, update, in that
+ * order): fsdp_adamw_prepare and fsdp_group_step_dev in one.  It advances
+ * the device step counter *step_dev, computes that step's AdamW scalars on
+ * the device (left in *scalars_dev) and runs the step.  A group with
+ * N*S <= FSDP_SMALL_STEP_ELEMS is one launch in all (its single CTA advances
+ * the counter and computes the scalars itself, while its first loads are in
+ * flight); a larger group is the prepare kernel and the four stage kernels.
+ * Same bits as fsdp_adamw_prepare followed by fsdp_group_step_dev.
+ *   hparams: lr, betas, eps, weight_decay as for fsdp_adamw_step (step is
+ *   ignored); step_dev: device int64, 8-byte aligned, 0 before the first
+ *   step; scalars_dev: device memory, 16-byte aligned; the other arguments
+ *   as for fsdp_group_step.
+ * Errors as for fsdp_adamw_prepare and fsdp_group_step. */
+FSDP_API int fsdp_group_step_graph(fsdp_group_t group, float* master, float* m, float* v,
+                                   const uint16_t* grads, int32_t op,
+                                   const fsdp_adamw_hparams* hparams, int64_t* step_dev,
+                                   fsdp_adamw_dev_scalars* scalars_dev, uint16_t* ag,
+                                   uint16_t* arena, float* reduced, fsdp_stream_t stream);
+
 /* Gradient accumulation without sync ([ML] Other controls:
  * set_requires_gradient_sync(False) accumulates the unsharded gradients and
  * skips the reduce-scatter).  Each rank's unsharded gradient is accumulated in

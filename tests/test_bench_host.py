@@ -125,3 +125,16 @@ def test_local_real_elems_split_the_group_across_devices(oracle):
                     want = sum(p.valid_rows(i, j) * int(p.cols[i])
                                for i in range(p.n) for j in range(d * L, (d + 1) * L))
                     assert parts[d] == want
+
+
+def test_profile_stages_byte_model_matches_the_bench():
+    """The single-stage profiler counts each stage's algorithmic bytes with
+    the bench's byte model (the fused update: reduce-scatter + AdamW + next
+    copy-in, 2N B per real element + 26 B per padded element)."""
+    from fully_sharded_shard_b200 import profile_stages as PS
+    for N, S, P in ((8, 1000, 8000), (6, 1001, 5990), (2, 7, 13)):
+        sb = bench.stage_bytes(N, S, P)
+        for k in ("copy_in", "copy_out", "rs_reduce", "adamw"):
+            assert PS.stage_bytes(k, N, S, P) == sb[k], k
+        assert PS.stage_bytes("rs_adamw", N, S, P) == sum(bench.fused_stage_bytes(N, S, P).values()) \
+            - bench.fused_stage_bytes(N, S, P)["copy_out"]

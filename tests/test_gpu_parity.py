@@ -414,9 +414,13 @@ def _group_step_case(H, wl, grp, steps, graph, full_init=None, grads_init=None):
         s.wait_stream(torch.cuda.current_stream())
         cg = torch.cuda.CUDAGraph()
         with torch.cuda.graph(cg, stream=s):
-            abi.fsdp_adamw_prepare(ds, **hp)
-            abi.fsdp_group_step_dev(g, a["p"], a["m"], a["v"], gbuf, op, ds, ag=a["ag"],
-                                    arena=a["arena"], reduced=a["red"])
+            if graph == "one_call":   # counter, scalars and step in one call
+                abi.fsdp_group_step_graph(g, a["p"], a["m"], a["v"], gbuf, op, ds, ag=a["ag"],
+                                          arena=a["arena"], reduced=a["red"], **hp)
+            else:
+                abi.fsdp_adamw_prepare(ds, **hp)
+                abi.fsdp_group_step_dev(g, a["p"], a["m"], a["v"], gbuf, op, ds, ag=a["ag"],
+                                        arena=a["arena"], reduced=a["red"])
     for t in range(1, steps + 1):
         torch.cuda.synchronize()
         pre = tuple(H.f32(a[k][:NS]) for k in ("p", "m", "v"))
@@ -464,6 +468,10 @@ def test_group_step_equals_the_four_stage_calls(H, wl):
              if wl.N * abi.fsdp_plan_group(grp.shapes, wl.N).S <= abi.FSDP_SMALL_STEP_ELEMS]
     for grp in small[:1]:
         _group_step_case(H, wl, grp, steps=3, graph=True)
+        _group_step_case(H, wl, grp, steps=3, graph="one_call")
+    big = [grp for grp in wl.groups if grp not in small]
+    for grp in big[:1]:   # the prepare kernel and the four stage kernels in one call
+        _group_step_case(H, wl, grp, steps=2, graph="one_call")
 
 
 @pytest.mark.parametrize("wl", GRID[:3], ids=[w.name for w in GRID[:3]])
