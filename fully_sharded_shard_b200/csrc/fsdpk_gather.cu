@@ -181,10 +181,11 @@ __device__ __forceinline__ void copy_unit(const T* src_run, T* dst_run, int len,
     if (t < len - done) dst_run[done + t] = src_run[done + t];
 }
 
-// CTAs [0, n_long) copy one long unit each (a team of 8 warps); the others
-// one pack of short units each, a warp per unit.  One launch: the packs'
-// CTAs are the last of the grid, so they are not a second, small grid that
-// waits for SM slots behind another stream's kernel.
+// CTAs [0, n_packs) copy one pack of short units each, a warp per unit; the
+// others one long unit each (a team of 8 warps).  One launch, so the packs
+// are not a second, small grid that waits for SM slots behind another
+// stream's kernel; and first in it, so that their CTAs -- a few dependent
+// round trips per warp -- run beside the long units rather than after them.
 // TAB: unit ui's rows come from unit_src[ui] (a pull from wherever that
 // rank's slot lives, resolved on the host), instead of ag + shard_pos.
 // A pack of short units, a warp per unit: not inlined into k_copy_out, so
@@ -206,11 +207,11 @@ __device__ __noinline__ void copy_out_pack(const T* __restrict__ ag,
 template <bool TAB, typename T>
 __global__ void __launch_bounds__(kThreads, 5)
 k_copy_out(const T* __restrict__ ag, const T* const* __restrict__ unit_src,
-           T* __restrict__ arena, const Unit* __restrict__ units, int64_t n_long,
+           T* __restrict__ arena, const Unit* __restrict__ units, int64_t n_packs,
            const int32_t* __restrict__ packs FSDPK_DBG_PARAM) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if ((int64_t)blockIdx.x < n_long) {
-        const int64_t ui = blockIdx.x;
+    if ((int64_t)blockIdx.x >= n_packs) {
+        const int64_t ui = (int64_t)blockIdx.x - n_packs;  // long units are units [0, n_long)
         const Unit u = units[ui];
 #ifdef FSDPK_DEBUG
         // a pulled unit's source is a pointer of the table, not a shard position
@@ -220,7 +221,7 @@ k_copy_out(const T* __restrict__ ag, const T* const* __restrict__ unit_src,
         copy_unit<kThreads / 32>(src, arena + u.arena_pos, u.len, warp, lane, threadIdx.x);
         return;
     }
-    const int p = (int)((int64_t)blockIdx.x - n_long);
+    const int p = (int)blockIdx.x;
     copy_out_pack<TAB>(ag, unit_src, arena, units, packs[p], packs[p + 1] FSDPK_DBG_ARG(dbg));
 }
 
@@ -230,8 +231,8 @@ cudaError_t launch_copy_out_units(const fsdp_group& g, const T* ag, const T* con
                                   T* arena, int32_t dbg_kernel, cudaStream_t st) {
     (void)dbg_kernel;
     const int64_t n_packs = (int64_t)g.packs.size() - 1;
-    k_copy_out<TAB, T><<<grid_for(g, nullptr, g.n_long_units + n_packs), kThreads, 0, st>>>(
-        ag, unit_src, arena, g.d_units, g.n_long_units, g.d_packs
+    k_copy_out<TAB, T><<<grid_for(g, nullptr, n_packs + g.n_long_units), kThreads, 0, st>>>(
+        ag, unit_src, arena, g.d_units, n_packs, g.d_packs
         FSDPK_DBG_ARG(debug_bounds(g, dbg_kernel)));
     return cudaGetLastError();
 }

@@ -71,7 +71,11 @@ def main(argv=None) -> int:
         for r in range(N):
             W.fill_grads_bf16(grads[r], wl, grp.name, "profile", r)
     if any(s in ("rs_reduce", "adamw") for s in stages):
-        red = torch.zeros(max(NS, 1), dtype=torch.float32, device=dev)
+        # a gradient-like reduced gradient: AdamW's arithmetic (its divisions
+        # in particular) takes different paths on zeros
+        red = torch.empty(max(NS, 1), dtype=torch.float32, device=dev)
+        W.fill_master(red, W.Workload(wl.name, N, [], wl.op, wl.seed, "normal",
+                                      wl.grad_sigma, wl.grad_sigma), grp.name, "profile_red")
     ag = torch.empty(max(NS, 1), dtype=torch.bfloat16, device=dev)
     if "copy_in" not in stages:
         ag.view(torch.int16).copy_(torch.randint(-16000, 16000, (max(NS, 1),), dtype=torch.int16,
