@@ -649,10 +649,13 @@ def run_fused(args, model, device, stream, ws, ms_unfused, peak):
     e1.record(stream)
     torch.cuda.synchronize(device)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
+    # per-stage times: events around every launch, averaged over a few steps
     events = {k: [] for k in ("copy_out", "rs_adamw_copy_in")}
-    model.fused_step(stream, events=events)
+    stage_steps = max(1, min(args.steps, 3))
+    for _ in range(stage_steps):
+        model.fused_step(stream, events=events)
     torch.cuda.synchronize(device)
-    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in events.items()}
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / stage_steps for k, v in events.items()}
     total = sum(model.fused_bytes.values())
     return {
         "ms_per_step": round(ms, 3),
@@ -746,9 +749,11 @@ def run_fused_fp8(args, model, device, stream, ws, ms_fused, peak):
     torch.cuda.synchronize(device)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
     events = {k: [] for k in ("copy_out", "rs_adamw_copy_in_fp8")}
-    one(events)
+    stage_steps = max(1, min(args.steps, 3))
+    for _ in range(stage_steps):
+        one(events)
     torch.cuda.synchronize(device)
-    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in events.items()}
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / stage_steps for k, v in events.items()}
     sb = {k: 0 for k in stage_ms}
     for i in model.instances:
         g = model.plans[i[0]]
@@ -1625,7 +1630,7 @@ def run_reference(args, wl):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b")

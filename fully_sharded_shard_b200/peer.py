@@ -284,12 +284,28 @@ class PipelinedPeerGroup:
     and a wait of phase A sees the records of phase B two steps back (the
     buffers of the other parity serve the step in between).  Ordering inside
     this process (for example an update before the next copy-in of the same
-    master) is the caller's, as with any two streams."""
+    master) is the caller's, as with any two streams.
+
+    With fp8=True the all-gather can also move E4M3 bytes (delayed scaling):
+    slot8[par] rows and partial amax arrays amax[par], double buffered too.
+      copy_in_fp8(par)        as copy_in, on slot8 ("in8", "out8")
+      copy_out_fp8(par)       as copy_out, on slot8
+      rs_adamw_step_fp8(par)  waits: every "gw{par}", every "out8{1 - par}"
+                              (slot8[1 - par] is rewritten) and every
+                              "sc{par}" (amax[par] is zeroed and refilled);
+                              records "gr{par}", "in8{1 - par}", "ax{par}"
+      fp8_scales(par)         waits: every "ax{par}"; the next scales from
+                              every device's amax[par]; records "sc{par}"
+    A step's fused update fills amax[par], and the scales it yields are the
+    next step's scales_prev: call fp8_scales(par) in phase B of the NEXT step
+    (after its host barrier, so that every device's "ax{par}" record is
+    enqueued), before that step's fused update."""
 
     EVENTS = tuple(f"{k}{p}" for k in ("in", "out", "gw", "gr") for p in (0, 1))
+    EVENTS_FP8 = tuple(f"{k}{p}" for k in ("in8", "out8", "ax", "sc") for p in (0, 1))
 
     def __init__(self, shapes: Sequence[Sequence[int]], N: int, *, group=None, device=None,
-                 grads: Optional["PipelinedPeerGroup"] = None):
+                 grads: Optional["PipelinedPeerGroup"] = None, fp8: bool = False):
         self.pg = group
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
@@ -320,7 +336,25 @@ class PipelinedPeerGroup:
             ag, gr = rank_pointer_tables([b + so for b in self.slot_buf.bases],
                                          [b + go for b in self.grad_buf.bases], L, S, A)
             abi.fsdp_peer_set_sources(self.pps[par], ag, gr)
-        self.ev = PeerEvents(self.EVENTS, group=group, device=self.device)
+        self.slot8_buf = self.amax_buf = None
+        self.ag8_slots, self.amax = [], []
+        if fp8:
+            self._slot8_half = _round_up(L * S, 256)
+            self._amax_half = _round_up(4 * self.g.n, 256)
+            self.slot8_buf = SharedBuffer(2 * self._slot8_half, group=group, device=self.device)
+            self.amax_buf = SharedBuffer(2 * self._amax_half, group=group, device=self.device)
+            for par in range(2):
+                so, ao = par * self._slot8_half, par * self._amax_half
+                self.ag8_slots.append(abi.device_tensor(self.slot8_buf.ptr + so, L * S,
+                                                        torch.uint8, self.device))
+                self.amax.append(abi.device_tensor(self.amax_buf.ptr + ao, self.g.n,
+                                                   torch.int32, self.device))
+                ag8 = [int(self.slot8_buf.bases[r // L]) + so + S * (r % L)
+                       for r in range(self.N)]
+                abi.fsdp_peer_set_fp8_sources(self.pps[par], ag8,
+                                              [b + ao for b in self.amax_buf.bases])
+        self.ev = PeerEvents(self.EVENTS + (self.EVENTS_FP8 if fp8 else ()), group=group,
+                             device=self.device)
         barrier(self.device, group)
 
     # phase A
@@ -362,8 +396,39 @@ class PipelinedPeerGroup:
         if next_copy_in:
             self.ev.record(f"in{nxt}", stream)
 
+    # the FP8 all-gather
+    def copy_in_fp8(self, par: int, master: torch.Tensor, scales: torch.Tensor, stream) -> None:
+        self.ev.wait_all(f"out8{par}", stream)
+        abi.fsdp_peer_copy_in_fp8_scaled(self.pps[par], master, scales, self.ag8_slots[par],
+                                         stream)
+        self.ev.record(f"in8{par}", stream)
+
+    def copy_out_fp8(self, par: int, arena8: torch.Tensor, stream) -> None:
+        self.ev.wait_all(f"in8{par}", stream)
+        abi.fsdp_peer_copy_out_fp8(self.pps[par], arena8, stream)
+        self.ev.record(f"out8{par}", stream)
+
+    def rs_adamw_step_fp8(self, par: int, op: int, master, m, v, *, scales_prev: torch.Tensor,
+                          stream, reduced: Optional[torch.Tensor] = None, **hp) -> None:
+        nxt = 1 - par
+        self.ev.wait_all(f"gw{par}", stream)
+        self.ev.wait_all(f"out8{nxt}", stream)
+        self.ev.wait_all(f"sc{par}", stream)
+        abi.fsdp_peer_rs_adamw_step_fp8(self.pps[par], op, master, m, v, scales_prev=scales_prev,
+                                        ag8_next=self.ag8_slots[nxt], amax_local=self.amax[par],
+                                        reduced=reduced, stream=stream, **hp)
+        self.ev.record(f"gr{par}", stream)
+        self.ev.record(f"in8{nxt}", stream)
+        self.ev.record(f"ax{par}", stream)
+
+    def fp8_scales(self, par: int, scales_next: torch.Tensor, stream) -> None:
+        self.ev.wait_all(f"ax{par}", stream)
+        abi.fsdp_peer_fp8_scales(self.pps[par], scales_next, stream)
+        self.ev.record(f"sc{par}", stream)
+
     def buffers(self) -> List[SharedBuffer]:
-        return [self.slot_buf] + ([self.grad_buf] if self._own_grads else [])
+        extra = [b for b in (self.slot8_buf, self.amax_buf) if b is not None]
+        return [self.slot_buf] + ([self.grad_buf] if self._own_grads else []) + extra
 
     def close(self) -> None:
         """Release the shared buffers (after barriers that drain every device,
@@ -372,6 +437,7 @@ class PipelinedPeerGroup:
         if self.pps is None:
             return
         self.ag_slots = self.grads = None
+        self.ag8_slots = self.amax = None
         release_all(self.buffers(), self.device, self.pg)
         self.ev = None
         for pp in self.pps:

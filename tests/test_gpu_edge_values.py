@@ -103,9 +103,9 @@ def full_init(N: int) -> np.ndarray:
 
 
 def grads_init(N: int):
-    """step -> bf16 bit patterns [N][P_arena]: seeded N(0, 1e-3) (N(0, 1)
-    for p0's tail), the fold cases at the heads of p0 and p4, and a negative
-    gradient on the amax elements of p2 and p3."""
+    """step -> bf16 bit patterns [N][P_arena]: seeded N(0, 1e-3), the fold
+    cases at the heads of p0 and p4, and a negative gradient on the amax
+    elements of p2 and p3."""
     p = _layout(N)
     u = [int(x) for x in p.arena_off]
 
@@ -210,3 +210,13 @@ def test_edge_values_single_launch_group_step(H, N):
                 gb[:, int(pb.arena_off[i]):int(pb.arena_off[i]) + n]
         return out
     _group_step_case(H, wl, g, steps=2, graph=False, full_init=full, grads_init=gi)
+
+
+@pytest.mark.parametrize("N,D", [(3, 3), (8, 2), (12, 4)])
+def test_edge_values_through_the_peer_pulls(H, N, D):
+    """The several-device pulls (copy-out, reduce-scatter, fused update) on
+    the special values, against the single-device path and the oracle."""
+    from tests.test_gpu_peer import run_group_peer
+    wl = _wl(N, W.AVG)
+    run_group_peer(H, wl, wl.groups[0], D, steps=2, full_init=full_init(N),
+                   grads_init=grads_init(N))

@@ -43,9 +43,11 @@ def H():
     return _harness
 
 
-def run_group_peer(H, wl, grp, D, *, steps=2, direct_oracle=False, tag=()):
+def run_group_peer(H, wl, grp, D, *, steps=2, direct_oracle=False, tag=(), full_init=None,
+                   grads_init=None):
     """Every stage of D emulated devices against the single-device group and
-    against the oracle on the GPU's own inputs."""
+    against the oracle on the GPU's own inputs.  full_init / grads_init
+    replace the seeded inputs as in the harness."""
     from fully_sharded_shard_b200 import abi
     from fully_sharded_shard_b200.peer import rank_pointer_tables
     import oracle
@@ -54,7 +56,11 @@ def run_group_peer(H, wl, grp, D, *, steps=2, direct_oracle=False, tag=()):
     g = abi.fsdp_plan_group(grp.shapes, N)
     S, A = g.S, g.P_arena
     full = torch.empty(max(A, 1), device="cuda")
-    W.fill_master(full, wl, grp.name, *tag)
+    if full_init is None:
+        W.fill_master(full, wl, grp.name, *tag)
+    else:
+        full.zero_()
+        full[:A].copy_(torch.from_numpy(np.ascontiguousarray(full_init, np.float32)))
     master = torch.empty(max(N * S, 1), device="cuda")
     abi.fsdp_shard_params(g, full, master)
     ref = {"p": master[:N * S].clone(), "m": torch.zeros(N * S, device="cuda"),
@@ -105,7 +111,7 @@ def run_group_peer(H, wl, grp, D, *, steps=2, direct_oracle=False, tag=()):
     torch.cuda.synchronize()
     gathered_and_copied_out(ag_ref)
     for step in range(1, steps + 1):
-        grads = H.make_grads(g, wl, grp, step, tag)
+        grads = H._grads_for(g, wl, grp, step, tag, grads_init)
         for d in range(D):
             gbufs[d].t.copy_(grads[d * L:(d + 1) * L].reshape(-1))
         # the reduce-scatter pulls
@@ -634,5 +640,115 @@ def test_pipelined_peer_group_over_cuda_ipc_events(H, tmp_path, D, case):
     import torch.multiprocessing as mp
     mp.spawn(_ipc_pipelined_worker, args=(_free_port(), D, case, 4, str(tmp_path)), nprocs=D,
              join=True)
+    for r in range(D):
+        assert open(tmp_path / f"r{r}.txt").read().strip() == "ok", f"process {r}"
+
+
+def _ipc_pipelined_fp8_worker(rank, port, D, case_name, steps, result_dir):
+    """The FP8 all-gather (delayed scaling) over D processes, event-ordered:
+    E4M3 slot rows and partial amax arrays double buffered, each step's
+    scales computed in the next step's phase B."""
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=D, timeout=datetime.timedelta(seconds=120))
+    msg = "ok"
+    try:
+        torch.cuda.set_device(0)
+        from fully_sharded_shard_b200 import abi
+        from fully_sharded_shard_b200.peer import PipelinedPeerGroup, host_barrier
+        from tests import _harness as H
+        import oracle
+        wl = {"uneven": W.uneven(16), "moe": W.moe(16)}[case_name]
+        grp = wl.groups[0]
+        N, op = wl.N, wl.op
+        p = oracle.plan(grp.shapes, N)
+        pgrp = PipelinedPeerGroup(grp.shapes, N, device="cuda:0", fp8=True)
+        g, S, A, L, r0, n = pgrp.g, pgrp.S, pgrp.P_arena, pgrp.L, pgrp.r0, pgrp.g.n
+        rows = slice(r0 * S, (r0 + L) * S)
+        full = torch.empty(max(A, 1), device="cuda")
+        W.fill_master(full, wl, grp.name)
+        master = torch.empty(max(N * S, 1), device="cuda")
+        abi.fsdp_shard_params(g, full, master)
+        hp = dict(W.ADAMW_DEFAULTS)
+        grads = [H.make_grads(g, wl, grp, t) for t in range(1, steps + 1)]
+        # single-device references of every step
+        ref = {"p": master[:N * S].clone(), "m": torch.zeros(N * S, device="cuda"),
+               "v": torch.zeros(N * S, device="cuda")}
+        mine = {k: t[rows].clone() for k, t in ref.items()}
+        ag8_ref = torch.empty(max(N * S, 1), dtype=torch.uint8, device="cuda")
+        scales_ref = [torch.empty(max(n, 1), device="cuda")]
+        abi.fsdp_copy_in_fp8(g, ref["p"], ag8_ref, scales_ref[0])
+        ar_ref = []
+        for t in range(1, steps + 1):
+            a8 = torch.full((max(A, 1),), 0xA5, dtype=torch.uint8, device="cuda")
+            abi.fsdp_copy_out_fp8(g, ag8_ref, a8[:A])
+            ar_ref.append(a8)
+            nxt = torch.empty(max(n, 1), device="cuda")
+            abi.fsdp_rs_adamw_step_fp8(g, grads[t - 1], op, ref["p"], ref["m"], ref["v"], step=t,
+                                       scales_prev=scales_ref[-1], ag8_next=ag8_ref,
+                                       scales_next=nxt, **hp)
+            scales_ref.append(nxt)
+        torch.cuda.synchronize()
+        # the pipelined run
+        sg, su = torch.cuda.Stream(), torch.cuda.Stream()
+        scales = [scales_ref[0].clone()] + [torch.full((max(n, 1),), -1.0, device="cuda")
+                                           for _ in range(steps)]
+        ar = [torch.full((max(A, 1),), 0xA5, dtype=torch.uint8, device="cuda")
+              for _ in range(steps)]
+        torch.cuda.synchronize()
+        host_barrier()
+        for t in range(1, steps + 1):
+            par = t % 2
+            if t == 1:
+                pgrp.copy_in_fp8(par, mine["p"], scales[0], sg)
+                read = torch.cuda.Event()
+                read.record(sg)
+                su.wait_event(read)
+            buf = pgrp.grads_begin(par, su)
+            with torch.cuda.stream(su):
+                buf.copy_(grads[t - 1][r0:r0 + L])
+            pgrp.grads_end(par, su)
+            host_barrier()
+            if t > 1:   # the previous step's scales, from every device's partial amax
+                pgrp.fp8_scales(1 - par, scales[t - 1], su)
+            pgrp.copy_out_fp8(par, ar[t - 1][:A], sg)
+            pgrp.rs_adamw_step_fp8(par, op, mine["p"], mine["m"], mine["v"],
+                                   scales_prev=scales[t - 1], stream=su, step=t, **hp)
+        host_barrier()
+        pgrp.fp8_scales(steps % 2, scales[steps], su)
+        torch.cuda.synchronize()
+        host_barrier()
+        for t in range(1, steps + 1):
+            if not torch.equal(ar[t - 1], ar_ref[t - 1]):
+                msg = f"FP8 copy-out differs at step {t}"
+                break
+            if not torch.equal(scales[t][:n].view(torch.int32), scales_ref[t][:n].view(torch.int32)):
+                msg = f"scales of step {t} differ"
+                break
+        if msg == "ok":
+            bad = [k for k in ("p", "m", "v")
+                   if not torch.equal(mine[k].view(torch.int32), ref[k][rows].view(torch.int32))]
+            if bad:
+                msg = f"state differs after {steps} steps: {bad}"
+            elif not torch.equal(pgrp.ag8_slots[(steps + 1) % 2], ag8_ref[rows]):
+                msg = "next E4M3 slot differs"
+            elif n and not H.bits_equal(H.f32(scales[steps])[:n],
+                                        oracle.fp8_scales(p, H.f32(ref["p"]))):
+                msg = "last scales differ from the oracle's"
+        pgrp.close()
+    except Exception as e:  # reported through the result file
+        msg = f"error: {type(e).__name__}: {e}"
+    finally:
+        with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+            f.write(msg + "\n")
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("D,case", [(2, "uneven"), (4, "moe")])
+def test_pipelined_peer_fp8_over_cuda_ipc_events(H, tmp_path, D, case):
+    import torch.multiprocessing as mp
+    mp.spawn(_ipc_pipelined_fp8_worker, args=(_free_port(), D, case, 4, str(tmp_path)),
+             nprocs=D, join=True)
     for r in range(D):
         assert open(tmp_path / f"r{r}.txt").read().strip() == "ok", f"process {r}"
