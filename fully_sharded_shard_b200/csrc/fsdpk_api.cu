@@ -103,6 +103,24 @@ namespace fsdpk {
 // [(r1 - r0)][S] of buffers that hold only those ranks' shards: real units of
 // every (rank j, parameter i), then pad units, the merged pad intervals and
 // the copy-in tile ranges.  Reads the per-parameter tables of g.
+// Packs of consecutive units [b, e): up to kPackUnits units and kPackElems
+// elements each (a single longer unit makes a pack of its own); out receives
+// the pack boundaries, out[0] = b and out.back() = e.
+void make_packs(const fsdp_group& g, int64_t b, int64_t e, std::vector<int32_t>* out) {
+    out->clear();
+    for (int64_t k = b; k < e;) {
+        out->push_back((int32_t)k);
+        int64_t elems = 0, cnt = 0;
+        while (k < e && cnt < fsdpk::kPackUnits &&
+               (cnt == 0 || elems + g.units[(size_t)k].len <= fsdpk::kPackElems)) {
+            elems += g.units[(size_t)k].len;
+            ++cnt;
+            ++k;
+        }
+    }
+    out->push_back((int32_t)e);
+}
+
 int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
     const int64_t S = g->S;
     const int32_t n_params = g->n;
@@ -137,18 +155,7 @@ int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
         while (g->n_long_units < g->n_real_units &&
                g->units[(size_t)g->n_long_units].len >= fsdpk::kShortRun)
             ++g->n_long_units;
-        g->packs.clear();
-        for (int64_t k = g->n_long_units; k < g->n_real_units;) {
-            g->packs.push_back((int32_t)k);
-            int64_t elems = 0, cnt = 0;
-            while (k < g->n_real_units && cnt < fsdpk::kPackUnits &&
-                   (cnt == 0 || elems + g->units[(size_t)k].len <= fsdpk::kPackElems)) {
-                elems += g->units[(size_t)k].len;
-                ++cnt;
-                ++k;
-            }
-        }
-        g->packs.push_back((int32_t)g->n_real_units);
+        make_packs(*g, g->n_long_units, g->n_real_units, &g->packs);
         for (int64_t j = r0; j < r1; ++j)
             for (int32_t i = 0; i < n_params; ++i) {
                 const int64_t v = std::clamp<int64_t>(g->d0[i] - j * g->c[i], 0, g->c[i]);
@@ -162,6 +169,7 @@ int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
                         g->intervals.push_back(Interval{lo, lo + len});
                 }
             }
+        make_packs(*g, g->n_long_units, (int64_t)g->units.size(), &g->rpacks);
         if (g->intervals.size() > (size_t)std::numeric_limits<int32_t>::max()) return FSDP_EINVAL;
         const int64_t NS = (r1 - r0) * S;
         g->n_tiles = (NS + fsdpk::kCopyInTile - 1) / fsdpk::kCopyInTile;
@@ -195,8 +203,10 @@ int upload_tables(fsdp_group* g) {
     const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
     const size_t b_up = g->unit_param.size() * sizeof(int32_t);
     const size_t b_pk = g->packs.size() * sizeof(int32_t);
+    const size_t b_rp = g->rpacks.size() * sizeof(int32_t);
     auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up) + up256(b_pk);
+    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up) + up256(b_pk) +
+                         up256(b_rp);
     if (total == 0) return FSDP_OK;
     e = cudaMalloc(&g->dev_mem, total);
     if (e != cudaSuccess) {
@@ -212,6 +222,8 @@ int upload_tables(fsdp_group* g) {
         reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) + up256(b_tr));
     g->d_packs = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
                                                   up256(b_tr) + up256(b_up));
+    g->d_rpacks = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
+                                                   up256(b_tr) + up256(b_up) + up256(b_pk));
     if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && b_iv)
         e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
@@ -222,6 +234,8 @@ int upload_tables(fsdp_group* g) {
         e = cudaMemcpy((void*)g->d_unit_param, g->unit_param.data(), b_up, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && b_pk)
         e = cudaMemcpy((void*)g->d_packs, g->packs.data(), b_pk, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && b_rp)
+        e = cudaMemcpy((void*)g->d_rpacks, g->rpacks.data(), b_rp, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
         cudaFree(g->dev_mem);
         g->dev_mem = nullptr;
@@ -438,6 +452,14 @@ int64_t check_tables(const fsdp_group& g) {
         ++bad;
     for (size_t p = 0; p + 1 < g.packs.size(); ++p) {
         const int64_t cnt = (int64_t)g.packs[p + 1] - g.packs[p];
+        if (cnt < 1 || cnt > fsdpk::kPackUnits) ++bad;
+    }
+    // the reduce-scatter's packs cover every unit after the long ones
+    if (g.rpacks.empty() || g.rpacks.front() != g.n_long_units ||
+        g.rpacks.back() != (int64_t)g.units.size())
+        ++bad;
+    for (size_t p = 0; p + 1 < g.rpacks.size(); ++p) {
+        const int64_t cnt = (int64_t)g.rpacks[p + 1] - g.rpacks[p];
         if (cnt < 1 || cnt > fsdpk::kPackUnits) ++bad;
     }
     std::sort(spans.begin(), spans.end());

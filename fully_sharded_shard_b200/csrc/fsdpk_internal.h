@@ -97,6 +97,8 @@ struct fsdp_group {
     int64_t n_long_units = 0;        // real units [0, n_long_units) are long
     std::vector<int32_t> packs;      // pack p = units [packs[p], packs[p + 1]),
                                      // packs[0] = n_long_units, back = n_real_units
+    std::vector<int32_t> rpacks;     // the reduce-scatter's packs: the short real
+                                     // units and every pad unit, [n_long_units, units)
     std::vector<fsdpk::Interval> intervals;
     std::vector<fsdpk::TileRange> tile_ranges;  // empty when no padding
     int64_t n_tiles = 0;                        // copy-in tiles over L*S
@@ -108,6 +110,7 @@ struct fsdp_group {
     const fsdpk::TileRange* d_tile_ranges = nullptr;
     const int32_t* d_unit_param = nullptr;
     const int32_t* d_packs = nullptr;
+    const int32_t* d_rpacks = nullptr;
 };
 
 // The opaque peer plan behind fsdp_peer_t: device `index` of `n_devices` holds the

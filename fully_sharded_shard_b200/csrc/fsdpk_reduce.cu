@@ -23,17 +23,25 @@ namespace {
 // NR = ranks known at compile time (1..8), 0 = any N (batches of 4).
 // ---------------------------------------------------------------------------
 
+// The threads that share one unit: the whole CTA (a long unit) or one warp
+// (a short or pad unit of a pack); t is this thread's index among them.
+struct Team {
+    int t, n;
+};
+
+__device__ __forceinline__ Team cta_team() { return Team{(int)threadIdx.x, (int)blockDim.x}; }
+
 // Compile-time rank count: all NR loads of a vector are issued before the fold.
 template <int NR, bool SHIFTED, int V, class Src>
 __device__ __forceinline__ void reduce_body(const Src& src_al, float* __restrict__ dst, int nvec,
-                                            int D, bool avg, float fN) {
+                                            int D, bool avg, float fN, Team tm) {
 #pragma unroll 1
-    for (int q0 = threadIdx.x; q0 < nvec; q0 += blockDim.x * V) {
+    for (int q0 = tm.t; q0 < nvec; q0 += tm.n * V) {
         uint4 a[V][NR];
         uint4 b[V][NR];
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            const int q = q0 + k * blockDim.x;
+            const int q = q0 + k * tm.n;
             if (q < nvec) {
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
@@ -45,7 +53,7 @@ __device__ __forceinline__ void reduce_body(const Src& src_al, float* __restrict
         }
 #pragma unroll
         for (int k = 0; k < V; ++k) {
-            const int q = q0 + k * blockDim.x;
+            const int q = q0 + k * tm.n;
             if (q < nvec) {
                 float acc[8];
                 unpack8(SHIFTED ? shift_bf16x8(a[k][0], b[k][0], D) : a[k][0], acc);
@@ -70,9 +78,9 @@ __device__ __forceinline__ void reduce_body(const Src& src_al, float* __restrict
 template <bool SHIFTED, class Src>
 __device__ __forceinline__ void reduce_body_any(const Src& src_al, int N,
                                                 float* __restrict__ dst, int nvec, int D,
-                                                bool avg, float fN) {
+                                                bool avg, float fN, Team tm) {
 #pragma unroll 1
-    for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+    for (int q = tm.t; q < nvec; q += tm.n) {
         float acc[8];
 #pragma unroll 1
         for (int r0 = 0; r0 < N; r0 += 4) {
@@ -110,23 +118,25 @@ __device__ __forceinline__ void reduce_body_any(const Src& src_al, int N,
 
 template <int NR, bool SHIFTED, class Src>
 __device__ __forceinline__ void reduce_body_dispatch(const Src& src_al, int N, float* dst,
-                                                     int nvec, int D, bool avg, float fN) {
+                                                     int nvec, int D, bool avg, float fN,
+                                                     Team tm) {
     if constexpr (NR == 0) {
-        reduce_body_any<SHIFTED>(src_al, N, dst, nvec, D, avg, fN);
+        reduce_body_any<SHIFTED>(src_al, N, dst, nvec, D, avg, fN, tm);
     } else {
         // keep about 4-8 independent 16-byte loads in flight per thread
         constexpr int V = NR >= 4 ? 1 : (4 / NR);
-        reduce_body<NR, SHIFTED, V>(src_al, dst, nvec, D, avg, fN);
+        reduce_body<NR, SHIFTED, V>(src_al, dst, nvec, D, avg, fN, tm);
     }
 }
 
 // One real unit: dst_run[e] = fold over ranks of src_run.rank(r)[e].
 template <int NR, class Src>
 __device__ __forceinline__ void reduce_unit(const Src& src_run, float* __restrict__ dst_run,
-                                            int len, int N, bool avg, float fN) {
+                                            int len, int N, bool avg, float fN,
+                                            Team tm = cta_team()) {
     const int head = (int)head_to_16B(dst_run, len);
-    if ((int)threadIdx.x < head)
-        dst_run[threadIdx.x] = finish(fold_scalar<NR>(src_run.at(threadIdx.x), N), avg, fN);
+    if (tm.t < head)
+        dst_run[tm.t] = finish(fold_scalar<NR>(src_run.at(tm.t), N), avg, fN);
     const int nvec = (len - head) >> 3;
     // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0, and
     // table pointers are checked on the host), so one phase D holds for all N
@@ -134,12 +144,43 @@ __device__ __forceinline__ void reduce_unit(const Src& src_run, float* __restric
     const int D = bf16_phase(src_run.rank(0) + head);
     const Src src_al = src_run.at(head - D);
     float* dst = dst_run + head;
-    if (D == 0) reduce_body_dispatch<NR, false>(src_al, N, dst, nvec, 0, avg, fN);
-    else reduce_body_dispatch<NR, true>(src_al, N, dst, nvec, D, avg, fN);
+    if (D == 0) reduce_body_dispatch<NR, false>(src_al, N, dst, nvec, 0, avg, fN, tm);
+    else reduce_body_dispatch<NR, true>(src_al, N, dst, nvec, D, avg, fN, tm);
     const int done = head + 8 * nvec;
-    if ((int)threadIdx.x < len - done)
-        dst_run[done + threadIdx.x] =
-            finish(fold_scalar<NR>(src_run.at(done + threadIdx.x), N), avg, fN);
+    if (tm.t < len - done)
+        dst_run[done + tm.t] = finish(fold_scalar<NR>(src_run.at(done + tm.t), N), avg, fN);
+}
+
+// Zero-fill `len` fp32 elements at dst (any alignment) by one warp.
+__device__ __forceinline__ void zero_f32_warp(float* __restrict__ dst, int64_t len, int lane) {
+    int64_t head = (4 - (reinterpret_cast<uintptr_t>(dst) >> 2 & 3)) & 3;
+    if (head > len) head = len;
+    if (lane < head) dst[lane] = 0.0f;
+    const int64_t nv = (len - head) >> 2;
+    float4* d4 = reinterpret_cast<float4*>(dst + head);
+    for (int64_t q = lane; q < nv; q += 32) __stcs(d4 + q, make_float4(0.f, 0.f, 0.f, 0.f));
+    const int64_t done = head + 4 * nv;
+    if (lane < len - done) dst[done + lane] = 0.0f;
+}
+
+// A pack of short real units and pad units, a warp per unit: not inlined into
+// k_reduce_units, so that its registers do not add to the long-unit path's.
+template <int NR>
+__device__ __noinline__ void reduce_pack(const uint16_t* __restrict__ gsrc, int64_t stride, int N,
+                                         float* __restrict__ gdst, const Unit* __restrict__ units,
+                                         int b, int e, bool avg, float fN FSDPK_DBG_PARAM) {
+    const int lane = threadIdx.x & 31;
+    for (int ui = b + (int)(threadIdx.x >> 5); ui < e; ui += kThreads / 32) {
+        const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
+        float* dst_run = gdst + u.shard_pos;
+        if (u.is_pad) {
+            zero_f32_warp(dst_run, u.len, lane);
+            continue;
+        }
+        reduce_unit<NR>(StrideSrc{gsrc + u.arena_pos, stride}, dst_run, u.len, N, avg, fN,
+                        Team{lane, 32});
+    }
 }
 
 // One launch covers every unit of the group.  blockIdx.y selects a source
@@ -149,16 +190,33 @@ __device__ __forceinline__ void reduce_unit(const Src& src_run, float* __restric
 // still 1.7 % faster on B200 than with three CTAs and no spill (more 16-byte
 // loads in flight per SM).  The pack (NR = 1), NR = 2 and the any-N path
 // would spill far more under that cap and keep three.
-template <int NR>
+// PACKS: the grid starts with n_rpacks CTAs of packed short and pad units.
+// Only a plan with many such units launches this form: the call to the pack
+// path costs the long-unit path a few registers.
+template <int NR, bool PACKS>
 __global__ void __launch_bounds__(kThreads, (NR >= 3 && NR <= 8) ? 4 : 3)
 k_reduce_units(const uint16_t* __restrict__ grads, int64_t stride, int N,
                float* __restrict__ out, int64_t y_src_step, int64_t y_dst_step,
-               const Unit* __restrict__ units, int64_t n_units, int op_avg FSDPK_DBG_PARAM) {
+               const Unit* __restrict__ units, int64_t n_units, int op_avg,
+               const int32_t* __restrict__ rpacks, int64_t n_rpacks FSDPK_DBG_PARAM) {
     const uint16_t* gsrc = grads + (int64_t)blockIdx.y * y_src_step;
     float* gdst = out + (int64_t)blockIdx.y * y_dst_step;
     const bool avg = op_avg != 0;
     const float fN = (float)N;
-    for (int64_t ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+    // CTAs [0, n_rpacks): one pack of short or pad units each; the others one
+    // unit of [0, n_units) each (the long units, or every unit without packs)
+    if constexpr (PACKS) {
+        if ((int64_t)blockIdx.x < n_rpacks) {
+            const int p = (int)blockIdx.x;
+            reduce_pack<NR>(gsrc, stride, N, gdst, units, rpacks[p], rpacks[p + 1], avg, fN
+                            FSDPK_DBG_ARG(dbg));
+            return;
+        }
+    } else {
+        (void)rpacks;
+    }
+    for (int64_t ui = (int64_t)blockIdx.x - n_rpacks; ui < n_units;
+         ui += (int64_t)gridDim.x - n_rpacks) {
         const Unit u = units[ui];
         FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
         const int len = u.len;
@@ -388,18 +446,42 @@ k_reduce_acc(const float* __restrict__ acc, const uint16_t* __restrict__ g, int6
     }
 }
 
+// n_units: the units one CTA each handles; rpacks / n_rpacks: the packs
+// (null / 0 when every unit gets a CTA).
 template <int NR>
 cudaError_t launch_reduce_nr(const fsdp_group& g, const uint16_t* grads, int64_t stride, int N,
                              float* out, int64_t y_src_step, int64_t y_dst_step,
                              unsigned ydim, const Unit* units, int64_t n_units, int avg,
-                             cudaStream_t st, const DebugBounds& dbg) {
+                             cudaStream_t st, const DebugBounds& dbg,
+                             const int32_t* rpacks = nullptr, int64_t n_rpacks = 0) {
     (void)dbg;
-    const void* kfn = (const void*)k_reduce_units<NR>;
-    dim3 grid(grid_for(g, kfn, n_units), ydim);
-    k_reduce_units<NR><<<grid, kThreads, 0, st>>>(grads, stride, N, out, y_src_step,
-                                                  y_dst_step, units, n_units, avg
-                                                  FSDPK_DBG_ARG(dbg));
+    dim3 grid(grid_for(g, nullptr, n_rpacks + n_units), ydim);
+    if (n_rpacks > 0)
+        k_reduce_units<NR, true><<<grid, kThreads, 0, st>>>(grads, stride, N, out, y_src_step,
+                                                            y_dst_step, units, n_units, avg,
+                                                            rpacks, n_rpacks FSDPK_DBG_ARG(dbg));
+    else
+        k_reduce_units<NR, false><<<grid, kThreads, 0, st>>>(grads, stride, N, out, y_src_step,
+                                                             y_dst_step, units, n_units, avg,
+                                                             nullptr, 0 FSDPK_DBG_ARG(dbg));
     return cudaGetLastError();
+}
+
+// The reduce-scatter packs its short and pad units when there are at least
+// this many of them (thousands of small parameters); otherwise every unit
+// gets a CTA of the plain kernel.
+constexpr int64_t kPackMinUnits = 2048;
+
+// (units a CTA each, packs) of g for the fused reduce-scatter kernels.
+inline void reduce_split(const fsdp_group& g, int64_t* n_cta_units, int64_t* n_packs) {
+    const int64_t n_small = (int64_t)g.units.size() - g.n_long_units;
+    if (n_small >= kPackMinUnits) {
+        *n_cta_units = g.n_long_units;
+        *n_packs = (int64_t)g.rpacks.size() - 1;
+    } else {
+        *n_cta_units = (int64_t)g.units.size();
+        *n_packs = 0;
+    }
 }
 
 }  // namespace
@@ -415,15 +497,18 @@ cudaError_t launch_rs_fused(const fsdp_group& g, const uint16_t* grads, int op, 
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
     const int64_t stride = g.P_arena;
     const DebugBounds dbg = debug_bounds(g, kDbgReduce);
+    int64_t nl, np;
+    reduce_split(g, &nl, &np);
+    (void)nu;
     switch (g.N) {
 #define FSDPK_CASE(K) \
-    case K: return launch_reduce_nr<K>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg, st, dbg);
+    case K: return launch_reduce_nr<K>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nl, avg, st, dbg, g.d_rpacks, np);
         FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
         FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
 #undef FSDPK_CASE
         default:
-            return launch_reduce_nr<0>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nu, avg,
-                                       st, dbg);
+            return launch_reduce_nr<0>(g, grads, stride, g.N, reduced, 0, 0, 1, g.d_units, nl, avg,
+                                       st, dbg, g.d_rpacks, np);
     }
 }
 
@@ -476,8 +561,11 @@ cudaError_t launch_rs_pack(const fsdp_group& g, const uint16_t* grads, float* pa
     const int64_t nu = (int64_t)g.units.size();
     if (nu == 0) return cudaSuccess;
     // blockIdx.y = source rank r: reads rank r's arena, writes packed[r]
+    int64_t nl, np;
+    reduce_split(g, &nl, &np);
     return launch_reduce_nr<1>(g, grads, 0, 1, packed, g.P_arena, (int64_t)g.N * g.S,
-                               (unsigned)g.N, g.d_units, nu, 0, st, debug_bounds(g, kDbgReduce));
+                               (unsigned)g.N, g.d_units, nl, 0, st, debug_bounds(g, kDbgReduce),
+                               g.d_rpacks, np);
 }
 
 cudaError_t launch_rs_reduce_packed(const fsdp_group& g, const float* packed, int op,

@@ -2,9 +2,10 @@
 FSDPK_DEBUG=1, so the binding loads libfsdpk_debug.so).
 
   python tests/_debug_run.py grid     every stage over the brute-force grid,
-                                      40 random groups and the emulated
-                                      several-device pulls; prints the error
-                                      words (all zero expected)
+                                      40 random groups, the emulated
+                                      several-device pulls and a group of 3000
+                                      small parameters (the packed paths);
+                                      prints the error words (all zero expected)
   python tests/_debug_run.py shrink   the copy-out and the fused reduce-scatter
                                       with every extent narrowed by one
                                       element; prints the error words and
@@ -44,6 +45,9 @@ def grid() -> dict:
                   (W.uneven(16), 3)):
         run_group_peer(H, wl, wl.groups[0], D, steps=1)
         cases += 1
+    wl = W.small_params()          # the packed copy-out and reduce-scatter paths
+    H.run_group(wl, wl.groups[0], steps=1, ops=ops, staged=True)
+    cases += 1
     torch.cuda.synchronize()
     abi.fsdp_debug_set_error_words(None)
     return {"words": [int(x) for x in words.cpu()], "cases": cases}

@@ -35,7 +35,7 @@ def _run(mode: str) -> dict:
 
 def test_debug_build_grid_has_no_violations():
     out = _run("grid")
-    assert out["cases"] == 51          # 9 grid groups, 40 random groups, 2 peer cases
+    assert out["cases"] == 52          # 9 grid groups, 40 random groups, 2 peer cases, 1 packed
     assert out["words"][0] == 0, f"violations: {out['words']}"
 
 

@@ -321,6 +321,21 @@ def test_random_groups_brute_force(H, wl):
     H.run_group_fused_fp8(wl, grp, steps=1)
 
 
+def test_many_small_parameters_packed_paths(H):
+    """3000 small parameters over 8 ranks: the copy-outs and the fused
+    reduce-scatter pack their short units (a warp each) -- every stage, the
+    staged pack, the fused update and the FP8 all-gather against the oracle."""
+    from fully_sharded_shard_b200 import abi
+    wl = W.small_params()
+    grp = wl.groups[0]
+    g = abi.fsdp_plan_group(grp.shapes, wl.N)
+    assert abi.fsdp_group_check(g) == 0
+    g.destroy()
+    H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
+    H.run_group_fused(wl, grp, steps=2)
+    H.run_group_fp8(wl, grp)
+
+
 GRID = [_wl(f"grid_n{N}", [((d0, c) if c > 1 else (d0,)) for d0 in range(21) for c in (1, 3, 8)], N,
             op=[W.SUM, W.AVG, W.SUM_THEN_DIV][N % 3]) for N in range(1, 10)]
 
