@@ -225,12 +225,21 @@ __device__ __forceinline__ void fold8(const Src& src_al, int N, int q, int D, fl
     }
 }
 
+// The threads that share one unit: the whole CTA, or one warp (a unit of a
+// pack); t is this thread's index among them.
+struct Team {
+    int t, n;
+};
+
+__device__ __forceinline__ Team cta_team() { return Team{(int)threadIdx.x, (int)blockDim.x}; }
+
 template <int NR, bool SHIFTED, bool FP8, class Src>
 __device__ __forceinline__ void fused_body(const Src& src_al, int N, int D, const FusedOut& o,
                                            int64_t k0, int nvec, bool avg, float fN,
-                                           const AdamScalars& sc, float scale, float& mx) {
+                                           const AdamScalars& sc, float scale, float& mx,
+                                           Team tm) {
 #pragma unroll 1
-    for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+    for (int q = tm.t; q < nvec; q += tm.n) {
         const int64_t k = k0 + 8 * (int64_t)q;
         float4 P[2], M[2], V[2];
         load_pmv8(o, k, P, M, V);
@@ -250,25 +259,82 @@ template <int NR, bool FP8, class Src>
 __device__ __forceinline__ void rs_adamw_real_unit(const Src& src_run, int N, const FusedOut& o,
                                                    int64_t k0, int len, int head, int nvec,
                                                    bool avg, float fN, const AdamScalars& sc,
-                                                   float scale, float& mx) {
+                                                   float scale, float& mx,
+                                                   Team tm = cta_team()) {
     const int done = head + 8 * nvec;
-    if ((int)threadIdx.x < head)
-        fused1<FP8>(o, k0 + threadIdx.x,
-                    finish(fold_scalar<NR>(src_run.at(threadIdx.x), N), avg, fN), false, sc,
-                    scale, mx);
+    if (tm.t < head)
+        fused1<FP8>(o, k0 + tm.t, finish(fold_scalar<NR>(src_run.at(tm.t), N), avg, fN), false,
+                    sc, scale, mx);
     // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0, and
     // table pointers are checked on the host), so one phase D holds for all N
     // source streams
     const int D = bf16_phase(src_run.rank(0) + head);
     const Src src_al = src_run.at(head - D);
     if (D == 0)
-        fused_body<NR, false, FP8>(src_al, N, 0, o, k0 + head, nvec, avg, fN, sc, scale, mx);
+        fused_body<NR, false, FP8>(src_al, N, 0, o, k0 + head, nvec, avg, fN, sc, scale, mx, tm);
     else
-        fused_body<NR, true, FP8>(src_al, N, D, o, k0 + head, nvec, avg, fN, sc, scale, mx);
-    if ((int)threadIdx.x < len - done)
-        fused1<FP8>(o, k0 + done + threadIdx.x,
-                    finish(fold_scalar<NR>(src_run.at(done + threadIdx.x), N), avg, fN), false,
-                    sc, scale, mx);
+        fused_body<NR, true, FP8>(src_al, N, D, o, k0 + head, nvec, avg, fN, sc, scale, mx, tm);
+    if (tm.t < len - done)
+        fused1<FP8>(o, k0 + done + tm.t,
+                    finish(fold_scalar<NR>(src_run.at(done + tm.t), N), avg, fN), false, sc,
+                    scale, mx);
+}
+
+// A pack of short real units and pad units, a warp per unit: the fused
+// update of a group of thousands of small parameters, launched before
+// k_rs_adamw, which then takes the long units only.  Same per-element
+// arithmetic, so the same bits.  FP8: each warp folds its unit's max into the
+// parameter's amax slot with one atomicMax.
+template <int NR, bool FP8>
+__global__ void __launch_bounds__(kThreads, 2)
+k_rs_adamw_packs(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o,
+                 const Unit* __restrict__ units, const int32_t* __restrict__ rpacks,
+                 int64_t n_rpacks, int op_avg, AdamScalars sc,
+                 const AdamScalars* __restrict__ sc_dev FSDPK_DBG_PARAM) {
+    if ((int64_t)blockIdx.x >= n_rpacks) return;
+    if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    const int lane = threadIdx.x & 31;
+    const Team tm{lane, 32};
+    const int b = rpacks[blockIdx.x], e = rpacks[blockIdx.x + 1];
+    for (int ui = b + (int)(threadIdx.x >> 5); ui < e; ui += kThreads / 32) {
+        const Unit u = units[ui];
+        FSDPK_UNIT_GUARD(u, ui, kChkShard | kChkArena);
+        if constexpr (FP8)
+            FSDPK_GUARD(u.is_pad || (o.unit_param[ui] >= 0 && o.unit_param[ui] < dbg.n_aux), ui);
+        const int len = u.len;
+        const int64_t k0 = u.shard_pos;
+        float scale = 0.0f, mx = 0.0f;
+        if constexpr (FP8) {
+            if (!u.is_pad) scale = o.scales[o.unit_param[ui]];
+        }
+        int head = (int)((8 - (k0 & 7)) & 7);
+        if (head > len) head = len;
+        const int nvec = (len - head) >> 3;
+        if (u.is_pad) {
+            const int done = head + 8 * nvec;
+            const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (lane < head) fused1<FP8>(o, k0 + lane, 0.0f, true, sc, scale, mx);
+#pragma unroll 1
+            for (int q = lane; q < nvec; q += 32) {
+                const int64_t k = k0 + head + 8 * (int64_t)q;
+                float4 P[2], M[2], V[2];
+                load_pmv8(o, k, P, M, V);
+                fused8<FP8>(o, k, zero8, P, M, V, true, sc, scale, mx);
+            }
+            if (lane < len - done) fused1<FP8>(o, k0 + done + lane, 0.0f, true, sc, scale, mx);
+            continue;
+        }
+        rs_adamw_real_unit<NR, FP8>(StrideSrc{grads + u.arena_pos, stride}, N, o, k0, len, head,
+                                    nvec, avg, fN, sc, scale, mx, tm);
+        if constexpr (FP8) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (lane == 0) atomicMax(o.amax_bits + o.unit_param[ui], __float_as_uint(mx));
+        }
+    }
 }
 
 // TAB: the N source arenas come from a table of per-rank pointers (rank_tab,
@@ -342,11 +408,25 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride,
     }
 }
 
+// The fused update packs its short and pad units when there are at least
+// this many of them (thousands of small parameters).
+constexpr int64_t kFusedPackMinUnits = 2048;
+
 template <int NR, bool FP8>
 cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const FusedOut& o,
                                int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
                                cudaStream_t st) {
-    const int64_t nu = (int64_t)g.units.size();
+    int64_t nu = (int64_t)g.units.size();
+    const int64_t n_small = nu - g.n_long_units;
+    if (n_small >= kFusedPackMinUnits) {
+        // thousands of short and pad units: packs first, then the long units
+        const int64_t np = (int64_t)g.rpacks.size() - 1;
+        k_rs_adamw_packs<NR, FP8><<<grid_for(g, nullptr, np), kThreads, 0, st>>>(
+            grads, g.P_arena, g.N, o, g.d_units, g.d_rpacks, np, avg, sc, sc_dev
+            FSDPK_DBG_ARG(debug_bounds(g, kDbgRsAdamw, g.n)));
+        nu = g.n_long_units;
+        if (nu == 0) return cudaGetLastError();
+    }
     k_rs_adamw<NR, FP8, false><<<grid_for(g, nullptr, nu), kThreads, 0, st>>>(
         grads, g.P_arena, nullptr, g.N, o, g.d_units, nu, avg, sc, sc_dev
         FSDPK_DBG_ARG(debug_bounds(g, kDbgRsAdamw, g.n)));

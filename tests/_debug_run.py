@@ -45,8 +45,10 @@ def grid() -> dict:
                   (W.uneven(16), 3)):
         run_group_peer(H, wl, wl.groups[0], D, steps=1)
         cases += 1
-    wl = W.small_params()          # the packed copy-out and reduce-scatter paths
+    wl = W.small_params()          # the packed copy-out, reduce-scatter and update paths
     H.run_group(wl, wl.groups[0], steps=1, ops=ops, staged=True)
+    H.run_group_fused(wl, wl.groups[0], steps=1)
+    H.run_group_fused_fp8(wl, wl.groups[0], steps=1)
     cases += 1
     torch.cuda.synchronize()
     abi.fsdp_debug_set_error_words(None)

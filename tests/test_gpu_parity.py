@@ -322,9 +322,10 @@ def test_random_groups_brute_force(H, wl):
 
 
 def test_many_small_parameters_packed_paths(H):
-    """3000 small parameters over 8 ranks: the copy-outs and the fused
-    reduce-scatter pack their short units (a warp each) -- every stage, the
-    staged pack, the fused update and the FP8 all-gather against the oracle."""
+    """3000 small parameters over 8 ranks: the copy-outs, the fused
+    reduce-scatter and the fused update pack their short units (a warp each)
+    -- every stage, the staged pack, the fused update (bf16 and FP8 next
+    all-gather input) and the FP8 all-gather against the oracle."""
     from fully_sharded_shard_b200 import abi
     wl = W.small_params()
     grp = wl.groups[0]
@@ -333,6 +334,7 @@ def test_many_small_parameters_packed_paths(H):
     g.destroy()
     H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=True)
     H.run_group_fused(wl, grp, steps=2)
+    H.run_group_fused_fp8(wl, grp, steps=2)
     H.run_group_fp8(wl, grp)
 
 
