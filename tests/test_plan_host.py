@@ -30,7 +30,8 @@ def _compare(abi, oracle, shapes, N):
 
 def test_workload_plans_on_host(abi, oracle):
     from fully_sharded_shard_b200 import workloads as W
-    for wl in (W.tiny_mlp(), W.llama_block(), W.uneven(), W.moe(), W.llama7b()):
+    for wl in (W.tiny_mlp(), W.llama_block(), W.uneven(), W.moe(), W.llama7b(),
+               W.small_params()):
         for grp in wl.groups:
             _compare(abi, oracle, grp.shapes, wl.N)
 
@@ -69,6 +70,15 @@ def test_data_calls_refuse_a_host_plan(abi):
 
 # Mistakes planted in a copy of the host plan builder (compiled on the CPU,
 # never run on a GPU): the consistency check must report each of them.
+MUTANTS_PACKS = [
+    ("pack one unit over the limit",
+     "while (k < e && cnt < fsdpk::kPackUnits &&",
+     "while (k < e && cnt <= fsdpk::kPackUnits &&"),
+    ("a short unit counted as long",
+     "return g->units[k].len >= fsdpk::kShortRun;",
+     "return g->units[k].len >= fsdpk::kShortRun / 2;"),
+]
+
 MUTANTS = [
     ("arena one row off",
      "g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);",
@@ -88,7 +98,8 @@ MUTANTS = [
 ]
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+@pytest.mark.parametrize("name,old,new", MUTANTS + MUTANTS_PACKS,
+                         ids=[m[0] for m in MUTANTS + MUTANTS_PACKS])
 def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
     import glob
     import os
@@ -116,6 +127,10 @@ def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
     # ragged rows on several ranks, pads that meet across parameters, a tile
     # boundary inside a pad run
     shapes = [(7, 3), (5,), (1, 32), (13, 9), (2, 2), (9001, 1), (3,)]
+    # and enough short runs to fill several packs
+    shapes += [(3 + k % 50, 1 + k % 7) for k in range(300)] + [(600, 1)] * 10
+    # runs of 512-1023 elements between long ones (700 at N = 2, 3, 4, 6)
+    shapes += [(1400, 1), (9001, 1), (2100, 1), (9001, 1), (2800, 1), (4200, 1), (9001, 1)]
     found = 0
     for N in (2, 3, 4, 6):
         _, arr = abi._descs(shapes)
