@@ -117,6 +117,9 @@ def _load() -> ctypes.CDLL:
     L.fsdp_plan_group_host.restype = ctypes.c_int
     L.fsdp_group_check.argtypes = [vp, ctypes.POINTER(i64)]
     L.fsdp_group_check.restype = ctypes.c_int
+    L.fsdp_group_flat.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(i64),
+                                  ctypes.POINTER(i64)]
+    L.fsdp_group_flat.restype = ctypes.c_int
     L.fsdp_group_step.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.POINTER(AdamWHparams), vp, vp,
                                   vp, vp]
     L.fsdp_group_step.restype = ctypes.c_int
@@ -245,6 +248,18 @@ def fsdp_group_check(g: Group) -> int:
     v = ctypes.c_int64()
     _check(_lib.fsdp_group_check(g.handle, ctypes.byref(v)), "fsdp_group_check")
     return v.value
+
+
+def fsdp_group_flat(g: Group) -> tuple:
+    """(flat, mixed shard-side vectors, mixed arena-side vectors) of a plan:
+    whether its copy-out, fused reduce-scatter and fused update take the flat
+    path, and how many of its vectors go element by element."""
+    f = ctypes.c_int32()
+    ms = ctypes.c_int64()
+    ma = ctypes.c_int64()
+    _check(_lib.fsdp_group_flat(g.handle, ctypes.byref(f), ctypes.byref(ms), ctypes.byref(ma)),
+           "fsdp_group_flat")
+    return bool(f.value), ms.value, ma.value
 
 
 def _stream(stream, t: torch.Tensor):

@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -27,6 +28,10 @@
 using fsdpk::Interval;
 using fsdpk::TileRange;
 using fsdpk::Unit;
+using fsdpk::FlatSeg;
+using fsdpk::kFlatMaxElems;
+using fsdpk::kFlatMinUnits;
+using fsdpk::kFlatPad;
 
 namespace {
 
@@ -121,6 +126,89 @@ void make_packs(const fsdp_group& g, int64_t b, int64_t e, std::vector<int32_t>*
     out->push_back((int32_t)e);
 }
 
+// Segments of a flat index space [0, end) from its runs (start, len, code),
+// sorted here; the space between runs gets kFlatPad.  Adjacent ranges with
+// one code merge, and a sentinel closes the table.
+std::vector<FlatSeg> flat_segments(std::vector<std::array<int64_t, 3>> runs, int64_t end) {
+    std::sort(runs.begin(), runs.end());
+    std::vector<FlatSeg> segs;
+    auto put = [&](int64_t start, int32_t code) {
+        if (segs.empty() || segs.back().code != code) segs.push_back(FlatSeg{(int32_t)start, code});
+    };
+    int64_t at = 0;
+    for (const auto& r : runs) {
+        if (r[1] <= 0) continue;
+        if (r[0] > at) put(at, kFlatPad);
+        put(r[0], (int32_t)r[2]);
+        at = r[0] + r[1];
+    }
+    if (at < end) put(at, kFlatPad);
+    segs.push_back(FlatSeg{(int32_t)end, kFlatPad});
+    return segs;
+}
+
+// One code per 8-element vector of [0, end) over its segments: the segment's
+// code when one segment holds all 8 elements, else 2 m + 1 for entry m of the
+// mixed list (mixq: the vector; mixc: its 8 elements' codes, kFlatPad past
+// the end).
+std::vector<int32_t> flat_codes(const std::vector<FlatSeg>& segs, int64_t end,
+                                std::vector<int32_t>* mixq, std::vector<int32_t>* mixc) {
+    std::vector<int32_t> codes((size_t)((end + 7) / 8));
+    mixq->clear();
+    mixc->clear();
+    size_t i = 0;
+    for (size_t q = 0; q < codes.size(); ++q) {
+        const int64_t lo = 8 * (int64_t)q, hi = lo + 8;
+        while (segs[i + 1].start <= lo) ++i;
+        if (hi <= end && segs[i + 1].start >= hi) {
+            codes[q] = segs[i].code;
+            continue;
+        }
+        codes[q] = (int32_t)(2 * mixq->size() + 1);
+        mixq->push_back((int32_t)q);
+        size_t t = i;
+        for (int64_t k = lo; k < hi; ++k) {
+            while (k < end && segs[t + 1].start <= k) ++t;
+            mixc->push_back(k < end ? segs[t].code : kFlatPad);
+        }
+    }
+    return codes;
+}
+
+// The flat path's tables, for a plan of all N ranks with at least
+// kFlatMinUnits short and pad units and both index spaces within the codes'
+// range; otherwise g->flat stays false.  Shard side: the real units (code
+// 2 * (arena_pos - shard_pos)) and the pad units over [N][S].  Arena side:
+// the real units (code 2 * (shard_pos - arena_pos)) over [P_arena], the
+// alignment gaps between parameters as kFlatPad.
+void build_flat_maps(fsdp_group* g) {
+    g->flat = false;
+    for (auto* v : {&g->smap, &g->amap, &g->smixq, &g->amixq, &g->smixc, &g->amixc}) v->clear();
+    g->ssegs.clear();
+    g->asegs.clear();
+    const int64_t LS = (int64_t)g->L * g->S;
+    const int64_t n_small = (int64_t)g->units.size() - g->n_long_units;
+    if (g->L != g->N || n_small < kFlatMinUnits || LS > kFlatMaxElems ||
+        g->P_arena > kFlatMaxElems)
+        return;
+    std::vector<std::array<int64_t, 3>> sruns, aruns;
+    sruns.reserve(g->units.size());
+    aruns.reserve((size_t)g->n_real_units);
+    for (const Unit& u : g->units) {
+        if (u.is_pad) {
+            sruns.push_back({u.shard_pos, u.len, kFlatPad});
+        } else {
+            sruns.push_back({u.shard_pos, u.len, 2 * (u.arena_pos - u.shard_pos)});
+            aruns.push_back({u.arena_pos, u.len, 2 * (u.shard_pos - u.arena_pos)});
+        }
+    }
+    g->ssegs = flat_segments(std::move(sruns), LS);
+    g->asegs = flat_segments(std::move(aruns), g->P_arena);
+    g->smap = flat_codes(g->ssegs, LS, &g->smixq, &g->smixc);
+    g->amap = flat_codes(g->asegs, g->P_arena, &g->amixq, &g->amixc);
+    g->flat = true;
+}
+
 int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
     const int64_t S = g->S;
     const int32_t n_params = g->n;
@@ -185,6 +273,7 @@ int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
                 g->tile_ranges[(size_t)t] = TileRange{(int32_t)a, (int32_t)b};
             }
         }
+        if (r0 == 0 && r1 == g->N) build_flat_maps(g);
     } catch (...) {
         return FSDP_ENOMEM;
     }
@@ -198,15 +287,31 @@ int upload_tables(fsdp_group* g) {
     if (e != cudaSuccess) return cuda_fail(e);
     e = cudaDeviceGetAttribute(&g->sm_count, cudaDevAttrMultiProcessorCount, g->device);
     if (e != cudaSuccess) return cuda_fail(e);
-    const size_t b_units = g->units.size() * sizeof(Unit);
-    const size_t b_iv = g->intervals.size() * sizeof(Interval);
-    const size_t b_tr = g->tile_ranges.size() * sizeof(TileRange);
-    const size_t b_up = g->unit_param.size() * sizeof(int32_t);
-    const size_t b_pk = g->packs.size() * sizeof(int32_t);
-    const size_t b_rp = g->rpacks.size() * sizeof(int32_t);
+    struct Table {
+        const void* host;
+        size_t bytes;
+        const void** dev;
+    };
+    auto table = [](const auto& v, const void** dev) {
+        return Table{v.data(), v.size() * sizeof(v[0]), dev};
+    };
+    const Table tables[] = {
+        table(g->units, reinterpret_cast<const void**>(&g->d_units)),
+        table(g->intervals, reinterpret_cast<const void**>(&g->d_intervals)),
+        table(g->tile_ranges, reinterpret_cast<const void**>(&g->d_tile_ranges)),
+        table(g->unit_param, reinterpret_cast<const void**>(&g->d_unit_param)),
+        table(g->packs, reinterpret_cast<const void**>(&g->d_packs)),
+        table(g->rpacks, reinterpret_cast<const void**>(&g->d_rpacks)),
+        table(g->smap, reinterpret_cast<const void**>(&g->d_smap)),
+        table(g->smixq, reinterpret_cast<const void**>(&g->d_smixq)),
+        table(g->smixc, reinterpret_cast<const void**>(&g->d_smixc)),
+        table(g->amap, reinterpret_cast<const void**>(&g->d_amap)),
+        table(g->amixq, reinterpret_cast<const void**>(&g->d_amixq)),
+        table(g->amixc, reinterpret_cast<const void**>(&g->d_amixc)),
+    };
     auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t total = up256(b_units) + up256(b_iv) + up256(b_tr) + up256(b_up) + up256(b_pk) +
-                         up256(b_rp);
+    size_t total = 0;
+    for (const Table& t : tables) total += up256(t.bytes);
     if (total == 0) return FSDP_OK;
     e = cudaMalloc(&g->dev_mem, total);
     if (e != cudaSuccess) {
@@ -214,28 +319,13 @@ int upload_tables(fsdp_group* g) {
         g->dev_mem = nullptr;
         return e == cudaErrorMemoryAllocation ? FSDP_ENOMEM : cuda_fail(e);
     }
-    char* base = static_cast<char*>(g->dev_mem);
-    g->d_units = reinterpret_cast<const Unit*>(base);
-    g->d_intervals = reinterpret_cast<const Interval*>(base + up256(b_units));
-    g->d_tile_ranges = reinterpret_cast<const TileRange*>(base + up256(b_units) + up256(b_iv));
-    g->d_unit_param =
-        reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) + up256(b_tr));
-    g->d_packs = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
-                                                  up256(b_tr) + up256(b_up));
-    g->d_rpacks = reinterpret_cast<const int32_t*>(base + up256(b_units) + up256(b_iv) +
-                                                   up256(b_tr) + up256(b_up) + up256(b_pk));
-    if (b_units) e = cudaMemcpy((void*)g->d_units, g->units.data(), b_units, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && b_iv)
-        e = cudaMemcpy((void*)g->d_intervals, g->intervals.data(), b_iv, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && b_tr)
-        e = cudaMemcpy((void*)g->d_tile_ranges, g->tile_ranges.data(), b_tr,
-                       cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && b_up)
-        e = cudaMemcpy((void*)g->d_unit_param, g->unit_param.data(), b_up, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && b_pk)
-        e = cudaMemcpy((void*)g->d_packs, g->packs.data(), b_pk, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && b_rp)
-        e = cudaMemcpy((void*)g->d_rpacks, g->rpacks.data(), b_rp, cudaMemcpyHostToDevice);
+    char* at = static_cast<char*>(g->dev_mem);
+    for (const Table& t : tables) {
+        *t.dev = at;
+        if (e == cudaSuccess && t.bytes)
+            e = cudaMemcpy(at, t.host, t.bytes, cudaMemcpyHostToDevice);
+        at += up256(t.bytes);
+    }
     if (e != cudaSuccess) {
         cudaFree(g->dev_mem);
         g->dev_mem = nullptr;
@@ -409,6 +499,98 @@ int plan_on_host(const fsdp_param_desc* params, int32_t n_params, int32_t world_
 // each real unit's arena position recomputed from its shard position (the
 // Shard(0) placement), the pad intervals against the pad units, and each
 // copy-in tile's interval range.  Returns the number of violations.
+// The flat path's segments, codes and mixed list of one index space
+// [0, end) against its runs (start, len, code): segments strictly increasing
+// from 0 with a sentinel at end and no two neighbours with one code; each run
+// inside a single segment of its code; as many elements in segments of real
+// codes as in real runs (so the rest is kFlatPad); each vector's code pure
+// exactly when one segment holds all 8 of its elements, else the next entry
+// of the mixed list, which names the vector and each element's code.
+int64_t check_flat_space(const std::vector<FlatSeg>& segs, const std::vector<int32_t>& codes,
+                         const std::vector<int32_t>& mixq, const std::vector<int32_t>& mixc,
+                         const std::vector<std::array<int64_t, 3>>& runs, int64_t end) {
+    int64_t bad = 0;
+    if (segs.size() < 2 || segs.front().start != 0 || segs.back().start != end ||
+        segs.back().code != kFlatPad)
+        return 1;
+    int64_t real = 0;
+    for (size_t i = 0; i + 1 < segs.size(); ++i) {
+        if (segs[i + 1].start <= segs[i].start) ++bad;
+        if (i + 2 < segs.size() && segs[i + 1].code == segs[i].code) ++bad;
+        if (segs[i].code != kFlatPad) {
+            if (segs[i].code & 1) ++bad;
+            real += (int64_t)segs[i + 1].start - segs[i].start;
+        }
+    }
+    if (bad) return bad;
+    auto seg_of = [&](int64_t k) {  // the segment holding element k < end
+        size_t lo = 0, hi = segs.size() - 1;
+        while (hi - lo > 1) {
+            const size_t mid = (lo + hi) / 2;
+            if (segs[mid].start <= k) lo = mid; else hi = mid;
+        }
+        return lo;
+    };
+    int64_t real_runs = 0;
+    for (const auto& r : runs) {
+        if (r[1] <= 0) continue;
+        if (r[0] < 0 || r[0] + r[1] > end) {
+            ++bad;
+            continue;
+        }
+        const size_t i = seg_of(r[0]);
+        if (segs[i].code != (int32_t)r[2] || segs[i + 1].start < r[0] + r[1]) ++bad;
+        if (r[2] != kFlatPad) real_runs += r[1];
+    }
+    if (real != real_runs) ++bad;
+    if ((int64_t)codes.size() != (end + 7) / 8 || mixc.size() != 8 * mixq.size()) return bad + 1;
+    size_t m = 0;
+    for (size_t q = 0; q < codes.size(); ++q) {
+        const int64_t lo = 8 * (int64_t)q, hi = lo + 8;
+        const size_t i = seg_of(lo);
+        const bool pure = hi <= end && segs[i + 1].start >= hi;
+        if (pure) {
+            if (codes[q] != segs[i].code) ++bad;
+            continue;
+        }
+        if (codes[q] != (int32_t)(2 * m + 1) || m >= mixq.size() || mixq[m] != (int32_t)q) {
+            ++bad;
+            continue;
+        }
+        for (int e = 0; e < 8; ++e) {
+            const int64_t k = lo + e;
+            const int32_t want = k < end ? segs[seg_of(k)].code : kFlatPad;
+            if (mixc[8 * m + (size_t)e] != want) ++bad;
+        }
+        ++m;
+    }
+    if (m != mixq.size()) ++bad;
+    return bad;
+}
+
+// The flat path of g: built exactly when the plan qualifies, and both
+// spaces' tables recomputed from the units.
+int64_t check_flat(const fsdp_group& g) {
+    const int64_t LS = (int64_t)g.L * g.S;
+    const int64_t n_small = (int64_t)g.units.size() - g.n_long_units;
+    const bool want = g.L == g.N && n_small >= kFlatMinUnits && LS <= kFlatMaxElems &&
+                      g.P_arena <= kFlatMaxElems;
+    if (want != g.flat) return 1;
+    if (!g.flat)
+        return (g.smap.empty() && g.amap.empty() && g.smixq.empty() && g.amixq.empty() &&
+                g.smixc.empty() && g.amixc.empty() && g.ssegs.empty() && g.asegs.empty())
+                   ? 0
+                   : 1;
+    std::vector<std::array<int64_t, 3>> sruns, aruns;
+    for (const Unit& u : g.units) {
+        sruns.push_back({u.shard_pos, u.len,
+                         u.is_pad ? (int64_t)kFlatPad : 2 * (u.arena_pos - u.shard_pos)});
+        if (!u.is_pad) aruns.push_back({u.arena_pos, u.len, -2 * (u.arena_pos - u.shard_pos)});
+    }
+    return check_flat_space(g.ssegs, g.smap, g.smixq, g.smixc, sruns, LS) +
+           check_flat_space(g.asegs, g.amap, g.amixq, g.amixc, aruns, g.P_arena);
+}
+
 int64_t check_tables(const fsdp_group& g) {
     int64_t bad = 0;
     const int64_t LS = (int64_t)g.L * g.S;
@@ -490,6 +672,7 @@ int64_t check_tables(const fsdp_group& g) {
             }
         }
     }
+    bad += check_flat(g);
     return bad;
 }
 
@@ -515,6 +698,14 @@ int fsdp_plan_group_host(const fsdp_param_desc* params, int32_t n_params, int32_
 int fsdp_group_check(fsdp_group_t g, int64_t* violations) {
     if (g == nullptr || violations == nullptr) return FSDP_EINVAL;
     *violations = check_tables(*g);
+    return FSDP_OK;
+}
+
+int fsdp_group_flat(fsdp_group_t g, int32_t* flat, int64_t* mixed_shard, int64_t* mixed_arena) {
+    if (g == nullptr) return FSDP_EINVAL;
+    if (flat) *flat = g->flat ? 1 : 0;
+    if (mixed_shard) *mixed_shard = (int64_t)g->smixq.size();
+    if (mixed_arena) *mixed_arena = (int64_t)g->amixq.size();
     return FSDP_OK;
 }
 

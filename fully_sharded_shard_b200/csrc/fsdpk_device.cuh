@@ -137,14 +137,125 @@ __device__ __forceinline__ float fold_scalar(const Src& src, int N) {
     return acc;
 }
 
+// x / N in binary32, round to nearest even.  For a rank count NR known at
+// compile time and a power of two, 1/NR is exact, so x * (1/NR) rounds the
+// same exact value as the division, for every x (subnormal results, zeros,
+// infinities and NaN included), and replaces it.
+template <int NR>
+__device__ __forceinline__ float div_n(float x, float fN) {
+    if constexpr (NR > 0 && (NR & (NR - 1)) == 0) {
+        (void)fN;
+        return __fmul_rn(x, 1.0f / (float)NR);
+    } else {
+        return __fdiv_rn(x, fN);
+    }
+}
+
+template <int NR = 0>
 __device__ __forceinline__ float finish(float acc, bool avg, float fN) {
-    return avg ? __fdiv_rn(acc, fN) : acc;
+    return avg ? div_n<NR>(acc, fN) : acc;
 }
 
 __device__ __forceinline__ void store8(float* __restrict__ dst, const float (&acc)[8]) {
     float4* o = reinterpret_cast<float4*>(dst);
     __stcs(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
     __stcs(o + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
+}
+
+// ---------------------------------------------------------------------------
+// flat path (groups of many small parameters): one CTA per tile of the flat
+// index space, kFlatV vectors of 8 elements per thread, one code per vector
+// ---------------------------------------------------------------------------
+constexpr int kFlatV = 4;
+constexpr int64_t kFlatTile = (int64_t)kThreads * 8 * kFlatV;
+
+// CTAs of a flat launch over `count` elements: one per tile.
+inline unsigned flat_grid(int64_t count) {
+    const int64_t t = (count + kFlatTile - 1) / kFlatTile;
+    return (unsigned)std::min<int64_t>(std::max<int64_t>(t, 1), 0x7FFFFFFF);
+}
+
+// Elements of the mixed vectors per thread, and the CTAs that take them:
+// thread t of that region has elements t + i * T (i < kFlatMixedPer; T the
+// region's threads), all its loads issued together.
+constexpr int kFlatMixedPer = 4;
+
+inline int64_t flat_mixed_ctas(int64_t n_mixed) {
+    return (8 * n_mixed + kThreads * kFlatMixedPer - 1) / (kThreads * kFlatMixedPer);
+}
+
+// The codes of this thread's kFlatV vectors of a flat tile (vector q0 + j *
+// kThreads for j < kFlatV), read before any of them is processed; entries
+// past the last vector read as mixed, which the vector loops skip.
+__device__ __forceinline__ void flat_tile_codes(const int32_t* __restrict__ map, int64_t q0,
+                                                int64_t nv, int32_t (&code)[kFlatV]) {
+#pragma unroll
+    for (int j = 0; j < kFlatV; ++j) {
+        const int64_t q = q0 + (int64_t)j * kThreads;
+        code[j] = q < nv ? __ldcs(map + q) : 1;
+    }
+}
+
+// code[j] for a loop index j that is not unrolled (selects, no local memory).
+__device__ __forceinline__ int32_t flat_pick(const int32_t (&code)[kFlatV], int j) {
+    int32_t c = code[0];
+#pragma unroll
+    for (int t = 1; t < kFlatV; ++t)
+        if (j == t) c = code[t];
+    return c;
+}
+
+// Rank-ordered fold of the 8 source elements a .. a+7 of every rank (rank r
+// at g + r * stride; stride a multiple of 8, so all N sources share the phase
+// D of a in its 16-byte vector): aligned loads at a - D and, for D != 0, at
+// a - D + 8, every rank's issued before the fold.  NR = 0: any N, ranks in
+// batches of 4.
+template <int NR>
+__device__ __forceinline__ void flat_fold8(const uint16_t* __restrict__ g, int64_t stride, int N,
+                                           int64_t a, float (&acc)[8]) {
+    const int D = (int)(a & 7);
+    const uint4* s = reinterpret_cast<const uint4*>(g + (a - D));
+    const int64_t st4 = stride >> 3;
+    if constexpr (NR != 0) {
+        uint4 x[NR], y[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            x[r] = __ldg(s + r * st4);
+            if (D != 0) y[r] = __ldg(s + r * st4 + 1);
+            else y[r] = x[r];
+        }
+        unpack8(shift_bf16x8(x[0], y[0], D), acc);
+#pragma unroll
+        for (int r = 1; r < NR; ++r) {
+            float t[8];
+            unpack8(shift_bf16x8(x[r], y[r], D), t);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], t[e]);
+        }
+    } else {
+#pragma unroll 1
+        for (int r0 = 0; r0 < N; r0 += 4) {
+            uint4 x[4], y[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r0 + r < N) {
+                    x[r] = __ldg(s + (r0 + r) * st4);
+                    if (D != 0) y[r] = __ldg(s + (r0 + r) * st4 + 1);
+                    else y[r] = x[r];
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r0 + r < N) {
+                    float t[8];
+                    unpack8(shift_bf16x8(x[r], y[r], D), t);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        acc[e] = (r0 + r == 0) ? t[e] : __fadd_rn(acc[e], t[e]);
+                }
+            }
+        }
+    }
 }
 
 // One AdamW step of one element in binary32.  Where (1 - b2) * g^2 overflows
@@ -214,11 +325,14 @@ __device__ __forceinline__ uint8_t e4m3(float x) {
     if (!unit_in_bounds(dbg, (u), (ui), (what))) continue
 #define FSDPK_GUARD(ok, where) \
     if (!debug_ok(dbg, (ok), (where))) continue
+#define FSDPK_THREAD_GUARD(ok, where) \
+    if (!debug_ok_thread(dbg, (ok), (where))) continue
 #else
 #define FSDPK_DBG_PARAM
 #define FSDPK_DBG_ARG(x)
 #define FSDPK_UNIT_GUARD(u, ui, what) ((void)0)
 #define FSDPK_GUARD(ok, where) ((void)0)
+#define FSDPK_THREAD_GUARD(ok, where) ((void)0)
 #endif
 
 constexpr int kChkShard = 1;  // shard_pos + len within [0, ns)
@@ -228,6 +342,19 @@ constexpr int kChkArena = 2;  // a real unit's arena_pos + len within [0, arena)
 // across the block; lane 0 of each warp that sees a violation records it.
 __device__ __forceinline__ bool debug_ok(const DebugBounds& b, bool ok, int64_t where) {
     if (!ok && (threadIdx.x & 31) == 0 && b.words != nullptr) {
+        if (atomicAdd(b.words, 1u) == 0u) {
+            b.words[1] = (uint32_t)b.kernel;
+            b.words[2] = (uint32_t)where;
+            b.words[3] = blockIdx.x;
+        }
+    }
+    return ok;
+}
+
+// The flat kernels check per thread (each thread its own vectors): every
+// thread that sees a violation counts it.
+__device__ __forceinline__ bool debug_ok_thread(const DebugBounds& b, bool ok, int64_t where) {
+    if (!ok && b.words != nullptr) {
         if (atomicAdd(b.words, 1u) == 0u) {
             b.words[1] = (uint32_t)b.kernel;
             b.words[2] = (uint32_t)where;

@@ -237,6 +237,83 @@ cudaError_t launch_copy_out_units(const fsdp_group& g, const T* ag, const T* con
     return cudaGetLastError();
 }
 
+// Flat copy-out (a group of many small parameters): one CTA per tile of
+// kFlatTile elements of the arena, kFlatV vectors of 8 per thread with their
+// codes read first.  A vector inside one real run takes its 8 elements from
+// the aligned 16-byte vectors of the buffer that hold them (shifted by the
+// run's phase) in one 16-byte store, every vector's loads issued before the
+// stores; a gap vector is left alone.  Mixed vectors go a thread per
+// element.
+// One launch: CTAs [0, mixed_ctas) take the mixed vectors' elements,
+// kFlatMixedPer a thread (element t + i * T, T the region's threads, is
+// element e = t % 8 of list entry m = t / 8: arena element k = 8 * mixq[m] + e
+// with code mixc[t]; gaps untouched), first in the grid; the others one tile
+// each.
+__global__ void __launch_bounds__(kThreads)
+k_copy_out_flat(const uint16_t* __restrict__ ag, uint16_t* __restrict__ arena, int64_t count,
+                const int32_t* __restrict__ amap, const int32_t* __restrict__ mixq,
+                const int32_t* __restrict__ mixc, int64_t n_mixed, int64_t mixed_ctas
+                FSDPK_DBG_PARAM) {
+    if ((int64_t)blockIdx.x < mixed_ctas) {
+        const int64_t t0 = (int64_t)blockIdx.x * kThreads + threadIdx.x, T = mixed_ctas * kThreads;
+        int64_t k[kFlatMixedPer];
+        uint16_t x[kFlatMixedPer];
+        bool on[kFlatMixedPer];
+#pragma unroll
+        for (int i = 0; i < kFlatMixedPer; ++i) {
+            const int64_t t = t0 + i * T;
+            on[i] = t < 8 * n_mixed;
+            k[i] = on[i] ? 8 * (int64_t)mixq[t >> 3] + (t & 7) : 0;
+            const int32_t c = on[i] ? mixc[t] : kFlatPad;
+            const int64_t src = k[i] + (c >> 1);
+            on[i] = on[i] && k[i] < count && c != kFlatPad;
+#ifdef FSDPK_DEBUG
+            if (on[i] && !debug_ok_thread(dbg, k[i] < dbg.arena && src >= 0 && src < dbg.ns, k[i]))
+                on[i] = false;
+#endif
+            if (on[i]) x[i] = ag[src];
+        }
+#pragma unroll
+        for (int i = 0; i < kFlatMixedPer; ++i)
+            if (on[i]) arena[k[i]] = x[i];
+        return;
+    }
+    const int64_t nv = (count + 7) >> 3;
+    const int64_t q0 = ((int64_t)blockIdx.x - mixed_ctas) * (kThreads * kFlatV) + threadIdx.x;
+    int32_t code[kFlatV];
+    flat_tile_codes(amap, q0, nv, code);
+    uint4 x[kFlatV], y[kFlatV];
+    int D[kFlatV];
+#pragma unroll
+    for (int j = 0; j < kFlatV; ++j) {
+        const int64_t k = 8 * (q0 + (int64_t)j * kThreads);
+        const int32_t c = code[j];
+        D[j] = 0;
+        if (!(c & 1) && c != kFlatPad) {
+            const int64_t src = k + (c >> 1);
+#ifdef FSDPK_DEBUG
+            if (!debug_ok_thread(dbg, k + 8 <= count && k + 8 <= dbg.arena && src >= 0 &&
+                                          src + 8 <= dbg.ns, k)) {
+                code[j] = kFlatPad;
+                continue;
+            }
+#endif
+            D[j] = (int)(src & 7);
+            const uint4* s = reinterpret_cast<const uint4*>(ag + (src - D[j]));
+            x[j] = __ldg(s);
+            if (D[j] != 0) y[j] = __ldg(s + 1);
+            else y[j] = x[j];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kFlatV; ++j) {
+        const int32_t c = code[j];
+        if (!(c & 1) && c != kFlatPad)
+            __stcs(reinterpret_cast<uint4*>(arena + 8 * (q0 + (int64_t)j * kThreads)),
+                   shift_bf16x8(x[j], y[j], D[j]));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // shard: master[shard_pos + e] = full[arena_pos + e]; pads +0 (set-up path)
 // ---------------------------------------------------------------------------
@@ -393,6 +470,14 @@ cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* a
 cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* arena,
                             cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
+    if (g.flat) {
+        const int64_t n_mixed = (int64_t)g.amixq.size();
+        const int64_t mixed_ctas = flat_mixed_ctas(n_mixed);
+        k_copy_out_flat<<<(unsigned)(flat_grid(g.P_arena) + mixed_ctas), kThreads, 0, st>>>(
+            ag, arena, g.P_arena, g.d_amap, g.d_amixq, g.d_amixc, n_mixed, mixed_ctas
+            FSDPK_DBG_ARG(debug_bounds(g, kDbgCopyOutFlat)));
+        return cudaGetLastError();
+    }
     return launch_copy_out_units<false, uint16_t>(g, ag, nullptr, arena, kDbgCopyOut, st);
 }
 

@@ -27,6 +27,34 @@ constexpr int64_t kShortRun = 1024;
 constexpr int64_t kPackUnits = 64;
 constexpr int64_t kPackElems = 16384;
 
+// Flat path of a group of many small parameters (at least kFlatMinUnits
+// short and pad units): the fused reduce-scatter, the fused update and the
+// copy-out run over fixed tiles of the flat index space instead of over
+// units, reading one code per 16-byte vector of 8 bf16 elements:
+//   even, not kFlatPad: all 8 elements are real rows of one run, and
+//                       element k's other-side position is k + code / 2
+//   kFlatPad:           all 8 elements are pad rows (shard side) or arena
+//                       gaps (arena side)
+//   odd, 2 m + 1:       mixed (several runs, a run and pads or gaps, or the
+//                       partial last vector): entry m of the mixed list, whose
+//                       vector index is mixq[m] and whose elements' codes
+//                       (2 * offset, or kFlatPad; kFlatPad past the end) are
+//                       mixc[8 m .. 8 m + 7].  A second launch takes the
+//                       mixed vectors, a thread per element.
+// Codes are int32, so both index spaces stay below kFlatMaxElems.
+constexpr int64_t kFlatMinUnits = 2048;
+constexpr int64_t kFlatMaxElems = (int64_t{1} << 30) - 64;
+constexpr int32_t kFlatPad = INT32_MIN;
+
+// A maximal range of a flat index space with one code (2 * offset to the
+// other side, or kFlatPad), running to the next segment's start; the last
+// segment of a table is a sentinel at the end of the space.  Host side only:
+// the codes and the mixed lists are built from these segments.
+struct FlatSeg {
+    int32_t start;
+    int32_t code;
+};
+
 // One contiguous run of a (rank j, parameter i) shard segment.
 //   shard_pos: first element in the rank-major [N][S] index space
 //   arena_pos: first element of the matching rows in an unsharded arena
@@ -71,7 +99,8 @@ struct DebugBounds {
 enum DebugKernel : int32_t {
     kDbgCopyIn = 1, kDbgCopyOut, kDbgCopyOutTab, kDbgShard, kDbgReduce, kDbgReduceTab,
     kDbgRsAdamw, kDbgRsAdamwTab, kDbgReduceAcc, kDbgFp8Amax, kDbgFp8CopyIn, kDbgFp8CopyOut,
-    kDbgFp8CopyOutTab, kDbgSmallStep, kDbgCopyInF32, kDbgCopyOutF32
+    kDbgFp8CopyOutTab, kDbgSmallStep, kDbgCopyInF32, kDbgCopyOutF32, kDbgReduceFlat,
+    kDbgRsAdamwFlat, kDbgCopyOutFlat
 };
 
 }  // namespace fsdpk
@@ -102,8 +131,15 @@ struct fsdp_group {
     std::vector<fsdpk::Interval> intervals;
     std::vector<fsdpk::TileRange> tile_ranges;  // empty when no padding
     int64_t n_tiles = 0;                        // copy-in tiles over L*S
+    // flat path (empty unless flat): codes of the shard-side vectors of
+    // [L][S] and of the arena-side vectors of [P_arena], with their segments
+    bool flat = false;
+    std::vector<int32_t> smap, amap;    // one code per vector
+    std::vector<int32_t> smixq, amixq;  // the mixed vectors
+    std::vector<int32_t> smixc, amixc;  // their elements' codes, 8 per vector
+    std::vector<fsdpk::FlatSeg> ssegs, asegs;
 
-    // one device allocation holding the three tables
+    // one device allocation holding the tables
     void* dev_mem = nullptr;
     const fsdpk::Unit* d_units = nullptr;
     const fsdpk::Interval* d_intervals = nullptr;
@@ -111,6 +147,12 @@ struct fsdp_group {
     const int32_t* d_unit_param = nullptr;
     const int32_t* d_packs = nullptr;
     const int32_t* d_rpacks = nullptr;
+    const int32_t* d_smap = nullptr;
+    const int32_t* d_smixq = nullptr;
+    const int32_t* d_smixc = nullptr;
+    const int32_t* d_amap = nullptr;
+    const int32_t* d_amixq = nullptr;
+    const int32_t* d_amixc = nullptr;
 };
 
 // The opaque peer plan behind fsdp_peer_t: device `index` of `n_devices` holds the

@@ -66,7 +66,7 @@ __device__ __forceinline__ void reduce_body(const Src& src_al, float* __restrict
                 }
                 if (avg) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[e] = __fdiv_rn(acc[e], fN);
+                    for (int e = 0; e < 8; ++e) acc[e] = div_n<NR>(acc[e], fN);
                 }
                 store8(dst + 8 * q, acc);
             }
@@ -136,7 +136,7 @@ __device__ __forceinline__ void reduce_unit(const Src& src_run, float* __restric
                                             Team tm = cta_team()) {
     const int head = (int)head_to_16B(dst_run, len);
     if (tm.t < head)
-        dst_run[tm.t] = finish(fold_scalar<NR>(src_run.at(tm.t), N), avg, fN);
+        dst_run[tm.t] = finish<NR>(fold_scalar<NR>(src_run.at(tm.t), N), avg, fN);
     const int nvec = (len - head) >> 3;
     // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0, and
     // table pointers are checked on the host), so one phase D holds for all N
@@ -148,7 +148,7 @@ __device__ __forceinline__ void reduce_unit(const Src& src_run, float* __restric
     else reduce_body_dispatch<NR, true>(src_al, N, dst, nvec, D, avg, fN, tm);
     const int done = head + 8 * nvec;
     if (tm.t < len - done)
-        dst_run[done + tm.t] = finish(fold_scalar<NR>(src_run.at(done + tm.t), N), avg, fN);
+        dst_run[done + tm.t] = finish<NR>(fold_scalar<NR>(src_run.at(done + tm.t), N), avg, fN);
 }
 
 // Zero-fill `len` fp32 elements at dst (any alignment) by one warp.
@@ -248,6 +248,109 @@ k_reduce_units_tab(const uint16_t* const* __restrict__ rank_tab, int N, float* _
             continue;
         }
         reduce_unit<NR>(TableSrc{s_tab, u.arena_pos}, dst_run, u.len, N, avg, fN);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// flat fused reduce-scatter (a group of many small parameters): one CTA per
+// tile of kFlatTile elements of [N][S].  Each thread reads the codes of its
+// kFlatV vectors first; a vector inside one real run folds its 8 elements
+// from aligned 16-byte loads of every rank (shifted by the run's phase), a
+// pad vector is +0.  Mixed vectors go a thread per element.  Same
+// arithmetic per element as k_reduce_units, so the same bits.
+// ---------------------------------------------------------------------------
+
+// This thread's elements of the mixed vectors: element t + i * T (T the
+// region's threads) is element e = t % 8 of list entry m = t / 8, i.e.
+// k = 8 * mixq[m] + e with code mixc[t]; every rank's loads of all of them
+// issued before the folds.
+template <int NR>
+__device__ __forceinline__ void reduce_flat_mixed(const uint16_t* __restrict__ grads,
+                                                  int64_t stride, int N, float* __restrict__ out,
+                                                  int64_t count, const int32_t* __restrict__ mixq,
+                                                  const int32_t* __restrict__ mixc,
+                                                  int64_t n_mixed, int64_t t0, int64_t T,
+                                                  bool avg, float fN FSDPK_DBG_PARAM) {
+    int64_t k[kFlatMixedPer];
+    int32_t c[kFlatMixedPer];
+    bool on[kFlatMixedPer];
+#pragma unroll
+    for (int i = 0; i < kFlatMixedPer; ++i) {
+        const int64_t t = t0 + i * T;
+        on[i] = t < 8 * n_mixed;
+        k[i] = on[i] ? 8 * (int64_t)mixq[t >> 3] + (t & 7) : 0;
+        c[i] = on[i] ? mixc[t] : kFlatPad;
+        on[i] = on[i] && k[i] < count;
+#ifdef FSDPK_DEBUG
+        if (on[i] && !debug_ok_thread(dbg, k[i] < dbg.ns &&
+                                               (c[i] == kFlatPad || (k[i] + (c[i] >> 1) >= 0 &&
+                                                                     k[i] + (c[i] >> 1) < dbg.arena)),
+                                      k[i]))
+            on[i] = false;
+#endif
+    }
+    float g[kFlatMixedPer];
+    const int n = NR ? NR : N;
+#pragma unroll
+    for (int i = 0; i < kFlatMixedPer; ++i) g[i] = 0.0f;
+#pragma unroll(NR ? NR : 1)
+    for (int r = 0; r < n; ++r) {
+        uint32_t h[kFlatMixedPer];
+#pragma unroll
+        for (int i = 0; i < kFlatMixedPer; ++i)
+            h[i] = (on[i] && c[i] != kFlatPad) ? (uint32_t)grads[r * stride + k[i] + (c[i] >> 1)]
+                                               : 0u;
+#pragma unroll
+        for (int i = 0; i < kFlatMixedPer; ++i)
+            g[i] = r == 0 ? bf16_bits_to_f32(h[i]) : __fadd_rn(g[i], bf16_bits_to_f32(h[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < kFlatMixedPer; ++i)
+        if (on[i]) out[k[i]] = c[i] == kFlatPad ? 0.0f : finish<NR>(g[i], avg, fN);
+}
+
+// One launch: CTAs [0, mixed_ctas) take the mixed vectors' elements,
+// kFlatMixedPer a thread (first in the grid, so that these few latency-bound
+// CTAs run beside the tiles rather than after them); the others one tile
+// each.
+template <int NR>
+__global__ void __launch_bounds__(kThreads, (NR >= 1 && NR <= 8) ? 3 : 2)
+k_reduce_flat(const uint16_t* __restrict__ grads, int64_t stride, int N, float* __restrict__ out,
+              int64_t count, const int32_t* __restrict__ smap, const int32_t* __restrict__ mixq,
+              const int32_t* __restrict__ mixc, int64_t n_mixed, int64_t mixed_ctas,
+              int op_avg FSDPK_DBG_PARAM) {
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    if ((int64_t)blockIdx.x < mixed_ctas) {
+        reduce_flat_mixed<NR>(grads, stride, N, out, count, mixq, mixc, n_mixed,
+                              (int64_t)blockIdx.x * kThreads + threadIdx.x, mixed_ctas * kThreads,
+                              avg, fN FSDPK_DBG_ARG(dbg));
+        return;
+    }
+    const int64_t nv = (count + 7) >> 3;
+    const int64_t q0 = ((int64_t)blockIdx.x - mixed_ctas) * (kThreads * kFlatV) + threadIdx.x;
+    int32_t code[kFlatV];
+    flat_tile_codes(smap, q0, nv, code);
+#pragma unroll 1
+    for (int j = 0; j < kFlatV; ++j) {
+        const int32_t c = flat_pick(code, j);
+        if (c & 1) continue;  // mixed, or past the end
+        const int64_t k = 8 * (q0 + (int64_t)j * kThreads);
+        FSDPK_THREAD_GUARD(k + 8 <= count && k + 8 <= dbg.ns, k);
+        float acc[8];
+        if (c == kFlatPad) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        } else {
+            const int64_t a = k + (c >> 1);
+            FSDPK_THREAD_GUARD(a >= 0 && a + 8 <= dbg.arena, k);
+            flat_fold8<NR>(grads, stride, N, a, acc);
+            if (avg) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = div_n<NR>(acc[e], fN);
+            }
+        }
+        store8(out + k, acc);
     }
 }
 
@@ -484,6 +587,32 @@ inline void reduce_split(const fsdp_group& g, int64_t* n_cta_units, int64_t* n_p
     }
 }
 
+template <int NR>
+cudaError_t launch_reduce_flat_nr(const fsdp_group& g, const uint16_t* grads, int avg,
+                                  float* reduced, cudaStream_t st) {
+    const int64_t count = (int64_t)g.L * g.S;
+    const int64_t n_mixed = (int64_t)g.smixq.size();
+    const int64_t mixed_ctas = flat_mixed_ctas(n_mixed);
+    k_reduce_flat<NR><<<(unsigned)(flat_grid(count) + mixed_ctas), kThreads, 0, st>>>(
+        grads, g.P_arena, g.N, reduced, count, g.d_smap, g.d_smixq, g.d_smixc, n_mixed,
+        mixed_ctas, avg FSDPK_DBG_ARG(debug_bounds(g, kDbgReduceFlat)));
+    return cudaGetLastError();
+}
+
+// The flat fused reduce-scatter of a plan with the flat tables.
+cudaError_t launch_reduce_flat(const fsdp_group& g, const uint16_t* grads, int avg,
+                               float* reduced, cudaStream_t st) {
+    switch (g.N) {
+#define FSDPK_CASE(K) \
+    case K: return launch_reduce_flat_nr<K>(g, grads, avg, reduced, st);
+        FSDPK_CASE(1) FSDPK_CASE(2) FSDPK_CASE(3) FSDPK_CASE(4)
+        FSDPK_CASE(5) FSDPK_CASE(6) FSDPK_CASE(7) FSDPK_CASE(8)
+#undef FSDPK_CASE
+        default:
+            return launch_reduce_flat_nr<0>(g, grads, avg, reduced, st);
+    }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -497,6 +626,7 @@ cudaError_t launch_rs_fused(const fsdp_group& g, const uint16_t* grads, int op, 
     const int avg = (op == FSDP_AVG || op == FSDP_SUM_THEN_DIV) ? 1 : 0;
     const int64_t stride = g.P_arena;
     const DebugBounds dbg = debug_bounds(g, kDbgReduce);
+    if (g.flat) return launch_reduce_flat(g, grads, avg, reduced, st);
     int64_t nl, np;
     reduce_split(g, &nl, &np);
     (void)nu;

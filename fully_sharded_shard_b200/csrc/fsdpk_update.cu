@@ -247,7 +247,7 @@ __device__ __forceinline__ void fused_body(const Src& src_al, int N, int D, cons
         fold8<NR, SHIFTED>(src_al, N, q, D, g);
         if (avg) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = __fdiv_rn(g[e], fN);
+            for (int e = 0; e < 8; ++e) g[e] = div_n<NR>(g[e], fN);
         }
         fused8<FP8>(o, k, g, P, M, V, false, sc, scale, mx);
     }
@@ -263,7 +263,7 @@ __device__ __forceinline__ void rs_adamw_real_unit(const Src& src_run, int N, co
                                                    Team tm = cta_team()) {
     const int done = head + 8 * nvec;
     if (tm.t < head)
-        fused1<FP8>(o, k0 + tm.t, finish(fold_scalar<NR>(src_run.at(tm.t), N), avg, fN), false,
+        fused1<FP8>(o, k0 + tm.t, finish<NR>(fold_scalar<NR>(src_run.at(tm.t), N), avg, fN), false,
                     sc, scale, mx);
     // every rank's arena starts on a 16-byte boundary (P_arena % 8 == 0, and
     // table pointers are checked on the host), so one phase D holds for all N
@@ -276,7 +276,7 @@ __device__ __forceinline__ void rs_adamw_real_unit(const Src& src_run, int N, co
         fused_body<NR, true, FP8>(src_al, N, D, o, k0 + head, nvec, avg, fN, sc, scale, mx, tm);
     if (tm.t < len - done)
         fused1<FP8>(o, k0 + done + tm.t,
-                    finish(fold_scalar<NR>(src_run.at(done + tm.t), N), avg, fN), false, sc,
+                    finish<NR>(fold_scalar<NR>(src_run.at(done + tm.t), N), avg, fN), false, sc,
                     scale, mx);
 }
 
@@ -408,6 +408,129 @@ k_rs_adamw(const uint16_t* __restrict__ grads, int64_t stride,
     }
 }
 
+// Flat fused update (a group of many small parameters, bf16 all-gather
+// input): one CTA per tile of kFlatTile elements of [N][S], kFlatV vectors of
+// 8 per thread with their codes read first.  A vector inside one real run
+// loads master/m/v and every rank's 8 source elements at once, a pad vector
+// updates with g = +0 and writes +0 to ag.  Mixed vectors go a thread per
+// element.  Same per-element arithmetic as k_rs_adamw, so the same bits.
+// This thread's elements of the mixed vectors (element t + i * T, T the
+// region's threads, is element t % 8 of list entry t / 8), every load of all
+// of them issued before the arithmetic.
+template <int NR>
+__device__ __forceinline__ void rs_adamw_flat_mixed(const uint16_t* __restrict__ grads,
+                                                    int64_t stride, int N, const FusedOut& o,
+                                                    int64_t count,
+                                                    const int32_t* __restrict__ mixq,
+                                                    const int32_t* __restrict__ mixc,
+                                                    int64_t n_mixed, int64_t t0, int64_t T,
+                                                    bool avg, float fN, const AdamScalars& sc
+                                                    FSDPK_DBG_PARAM) {
+    int64_t k[kFlatMixedPer];
+    int32_t c[kFlatMixedPer];
+    bool on[kFlatMixedPer];
+    float pp[kFlatMixedPer], mm[kFlatMixedPer], vv[kFlatMixedPer];
+#pragma unroll
+    for (int i = 0; i < kFlatMixedPer; ++i) {
+        const int64_t t = t0 + i * T;
+        on[i] = t < 8 * n_mixed;
+        k[i] = on[i] ? 8 * (int64_t)mixq[t >> 3] + (t & 7) : 0;
+        c[i] = on[i] ? mixc[t] : kFlatPad;
+        on[i] = on[i] && k[i] < count;
+#ifdef FSDPK_DEBUG
+        if (on[i] && !debug_ok_thread(dbg, k[i] < dbg.ns &&
+                                               (c[i] == kFlatPad || (k[i] + (c[i] >> 1) >= 0 &&
+                                                                     k[i] + (c[i] >> 1) < dbg.arena)),
+                                      k[i]))
+            on[i] = false;
+#endif
+        if (on[i]) {
+            pp[i] = o.p[k[i]];
+            mm[i] = o.m[k[i]];
+            vv[i] = o.v[k[i]];
+        }
+    }
+    float g[kFlatMixedPer];
+    const int n = NR ? NR : N;
+#pragma unroll
+    for (int i = 0; i < kFlatMixedPer; ++i) g[i] = 0.0f;
+#pragma unroll(NR ? NR : 1)
+    for (int r = 0; r < n; ++r) {
+        uint32_t h[kFlatMixedPer];
+#pragma unroll
+        for (int i = 0; i < kFlatMixedPer; ++i)
+            h[i] = (on[i] && c[i] != kFlatPad) ? (uint32_t)grads[r * stride + k[i] + (c[i] >> 1)]
+                                               : 0u;
+#pragma unroll
+        for (int i = 0; i < kFlatMixedPer; ++i)
+            g[i] = r == 0 ? bf16_bits_to_f32(h[i]) : __fadd_rn(g[i], bf16_bits_to_f32(h[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < kFlatMixedPer; ++i) {
+        if (!on[i]) continue;
+        const bool pad = c[i] == kFlatPad;
+        const float gi = pad ? 0.0f : finish<NR>(g[i], avg, fN);
+        adamw1(pp[i], mm[i], vv[i], gi, sc);
+        o.p[k[i]] = pp[i];
+        o.m[k[i]] = mm[i];
+        o.v[k[i]] = vv[i];
+        if (o.red) o.red[k[i]] = gi;
+        if (o.ag) {
+            __nv_bfloat16 h = __float2bfloat16_rn(pad ? 0.0f : pp[i]);
+            o.ag[k[i]] = *reinterpret_cast<uint16_t*>(&h);
+        }
+    }
+}
+
+// One launch: CTAs [0, mixed_ctas) take the mixed vectors' elements,
+// kFlatMixedPer a thread, first in the grid; the others one tile each.
+template <int NR>
+__global__ void __launch_bounds__(kThreads, 2)
+k_rs_adamw_flat(const uint16_t* __restrict__ grads, int64_t stride, int N, FusedOut o,
+                int64_t count, const int32_t* __restrict__ smap, const int32_t* __restrict__ mixq,
+                const int32_t* __restrict__ mixc, int64_t n_mixed, int64_t mixed_ctas,
+                int op_avg, AdamScalars sc, const AdamScalars* __restrict__ sc_dev
+                FSDPK_DBG_PARAM) {
+    if (sc_dev != nullptr) sc = *sc_dev;  // scalars of a graph-replayed step
+    const bool avg = op_avg != 0;
+    const float fN = (float)N;
+    if ((int64_t)blockIdx.x < mixed_ctas) {
+        rs_adamw_flat_mixed<NR>(grads, stride, N, o, count, mixq, mixc, n_mixed,
+                                (int64_t)blockIdx.x * kThreads + threadIdx.x,
+                                mixed_ctas * kThreads, avg, fN, sc FSDPK_DBG_ARG(dbg));
+        return;
+    }
+    const int64_t nv = (count + 7) >> 3;
+    const int64_t q0 = ((int64_t)blockIdx.x - mixed_ctas) * (kThreads * kFlatV) + threadIdx.x;
+    int32_t code[kFlatV];
+    flat_tile_codes(smap, q0, nv, code);
+#pragma unroll 1
+    for (int j = 0; j < kFlatV; ++j) {
+        const int32_t c = flat_pick(code, j);
+        if (c & 1) continue;  // mixed, or past the end
+        const int64_t k = 8 * (q0 + (int64_t)j * kThreads);
+        FSDPK_THREAD_GUARD(k + 8 <= count && k + 8 <= dbg.ns, k);
+        float4 P[2], M[2], V[2];
+        load_pmv8(o, k, P, M, V);
+        float g[8];
+        const bool pad = c == kFlatPad;
+        if (pad) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = 0.0f;
+        } else {
+            const int64_t a = k + (c >> 1);
+            FSDPK_THREAD_GUARD(a >= 0 && a + 8 <= dbg.arena, k);
+            flat_fold8<NR>(grads, stride, N, a, g);
+            if (avg) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) g[e] = div_n<NR>(g[e], fN);
+            }
+        }
+        float mx = 0.0f;
+        fused8<false>(o, k, g, P, M, V, pad, sc, 0.0f, mx);
+    }
+}
+
 // The fused update packs its short and pad units when there are at least
 // this many of them (thousands of small parameters).
 constexpr int64_t kFusedPackMinUnits = 2048;
@@ -416,6 +539,17 @@ template <int NR, bool FP8>
 cudaError_t launch_rs_adamw_nr(const fsdp_group& g, const uint16_t* grads, const FusedOut& o,
                                int avg, const AdamScalars& sc, const AdamScalars* sc_dev,
                                cudaStream_t st) {
+    if constexpr (!FP8) {
+        if (g.flat) {
+            const int64_t count = (int64_t)g.L * g.S;
+            const int64_t n_mixed = (int64_t)g.smixq.size();
+            const int64_t mixed_ctas = flat_mixed_ctas(n_mixed);
+            k_rs_adamw_flat<NR><<<(unsigned)(flat_grid(count) + mixed_ctas), kThreads, 0, st>>>(
+                grads, g.P_arena, g.N, o, count, g.d_smap, g.d_smixq, g.d_smixc, n_mixed,
+                mixed_ctas, avg, sc, sc_dev FSDPK_DBG_ARG(debug_bounds(g, kDbgRsAdamwFlat)));
+            return cudaGetLastError();
+        }
+    }
     int64_t nu = (int64_t)g.units.size();
     const int64_t n_small = nu - g.n_long_units;
     if (n_small >= kFusedPackMinUnits) {

@@ -154,9 +154,25 @@ FSDP_API int fsdp_plan_group_host(const fsdp_param_desc* params, int32_t n_param
  * shard, the units covering [N][S] exactly once, each real unit's arena
  * position recomputed from its shard position (the Shard(0) placement), pad
  * units on the pad rows, the pad intervals matching the pad units, and each
- * copy-in tile's interval range.  *violations receives the number of failed
- * checks (0 for every plan this library builds).  Host only. */
+ * copy-in tile's interval range, the pack tables, and the flat path's
+ * segment and vector-code tables recomputed from the units.  *violations
+ * receives the number of failed checks (0 for every plan this library
+ * builds).  Host only. */
 FSDP_API int fsdp_group_check(fsdp_group_t group, int64_t* violations);
+
+/* Which work tables the data calls of a plan use.  A group of many small
+ * parameters (at least 2048 short and pad runs, both index spaces below 2^30
+ * elements) takes the flat path in the bf16 copy-out, the fused
+ * reduce-scatter and the bf16 fused update: fixed tiles of the index space,
+ * one code per 8-element vector, instead of one work unit per (rank,
+ * parameter) run -- the same results, bit for bit.  *flat receives 1 for
+ * such a plan, else 0; *mixed_shard and *mixed_arena the vectors of the
+ * [N][S] and of the arena index space that hold more than one run (or a run
+ * and padding, or the ragged end), which go element by element (0 when not
+ * flat).  Host only; any output pointer may be NULL.
+ * Errors: FSDP_EINVAL (NULL group). */
+FSDP_API int fsdp_group_flat(fsdp_group_t group, int32_t* flat, int64_t* mixed_shard,
+                             int64_t* mixed_arena);
 
 /* S (per-rank padded shard elements), P (real elements), P_arena of a plan:
  * the sizes of one rank's padded shard of the group and of the unsharded

@@ -35,7 +35,7 @@ def _run(mode: str) -> dict:
 
 def test_debug_build_grid_has_no_violations():
     out = _run("grid")
-    assert out["cases"] == 52          # 9 grid groups, 40 random groups, 2 peer cases, 1 packed
+    assert out["cases"] == 54          # 9 grid groups, 40 random groups, 2 peer cases, 3 flat
     assert out["words"][0] == 0, f"violations: {out['words']}"
 
 
@@ -44,3 +44,10 @@ def test_debug_build_checks_fire_on_narrowed_extents():
     assert out["copy_out"][0] > 0 and out["copy_out"][1] == 2, out   # kDbgCopyOut
     assert out["tail_kept"], "a skipped unit was written"
     assert out["reduce"][0] > 0 and out["reduce"][1] == 5, out       # kDbgReduce
+    # the flat path of a group of many small parameters
+    assert out["flat_copy_out"][0] > 0 and out["flat_copy_out"][1] == 19, out  # kDbgCopyOutFlat
+    assert out["flat_tail_kept"], "a skipped element was written"
+    assert out["flat_reduce"][0] > 0 and out["flat_reduce"][1] == 17, out      # kDbgReduceFlat
+    assert out["flat_reduce_kept"], out
+    assert out["flat_update"][0] > 0 and out["flat_update"][1] == 18, out      # kDbgRsAdamwFlat
+    assert out["flat_update_kept"], out

@@ -81,15 +81,21 @@ def _u16_of(x: np.ndarray) -> np.ndarray:
         .view(torch.int16).numpy().view(np.uint16)
 
 
-def _layout(N):
+# The edge group followed by 800 small parameters: at least 2048 short and
+# pad runs at every N here, so the copy-out, the fused reduce-scatter and the
+# fused update take the flat path (fixed tiles, one code per 8 elements).
+FLAT_SHAPES = SHAPES + [(3 + k % 23, 1 + k % 5) for k in range(800)]
+
+
+def _layout(N, shapes=SHAPES):
     import oracle
-    return oracle.plan(SHAPES, N)
+    return oracle.plan(shapes, N)
 
 
-def full_init(N: int) -> np.ndarray:
+def full_init(N: int, shapes=SHAPES) -> np.ndarray:
     """The full fp32 parameters in the arena layout: seeded N(0, 0.02), the
     listed values at the head of each parameter."""
-    p = _layout(N)
+    p = _layout(N, shapes)
     rng = np.random.default_rng(11)
     full = (rng.standard_normal(p.P_arena) * 0.02).astype(np.float32)
     u = [int(x) for x in p.arena_off]
@@ -102,11 +108,11 @@ def full_init(N: int) -> np.ndarray:
     return full
 
 
-def grads_init(N: int):
+def grads_init(N: int, shapes=SHAPES):
     """step -> bf16 bit patterns [N][P_arena]: seeded N(0, 1e-3), the fold
     cases at the heads of p0 and p4, and a negative gradient on the amax
     elements of p2 and p3."""
-    p = _layout(N)
+    p = _layout(N, shapes)
     u = [int(x) for x in p.arena_off]
 
     def make(step: int) -> np.ndarray:
@@ -122,8 +128,8 @@ def grads_init(N: int):
     return make
 
 
-def _wl(N, op):
-    g = W.Group("edge", list(SHAPES), [f"p{i}" for i in range(len(SHAPES))])
+def _wl(N, op, shapes=SHAPES):
+    g = W.Group("edge", list(shapes), [f"p{i}" for i in range(len(shapes))])
     return W.Workload(f"edge_n{N}", N, [g], op, 0, "normal", 0.02, 1e-3, steps=2)
 
 
@@ -152,6 +158,24 @@ def test_edge_values_through_the_five_stages(H, N):
     wl = _wl(N, W.AVG)
     H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=True,
                 full_init=full_init(N), grads_init=grads_init(N))
+
+
+@pytest.mark.parametrize("N", NS)
+def test_edge_values_through_the_flat_path(H, N):
+    """The same values in a group of many small parameters: the flat
+    copy-out, fused reduce-scatter (all ops) and fused update."""
+    from fully_sharded_shard_b200 import abi
+    g = abi.fsdp_plan_group(FLAT_SHAPES, N)
+    flat, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
+    g.destroy()
+    assert flat and mixed_shard > 0 and mixed_arena > 0
+    fi, gi = full_init(N, FLAT_SHAPES), grads_init(N, FLAT_SHAPES)
+    wl = _wl(N, W.AVG, FLAT_SHAPES)
+    H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=False, full_init=fi,
+                grads_init=gi)
+    for op in ALL_OPS:
+        wl = _wl(N, op, FLAT_SHAPES)
+        H.run_group_fused(wl, wl.groups[0], steps=2, full_init=fi, grads_init=gi)
 
 
 @pytest.mark.parametrize("N", NS)

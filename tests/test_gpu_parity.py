@@ -338,6 +338,40 @@ def test_many_small_parameters_packed_paths(H):
     H.run_group_fp8(wl, grp)
 
 
+def _small(count, seed):
+    return W.small_params(count=count, seed=seed).groups[0].shapes
+
+
+# Groups of many small parameters, which take the flat path: N = 1 (no pads),
+# an odd [N][S] (a partial last vector), long runs beside the small ones, and
+# the any-N kernels (N = 11).
+FLAT = [
+    _wl("flat_n1", _small(4000, 15), 1, op=W.SUM),
+    _wl("flat_n3", _small(1000, 11), 3, op=W.SUM),
+    _wl("flat_n5_long", _small(700, 12) + [(30001, 64), (4097,), (0, 5), (1, 1)], 5),
+    _wl("flat_n8", _small(600, 13), 8, op=W.SUM_THEN_DIV),
+    _wl("flat_n11", _small(400, 14), 11),
+]
+
+
+@pytest.mark.parametrize("wl", FLAT, ids=[w.name for w in FLAT])
+def test_many_small_parameters_flat_path(H, wl):
+    """The flat copy-out, fused reduce-scatter (every op) and fused update
+    against the oracle; the FP8 paths of the same group keep the packs."""
+    from fully_sharded_shard_b200 import abi
+    grp = wl.groups[0]
+    g = abi.fsdp_plan_group(grp.shapes, wl.N)
+    flat, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
+    assert abi.fsdp_group_check(g) == 0
+    g.destroy()
+    assert flat and mixed_shard > 0 and mixed_arena > 0
+    if wl.name == "flat_n3":
+        assert (wl.N * g.S) % 8 != 0, "the partial last vector"
+    H.run_group(wl, grp, steps=2, ops=ALL_OPS, staged=False)
+    H.run_group_fused(wl, grp, steps=2)
+    H.run_group_fused_fp8(wl, grp, steps=1)
+
+
 GRID = [_wl(f"grid_n{N}", [((d0, c) if c > 1 else (d0,)) for d0 in range(21) for c in (1, 3, 8)], N,
             op=[W.SUM, W.AVG, W.SUM_THEN_DIV][N % 3]) for N in range(1, 10)]
 

@@ -57,6 +57,22 @@ def test_brute_force_grid_plans_on_host(abi, oracle):
         _compare(abi, oracle, shapes, N)
 
 
+def test_flat_path_for_groups_of_many_small_parameters(abi):
+    """The flat tables exist for a group of thousands of small parameters
+    (and pass the check), not for the transformer groups."""
+    from fully_sharded_shard_b200 import workloads as W
+    wl = W.small_params()
+    g = abi.fsdp_plan_group_host(wl.groups[0].shapes, wl.N)
+    flat, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
+    assert flat and 0 < mixed_shard < wl.N * g.S // 8 // 20 and 0 < mixed_arena
+    assert abi.fsdp_group_check(g) == 0
+    g.destroy()
+    for wl in (W.llama_block(), W.uneven(), W.moe(), W.tiny_mlp()):
+        g = abi.fsdp_plan_group_host(wl.groups[0].shapes, wl.N)
+        assert abi.fsdp_group_flat(g) == (False, 0, 0)
+        g.destroy()
+
+
 def test_data_calls_refuse_a_host_plan(abi):
     L = abi.lib()
     g = abi.fsdp_plan_group_host([(7, 3), (5,)], 2)
@@ -79,6 +95,30 @@ MUTANTS_PACKS = [
      "return g->units[k].len >= fsdpk::kShortRun / 2;"),
 ]
 
+MUTANTS_FLAT = [
+    ("flat shard code one element off",
+     "sruns.push_back({u.shard_pos, u.len, 2 * (u.arena_pos - u.shard_pos)});",
+     "sruns.push_back({u.shard_pos, u.len, 2 * (u.arena_pos - u.shard_pos + 1)});"),
+    ("flat arena code one element off",
+     "aruns.push_back({u.arena_pos, u.len, 2 * (u.shard_pos - u.arena_pos)});",
+     "aruns.push_back({u.arena_pos, u.len, 2 * (u.shard_pos - u.arena_pos) + 2});"),
+    ("a mixed vector coded pure",
+     "if (hi <= end && segs[i + 1].start >= hi) {",
+     "if (hi <= end && segs[i + 1].start >= lo + 4) {"),
+    ("a mixed vector's elements all given its first code",
+     "while (k < end && segs[t + 1].start <= k) ++t;",
+     "while (false) ++t;"),
+    ("arena gaps not marked",
+     "if (r[0] > at) put(at, kFlatPad);",
+     "(void)0;"),
+    ("flat segments not merged",
+     "if (segs.empty() || segs.back().code != code)",
+     "if (true)"),
+    ("flat path below its threshold",
+     "n_small < kFlatMinUnits ||",
+     "n_small < kFlatMinUnits / 4 ||"),
+]
+
 MUTANTS = [
     ("arena one row off",
      "g->u[i] + j * g->c[i] * g->cols[i], v * g->cols[i], 0);",
@@ -98,8 +138,10 @@ MUTANTS = [
 ]
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS + MUTANTS_PACKS,
-                         ids=[m[0] for m in MUTANTS + MUTANTS_PACKS])
+ALL_MUTANTS = MUTANTS + MUTANTS_PACKS + MUTANTS_FLAT
+
+
+@pytest.mark.parametrize("name,old,new", ALL_MUTANTS, ids=[m[0] for m in ALL_MUTANTS])
 def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
     import glob
     import os
@@ -131,6 +173,9 @@ def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
     shapes += [(3 + k % 50, 1 + k % 7) for k in range(300)] + [(600, 1)] * 10
     # runs of 512-1023 elements between long ones (700 at N = 2, 3, 4, 6)
     shapes += [(1400, 1), (9001, 1), (2100, 1), (9001, 1), (2800, 1), (4200, 1), (9001, 1)]
+    # and tiny ones: the flat path at N = 4 (a partial last vector) and 6, not
+    # at N = 2 and 3
+    shapes += [(1 + k % 13, 1 + k % 3) for k in range(150)]
     found = 0
     for N in (2, 3, 4, 6):
         _, arr = abi._descs(shapes)
