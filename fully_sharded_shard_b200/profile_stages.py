@@ -12,7 +12,10 @@ unsharded arena), rs_reduce (fused reduce-scatter), adamw, rs_adamw (fused
 reduce-scatter + AdamW + next copy-in).  Every buffer is allocated once and
 filled with seeded values; each iteration runs the stages in that order, and
 the per-stage CUDA-event times (median over the iterations) are printed as
-one JSON line with the algorithmic bytes and GB/s of each stage.
+one JSON line with the algorithmic bytes and GB/s of each stage.  Before
+every stage a 256 MB buffer (twice the L2) is written outside the timed
+events, so a stage never reads what the previous one left in L2 (a group of
+small parameters fits there); --no-flush leaves L2 alone.
 """
 from __future__ import annotations
 
@@ -42,6 +45,8 @@ def main(argv=None) -> int:
     ap.add_argument("--group", type=int, default=0)
     ap.add_argument("--stages", default="copy_in,copy_out")
     ap.add_argument("--iters", type=int, default=5)
+    ap.add_argument("--no-flush", action="store_true",
+                    help="do not write a buffer larger than L2 before each stage")
     args = ap.parse_args(argv)
     stages = [s for s in args.stages.split(",") if s]
     for s in stages:
@@ -91,9 +96,12 @@ def main(argv=None) -> int:
         "rs_adamw": lambda t: abi.fsdp_rs_adamw_step(g, grads, wl.op, master, m, v, step=t,
                                                      ag_next=ag, **hp),
     }
+    flush = None if args.no_flush else torch.empty(64 << 20, dtype=torch.float32, device=dev)
     times = {s: [] for s in stages}
     for t in range(1, args.iters + 1):
         for s in stages:
+            if flush is not None:
+                flush.zero_()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -102,6 +110,7 @@ def main(argv=None) -> int:
             times[s].append((e0, e1))
     torch.cuda.synchronize()
     out = {"workload": wl.name, "group": grp.name, "N": N, "S": g.S, "P": g.P,
+           "l2": "not flushed" if flush is None else "256 MB written before each stage",
            "device_bytes": int(torch.cuda.max_memory_allocated(dev)), "stages": {}}
     for s in stages:
         ms = statistics.median(a.elapsed_time(b) for a, b in times[s])
