@@ -251,15 +251,16 @@ def fsdp_group_check(g: Group) -> int:
 
 
 def fsdp_group_flat(g: Group) -> tuple:
-    """(flat, mixed shard-side vectors, mixed arena-side vectors) of a plan:
-    whether its copy-out, fused reduce-scatter and fused update take the flat
-    path, and how many of its vectors go element by element."""
+    """(flat, flat_copy_out, mixed shard-side vectors, mixed arena-side
+    vectors) of a plan: whether its fused reduce-scatter and fused update take
+    the flat path, whether its copy-out does, and how many vectors of each
+    side go element by element."""
     f = ctypes.c_int32()
     ms = ctypes.c_int64()
     ma = ctypes.c_int64()
     _check(_lib.fsdp_group_flat(g.handle, ctypes.byref(f), ctypes.byref(ms), ctypes.byref(ma)),
            "fsdp_group_flat")
-    return bool(f.value), ms.value, ma.value
+    return bool(f.value & 1), bool(f.value & 2), ms.value, ma.value
 
 
 def _stream(stream, t: torch.Tensor):

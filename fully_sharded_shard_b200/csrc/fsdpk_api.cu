@@ -29,6 +29,7 @@ using fsdpk::Interval;
 using fsdpk::TileRange;
 using fsdpk::Unit;
 using fsdpk::FlatSeg;
+using fsdpk::kFlatCopyOutShare;
 using fsdpk::kFlatMaxElems;
 using fsdpk::kFlatMinUnits;
 using fsdpk::kFlatPad;
@@ -178,11 +179,13 @@ std::vector<int32_t> flat_codes(const std::vector<FlatSeg>& segs, int64_t end,
 // The flat path's tables, for a plan of all N ranks with at least
 // kFlatMinUnits short and pad units and both index spaces within the codes'
 // range; otherwise g->flat stays false.  Shard side: the real units (code
-// 2 * (arena_pos - shard_pos)) and the pad units over [N][S].  Arena side:
-// the real units (code 2 * (shard_pos - arena_pos)) over [P_arena], the
+// 2 * (arena_pos - shard_pos)) and the pad units over [N][S].  Arena side,
+// when the short runs hold enough of the elements for the flat copy-out: the
+// real units (code 2 * (shard_pos - arena_pos)) over [P_arena], the
 // alignment gaps between parameters as kFlatPad.
 void build_flat_maps(fsdp_group* g) {
     g->flat = false;
+    g->flat_copy_out = false;
     for (auto* v : {&g->smap, &g->amap, &g->smixq, &g->amixq, &g->smixc, &g->amixc}) v->clear();
     g->ssegs.clear();
     g->asegs.clear();
@@ -194,6 +197,8 @@ void build_flat_maps(fsdp_group* g) {
     std::vector<std::array<int64_t, 3>> sruns, aruns;
     sruns.reserve(g->units.size());
     aruns.reserve((size_t)g->n_real_units);
+    int64_t short_elems = 0;
+    for (int64_t k = g->n_long_units; k < g->n_real_units; ++k) short_elems += g->units[(size_t)k].len;
     for (const Unit& u : g->units) {
         if (u.is_pad) {
             sruns.push_back({u.shard_pos, u.len, kFlatPad});
@@ -203,10 +208,13 @@ void build_flat_maps(fsdp_group* g) {
         }
     }
     g->ssegs = flat_segments(std::move(sruns), LS);
-    g->asegs = flat_segments(std::move(aruns), g->P_arena);
     g->smap = flat_codes(g->ssegs, LS, &g->smixq, &g->smixc);
-    g->amap = flat_codes(g->asegs, g->P_arena, &g->amixq, &g->amixc);
     g->flat = true;
+    if (short_elems * kFlatCopyOutShare >= g->P) {
+        g->asegs = flat_segments(std::move(aruns), g->P_arena);
+        g->amap = flat_codes(g->asegs, g->P_arena, &g->amixq, &g->amixc);
+        g->flat_copy_out = true;
+    }
 }
 
 int build_rank_tables(fsdp_group* g, int64_t r0, int64_t r1) {
@@ -576,9 +584,15 @@ int64_t check_flat(const fsdp_group& g) {
     const bool want = g.L == g.N && n_small >= kFlatMinUnits && LS <= kFlatMaxElems &&
                       g.P_arena <= kFlatMaxElems;
     if (want != g.flat) return 1;
+    int64_t short_elems = 0;
+    for (int64_t k = g.n_long_units; k < g.n_real_units && k < (int64_t)g.units.size(); ++k)
+        short_elems += g.units[(size_t)k].len;
+    const bool want_copy_out = want && short_elems * kFlatCopyOutShare >= g.P;
+    if (want_copy_out != g.flat_copy_out) return 1;
+    const bool arena_empty = g.amap.empty() && g.amixq.empty() && g.amixc.empty() && g.asegs.empty();
     if (!g.flat)
-        return (g.smap.empty() && g.amap.empty() && g.smixq.empty() && g.amixq.empty() &&
-                g.smixc.empty() && g.amixc.empty() && g.ssegs.empty() && g.asegs.empty())
+        return (g.smap.empty() && g.smixq.empty() && g.smixc.empty() && g.ssegs.empty() &&
+                arena_empty)
                    ? 0
                    : 1;
     std::vector<std::array<int64_t, 3>> sruns, aruns;
@@ -587,8 +601,9 @@ int64_t check_flat(const fsdp_group& g) {
                          u.is_pad ? (int64_t)kFlatPad : 2 * (u.arena_pos - u.shard_pos)});
         if (!u.is_pad) aruns.push_back({u.arena_pos, u.len, -2 * (u.arena_pos - u.shard_pos)});
     }
-    return check_flat_space(g.ssegs, g.smap, g.smixq, g.smixc, sruns, LS) +
-           check_flat_space(g.asegs, g.amap, g.amixq, g.amixc, aruns, g.P_arena);
+    const int64_t bad = check_flat_space(g.ssegs, g.smap, g.smixq, g.smixc, sruns, LS);
+    if (!g.flat_copy_out) return bad + (arena_empty ? 0 : 1);
+    return bad + check_flat_space(g.asegs, g.amap, g.amixq, g.amixc, aruns, g.P_arena);
 }
 
 int64_t check_tables(const fsdp_group& g) {
@@ -703,7 +718,7 @@ int fsdp_group_check(fsdp_group_t g, int64_t* violations) {
 
 int fsdp_group_flat(fsdp_group_t g, int32_t* flat, int64_t* mixed_shard, int64_t* mixed_arena) {
     if (g == nullptr) return FSDP_EINVAL;
-    if (flat) *flat = g->flat ? 1 : 0;
+    if (flat) *flat = (g->flat ? 1 : 0) | (g->flat_copy_out ? 2 : 0);
     if (mixed_shard) *mixed_shard = (int64_t)g->smixq.size();
     if (mixed_arena) *mixed_arena = (int64_t)g->amixq.size();
     return FSDP_OK;

@@ -470,7 +470,7 @@ cudaError_t launch_copy_in(const fsdp_group& g, const float* master, uint16_t* a
 cudaError_t launch_copy_out(const fsdp_group& g, const uint16_t* ag, uint16_t* arena,
                             cudaStream_t st) {
     if (g.n_real_units == 0) return cudaSuccess;
-    if (g.flat) {
+    if (g.flat_copy_out) {
         const int64_t n_mixed = (int64_t)g.amixq.size();
         const int64_t mixed_ctas = flat_mixed_ctas(n_mixed);
         k_copy_out_flat<<<(unsigned)(flat_grid(g.P_arena) + mixed_ctas), kThreads, 0, st>>>(

@@ -43,6 +43,11 @@ constexpr int64_t kPackElems = 16384;
 //                       mixed vectors, a thread per element.
 // Codes are int32, so both index spaces stay below kFlatMaxElems.
 constexpr int64_t kFlatMinUnits = 2048;
+// The copy-out reads 2 B and writes 2 B per element, so a code's 0.5 B per
+// element weighs more there: it takes the flat path only when runs shorter
+// than kShortRun hold at least 1 / kFlatCopyOutShare of the real elements
+// (with mostly long runs the per-unit copy-out is the faster one).
+constexpr int64_t kFlatCopyOutShare = 10;
 constexpr int64_t kFlatMaxElems = (int64_t{1} << 30) - 64;
 constexpr int32_t kFlatPad = INT32_MIN;
 
@@ -133,7 +138,8 @@ struct fsdp_group {
     int64_t n_tiles = 0;                        // copy-in tiles over L*S
     // flat path (empty unless flat): codes of the shard-side vectors of
     // [L][S] and of the arena-side vectors of [P_arena], with their segments
-    bool flat = false;
+    bool flat = false;           // reduce-scatter and update
+    bool flat_copy_out = false;  // the copy-out too (amap, amixq, amixc)
     std::vector<int32_t> smap, amap;    // one code per vector
     std::vector<int32_t> smixq, amixq;  // the mixed vectors
     std::vector<int32_t> smixc, amixc;  // their elements' codes, 8 per vector

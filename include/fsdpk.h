@@ -165,11 +165,15 @@ FSDP_API int fsdp_group_check(fsdp_group_t group, int64_t* violations);
  * elements) takes the flat path in the bf16 copy-out, the fused
  * reduce-scatter and the bf16 fused update: fixed tiles of the index space,
  * one code per 8-element vector, instead of one work unit per (rank,
- * parameter) run -- the same results, bit for bit.  *flat receives 1 for
- * such a plan, else 0; *mixed_shard and *mixed_arena the vectors of the
- * [N][S] and of the arena index space that hold more than one run (or a run
- * and padding, or the ragged end), which go element by element (0 when not
- * flat).  Host only; any output pointer may be NULL.
+ * parameter) run -- the same results, bit for bit.  The copy-out takes it
+ * only when runs shorter than 1024 elements hold at least a tenth of the real
+ * elements (with mostly long runs the per-run copy-out is faster).  *flat
+ * receives bit 0 set for a plan whose reduce-scatter and update are flat,
+ * bit 1 for a flat copy-out, else 0; *mixed_shard and *mixed_arena the
+ * vectors of the [N][S] and of the arena index space that hold more than one
+ * run (or a run and padding, or the ragged end), which go element by element
+ * (0 where that side is not flat).  Host only; any output pointer may be
+ * NULL.
  * Errors: FSDP_EINVAL (NULL group). */
 FSDP_API int fsdp_group_flat(fsdp_group_t group, int32_t* flat, int64_t* mixed_shard,
                              int64_t* mixed_arena);

@@ -84,7 +84,7 @@ def shrink() -> dict:
     # a group of many small parameters (the flat path), the same last parameter
     shapes = [(3 + k % 23, 1 + k % 5) for k in range(800)] + [(16386,)]
     g = abi.fsdp_plan_group(shapes, N)
-    assert abi.fsdp_group_flat(g)[0]
+    assert abi.fsdp_group_flat(g)[:2] == (True, True)
     NS = N * g.S
     last = int(g.arena_off[-1]) + 16385          # the last real element of the arena
     words.zero_()

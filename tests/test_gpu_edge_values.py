@@ -166,9 +166,9 @@ def test_edge_values_through_the_flat_path(H, N):
     copy-out, fused reduce-scatter (all ops) and fused update."""
     from fully_sharded_shard_b200 import abi
     g = abi.fsdp_plan_group(FLAT_SHAPES, N)
-    flat, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
+    flat, flat_copy_out, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
     g.destroy()
-    assert flat and mixed_shard > 0 and mixed_arena > 0
+    assert flat and flat_copy_out and mixed_shard > 0 and mixed_arena > 0
     fi, gi = full_init(N, FLAT_SHAPES), grads_init(N, FLAT_SHAPES)
     wl = _wl(N, W.AVG, FLAT_SHAPES)
     H.run_group(wl, wl.groups[0], steps=2, ops=ALL_OPS, staged=False, full_init=fi,

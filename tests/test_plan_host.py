@@ -63,13 +63,13 @@ def test_flat_path_for_groups_of_many_small_parameters(abi):
     from fully_sharded_shard_b200 import workloads as W
     wl = W.small_params()
     g = abi.fsdp_plan_group_host(wl.groups[0].shapes, wl.N)
-    flat, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
-    assert flat and 0 < mixed_shard < wl.N * g.S // 8 // 20 and 0 < mixed_arena
+    flat, flat_copy_out, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
+    assert flat and flat_copy_out and 0 < mixed_shard < wl.N * g.S // 8 // 20 and 0 < mixed_arena
     assert abi.fsdp_group_check(g) == 0
     g.destroy()
     for wl in (W.llama_block(), W.uneven(), W.moe(), W.tiny_mlp()):
         g = abi.fsdp_plan_group_host(wl.groups[0].shapes, wl.N)
-        assert abi.fsdp_group_flat(g) == (False, 0, 0)
+        assert abi.fsdp_group_flat(g) == (False, False, 0, 0)
         g.destroy()
 
 
@@ -117,6 +117,9 @@ MUTANTS_FLAT = [
     ("flat path below its threshold",
      "n_small < kFlatMinUnits ||",
      "n_small < kFlatMinUnits / 4 ||"),
+    ("flat copy-out below its share of short runs",
+     "if (short_elems * kFlatCopyOutShare >= g->P) {",
+     "if (short_elems * kFlatCopyOutShare * 100 >= g->P) {"),
 ]
 
 MUTANTS = [
@@ -177,12 +180,15 @@ def test_group_check_reports_planted_mistakes(abi, tmp_path, name, old, new):
     # at N = 2 and 3
     shapes += [(1 + k % 13, 1 + k % 3) for k in range(150)]
     found = 0
-    for N in (2, 3, 4, 6):
-        _, arr = abi._descs(shapes)
-        h = ctypes.c_void_p()
-        assert L.fsdp_plan_group_host(arr, len(shapes), N, ctypes.byref(h)) == 0
-        v = ctypes.c_int64()
-        assert L.fsdp_group_check(h, ctypes.byref(v)) == 0
-        found += v.value
-        L.fsdp_destroy_group(h)
+    # the same with one large parameter: the flat reduce-scatter, the per-run
+    # copy-out (short runs under a tenth of the elements)
+    for sh in (shapes, shapes + [(400000, 1)]):
+        for N in (2, 3, 4, 6):
+            _, arr = abi._descs(sh)
+            h = ctypes.c_void_p()
+            assert L.fsdp_plan_group_host(arr, len(sh), N, ctypes.byref(h)) == 0
+            v = ctypes.c_int64()
+            assert L.fsdp_group_check(h, ctypes.byref(v)) == 0
+            found += v.value
+            L.fsdp_destroy_group(h)
     assert found > 0, f"planted mistake not reported: {name}"
