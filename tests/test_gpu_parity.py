@@ -511,7 +511,8 @@ def _group_step_case(H, wl, grp, steps, graph, full_init=None, grads_init=None):
     g.destroy()
 
 
-GROUP_STEP = SMALL + [W.tiny_mlp(), W.uneven(64), W.moe(64)]
+# + two groups of many small parameters (the flat kernels inside the one call)
+GROUP_STEP = SMALL + [W.tiny_mlp(), W.uneven(64), W.moe(64), FLAT[1], FLAT[4]]
 
 
 @pytest.mark.parametrize("wl", GROUP_STEP, ids=[w.name for w in GROUP_STEP])
