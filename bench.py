@@ -380,9 +380,11 @@ class Model:
                     e1.record(stream)
                     events[name].append((e0, e1))
 
-    def run_group(self, idx, stream, step, grads=None, events=None):
+    def run_group(self, idx, stream, step, grads=None, events=None, spacer=None):
         """Enqueue the four stages of group instance `idx` on `stream`.
-        events: optional dict stage -> list receiving (start, end) events."""
+        events: optional dict stage -> list receiving (start, end) events.
+        spacer: optional callable enqueued before each stage's start event
+        (outside the timed pair)."""
         import torch
         from fully_sharded_shard_b200 import abi
         from fully_sharded_shard_b200 import workloads as W
@@ -403,6 +405,8 @@ class Model:
             if events is None:
                 fn()
             else:
+                if spacer is not None:
+                    spacer()
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
@@ -410,11 +414,11 @@ class Model:
                 e1.record(stream)
                 events[name].append((e0, e1))
 
-    def step(self, stream, events=None):
+    def step(self, stream, events=None, spacer=None):
         """Enqueue one full step (every group, in order) on `stream`."""
         self.step_count += 1
         for idx in range(len(self.instances)):
-            self.run_group(idx, stream, self.step_count, events=events)
+            self.run_group(idx, stream, self.step_count, events=events, spacer=spacer)
 
     def step_two_streams(self, s_gather, s_update, events=None):
         """One full step on two streams, as FSDP2 splits communication from
@@ -510,12 +514,19 @@ def run_ours(args, wl, device, rank, ws):
     per_step = [a.elapsed_time(b) for a, b in zip([e_start] + marks[:-1], marks)]
     ms_median = max_over_ranks(float(statistics.median(per_step)), device)
 
-    # per-stage times: the same steps again with events around every launch
+    # per-stage times: the same steps again, one stream, events around every
+    # launch.  Before each start event a 256 MB buffer (twice the L2) is
+    # written: no stage reads what the previous one left in L2, and the GPU
+    # stays ahead of the host, so a short launch's time does not include the
+    # host's call overhead.
     events = {k: [] for k in ("copy_in", "copy_out", "rs_reduce", "adamw")}
     stage_steps = max(1, min(args.steps, 3))
-    for _ in range(stage_steps):
-        model.step(stream, events=events)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(stage_steps):
+            model.step(stream, events=events, spacer=flush.zero_)
     torch.cuda.synchronize(device)
+    del flush
     stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / stage_steps for k, v in events.items()}
 
     peak, peak_kind = hbm_peak()
@@ -601,7 +612,8 @@ def run_ours(args, wl, device, rank, ws):
             "bytes_per_step": model.bytes_per_step,
             "reduce_op": W.OP_NAMES[wl.op],
             "grad_pool_per_plan": args.grad_pool,
-            "l2": "inputs larger than L2 (every group's state >> 126 MB)",
+            "l2": "inputs larger than L2 (every group's state >> 126 MB); the per-stage pass "
+                  "writes 256 MB before each launch",
             "parallelism": f"{ws} GPU(s), each a full {wl.N}-virtual-rank replica",
             "schedule": "one stream" if args.one_stream else
                         "two streams: all-gather half / reduce-scatter + update half",
@@ -1643,7 +1655,7 @@ def main(argv=None):
     ap.add_argument("--no-staged", action="store_true")
     ap.add_argument("--one-stream", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--extra-workloads", default="uneven,moe",
+    ap.add_argument("--extra-workloads", default="uneven,moe,small_params",
                     help="comma-separated workloads timed after the headline one (per-stage "
                          "GB/s of the five-stage and the fused step); empty for none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
