@@ -73,6 +73,27 @@ def test_flat_path_for_groups_of_many_small_parameters(abi):
         g.destroy()
 
 
+def test_random_flat_plans_on_host(abi, oracle):
+    """Random groups of thousands of small parameters (with and without a
+    large one, N from 1 to 24): the flat tables pass the check and the layout
+    matches the oracle's."""
+    rng = np.random.default_rng(23)
+    seen = set()
+    for k in range(24):
+        N = int(rng.integers(1, 25))
+        count = int(rng.integers(2100 // N + 1, 2600))
+        shapes = [(int(rng.integers(0, 200)),) if rng.random() < 0.3 else
+                  (int(rng.integers(0, 120)), int(rng.integers(1, 20))) for _ in range(count)]
+        if k % 3 == 0:
+            shapes.insert(int(rng.integers(0, count)), (int(rng.integers(4000, 16000)), 1000))
+        g = abi.fsdp_plan_group_host(shapes, N)
+        flat, flat_copy_out, _, _ = abi.fsdp_group_flat(g)
+        seen.add((flat, flat_copy_out))
+        g.destroy()
+        _compare(abi, oracle, shapes, N)
+    assert (True, True) in seen and (True, False) in seen
+
+
 def test_data_calls_refuse_a_host_plan(abi):
     L = abi.lib()
     g = abi.fsdp_plan_group_host([(7, 3), (5,)], 2)
