@@ -21,6 +21,12 @@ Workload shapes follow the pages' examples:
 * ``llama7b`` -- 32 Llama-2-7B-shaped blocks plus the root group (embedding,
   final norm, LM head), N = 8.  The 7B figure is the 16 bytes/param example
   of the Sharded Training page's opening paragraph.
+* ``toy_llm`` -- the demo transformer of the DTensor guide's section
+  "End-to-End Implementation: Sharding a Transformer with PyTorch FSDP2"
+  (vocabulary 1000, hidden size 256, 4 blocks, each block its own group and
+  the embedding, final norm and LM head the root's), N = 8: its SwiGLU
+  projections [1364, 256] and [256, 682] do not divide into 8 row chunks of
+  equal size.
 
 Values: fp32 master parameters ~ N(0, 0.02) (tiny_mlp: U(-0.25, 0.25));
 per-rank bf16 gradients ~ N(0, sigma) with sigma = 1e-3 (tiny_mlp: 1), drawn in
@@ -86,6 +92,24 @@ def tiny_mlp() -> Workload:
     g = Group("root", [(32, 16), (32,), (4, 32), (4,)],
               ["0.weight", "0.bias", "2.weight", "2.bias"])
     return Workload("tiny_mlp", 2, [g], AVG, 0, "uniform", 0.25, 1.0, steps=3)
+
+
+def toy_llm() -> Workload:
+    """The DTensor guide's demo model, SimpleLLM(vocab_size=1000, hidden_dim=256,
+    num_layers=4): per block two LayerNorms (weight and bias), the fused QKV
+    projection [3 * 256, 256], the output projection [256, 256], the SwiGLU
+    gate/up projection [2 * int(4 * 256 * 2 / 3), 256] = [1364, 256] and the
+    down projection [256, 682], all without biases; the root group holds the
+    embedding [1000, 256], the final LayerNorm and the output (LM head)
+    projection [1000, 256]."""
+    d, ffn, vocab = 256, int(4 * 256 * 2 / 3), 1000
+    blk = Group("block", [(d,), (d,), (3 * d, d), (d, d), (d,), (d,), (2 * ffn, d), (d, ffn)],
+                ["norm1.weight", "norm1.bias", "qkv_proj.weight", "out_proj.weight",
+                 "norm2.weight", "norm2.bias", "mlp_gate_up.weight", "mlp_down.weight"])
+    blk.repeat = 4
+    root = Group("root", [(vocab, d), (d,), (d,), (vocab, d)],
+                 ["tok_embeddings.weight", "norm.weight", "norm.bias", "output.weight"])
+    return Workload("toy_llm", 8, [blk, root], AVG, 3, "normal", 0.02, 1e-3)
 
 
 def llama_block(scale: int = 1) -> Workload:
@@ -169,6 +193,7 @@ def by_name(name: str) -> Workload:
         "moe": moe,
         "llama7b": llama7b,
         "small_params": small_params,
+        "toy_llm": toy_llm,
     }
     if name in table:
         return table[name]()

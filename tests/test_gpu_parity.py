@@ -68,6 +68,18 @@ def test_scaled_workloads(H, wl):
         H.run_group(wl, g, steps=2, ops=ALL_OPS, staged=True)
 
 
+def test_toy_llm_block_and_root(H):
+    """The DTensor guide's demo transformer at N = 8 (SwiGLU rows 1364 and
+    256 x 682: the gate/up projection pads its last rank): every stage and
+    op, the fused update and the FP8 all-gather, for the block and the root
+    group."""
+    wl = W.toy_llm()
+    for g in wl.groups:
+        H.run_group(wl, g, steps=2, ops=ALL_OPS, staged=True)
+        H.run_group_fused(wl, g, steps=2)
+        H.run_group_fp8(wl, g)
+
+
 FULL = [W.tiny_mlp(), W.llama_block(), W.uneven(), W.moe()]
 
 

@@ -31,7 +31,7 @@ def _compare(abi, oracle, shapes, N):
 def test_workload_plans_on_host(abi, oracle):
     from fully_sharded_shard_b200 import workloads as W
     for wl in (W.tiny_mlp(), W.llama_block(), W.uneven(), W.moe(), W.llama7b(),
-               W.small_params()):
+               W.small_params(), W.toy_llm()):
         for grp in wl.groups:
             _compare(abi, oracle, grp.shapes, wl.N)
 
