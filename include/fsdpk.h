@@ -160,7 +160,10 @@ FSDP_API int fsdp_plan_group_host(const fsdp_param_desc* params, int32_t n_param
  * builds).  Host only. */
 FSDP_API int fsdp_group_check(fsdp_group_t group, int64_t* violations);
 
-/* Which work tables the data calls of a plan use.  A group of many small
+/* Which work tables the data calls of a plan use -- an inspection of the
+ * group plan of "Sharded Training: FSDP2, DTensor, Tensor and Pipeline
+ * Parallelism", fully_shard paragraph (one group per call, rows chunked and
+ * padded per rank); the pages describe no such choice.  A group of many small
  * parameters (at least 2048 short and pad runs, both index spaces below 2^30
  * elements) takes the flat path in the bf16 copy-out, the fused
  * reduce-scatter and the bf16 fused update: fixed tiles of the index space,
