@@ -73,6 +73,23 @@ def test_flat_path_for_groups_of_many_small_parameters(abi):
         g.destroy()
 
 
+def test_flat_path_thresholds_on_host(abi):
+    """The flat path starts at 2048 short and pad runs, and stops where an
+    index space exceeds the codes' range (2^30 elements)."""
+    for n, want in ((2047, False), (2048, True)):
+        g = abi.fsdp_plan_group_host([(1,)] * n, 1)        # one 1-element run each
+        flat, flat_copy_out, mixed_shard, mixed_arena = abi.fsdp_group_flat(g)
+        assert (flat, flat_copy_out) == (want, want)
+        if want:   # every vector holds several runs (shard side) or a run and gaps (arena)
+            assert (mixed_shard, mixed_arena) == (n // 8, n)
+        assert abi.fsdp_group_check(g) == 0
+        g.destroy()
+    g = abi.fsdp_plan_group_host([(3,)] * 2100 + [((1 << 30) // 8 + 8, 8)], 1)
+    assert g.S > (1 << 30) and abi.fsdp_group_flat(g) == (False, False, 0, 0)
+    assert abi.fsdp_group_check(g) == 0
+    g.destroy()
+
+
 def test_random_flat_plans_on_host(abi, oracle):
     """Random groups of thousands of small parameters (with and without a
     large one, N from 1 to 24): the flat tables pass the check and the layout
